@@ -1,0 +1,443 @@
+"""Benchmark of the KDA hot path on B200: one JSON line per run.
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+  1. kda_prefill  - chunked prefill of 8192 tokens x 64 heads, d_k = d_v = 128,
+                    chunk 64, bf16 q/k/v/o, fp32 state, snapshots every 256 tokens;
+  2. kda_decode   - one token for 512 sequences x 64 heads against fp32 states;
+  3. kda_verify   - 1..8 draft tokens per sequence (seeded uniform), writing the
+                    state after every token;
+  4. kda_snapshot - commit the state of each sequence's last accepted token
+                    (seeded acceptance) into its live slot.
+Inputs are seeded (synth.py) and resident in HBM before timing; every input set
+is larger than the 126 MB L2 (prefill 0.94 GB, decode 2.1 GB, verify 12 GB), so
+no L2 flush is needed between steps.
+
+`value` is prefill tokens per second (tokens of all 64 heads), summed over
+ranks; the decode and verify rows are reported in state-steps per second (one
+(sequence, head) state advanced by one token) under "components". Times are
+CUDA events on the launching stream; for N > 1 the max over ranks. With
+--gpus N > 1 the ranks are independent replicas (the layer has no exchange).
+
+--impl reference times the fp64 CPU oracle (the test oracle, untuned) on a
+bounded sample of the same prefill workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+from pathlib import Path
+
+import numpy as np
+import torch
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+import synth  # noqa: E402
+
+METRIC = "KDA prefill tok/s + decode state-steps/s on 1 B200; % of TC/HBM roofline"
+H, D, C = 64, 128, 64
+PREFILL_T = 8192
+SNAP = 256
+N_SEQ = 512
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+# ----------------------------------------------------------------------------
+def load_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {**FALLBACK, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in sorted((ROOT / "hybrid_linear_attention_04_b200" / "csrc").glob("*")):
+        h.update(f.read_bytes())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    p = ROOT / "profiles" / "dram_traffic.json"
+    if not p.exists():
+        return {}
+    d = json.loads(p.read_text())
+    if d.get("csrc_hash") != kernel_source_hash():
+        return {}
+    return d.get("kernels", {})
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = Path(f"/tmp/kda_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not self.path.exists():
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.path.read_text().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() in ("active", "1"):
+                    reasons.add(n)
+        self.path.unlink(missing_ok=True)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+def prefill_bytes(T, n_seq, n_snap, with_state_in):
+    per_tok = H * (3 * D * 2 + D * 2 + D * 4 + 4)     # q,k,v,o bf16 + g fp32 + beta
+    state = H * D * D * 4
+    return T * per_tok + (n_snap + n_seq * (2 if with_state_in else 1)) * state
+
+
+def prefill_flops(T):
+    # chunk form per token-head, d_k = d_v = d, chunk C (causal halves):
+    # 6 d^2 (S_0 products and state update) + C (3 d_k + 2 d_v) + C^2 / 3
+    return T * H * (6 * D * D + C * (3 * D + 2 * D) + C * C / 3)
+
+
+def decode_bytes(n):
+    return n * H * (2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 2)
+
+
+def verify_bytes(n_seq, n_tok):
+    return n_seq * H * D * D * 4 + n_tok * H * (D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 2)
+
+
+def commit_bytes(n):
+    return n * H * D * D * 4 * 2
+
+
+class Workload:
+    """The serving-step workload, resident on one device."""
+
+    def __init__(self, dev):
+        from hybrid_linear_attention_04_b200 import kda as K
+        self.K = K
+        self.dev = dev
+        x = synth.token_inputs(1001, PREFILL_T, H, D, D, io="bf16")
+        self.host_prefill = x
+        self.p = {k: v.to(dev) for k, v in x.items()}
+        self.cu = np.array([0, PREFILL_T], dtype=np.int32)
+        offs, _ = K.kda_snapshot_plan(self.cu, None, SNAP)
+        self.n_snap = int(offs[-1])
+        self.p_o = torch.empty((PREFILL_T, H, D), dtype=torch.bfloat16, device=dev)
+        self.p_sout = torch.empty((1, H, D, D), device=dev)
+        self.p_snaps = torch.empty((self.n_snap, H, D, D), device=dev)
+        # decode + verify
+        self.pool = synth.states(1002, N_SEQ, H, D, D, std=0.1).to(dev)
+        self.slots = torch.arange(N_SEQ, dtype=torch.int32, device=dev)
+        y = synth.token_inputs(1002, N_SEQ, H, D, D, io="bf16")
+        self.d = {k: v.to(dev) for k, v in y.items()}
+        self.d_o = torch.empty((N_SEQ, H, D), dtype=torch.bfloat16, device=dev)
+        lens = synth.draft_lengths(1002, N_SEQ, 1, 8)
+        self.cu_draft = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+        self.n_tok = int(self.cu_draft[-1])
+        z = synth.token_inputs(1002, self.n_tok, H, D, D, io="bf16", t0=N_SEQ)
+        self.v = {k: v.to(dev) for k, v in z.items()}
+        self.v_o = torch.empty((self.n_tok, H, D), dtype=torch.bfloat16, device=dev)
+        self.ts = torch.empty((self.n_tok, H, D, D), device=dev)
+        acc = synth.randint(1002, "misc", N_SEQ, 0, 8)
+        src, dst = [], []
+        for s in range(N_SEQ):
+            a = min(acc[s], lens[s])
+            if a > 0:
+                src.append(int(self.cu_draft[s]) + a - 1)
+                dst.append(s)
+        self.c_src = torch.tensor(src, dtype=torch.int64, device=dev)
+        self.c_dst = torch.tensor(dst, dtype=torch.int64, device=dev)
+        self.n_commit = len(src)
+
+    def prefill(self):
+        K, p = self.K, self.p
+        K.kda_prefill(p["q"], p["k"], p["v"], p["g"], p["beta"], self.cu, self.p_o,
+                      state_out=self.p_sout, snap_interval=SNAP, snapshots=self.p_snaps, chunk=C)
+
+    def decode(self):
+        d = self.d
+        self.K.kda_decode(d["q"], d["k"], d["v"], d["g"], d["beta"], self.slots, self.pool, self.d_o)
+
+    def verify(self):
+        v = self.v
+        self.K.kda_verify(v["q"], v["k"], v["v"], v["g"], v["beta"], self.cu_draft, self.slots,
+                          self.pool, self.ts, self.v_o)
+
+    def commit(self):
+        self.K.kda_snapshot(self.c_src, self.c_dst, self.ts, self.pool)
+
+
+def dist_setup(n_gpus):
+    if n_gpus > 1 or int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        import datetime
+        import torch.distributed as dist
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        return dist, dist.get_rank(), dist.get_world_size(), local
+    return None, 0, 1, 0
+
+
+def max_over_ranks(dist, x, dev):
+    if dist is None:
+        return x
+    t = torch.tensor(x, dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def cpu_baseline_prefill(tokens, heads):
+    """The oracle, as it stands, on `tokens` x `heads` of the prefill workload."""
+    from oracle import native
+    x = synth.token_inputs(1001, tokens, H, D, D, io="bf16")
+    sl = {k: v[:, :heads].contiguous() for k, v in x.items()}
+    native.load()
+    t0 = time.perf_counter()
+    native.oracle_sequence(sl["q"], sl["k"], sl["v"], sl["g"], sl["beta"], None, None, 0, SNAP,
+                           out_dtype=np.float32)
+    dt = time.perf_counter() - t0
+    return dt, native.max_threads()
+
+
+# ----------------------------------------------------------------------------
+def run_ours(args):
+    dist, rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from hybrid_linear_attention_04_b200 import build as kbuild
+    if rank == 0:
+        kbuild.build()
+    if dist is not None:
+        dist.barrier()
+    from hybrid_linear_attention_04_b200 import kda as K
+    wl = Workload(dev)
+    stream = torch.cuda.current_stream(dev)
+    comps = ["prefill", "decode", "verify", "commit"]
+    fns = [wl.prefill, wl.decode, wl.verify, wl.commit]
+
+    def step(ev=None):
+        for i, f in enumerate(fns):
+            if ev is not None:
+                ev[i][0].record(stream)
+            f()
+            if ev is not None:
+                ev[i][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    st = K.kda_check_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {K.kda_status_string(st)} after warm-up")
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in comps]
+           for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = K.kda_launch_count()
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        t_start.record(stream)
+        for s in range(args.steps):
+            step(evs[s])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    launches = K.kda_launch_count() - launches0
+    if dist is not None:
+        dist.barrier()
+    st = K.kda_check_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {K.kda_status_string(st)} after timing")
+    total_ms = t_start.elapsed_time(t_end)
+    comp_ms = [sum(evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(args.steps)) / args.steps
+               for i in range(len(comps))]
+    vals = max_over_ranks(dist, [total_ms] + comp_ms, dev)
+    total_ms, comp_ms = vals[0], vals[1:]
+
+    # end to end through the same C-ABI call, host buffers: H2D of the step's
+    # prefill inputs from pinned memory, the call, D2H of its outputs
+    hp = {k: v.pin_memory() for k, v in wl.host_prefill.items()}
+    ho = torch.empty(wl.p_o.shape, dtype=wl.p_o.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in hp.values())
+    d2h = ho.numel() * ho.element_size()
+
+    def e2e_step():
+        for k in hp:
+            wl.p[k].copy_(hp[k], non_blocking=True)
+        wl.prefill()
+        ho.copy_(wl.p_o, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(dist, [e0.elapsed_time(e1) / args.steps], dev)[0]
+
+    result = None
+    if rank == 0:
+        peaks = load_peaks()
+        hbm = peaks["hbm_gbs"]
+        comp = {}
+        units = {
+            "prefill": (PREFILL_T, "tok/s", prefill_bytes(PREFILL_T, 1, wl.n_snap, False)),
+            "decode": (N_SEQ * H, "state-steps/s", decode_bytes(N_SEQ)),
+            "verify": (wl.n_tok * H, "state-steps/s", verify_bytes(N_SEQ, wl.n_tok)),
+            "commit": (wl.n_commit, "states/s", commit_bytes(wl.n_commit)),
+        }
+        traffic = ncu_traffic()
+        for name, ms in zip(comps, comp_ms):
+            n_units, unit, byts = units[name]
+            gbs = byts / (ms * 1e-3) / 1e9
+            comp[name] = {"ms": round(ms, 4), "value": world * n_units / (ms * 1e-3), "unit": unit,
+                          "algorithmic_bytes": byts, "achieved_gbs": round(gbs, 1),
+                          "hbm_frac": round(gbs / hbm, 4)}
+        pf = prefill_flops(PREFILL_T)
+        comp["prefill"]["algorithmic_flops"] = pf
+        comp["prefill"]["tc_frac"] = round(pf / (comp_ms[0] * 1e-3) / (peaks["bf16_tflops"] * 1e12), 4)
+        dom = max(comps, key=lambda c: comp[c]["ms"])
+        kname = {"prefill": "prefill", "decode": "decode_kernel", "verify": "verify_kernel",
+                 "commit": "snapshot_kernel"}[dom]
+        tr = traffic.get(kname)
+        roof = {"bound": "hbm", "kernel": kname, "achieved": comp[dom]["achieved_gbs"],
+                "peak": hbm, "unit": "GB/s", "frac": comp[dom]["hbm_frac"],
+                "traffic": tr, "peak_source": peaks["source"]}
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            tok = args.cpu_tokens
+            dt, cores = cpu_baseline_prefill(tok, H)
+            cpu = {"value": tok / dt, "unit": "tok/s", "cores": cores, "kind": "oracle",
+                   "sample": f"fp64 token recurrence, first {tok} tokens x {H} heads of the "
+                             f"prefill workload ({dt:.1f} s)"}
+        clocks = clk.summary()
+        result = {
+            "metric": METRIC,
+            "value": world * PREFILL_T / (comp_ms[0] * 1e-3),
+            "unit": "tok/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "prefill 8192 tok x 64 heads (d=128, chunk 64, snapshots /256)"
+                                   " + decode/verify/commit 512 seq x 64 heads (drafts 1..8)",
+                       "global_batch": world * (1 + N_SEQ), "seq_len": PREFILL_T,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (no flush)"},
+            "components": comp,
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * PREFILL_T / (e2e_ms * 1e-3), "unit": "tok/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "scope": "prefill call with pinned-host inputs and outputs"},
+            "gpu_launches": launches,
+            "clocks": clocks,
+        }
+        print(json.dumps(result), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return None
+    tok = args.ref_tokens
+    for _ in range(args.warmup):
+        cpu_baseline_prefill(tok, H)
+    times, cores = [], 1
+    for _ in range(args.steps):
+        dt, cores = cpu_baseline_prefill(tok, H)
+        times.append(dt)
+    total = sum(times)
+    val = args.steps * tok / total
+    sample = f"fp64 token recurrence (the test oracle), first {tok} tokens x {H} heads of the " \
+             f"prefill workload per step"
+    result = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "tok/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "prefill 8192 tok x 64 heads (d=128, chunk 64, snapshots /256)"
+                               " + decode/verify/commit 512 seq x 64 heads (drafts 1..8)",
+                   "global_batch": 1 + N_SEQ, "seq_len": PREFILL_T, "parallelism": "cpu"},
+        "cpu_baseline": {"value": val, "unit": "tok/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": val, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(result), flush=True)
+    return result
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-tokens", type=int, default=2048)
+    ap.add_argument("--ref-tokens", type=int, default=512)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,227 @@
+// KDA decode and speculative-verify kernels (sm_100a, SIMT, HBM-bound).
+//
+// One CTA owns one (sequence, head) state S [D x D] fp32 (d_v contiguous) and
+// streams it through registers once: 128-bit loads, gate, rank-1 delta
+// correction and output read in one pass, 128-bit stores.
+//
+// Per token (Kimi K3 technical FAQ, "What is KDA": delta rule with a
+// per-channel forget gate; standard gated-delta form):
+//     S' = Diag(alpha) S                    alpha = exp(g), per key channel
+//     x  = S'^T k,   y = S'^T q             (one pass, shared reduction over d_k)
+//     w  = beta (v - x)
+//     S  = S' + k w^T
+//     o  = scale (y + (k . q) w)            (= scale * S^T q, read after update)
+//
+// Thread map: thread t owns column group cg = t % (D/4) (four adjacent d_v
+// columns, one float4) and rows rs, rs + RS, ... with rs = t / (D/4). Column
+// sums over d_k reduce first across lanes of a warp that share cg (shuffles),
+// then across warps through shared memory in a fixed order (deterministic).
+// Decode and verify run the same step function, so verify's state after its
+// j-th token is bit-identical to j decode calls.
+#pragma once
+#include "common.cuh"
+
+namespace kda {
+
+constexpr int kMaxSeqsPerLaunch = KDA_SEQS_PER_LAUNCH;
+
+template <int D> struct DecodeShape {
+    static constexpr int NT = D == 128 ? 256 : (D == 64 ? 128 : 64);  // threads per CTA
+    static constexpr int CG = D / 4;                                    // column groups
+    static constexpr int RS = NT / CG;                                  // row slots
+    static constexpr int R = D / RS;                                    // rows per thread
+    static constexpr int NW = NT / 32;                                  // warps
+    static_assert(CG <= 32 && 32 % CG == 0, "column groups must tile a warp");
+};
+
+struct DecodeParams {
+    const void *q, *k, *v;
+    const float *g, *beta;
+    const int32_t *slots;
+    float *pool;             // decode: read/write; verify: read-only source
+    float *token_states;     // verify only
+    void *o;
+    int32_t n_seq, H, n_slots;
+    float scale;
+    int32_t tok0[kMaxSeqsPerLaunch + 1];  // verify: packed token offsets (relative)
+    int64_t tok_base;                     // verify: absolute offset of tok0[0]
+};
+
+// Per-token vectors staged in shared memory.
+template <int D> struct TokVec {
+    float k[D], q[D], a[D], v[D];
+    float beta, kq;
+};
+
+template <int D, typename TIO>
+__device__ __forceinline__ void load_token(TokVec<D> &tv, const DecodeParams &p, int64_t row) {
+    // row = token * H + head; D threads (or fewer, looping) fill the vectors.
+    const TIO *q = static_cast<const TIO *>(p.q) + row * D;
+    const TIO *k = static_cast<const TIO *>(p.k) + row * D;
+    const TIO *v = static_cast<const TIO *>(p.v) + row * D;
+    const float *g = p.g + row * D;
+    for (int i = threadIdx.x; i < D; i += blockDim.x) {
+        tv.k[i] = IO<TIO>::ld(k + i);
+        tv.q[i] = IO<TIO>::ld(q + i);
+        tv.v[i] = IO<TIO>::ld(v + i);
+        tv.a[i] = expf(g[i]);
+    }
+    if (threadIdx.x == 0) tv.beta = p.beta[row];
+}
+
+// k . q for a staged token, by one warp, fixed reduction order.
+template <int D>
+__device__ __forceinline__ void token_kq(TokVec<D> &tv) {
+    int lane = threadIdx.x & 31;
+    float s = 0.f;
+#pragma unroll
+    for (int i = lane; i < D; i += 32) s = fmaf(tv.k[i], tv.q[i], s);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (lane == 0) tv.kq = s;
+}
+
+// One recurrence step on the register-resident state. red: [NW][2][D] scratch
+// in shared memory; the caller separates reuses of `red` by a barrier.
+template <int D>
+__device__ __forceinline__ float4 kda_step(float4 (&st)[DecodeShape<D>::R], const TokVec<D> &tv,
+                                           float *red, float scale) {
+    using Sh = DecodeShape<D>;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int cg = t % Sh::CG, rs = t / Sh::CG;
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
+#pragma unroll
+    for (int m = 0; m < Sh::R; ++m) {
+        const int r = rs + Sh::RS * m;
+        const float a = tv.a[r], kr = tv.k[r], qr = tv.q[r];
+        float4 s = st[m];
+        s.x *= a; s.y *= a; s.z *= a; s.w *= a;
+        st[m] = s;
+        x.x = fmaf(kr, s.x, x.x); x.y = fmaf(kr, s.y, x.y);
+        x.z = fmaf(kr, s.z, x.z); x.w = fmaf(kr, s.w, x.w);
+        y.x = fmaf(qr, s.x, y.x); y.y = fmaf(qr, s.y, y.y);
+        y.z = fmaf(qr, s.z, y.z); y.w = fmaf(qr, s.w, y.w);
+    }
+#pragma unroll
+    for (int off = Sh::CG; off < 32; off <<= 1) {
+        x.x += __shfl_xor_sync(0xffffffffu, x.x, off);
+        x.y += __shfl_xor_sync(0xffffffffu, x.y, off);
+        x.z += __shfl_xor_sync(0xffffffffu, x.z, off);
+        x.w += __shfl_xor_sync(0xffffffffu, x.w, off);
+        y.x += __shfl_xor_sync(0xffffffffu, y.x, off);
+        y.y += __shfl_xor_sync(0xffffffffu, y.y, off);
+        y.z += __shfl_xor_sync(0xffffffffu, y.z, off);
+        y.w += __shfl_xor_sync(0xffffffffu, y.w, off);
+    }
+    if (lane < Sh::CG) {
+        *reinterpret_cast<float4 *>(red + (warp * 2 + 0) * D + cg * 4) = x;
+        *reinterpret_cast<float4 *>(red + (warp * 2 + 1) * D + cg * 4) = y;
+    }
+    __syncthreads();
+    float4 X = make_float4(0.f, 0.f, 0.f, 0.f), Y = X;
+#pragma unroll
+    for (int w = 0; w < Sh::NW; ++w) {
+        float4 a = *reinterpret_cast<const float4 *>(red + (w * 2 + 0) * D + cg * 4);
+        float4 b = *reinterpret_cast<const float4 *>(red + (w * 2 + 1) * D + cg * 4);
+        X.x += a.x; X.y += a.y; X.z += a.z; X.w += a.w;
+        Y.x += b.x; Y.y += b.y; Y.z += b.z; Y.w += b.w;
+    }
+    const float4 vv = *reinterpret_cast<const float4 *>(tv.v + cg * 4);
+    float4 wv;
+    wv.x = tv.beta * (vv.x - X.x); wv.y = tv.beta * (vv.y - X.y);
+    wv.z = tv.beta * (vv.z - X.z); wv.w = tv.beta * (vv.w - X.w);
+#pragma unroll
+    for (int m = 0; m < Sh::R; ++m) {
+        const float kr = tv.k[rs + Sh::RS * m];
+        float4 s = st[m];
+        s.x = fmaf(kr, wv.x, s.x); s.y = fmaf(kr, wv.y, s.y);
+        s.z = fmaf(kr, wv.z, s.z); s.w = fmaf(kr, wv.w, s.w);
+        st[m] = s;
+    }
+    float4 o;
+    o.x = scale * fmaf(tv.kq, wv.x, Y.x); o.y = scale * fmaf(tv.kq, wv.y, Y.y);
+    o.z = scale * fmaf(tv.kq, wv.z, Y.z); o.w = scale * fmaf(tv.kq, wv.w, Y.w);
+    return o;
+}
+
+template <int D, typename TIO>
+__global__ void __launch_bounds__(DecodeShape<D>::NT)
+decode_kernel(const __grid_constant__ DecodeParams p) {
+    using Sh = DecodeShape<D>;
+    __shared__ TokVec<D> tv;
+    __shared__ __align__(16) float red[Sh::NW * 2 * D];
+    const int s = blockIdx.x / p.H, h = blockIdx.x % p.H;
+    const int32_t slot = p.slots[s];
+    if (slot < 0 || slot >= p.n_slots) {
+        if (threadIdx.x == 0) record_status(KDA_ERR_RANGE);
+        return;
+    }
+    const int t = threadIdx.x, cg = t % Sh::CG, rs = t / Sh::CG;
+    float *S = p.pool + ((int64_t)slot * p.H + h) * (int64_t)D * D;
+    float4 st[Sh::R];
+#pragma unroll
+    for (int m = 0; m < Sh::R; ++m) {
+        const float *src = S + (int64_t)(rs + Sh::RS * m) * D + cg * 4;
+        asm volatile("ld.global.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
+                     : "=f"(st[m].x), "=f"(st[m].y), "=f"(st[m].z), "=f"(st[m].w)
+                     : "l"(src));
+    }
+    const int64_t row = (int64_t)s * p.H + h;
+    load_token<D, TIO>(tv, p, row);
+    __syncthreads();
+    if (t < 32) token_kq<D>(tv);
+    __syncthreads();
+    const float4 o = kda_step<D>(st, tv, red, p.scale);
+#pragma unroll
+    for (int m = 0; m < Sh::R; ++m)
+        st_stream(S + (int64_t)(rs + Sh::RS * m) * D + cg * 4, st[m]);
+    if (rs == 0) IO<TIO>::st4(static_cast<TIO *>(p.o) + row * D + cg * 4, o);
+}
+
+// Verify: tokens are processed in batches of kTokBatch staged in shared memory.
+constexpr int kTokBatch = 8;
+
+template <int D, typename TIO>
+__global__ void __launch_bounds__(DecodeShape<D>::NT)
+verify_kernel(const __grid_constant__ DecodeParams p) {
+    using Sh = DecodeShape<D>;
+    __shared__ TokVec<D> tv[kTokBatch];
+    __shared__ __align__(16) float red[2][Sh::NW * 2 * D];
+    const int s = blockIdx.x / p.H, h = blockIdx.x % p.H;
+    const int32_t slot = p.slots[s];
+    if (slot < 0 || slot >= p.n_slots) {
+        if (threadIdx.x == 0) record_status(KDA_ERR_RANGE);
+        return;
+    }
+    const int n_tok = p.tok0[s + 1] - p.tok0[s];
+    const int64_t tok_first = p.tok_base + p.tok0[s];
+    const int t = threadIdx.x, cg = t % Sh::CG, rs = t / Sh::CG, warp = t >> 5;
+    const float *S = p.pool + ((int64_t)slot * p.H + h) * (int64_t)D * D;
+    float4 st[Sh::R];
+#pragma unroll
+    for (int m = 0; m < Sh::R; ++m) st[m] = ld_stream(S + (int64_t)(rs + Sh::RS * m) * D + cg * 4);
+    int parity = 0;
+    for (int j0 = 0; j0 < n_tok; j0 += kTokBatch) {
+        const int nb = min(kTokBatch, n_tok - j0);
+        __syncthreads();  // previous batch's vectors are no longer read
+        for (int j = 0; j < nb; ++j)
+            load_token<D, TIO>(tv[j], p, (tok_first + j0 + j) * p.H + h);
+        __syncthreads();
+        if (warp < nb) token_kq<D>(tv[warp]);
+        for (int j = Sh::NW; j < nb; ++j)
+            if (warp == 0) token_kq<D>(tv[j]);
+        __syncthreads();
+        for (int j = 0; j < nb; ++j) {
+            const float4 o = kda_step<D>(st, tv[j], red[parity], p.scale);
+            parity ^= 1;
+            const int64_t row = (tok_first + j0 + j) * p.H + h;
+            float *dst = p.token_states + row * (int64_t)D * D;
+#pragma unroll
+            for (int m = 0; m < Sh::R; ++m)
+                st_stream(dst + (int64_t)(rs + Sh::RS * m) * D + cg * 4, st[m]);
+            if (rs == 0) IO<TIO>::st4(static_cast<TIO *>(p.o) + row * D + cg * 4, o);
+        }
+    }
+}
+
+}  // namespace kda

@@ -1,0 +1,343 @@
+// libkda: the C ABI of the KDA hot path (declared in include/kda.h).
+//
+// Host side: argument validation (every error returns before any launch), the
+// ragged-batch plan (snapshot rows, longest-first sequence order, launches of
+// at most KDA_SEQS_PER_LAUNCH sequences), kernel dispatch and the device
+// status word. All kernels of the library live in this translation unit.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <numeric>
+#include <vector>
+
+#include "common.cuh"
+#include "decode.cuh"
+#include "prefill_simt.cuh"
+#include "prefill_tc.cuh"
+#include "snapshot.cuh"
+
+namespace kda {
+
+static std::atomic<int64_t> g_launches{0};
+static std::atomic<int32_t> g_fail_next{0};
+
+// Count a launch, or simulate a failed one (failure-injection hook).
+static bool launch_gate() {
+    int32_t n = g_fail_next.load();
+    while (n > 0) {
+        if (g_fail_next.compare_exchange_weak(n, n - 1)) return false;
+    }
+    g_launches.fetch_add(1);
+    return true;
+}
+
+static kda_status last_launch_status() {
+    return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static kda_status check_dims(const kda_dims *d, bool need_chunk) {
+    if (!d) return KDA_ERR_INVALID;
+    if (d->H < 1 || d->dk < 1 || d->dv < 1) return KDA_ERR_INVALID;
+    if (d->io != KDA_IO_BF16 && d->io != KDA_IO_FP32) return KDA_ERR_INVALID;
+    if (!std::isfinite(d->scale)) return KDA_ERR_INVALID;
+    if (d->dk != d->dv) return KDA_ERR_UNSUPPORTED;
+    if (d->dk != 32 && d->dk != 64 && d->dk != 128) return KDA_ERR_UNSUPPORTED;
+    if (need_chunk && d->chunk != 16 && d->chunk != 32 && d->chunk != 64) return KDA_ERR_UNSUPPORTED;
+    return KDA_OK;
+}
+
+static float eff_scale(const kda_dims *d) {
+    return d->scale != 0.f ? d->scale : 1.0f / std::sqrt((float)d->dk);
+}
+
+// ---------------------------------------------------------------- decode ----
+template <int D, typename TIO>
+static kda_status launch_decode(DecodeParams &p, int n_blocks, cudaStream_t st, bool verify) {
+    if (!launch_gate()) return KDA_ERR_CUDA;
+    if (verify)
+        verify_kernel<D, TIO><<<n_blocks, DecodeShape<D>::NT, 0, st>>>(p);
+    else
+        decode_kernel<D, TIO><<<n_blocks, DecodeShape<D>::NT, 0, st>>>(p);
+    return last_launch_status();
+}
+
+template <typename TIO>
+static kda_status dispatch_decode(int D, DecodeParams &p, int n_blocks, cudaStream_t st, bool verify) {
+    switch (D) {
+    case 32: return launch_decode<32, TIO>(p, n_blocks, st, verify);
+    case 64: return launch_decode<64, TIO>(p, n_blocks, st, verify);
+    case 128: return launch_decode<128, TIO>(p, n_blocks, st, verify);
+    }
+    return KDA_ERR_UNSUPPORTED;
+}
+
+// --------------------------------------------------------------- prefill ----
+template <int D, int C, typename TIO>
+static kda_status launch_simt(const PrefillParams &p, cudaStream_t st) {
+    using Sh = SimtShape<D, C>;
+    static bool attr_done = false;
+    if (!attr_done) {
+        if (cudaFuncSetAttribute(prefill_simt_kernel<D, C, TIO>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)Sh::smem_bytes) != cudaSuccess)
+            return KDA_ERR_CUDA;
+        attr_done = true;
+    }
+    if (!launch_gate()) return KDA_ERR_CUDA;
+    prefill_simt_kernel<D, C, TIO><<<p.n_items, Sh::NT, Sh::smem_bytes, st>>>(p);
+    return last_launch_status();
+}
+
+template <typename TIO>
+static kda_status dispatch_simt(int D, int C, const PrefillParams &p, cudaStream_t st) {
+#define KDA_CASE(d, c) \
+    if (D == d && C == c) return launch_simt<d, c, TIO>(p, st);
+    KDA_CASE(32, 16) KDA_CASE(32, 32) KDA_CASE(32, 64)
+    KDA_CASE(64, 16) KDA_CASE(64, 32) KDA_CASE(64, 64)
+    KDA_CASE(128, 16) KDA_CASE(128, 32) KDA_CASE(128, 64)
+#undef KDA_CASE
+    return KDA_ERR_UNSUPPORTED;
+}
+
+// Forced path selection for tests: 0 = automatic, 1 = CUDA-core path only.
+static std::atomic<int> g_prefill_path{0};
+
+}  // namespace kda
+
+using namespace kda;
+
+extern "C" {
+
+const char *kda_status_string(kda_status s) {
+    switch (s) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID: return "KDA_ERR_INVALID: invalid argument";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: unsupported dimensions";
+    case KDA_ERR_ALIGN: return "KDA_ERR_ALIGN: device pointer not 16-byte aligned";
+    case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE: reserved";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA: CUDA call or launch failed";
+    case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: device wait ran out of iterations";
+    case KDA_ERR_RANGE: return "KDA_ERR_RANGE: device-side range check failed";
+    }
+    return "KDA_ERR_UNKNOWN";
+}
+
+int64_t kda_launch_count(void) { return g_launches.load(); }
+
+void kda_test_fail_next_launches(int32_t n) { g_fail_next.store(n > 0 ? n : 0); }
+
+kda_status kda_snapshot_plan(int32_t n_seq, const int32_t *cu, const int64_t *start_pos,
+                             int32_t snap_interval, int64_t *offsets, int64_t *positions) {
+    if (n_seq < 0 || !cu || !offsets || snap_interval < 0) return KDA_ERR_INVALID;
+    if (cu[0] != 0) return KDA_ERR_INVALID;
+    for (int s = 0; s < n_seq; ++s) {
+        if (cu[s + 1] < cu[s]) return KDA_ERR_INVALID;
+        if (start_pos && start_pos[s] < 0) return KDA_ERR_INVALID;
+    }
+    int64_t total = 0;
+    offsets[0] = 0;
+    for (int s = 0; s < n_seq; ++s) {
+        const int64_t p0 = start_pos ? start_pos[s] : 0, len = cu[s + 1] - cu[s];
+        int64_t cnt = 0;
+        if (snap_interval > 0) {
+            cnt = (p0 + len) / snap_interval - p0 / snap_interval;
+            if (positions) {
+                int64_t p = (p0 / snap_interval + 1) * snap_interval;
+                for (int64_t j = 0; j < cnt; ++j, p += snap_interval) positions[total + j] = p;
+            }
+        }
+        total += cnt;
+        offsets[s + 1] = total;
+    }
+    return KDA_OK;
+}
+
+kda_status kda_prefill(const kda_dims *dims, int32_t n_seq, const int32_t *cu,
+                       const int64_t *start_pos, const void *q, const void *k, const void *v,
+                       const float *g, const float *beta, const float *state_in,
+                       float *state_out, void *o, int32_t snap_interval, float *snapshots,
+                       kda_stream_t stream) {
+    kda_status st = check_dims(dims, true);
+    if (st != KDA_OK) return st;
+    if (n_seq < 0 || snap_interval < 0) return KDA_ERR_INVALID;
+    if (n_seq == 0) return KDA_OK;
+    if (!cu) return KDA_ERR_INVALID;
+    const int C = dims->chunk, D = dims->dk, H = dims->H;
+    std::vector<int64_t> offs(n_seq + 1);
+    st = kda_snapshot_plan(n_seq, cu, start_pos, snap_interval, offs.data(), nullptr);
+    if (st != KDA_OK) return st;
+    if (snap_interval > 0) {
+        if (snap_interval % C != 0) return KDA_ERR_INVALID;
+        for (int s = 0; s < n_seq && start_pos; ++s)
+            if (start_pos[s] % C != 0) return KDA_ERR_INVALID;
+    }
+    const int64_t T = cu[n_seq];
+    if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID;
+    if (offs[n_seq] > 0 && !snapshots) return KDA_ERR_INVALID;
+    const void *ptrs[] = {q, k, v, g, beta, state_in, state_out, o, snapshots};
+    for (const void *ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
+
+    // longest-first order: the hardware block scheduler hands out CTAs in
+    // index order, so long chains start first and short ones fill the tail.
+    std::vector<int> order(n_seq);
+    std::iota(order.begin(), order.end(), 0);
+    std::stable_sort(order.begin(), order.end(),
+                     [&](int a, int b) { return cu[a + 1] - cu[a] > cu[b + 1] - cu[b]; });
+
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    const bool tc = g_prefill_path.load() == 0 && tc_prefill_supported(*dims);
+    static thread_local PrefillParams p;  // ~27 KB: keep it off the stack
+    for (int g0 = 0; g0 < n_seq; g0 += kPrefillSeqs) {
+        const int ng = std::min(kPrefillSeqs, n_seq - g0);
+        std::memset(&p, 0, sizeof(p));
+        p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.o = o; p.snapshots = snapshots;
+        const int64_t state_stride = (int64_t)H * D * D;
+        p.state_in = state_in ? state_in + g0 * state_stride : nullptr;
+        p.state_out = state_out ? state_out + g0 * state_stride : nullptr;
+        p.H = H; p.n_seq = ng; p.snap_interval = snap_interval; p.scale = eff_scale(dims);
+        int r = 0;
+        for (int idx : order)
+            if (idx >= g0 && idx < g0 + ng) p.order[r++] = (int16_t)(idx - g0);
+        for (int i = 0; i < ng; ++i) {
+            const int s = g0 + i;
+            p.seq[i].tok0 = cu[s];
+            p.seq[i].len = cu[s + 1] - cu[s];
+            p.seq[i].start_pos = start_pos ? start_pos[s] : 0;
+            p.seq[i].snap_off = offs[s];
+        }
+        if (tc) {
+            st = launch_prefill_tc(p, *dims, T, cs, launch_gate);
+        } else {
+            p.n_items = ng * H * (D / SimtShape<32, 16>::DVS);
+            st = dims->io == KDA_IO_BF16 ? dispatch_simt<__nv_bfloat16>(D, C, p, cs)
+                                         : dispatch_simt<float>(D, C, p, cs);
+        }
+        if (st != KDA_OK) return st;
+    }
+    return KDA_OK;
+}
+
+kda_status kda_decode(const kda_dims *dims, int32_t n_seq, const void *q, const void *k,
+                      const void *v, const float *g, const float *beta, const int32_t *slots,
+                      int32_t n_slots, float *pool, void *o, kda_stream_t stream) {
+    kda_status st = check_dims(dims, false);
+    if (st != KDA_OK) return st;
+    if (n_seq < 0 || n_slots < 0) return KDA_ERR_INVALID;
+    if (n_seq == 0) return KDA_OK;
+    if (!q || !k || !v || !g || !beta || !slots || !pool || !o) return KDA_ERR_INVALID;
+    const void *ptrs[] = {q, k, v, g, beta, slots, pool, o};
+    for (const void *ptr : ptrs)
+        if (!aligned16(ptr)) return KDA_ERR_ALIGN;
+    if ((int64_t)n_seq * dims->H > 0x7fffffffLL) return KDA_ERR_INVALID;
+    static thread_local DecodeParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.slots = slots; p.pool = pool; p.o = o;
+    p.n_seq = n_seq; p.H = dims->H; p.n_slots = n_slots; p.scale = eff_scale(dims);
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    return dims->io == KDA_IO_BF16
+               ? dispatch_decode<__nv_bfloat16>(dims->dk, p, n_seq * dims->H, cs, false)
+               : dispatch_decode<float>(dims->dk, p, n_seq * dims->H, cs, false);
+}
+
+kda_status kda_verify(const kda_dims *dims, int32_t n_seq, const int32_t *cu_draft,
+                      const void *q, const void *k, const void *v, const float *g,
+                      const float *beta, const int32_t *slots, int32_t n_slots,
+                      const float *pool, float *token_states, void *o, kda_stream_t stream) {
+    kda_status st = check_dims(dims, false);
+    if (st != KDA_OK) return st;
+    if (n_seq < 0 || n_slots < 0) return KDA_ERR_INVALID;
+    if (n_seq == 0) return KDA_OK;
+    if (!cu_draft || cu_draft[0] != 0) return KDA_ERR_INVALID;
+    for (int s = 0; s < n_seq; ++s)
+        if (cu_draft[s + 1] < cu_draft[s]) return KDA_ERR_INVALID;
+    const int64_t T = cu_draft[n_seq];
+    if (!slots || !pool) return KDA_ERR_INVALID;
+    if (T > 0 && (!q || !k || !v || !g || !beta || !token_states || !o)) return KDA_ERR_INVALID;
+    const void *ptrs[] = {q, k, v, g, beta, slots, pool, token_states, o};
+    for (const void *ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    static thread_local DecodeParams p;
+    for (int g0 = 0; g0 < n_seq; g0 += kMaxSeqsPerLaunch) {
+        const int ng = std::min(kMaxSeqsPerLaunch, n_seq - g0);
+        std::memset(&p, 0, sizeof(p));
+        p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.slots = slots + g0;
+        p.pool = const_cast<float *>(pool); p.token_states = token_states; p.o = o;
+        p.n_seq = ng; p.H = dims->H; p.n_slots = n_slots; p.scale = eff_scale(dims);
+        p.tok_base = cu_draft[g0];
+        for (int i = 0; i <= ng; ++i) p.tok0[i] = cu_draft[g0 + i] - cu_draft[g0];
+        st = dims->io == KDA_IO_BF16
+                 ? dispatch_decode<__nv_bfloat16>(dims->dk, p, ng * dims->H, cs, true)
+                 : dispatch_decode<float>(dims->dk, p, ng * dims->H, cs, true);
+        if (st != KDA_OK) return st;
+    }
+    return KDA_OK;
+}
+
+kda_status kda_snapshot(int32_t n, const int64_t *src_idx, const int64_t *dst_idx,
+                        const float *src, int64_t n_src, float *dst, int64_t n_dst, int32_t H,
+                        int32_t dk, int32_t dv, kda_stream_t stream) {
+    if (n < 0 || n_src < 0 || n_dst < 0 || H < 1 || dk < 1 || dv < 1) return KDA_ERR_INVALID;
+    if (n == 0) return KDA_OK;
+    if (!src_idx || !dst_idx || !src || !dst) return KDA_ERR_INVALID;
+    const int64_t elems = (int64_t)H * dk * dv;
+    if (elems % 4 != 0) return KDA_ERR_UNSUPPORTED;
+    const void *ptrs[] = {src_idx, dst_idx, src, dst};
+    for (const void *ptr : ptrs)
+        if (!aligned16(ptr)) return KDA_ERR_ALIGN;
+    SnapshotParams p;
+    p.src = src; p.dst = dst; p.n_src = n_src; p.n_dst = n_dst; p.elems4 = elems / 4;
+    const int per_copy = (int)std::min<int64_t>(128, (p.elems4 + 1023) / 1024);
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    for (int i0 = 0; i0 < n; i0 += 65535) {
+        const int ni = std::min(65535, n - i0);
+        p.src_idx = src_idx + i0;
+        p.dst_idx = dst_idx + i0;
+        if (!launch_gate()) return KDA_ERR_CUDA;
+        snapshot_kernel<<<dim3(per_copy, ni), 256, 0, cs>>>(p);
+        if (last_launch_status() != KDA_OK) return KDA_ERR_CUDA;
+    }
+    return KDA_OK;
+}
+
+kda_status kda_check_device_status(kda_stream_t stream) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return KDA_ERR_CUDA;
+    if (v != 0 && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    return static_cast<kda_status>(v);
+}
+
+// Forces the CUDA-core prefill path (1) or restores automatic selection (0).
+// Not in the public header: used by the parity tests to check both paths.
+void kda_internal_force_prefill_path(int32_t path) { g_prefill_path.store(path); }
+
+}  // extern "C"
+
+// ------------------------------------------------ failure-injection hook ----
+namespace kda {
+__device__ int g_never_set;
+
+__global__ void wait_timeout_kernel(int32_t iters) {
+    if (threadIdx.x != 0) return;
+    volatile int *flag = &g_never_set;
+    for (int32_t i = 0; i < iters; ++i) {
+        if (*flag != 0) return;
+        __nanosleep(1000);
+    }
+    record_status(KDA_ERR_TIMEOUT);
+}
+}  // namespace kda
+
+extern "C" kda_status kda_test_wait_timeout(int32_t iters, kda_stream_t stream) {
+    if (iters < 0) return KDA_ERR_INVALID;
+    if (!launch_gate()) return KDA_ERR_CUDA;
+    wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(iters);
+    return last_launch_status();
+}

@@ -1,0 +1,186 @@
+"""Python binding of libkda (include/kda.h): argument marshalling only.
+
+Each function takes torch tensors that already live where the C ABI wants
+them (device tensors for device pointers, Python sequences or CPU tensors for
+the _h host arrays), reads their shapes into a ``kda_dims``, and calls the
+library function of the same name on the current CUDA stream. Every step of
+the computation runs in libkda's kernels; there is no fallback of any kind. A
+missing library raises ``KDAError`` at import of this module's first call.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+import numpy as np
+import torch
+
+_LIB_PATH = Path(__file__).resolve().parent / "libkda.so"
+_lib = None
+
+KDA_OK = 0
+KDA_IO_BF16, KDA_IO_FP32 = 0, 1
+STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID", 2: "KDA_ERR_UNSUPPORTED", 3: "KDA_ERR_ALIGN",
+                4: "KDA_ERR_WORKSPACE", 5: "KDA_ERR_CUDA", 6: "KDA_ERR_TIMEOUT", 7: "KDA_ERR_RANGE"}
+
+
+class KDAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+class kda_dims(ctypes.Structure):
+    _fields_ = [("H", ctypes.c_int32), ("dk", ctypes.c_int32), ("dv", ctypes.c_int32),
+                ("chunk", ctypes.c_int32), ("io", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+_P = ctypes.c_void_p
+_I32, _I64 = ctypes.c_int32, ctypes.c_int64
+
+_SIGNATURES = {
+    "kda_snapshot_plan": (_I32, [_I32, _P, _P, _I32, _P, _P]),
+    "kda_prefill": (_I32, [_P, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P]),
+    "kda_decode": (_I32, [_P, _I32, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P]),
+    "kda_verify": (_I32, [_P, _I32, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P]),
+    "kda_snapshot": (_I32, [_I32, _P, _P, _P, _I64, _P, _I64, _I32, _I32, _I32, _P]),
+    "kda_status_string": (ctypes.c_char_p, [_I32]),
+    "kda_check_device_status": (_I32, [_P]),
+    "kda_launch_count": (_I64, []),
+    "kda_test_fail_next_launches": (None, [_I32]),
+    "kda_test_wait_timeout": (_I32, [_I32, _P]),
+    "kda_internal_force_prefill_path": (None, [_I32]),
+}
+
+
+def library_path() -> Path:
+    return _LIB_PATH
+
+
+def lib():
+    """The loaded libkda (ctypes). Raises KDAError if the library is missing."""
+    global _lib
+    if _lib is None:
+        if not _LIB_PATH.exists():
+            raise KDAError(-1, f"libkda.so not built at {_LIB_PATH} "
+                               "(python -m hybrid_linear_attention_04_b200.build)")
+        L = ctypes.CDLL(str(_LIB_PATH))
+        for name, (res, args) in _SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != KDA_OK:
+        raise KDAError(status, where)
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _dptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise KDAError(1, "device tensor expected")
+    if not t.is_contiguous():
+        raise KDAError(1, "contiguous tensor expected")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _host_array(x, dtype):
+    if x is None:
+        return None
+    if isinstance(x, torch.Tensor):
+        x = x.detach().cpu().numpy()
+    return np.ascontiguousarray(np.asarray(x), dtype=dtype)
+
+
+def _hptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _io(t):
+    if t.dtype == torch.bfloat16:
+        return KDA_IO_BF16
+    if t.dtype == torch.float32:
+        return KDA_IO_FP32
+    raise KDAError(2, f"unsupported io dtype {t.dtype}")
+
+
+def _dims(q, v, chunk=0, scale=0.0):
+    H, dk = q.shape[-2], q.shape[-1]
+    return kda_dims(H, dk, v.shape[-1], chunk, _io(q), float(scale))
+
+
+def kda_snapshot_plan(cu_seqlens, start_pos=None, snap_interval=0):
+    """Snapshot rows per sequence: returns (offsets int64 [n_seq+1], positions int64 [total])."""
+    cu = _host_array(cu_seqlens, np.int32)
+    n_seq = len(cu) - 1
+    sp = _host_array(start_pos, np.int64)
+    offs = np.zeros(n_seq + 1, dtype=np.int64)
+    _check(lib().kda_snapshot_plan(n_seq, _hptr(cu), _hptr(sp), snap_interval, _hptr(offs), None),
+           "kda_snapshot_plan")
+    pos = np.zeros(int(offs[-1]), dtype=np.int64)
+    _check(lib().kda_snapshot_plan(n_seq, _hptr(cu), _hptr(sp), snap_interval, _hptr(offs),
+                                   _hptr(pos)), "kda_snapshot_plan")
+    return offs, pos
+
+
+def kda_prefill(q, k, v, g, beta, cu_seqlens, o, state_out=None, state_in=None, start_pos=None,
+                snap_interval=0, snapshots=None, chunk=64, scale=0.0, stream=None):
+    """Packed variable-length chunked prefill (see include/kda.h)."""
+    cu = _host_array(cu_seqlens, np.int32)
+    sp = _host_array(start_pos, np.int64)
+    dims = _dims(q, v, chunk, scale)
+    _check(lib().kda_prefill(ctypes.byref(dims), len(cu) - 1, _hptr(cu), _hptr(sp), _dptr(q),
+                             _dptr(k), _dptr(v), _dptr(g), _dptr(beta), _dptr(state_in),
+                             _dptr(state_out), _dptr(o), int(snap_interval), _dptr(snapshots),
+                             _stream(stream)), "kda_prefill")
+
+
+def kda_decode(q, k, v, g, beta, slots, state_pool, o, scale=0.0, stream=None):
+    """One decode token per sequence, states updated in place (see include/kda.h)."""
+    dims = _dims(q, v, 0, scale)
+    _check(lib().kda_decode(ctypes.byref(dims), q.shape[0], _dptr(q), _dptr(k), _dptr(v),
+                            _dptr(g), _dptr(beta), _dptr(slots), state_pool.shape[0],
+                            _dptr(state_pool), _dptr(o), _stream(stream)), "kda_decode")
+
+
+def kda_verify(q, k, v, g, beta, cu_draft, slots, state_pool, token_states, o, scale=0.0,
+               stream=None):
+    """Speculative verify with per-token states (see include/kda.h)."""
+    cu = _host_array(cu_draft, np.int32)
+    dims = _dims(q, v, 0, scale)
+    _check(lib().kda_verify(ctypes.byref(dims), len(cu) - 1, _hptr(cu), _dptr(q), _dptr(k),
+                            _dptr(v), _dptr(g), _dptr(beta), _dptr(slots), state_pool.shape[0],
+                            _dptr(state_pool), _dptr(token_states), _dptr(o), _stream(stream)),
+           "kda_verify")
+
+
+def kda_snapshot(src_idx, dst_idx, src, dst, stream=None):
+    """dst[dst_idx[i]] = src[src_idx[i]] for whole [H, dk, dv] states (see include/kda.h)."""
+    n, H, dk, dv = src_idx.shape[0], src.shape[1], src.shape[2], src.shape[3]
+    _check(lib().kda_snapshot(n, _dptr(src_idx), _dptr(dst_idx), _dptr(src), src.shape[0],
+                              _dptr(dst), dst.shape[0], H, dk, dv, _stream(stream)), "kda_snapshot")
+
+
+def kda_check_device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status code."""
+    return int(lib().kda_check_device_status(_stream(stream)))
+
+
+def kda_launch_count() -> int:
+    return int(lib().kda_launch_count())
+
+
+def kda_status_string(status: int) -> str:
+    return lib().kda_status_string(status).decode()

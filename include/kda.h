@@ -1,0 +1,192 @@
+/*
+ * libkda — Kimi Delta Attention (KDA) hot path on NVIDIA B200 (sm_100a).
+ *
+ * The operation (Kimi K3 technical FAQ, runpod.io, "What is KDA, and why does a
+ * serving engineer care?": a delta-rule linear-attention recurrence with a
+ * per-channel forget gate and a fixed d_k x d_v state per head, computed
+ * parallel within a chunk and recurrent across chunks), in the standard
+ * gated-delta form, per sequence and head:
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = scale * S_t^T q_t,        alpha_t = exp(g_t) in (0, 1]^{d_k}
+ *
+ * State snapshots (vLLM day-0 blog, "Kimi Delta Attention": prefix caching over
+ * recurrent state reuses state snapshots taken at block boundaries): the state
+ * after absolute position p is a snapshot when p % snap_interval == 0.
+ *
+ * Conventions shared by every call
+ *  - Layouts (row-major, innermost last): q, k, g: [tokens, H, d_k];
+ *    v, o: [tokens, H, d_v]; beta: [tokens, H]; a state: [H, d_k, d_v] fp32 with
+ *    d_v contiguous; pools of states: [n, H, d_k, d_v].
+ *  - q, k, v, o are bf16 (KDA_IO_BF16) or fp32 (KDA_IO_FP32); g (= log alpha,
+ *    must be <= 0), beta (in [0, 1]) and states are always fp32. q and k are
+ *    used as given: the library does not normalise them.
+ *  - Pointers suffixed _h are host memory read during the call only. All other
+ *    pointers are device memory owned by the caller; the library allocates no
+ *    memory and keeps no state between calls except a device status word.
+ *  - Every device pointer must be 16-byte aligned (KDA_ERR_ALIGN otherwise).
+ *  - Calls are asynchronous on `stream`: argument errors return synchronously
+ *    before anything is launched; device-side range errors and bounded-wait
+ *    timeouts are recorded in the status word read by kda_check_device_status.
+ *  - Element offsets are 64-bit; tokens per call must be < 2^31.
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (the same handle type); NULL is the legacy default stream. */
+typedef struct CUstream_st *kda_stream_t;
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID = 1,     /* bad argument: null pointer, negative size, bad cu_seqlens ... */
+    KDA_ERR_UNSUPPORTED = 2, /* dimensions outside the compiled set (see kda_dims) */
+    KDA_ERR_ALIGN = 3,       /* a device pointer is not 16-byte aligned */
+    KDA_ERR_WORKSPACE = 4,   /* reserved */
+    KDA_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
+    KDA_ERR_TIMEOUT = 6,     /* a device-side wait ran out of iterations (device status) */
+    KDA_ERR_RANGE = 7        /* device-side check failed: a slot or index out of range, or a
+                                gate whose decay over one chunk is outside the supported
+                                range of the tensor-core prefill (device status) */
+} kda_status;
+
+typedef enum { KDA_IO_BF16 = 0, KDA_IO_FP32 = 1 } kda_io;
+
+typedef struct {
+    int32_t H;     /* heads, >= 1 */
+    int32_t dk;    /* key head dim;   supported: dk == dv in {32, 64, 128} */
+    int32_t dv;    /* value head dim */
+    int32_t chunk; /* prefill chunk length C in {16, 32, 64}; unused by decode/verify */
+    int32_t io;    /* kda_io: element type of q, k, v, o */
+    float scale;   /* output scale; 0 selects 1/sqrt(dk) */
+} kda_dims;
+
+/* Maximum sequences per kernel launch; larger batches are split by the library
+ * into several launches on the same stream. */
+#define KDA_SEQS_PER_LAUNCH 1024
+
+/*
+ * kda_snapshot_plan — where each sequence's snapshots go (host only, no GPU).
+ * Snapshot rule of the vLLM day-0 blog, "Kimi Delta Attention" (snapshots at
+ * block boundaries): sequence s (tokens cu_seqlens_h[s] .. cu_seqlens_h[s+1]-1,
+ * with start_pos_h[s] tokens already absorbed by its initial state; NULL means
+ * all zero) takes a snapshot after each absolute position p with
+ * start_pos < p <= start_pos + len and p % snap_interval == 0, ascending.
+ *   snap_offsets_h [n_seq+1] (out): exclusive prefix sum of per-sequence counts;
+ *                                   snapshot j of sequence s is row
+ *                                   snap_offsets_h[s] + j of the snapshot pool.
+ *   snap_pos_h     [snap_offsets_h[n_seq]] (out, nullable): the positions p.
+ * snap_interval == 0 means no snapshots (all offsets 0).
+ * Errors: KDA_ERR_INVALID for n_seq < 0, null cu_seqlens_h / snap_offsets_h,
+ * cu_seqlens_h[0] != 0, decreasing cu_seqlens_h, negative start_pos or interval.
+ */
+kda_status kda_snapshot_plan(int32_t n_seq, const int32_t *cu_seqlens_h,
+                             const int64_t *start_pos_h, int32_t snap_interval,
+                             int64_t *snap_offsets_h, int64_t *snap_pos_h);
+
+/*
+ * kda_prefill — packed variable-length chunked prefill (Kimi K3 technical FAQ,
+ * "What is KDA": parallel within a chunk, recurrent across chunks; the
+ * chunk-form algebra is derived from the recurrence in the library's design
+ * notes). Sequence s is tokens [cu_seqlens_h[s], cu_seqlens_h[s+1]) of the
+ * packed q, k, v, g, beta, o arrays (T_total = cu_seqlens_h[n_seq] tokens).
+ *   start_pos_h [n_seq] (nullable = zeros): tokens already absorbed by the
+ *               initial state; sets the absolute positions of snapshots.
+ *   state_in  [n_seq, H, dk, dv] (nullable = zero states): initial states.
+ *   state_out [n_seq, H, dk, dv] (nullable): state after each sequence's last
+ *               token. May alias state_in (in-place update).
+ *   o         [T_total, H, dv]: outputs, written for every token.
+ *   snap_interval: 0 (none) or a multiple of dims->chunk; with snapshots on,
+ *               every start_pos must be a multiple of dims->chunk.
+ *   snapshots [kda_snapshot_plan total, H, dk, dv] (required when any
+ *               snapshot is due): fp32 states, rows as kda_snapshot_plan says.
+ * A zero-length sequence writes state_out = state_in and no snapshots.
+ * Errors (before launch): KDA_ERR_INVALID, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGN.
+ * Device status KDA_ERR_RANGE: a chunk whose per-channel decay exceeds the
+ * tensor-core path's range (sum of g over one chunk below -170 in some channel;
+ * the outputs of that chunk are then not reliable).
+ */
+kda_status kda_prefill(const kda_dims *dims, int32_t n_seq, const int32_t *cu_seqlens_h,
+                       const int64_t *start_pos_h, const void *q, const void *k,
+                       const void *v, const float *g, const float *beta,
+                       const float *state_in, float *state_out, void *o,
+                       int32_t snap_interval, float *snapshots, kda_stream_t stream);
+
+/*
+ * kda_decode — one token per sequence against a pool of live states (the
+ * recurrence above for a single t), updating each state in place with one
+ * read and one write of it.
+ *   q, k, g [n_seq, H, dk]; v, o [n_seq, H, dv]; beta [n_seq, H].
+ *   slots [n_seq] (device int32): row of state_pool used by each sequence;
+ *               slots must be distinct (a repeated slot is a data race).
+ *   state_pool [n_slots, H, dk, dv]: read and written in place.
+ * Device status KDA_ERR_RANGE if a slot is outside [0, n_slots) (that
+ * sequence is skipped).
+ */
+kda_status kda_decode(const kda_dims *dims, int32_t n_seq, const void *q, const void *k,
+                      const void *v, const float *g, const float *beta, const int32_t *slots,
+                      int32_t n_slots, float *state_pool, void *o, kda_stream_t stream);
+
+/*
+ * kda_verify — speculative verify: sequence s runs its draft tokens
+ * [cu_draft_h[s], cu_draft_h[s+1]) (packed like prefill) from the state
+ * state_pool[slots[s]], which is only read, and writes the output and the
+ * state after every token, so that the caller can commit the state of the
+ * last accepted token with kda_snapshot (rollback of rejected drafts).
+ *   token_states [cu_draft_h[n_seq], H, dk, dv]: state after each token.
+ * Errors as kda_decode.
+ */
+kda_status kda_verify(const kda_dims *dims, int32_t n_seq, const int32_t *cu_draft_h,
+                      const void *q, const void *k, const void *v, const float *g,
+                      const float *beta, const int32_t *slots, int32_t n_slots,
+                      const float *state_pool, float *token_states, void *o,
+                      kda_stream_t stream);
+
+/*
+ * kda_snapshot — bit-exact copies of whole states between pools: for i < n,
+ * dst[dst_idx[i]] = src[src_idx[i]] (each an [H, dk, dv] fp32 state). Used to
+ * commit a verified token's state, restore a cached prefix snapshot into a
+ * live slot, or save a live state (vLLM day-0 blog, prefix caching over
+ * recurrent state).
+ *   src_idx, dst_idx [n] (device int64); src [n_src, ...], dst [n_dst, ...].
+ * Destinations must be distinct and must not overlap the sources read.
+ * Device status KDA_ERR_RANGE for an index outside its pool (copy skipped).
+ */
+kda_status kda_snapshot(int32_t n, const int64_t *src_idx, const int64_t *dst_idx,
+                        const float *src, int64_t n_src, float *dst, int64_t n_dst,
+                        int32_t H, int32_t dk, int32_t dv, kda_stream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *kda_status_string(kda_status s);
+
+/*
+ * kda_check_device_status — synchronises `stream`, then returns and clears the
+ * device status word of the current device (KDA_OK, KDA_ERR_RANGE or
+ * KDA_ERR_TIMEOUT; the first error recorded since the last check), or
+ * KDA_ERR_CUDA if the synchronisation itself failed.
+ */
+kda_status kda_check_device_status(kda_stream_t stream);
+
+/* Number of kernel launches the library has issued in this process (for
+ * launch accounting in benchmarks). */
+int64_t kda_launch_count(void);
+
+/* ---- Failure-injection hooks (tests) -------------------------------------
+ * kda_test_fail_next_launches(n): the next n launches are not issued and
+ *   report KDA_ERR_CUDA, as a failed launch would.
+ * kda_test_wait_timeout(iters, stream): launches one kernel that waits on a
+ *   flag that nothing sets, giving up after `iters` polls (bounded); it then
+ *   records KDA_ERR_TIMEOUT in the device status word and returns. */
+void kda_test_fail_next_launches(int32_t n);
+kda_status kda_test_wait_timeout(int32_t iters, kda_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KDA_H */

@@ -1,0 +1,149 @@
+"""Host-side tests of the C ABI (no GPU): the library loads, exports every
+function include/kda.h declares, plans snapshots as the block-boundary rule
+says (vLLM day-0 blog, "Kimi Delta Attention"), and rejects bad arguments
+before anything is launched. Every call here fails validation or is host-only,
+so no kernel is ever launched with the fake pointers these tests pass.
+"""
+from __future__ import annotations
+
+import ctypes
+import re
+from pathlib import Path
+
+import numpy as np
+import pytest
+
+import synth
+from hybrid_linear_attention_04_b200 import build as kbuild
+from hybrid_linear_attention_04_b200 import kda as K
+
+ROOT = Path(__file__).resolve().parents[1]
+HEADER = ROOT / "include" / "kda.h"
+
+# aligned and misaligned fake device addresses: never dereferenced, because
+# every call that receives them fails validation on the host first.
+A = ctypes.c_void_p(0x10000)
+MIS = ctypes.c_void_p(0x10004)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    kbuild.build()
+
+
+def declared_functions():
+    text = HEADER.read_text()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol():
+    names = declared_functions()
+    assert {"kda_prefill", "kda_decode", "kda_verify", "kda_snapshot", "kda_snapshot_plan",
+            "kda_check_device_status", "kda_status_string"} <= set(names)
+    L = ctypes.CDLL(str(K.library_path()))
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings():
+    for code, name in K.STATUS_NAMES.items():
+        assert K.kda_status_string(code).startswith(name)
+
+
+def _plan_ref(cu, start, interval):
+    offs, pos = [0], []
+    for s in range(len(cu) - 1):
+        p0, n = start[s], cu[s + 1] - cu[s]
+        ps = [p for p in range(p0 + 1, p0 + n + 1) if interval and p % interval == 0]
+        pos += ps
+        offs.append(offs[-1] + len(ps))
+    return offs, pos
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_snapshot_plan_matches_restatement(seed):
+    n = 1 + seed * 7
+    lens = synth.randint(seed, "lens", n, 0, 700)
+    lens[0] = 0                                   # zero-length sequence
+    if n > 2:
+        lens[1] = 512                             # boundary-aligned end
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    start = [64 * m for m in synth.randint(seed, "resume", n, 0, 12)]
+    for interval in (0, 64, 256):
+        offs, pos = K.kda_snapshot_plan(cu, start, interval)
+        ro, rp = _plan_ref(cu.tolist(), start, interval)
+        assert offs.tolist() == ro
+        assert pos.tolist() == rp
+
+
+def test_snapshot_plan_rejects_bad_input():
+    with pytest.raises(K.KDAError) as e:
+        K.kda_snapshot_plan([1, 5], None, 4)
+    assert e.value.status == 1
+    with pytest.raises(K.KDAError):
+        K.kda_snapshot_plan([0, 5, 3], None, 4)
+    with pytest.raises(K.KDAError):
+        K.kda_snapshot_plan([0, 5], [-1], 4)
+
+
+def _dims(H=4, d=128, chunk=64, io=0, scale=0.0):
+    return K.kda_dims(H, d, d, chunk, io, scale)
+
+
+def _prefill(dims, cu, start=None, snap=0, ptr=A, snapshots=A, n_seq=None):
+    cu = np.asarray(cu, dtype=np.int32)
+    sp = None if start is None else np.asarray(start, dtype=np.int64)
+    L = K.lib()
+    return L.kda_prefill(ctypes.byref(dims), len(cu) - 1 if n_seq is None else n_seq,
+                         cu.ctypes.data_as(ctypes.c_void_p),
+                         None if sp is None else sp.ctypes.data_as(ctypes.c_void_p),
+                         ptr, A, A, A, A, None, A, A, snap, snapshots, None)
+
+
+def test_prefill_validation():
+    assert _prefill(_dims(d=96), [0, 64]) == 2                 # unsupported head dim
+    assert _prefill(K.kda_dims(4, 128, 64, 64, 0, 0.0), [0, 64]) == 2   # dk != dv
+    assert _prefill(_dims(chunk=48), [0, 64]) == 2             # unsupported chunk
+    assert _prefill(_dims(io=7), [0, 64]) == 1                 # bad io type
+    assert _prefill(_dims(H=0), [0, 64]) == 1
+    assert _prefill(_dims(), [0, 64], n_seq=-1) == 1
+    assert _prefill(_dims(), [3, 64]) == 1                     # cu_seqlens[0] != 0
+    assert _prefill(_dims(), [0, 64, 10]) == 1                 # decreasing
+    assert _prefill(_dims(), [0, 300], snap=100) == 1          # interval % chunk != 0
+    assert _prefill(_dims(), [0, 300], start=[32], snap=256) == 1   # start % chunk != 0
+    assert _prefill(_dims(), [0, 300], start=[-64]) == 1
+    assert _prefill(_dims(), [0, 300], snap=256, snapshots=None) == 1   # missing pool
+    assert _prefill(_dims(), [0, 64], ptr=MIS) == 3            # misaligned q
+    assert _prefill(_dims(), [0, 64], ptr=None) == 1           # null q
+    assert _prefill(_dims(), [0], n_seq=0) == 0                # nothing to do
+
+
+def test_decode_verify_snapshot_validation():
+    L = K.lib()
+    d = _dims()
+    assert L.kda_decode(ctypes.byref(_dims(d=48)), 4, A, A, A, A, A, A, 8, A, A, None) == 2
+    assert L.kda_decode(ctypes.byref(d), -1, A, A, A, A, A, A, 8, A, A, None) == 1
+    assert L.kda_decode(ctypes.byref(d), 4, None, A, A, A, A, A, 8, A, A, None) == 1
+    assert L.kda_decode(ctypes.byref(d), 4, A, A, A, A, A, MIS, 8, A, A, None) == 3
+    assert L.kda_decode(ctypes.byref(d), 0, None, None, None, None, None, None, 0, None, None,
+                        None) == 0
+    cu = np.array([1, 3], dtype=np.int32)
+    assert L.kda_verify(ctypes.byref(d), 1, cu.ctypes.data_as(ctypes.c_void_p), A, A, A, A, A, A,
+                        8, A, A, A, None) == 1
+    cu = np.array([0, 3, 2], dtype=np.int32)
+    assert L.kda_verify(ctypes.byref(d), 2, cu.ctypes.data_as(ctypes.c_void_p), A, A, A, A, A, A,
+                        8, A, A, A, None) == 1
+    cu = np.array([0, 3], dtype=np.int32)
+    assert L.kda_verify(ctypes.byref(d), 1, cu.ctypes.data_as(ctypes.c_void_p), A, A, A, A, A, A,
+                        8, A, MIS, A, None) == 3
+    assert L.kda_snapshot(-1, A, A, A, 4, A, 4, 4, 128, 128, None) == 1
+    assert L.kda_snapshot(2, A, A, A, 4, A, 4, 1, 3, 1, None) == 2
+    assert L.kda_snapshot(2, A, MIS, A, 4, A, 4, 4, 128, 128, None) == 3
+    assert L.kda_snapshot(2, None, A, A, 4, A, 4, 4, 128, 128, None) == 1
+    assert L.kda_snapshot(0, None, None, None, 0, None, 0, 4, 128, 128, None) == 0
+
+
+def test_no_launch_issued_by_host_tests():
+    # the validation failures above must not have launched anything
+    assert K.kda_launch_count() == 0

@@ -1,0 +1,131 @@
+"""GPU parity of kda_prefill against the fp64 oracle (token recurrence), through
+the C ABI: packed ragged batches, initial states, start positions and
+block-boundary snapshots (vLLM day-0 blog, "Kimi Delta Attention"), on both
+prefill paths (tensor-core and CUDA-core) where the dims allow.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from hybrid_linear_attention_04_b200 import kda as K
+from kda_cases import blockwise_err, oracle_prefill, packed_inputs, to_np, tol_for
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(params=["auto", "simt"])
+def path(request):
+    K.lib().kda_internal_force_prefill_path(1 if request.param == "simt" else 0)
+    yield request.param
+    K.lib().kda_internal_force_prefill_path(0)
+
+
+def run_prefill(dev, cu, H, d, chunk, io, start=None, s0=None, snap=0, device=None):
+    n_seq = len(cu) - 1
+    T = int(cu[-1])
+    o = torch.empty((T, H, d), dtype=dev["v"].dtype, device=device)
+    sout = torch.empty((n_seq, H, d, d), dtype=torch.float32, device=device)
+    offs, pos = K.kda_snapshot_plan(cu, start, snap)
+    n_snap = int(offs[-1])
+    # sentinel-filled snapshot pool with one spare row: only planned rows change
+    snaps = torch.full((n_snap + 1, H, d, d), float("nan"), device=device)
+    K.kda_prefill(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], cu, o, state_out=sout,
+                  state_in=s0, start_pos=start, snap_interval=snap, snapshots=snaps, chunk=chunk)
+    assert K.kda_check_device_status() == 0
+    return o, sout, snaps, offs
+
+
+def check(o, sout, snaps, offs, ref, io):
+    tol = tol_for(io)
+    o_ref, s_ref, sn_ref = ref
+    assert blockwise_err(to_np(o), o_ref, (2,)) <= tol
+    assert blockwise_err(to_np(sout), s_ref, (2, 3)) <= tol
+    n_snap = int(offs[-1])
+    got = snaps.cpu().numpy()
+    assert sn_ref.shape[0] == n_snap
+    assert torch.isnan(snaps[n_snap]).all()                      # spare row untouched
+    if n_snap:
+        assert not np.isnan(got[:n_snap]).any()
+        assert blockwise_err(got[:n_snap], sn_ref, (2, 3)) <= tol
+
+
+def test_tiny_fp32_workload(cuda_device, path):
+    """B=1, H=2, T=64, d=32, chunk 16, fp32 throughout, zero initial state."""
+    x, dev, cu = packed_inputs(1000, [64], 2, 32, "fp32", cuda_device)
+    o, sout, snaps, offs = run_prefill(dev, cu, 2, 32, 16, "fp32", device=cuda_device)
+    check(o, sout, snaps, offs, oracle_prefill(x, cu), "fp32")
+
+
+@pytest.mark.parametrize("d,chunk,io", [(128, 64, "bf16"), (128, 64, "fp32"), (64, 32, "bf16"),
+                                        (32, 16, "fp32"), (128, 16, "bf16")])
+def test_ragged_with_state_and_snapshots(cuda_device, path, d, chunk, io):
+    lens = [1, chunk - 1, chunk, chunk + 1, 5 * chunk + 7, 0, 8 * chunk]
+    H = 3
+    x, dev, cu = packed_inputs(400 + d + chunk, lens, H, d, io, cuda_device)
+    start = [0, chunk, 0, 3 * chunk, 2 * chunk, chunk, 4 * chunk]
+    s0 = synth.states(401, len(lens), H, d, d, std=0.1)
+    snap = 2 * chunk
+    o, sout, snaps, offs = run_prefill(dev, cu, H, d, chunk, io, start, s0.to(cuda_device), snap,
+                                       cuda_device)
+    check(o, sout, snaps, offs, oracle_prefill(x, cu, start, s0, snap), io)
+
+
+def test_zero_length_sequence_passes_state_through(cuda_device, path):
+    H, d = 2, 128
+    x, dev, cu = packed_inputs(9, [0, 70, 0], H, d, "bf16", cuda_device)
+    s0 = synth.states(9, 3, H, d, d, std=0.1).to(cuda_device)
+    o, sout, snaps, offs = run_prefill(dev, cu, H, d, 64, "bf16", None, s0, 0, cuda_device)
+    assert torch.equal(sout[0], s0[0]) and torch.equal(sout[2], s0[2])
+
+
+def test_prefill_is_deterministic(cuda_device, path):
+    H, d = 4, 128
+    lens = [300, 129, 64]
+    x, dev, cu = packed_inputs(11, lens, H, d, "bf16", cuda_device)
+    a = run_prefill(dev, cu, H, d, 64, "bf16", None, None, 64, cuda_device)
+    b = run_prefill(dev, cu, H, d, 64, "bf16", None, None, 64, cuda_device)
+    for u, v in zip(a[:3], b[:3]):
+        assert torch.equal(torch.nan_to_num(u), torch.nan_to_num(v))
+
+
+def test_resume_from_gpu_snapshot_equals_full_run(cuda_device, path):
+    """Prefix caching: resuming from the GPU's own block-boundary snapshot gives
+    the same outputs and final state as the uninterrupted GPU run, bit for bit
+    (same chunk grid, deterministic kernels)."""
+    H, d, C = 4, 128, 64
+    T = 1000
+    x, dev, cu = packed_inputs(12, [T], H, d, "bf16", cuda_device)
+    o, sout, snaps, offs = run_prefill(dev, cu, H, d, C, "bf16", None, None, 256, cuda_device)
+    for m in range(int(offs[-1])):
+        p = 256 * (m + 1)
+        sub = {k: v[p:].contiguous() for k, v in dev.items()}
+        cu2 = np.array([0, T - p], dtype=np.int32)
+        o2, s2, sn2, offs2 = run_prefill(sub, cu2, H, d, C, "bf16", [p], snaps[m:m + 1].clone(),
+                                         256, cuda_device)
+        assert torch.equal(o2, o[p:])
+        assert torch.equal(s2, sout)
+        assert torch.equal(sn2[:int(offs2[-1])], snaps[m + 1:int(offs[-1])])
+
+
+def test_segment_handoff_equals_one_shot(cuda_device, path):
+    """A long sequence processed in segments, each call taking the previous
+    call's final state and start position, equals one call, bit for bit."""
+    H, d, C, seg = 2, 128, 64, 512
+    T = 4 * seg
+    x, dev, cu = packed_inputs(13, [T], H, d, "bf16", cuda_device)
+    o, sout, snaps, offs = run_prefill(dev, cu, H, d, C, "bf16", None, None, 256, cuda_device)
+    state = None
+    outs, sn_all = [], []
+    for i in range(4):
+        sub = {k: v[i * seg:(i + 1) * seg].contiguous() for k, v in dev.items()}
+        o2, s2, sn2, offs2 = run_prefill(sub, np.array([0, seg], dtype=np.int32), H, d, C, "bf16",
+                                         [i * seg], state, 256, cuda_device)
+        outs.append(o2)
+        sn_all.append(sn2[:int(offs2[-1])])
+        state = s2
+    assert torch.equal(torch.cat(outs), o)
+    assert torch.equal(state, sout)
+    assert torch.equal(torch.cat(sn_all), snaps[:int(offs[-1])])
