@@ -47,11 +47,13 @@ struct DecodeParams {
     int64_t tok_base;                     // verify: absolute offset of tok0[0]
 };
 
-// Per-token vectors staged in shared memory.
-template <int D> struct TokVec {
+// Per-token vectors staged in shared memory. 16-byte aligned (and padded to a
+// multiple of 16 bytes) because the step reads v with float4 loads.
+template <int D> struct __align__(16) TokVec {
     float k[D], q[D], a[D], v[D];
     float beta, kq;
 };
+static_assert(sizeof(TokVec<128>) % 16 == 0 && sizeof(TokVec<32>) % 16 == 0, "TokVec padding");
 
 template <int D, typename TIO>
 __device__ __forceinline__ void load_token(TokVec<D> &tv, const DecodeParams &p, int64_t row) {

@@ -21,6 +21,12 @@ namespace kda {
 
 static std::atomic<int64_t> g_launches{0};
 static std::atomic<int32_t> g_fail_next{0};
+static std::atomic<int> g_last_cuda_error{0};
+
+static kda_status cuda_fail(cudaError_t e) {
+    g_last_cuda_error.store((int)e);
+    return KDA_ERR_CUDA;
+}
 
 // Count a launch, or simulate a failed one (failure-injection hook).
 static bool launch_gate() {
@@ -33,7 +39,8 @@ static bool launch_gate() {
 }
 
 static kda_status last_launch_status() {
-    return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e);
 }
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -305,13 +312,20 @@ kda_status kda_snapshot(int32_t n, const int64_t *src_idx, const int64_t *dst_id
 }
 
 kda_status kda_check_device_status(kda_stream_t stream) {
-    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-        return KDA_ERR_CUDA;
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e);
     unsigned int v = 0, zero = 0;
-    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return KDA_ERR_CUDA;
-    if (v != 0 && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess)
-        return KDA_ERR_CUDA;
+    e = cudaMemcpyFromSymbol(&v, g_status, sizeof(v));
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (v != 0) {
+        e = cudaMemcpyToSymbol(g_status, &zero, sizeof(zero));
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
     return static_cast<kda_status>(v);
+}
+
+const char *kda_last_cuda_error(void) {
+    return cudaGetErrorString(static_cast<cudaError_t>(g_last_cuda_error.load()));
 }
 
 // Forces the CUDA-core prefill path (1) or restores automatic selection (0).

@@ -47,6 +47,7 @@ _SIGNATURES = {
     "kda_status_string": (ctypes.c_char_p, [_I32]),
     "kda_check_device_status": (_I32, [_P]),
     "kda_launch_count": (_I64, []),
+    "kda_last_cuda_error": (ctypes.c_char_p, []),
     "kda_test_fail_next_launches": (None, [_I32]),
     "kda_test_wait_timeout": (_I32, [_I32, _P]),
     "kda_internal_force_prefill_path": (None, [_I32]),
@@ -75,6 +76,8 @@ def lib():
 
 def _check(status: int, where: str):
     if status != KDA_OK:
+        if status == 5:
+            where = f"{where} ({lib().kda_last_cuda_error().decode()})"
         raise KDAError(status, where)
 
 
@@ -176,6 +179,10 @@ def kda_snapshot(src_idx, dst_idx, src, dst, stream=None):
 def kda_check_device_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status code."""
     return int(lib().kda_check_device_status(_stream(stream)))
+
+
+def kda_last_cuda_error() -> str:
+    return lib().kda_last_cuda_error().decode()
 
 
 def kda_launch_count() -> int:

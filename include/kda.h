@@ -173,6 +173,10 @@ const char *kda_status_string(kda_status s);
  */
 kda_status kda_check_device_status(kda_stream_t stream);
 
+/* Text of the CUDA error behind the most recent KDA_ERR_CUDA (static storage;
+ * "no error" if there was none). */
+const char *kda_last_cuda_error(void);
+
 /* Number of kernel launches the library has issued in this process (for
  * launch accounting in benchmarks). */
 int64_t kda_launch_count(void);
