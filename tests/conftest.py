@@ -14,6 +14,13 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "slow: long-running CPU test")
 
 
+@pytest.fixture(scope="session", autouse=True)
+def built_library():
+    """Rebuild libkda.so if any CUDA source is newer than it (no-op otherwise)."""
+    from hybrid_linear_attention_04_b200 import build
+    build.build()
+
+
 @pytest.fixture(scope="session")
 def cuda_device():
     import torch
