@@ -36,7 +36,7 @@ struct TcParams {
 };
 
 namespace tcp {
-constexpr int C = 64, D = 128, DVS = 64, NT = 128;
+constexpr int C = 64, D = 128, DVS = 64, NT = 256;
 // shared memory map (bytes from a 1024-aligned base)
 constexpr uint32_t STG_Q = 0;          // q   [64 tok x 128 ch] bf16: 2 slabs of 64 rows
 constexpr uint32_t STG_K = 16384;      // k   same
@@ -44,20 +44,21 @@ constexpr uint32_t STG_V = 32768;      // v   slice, 2 buffers of 1 slab [64 tok
 constexpr uint32_t OP_AK = 49152;      // [Qh; Ka]: 2 slabs of 128 rows (channels 0-63, 64-127)
 constexpr uint32_t OP_KB = 81920;      // Kb: 2 slabs of 64 rows
 constexpr uint32_t OP_T = 98304;       // T  [64 x 64]
-constexpr uint32_t OP_WK = 106496;     // Wk [64 tok x 128 ch]: 2 slabs of 64 rows
+constexpr uint32_t OP_WK = 106496;     // Wk [64 tok x 128 ch]: 2 slabs; solve scratch before that
 constexpr uint32_t OP_AQK = 122880;    // A_qk masked [64 x 64]
 constexpr uint32_t OP_W = 131072;      // W  [64 tok x 64 dv]
 constexpr uint32_t OP_SM = 139264;     // Sm [128 ch x 64 dv]: 1 slab of 128 rows
-constexpr uint32_t STG_G = 155648;     // g -> b, fp32 [64][128]
-constexpr uint32_t SOLVE = 188416;     // fp32 [64][65]: L, then X
-constexpr uint32_t VEC = SOLVE + 64 * 65 * 4;  // mC, eM, eC, gC [128] + bet [64]
-constexpr uint32_t BARS = VEC + (4 * 128 + 64) * 4;
+constexpr uint32_t STG_G = 155648;     // g, fp32 [64][128]
+constexpr uint32_t SOLVE = 188416;     // fp32 [64][65]: L off the diagonal, X on it
+constexpr uint32_t VEC = SOLVE + 64 * 65 * 4;  // eM, eC, gC [128] + bet [64]
+constexpr uint32_t BARS = VEC + (3 * 128 + 64) * 4;
 constexpr uint32_t SMEM_USED = BARS + 32;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
 // TMEM columns
 constexpr uint32_t COL_A = 0, COL_WK = 64, COL_W = 192, COL_O = 256, COL_S = 320, TMEM_COLS = 512;
 constexpr uint32_t CHUNK_TX = 16384 + 16384 + 32768 + 8192;   // bytes per chunk of loads
-constexpr float RANGE_LIMIT = 80.f;
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float RANGE_LIMIT2 = 80.f * LOG2E;    // 80 nats, in log2 units
 }  // namespace tcp
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -67,8 +68,15 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
     return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&u));
 }
+__device__ __forceinline__ uint4 pack8(const float *a, float s) {
+    return make_uint4(pack_bf16(s * a[0], s * a[1]), pack_bf16(s * a[2], s * a[3]),
+                      pack_bf16(s * a[4], s * a[5]), pack_bf16(s * a[6], s * a[7]));
+}
 
-__global__ void __launch_bounds__(128, 1) prefill_tc_kernel(const __grid_constant__ TcParams P) {
+// slot of the off-diagonal 16x16 block X[Cb + dist][Cb] in the solve scratch
+__device__ __forceinline__ int xslot(int dist, int cb) { return (dist == 1 ? 0 : dist == 2 ? 3 : 5) + cb; }
+
+__global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constant__ TcParams P) {
     using namespace tcp;
     const PrefillParams &p = P.p;
     extern __shared__ uint8_t smem_raw[];
@@ -76,13 +84,16 @@ __global__ void __launch_bounds__(128, 1) prefill_tc_kernel(const __grid_constan
     const uint32_t sbase = tc::smem_u32(sm);
     float *Gs = reinterpret_cast<float *>(sm + STG_G);
     float *Ls = reinterpret_cast<float *>(sm + SOLVE);
-    float *mC = reinterpret_cast<float *>(sm + VEC);
-    float *eM = mC + 128, *eC = mC + 256, *gC = mC + 384, *bet = mC + 512;
+    float *eM = reinterpret_cast<float *>(sm + VEC);
+    float *eC = eM + 128, *gC = eM + 256, *bet = eM + 384;
+    float *Xo = reinterpret_cast<float *>(sm + OP_WK);     // 6 blocks 16x16 (solve only)
+    float *Yw = Xo + 6 * 256;                                // 3 per-warp 16x16 blocks
     uint64_t *tma_bar = reinterpret_cast<uint64_t *>(sm + BARS);   // [2]
     uint64_t *mma_bar = tma_bar + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_bar + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wq = warp & 3, wh = warp >> 2;          // TMEM sub-partition, column half
     const int H = p.H;
     const int item = blockIdx.x;
     const int rank = item / (H * 2);
@@ -110,14 +121,16 @@ __global__ void __launch_bounds__(128, 1) prefill_tc_kernel(const __grid_constan
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tbase = *tmem_slot;
-    const uint32_t tlane = (uint32_t)(32 * warp) << 16;   // this warp's TMEM sub-partition
+    const uint32_t tlane = (uint32_t)(32 * wq) << 16;   // this warp's TMEM sub-partition
 
-    // fp32 master state: thread tid owns row tid (a d_k channel), 64 columns
-    float S[DVS];
+    // fp32 master state: thread owns d_k row c_own, columns [32 wh, 32 wh + 32) of the slice
+    const int c_own = tid & 127;
+    float S[32];
     {
-        const float *src = p.state_in ? p.state_in + (((int64_t)s * H + h) * D + tid) * D + j0 : nullptr;
+        const float *src =
+            p.state_in ? p.state_in + (((int64_t)s * H + h) * D + c_own) * D + j0 + 32 * wh : nullptr;
 #pragma unroll
-        for (int j = 0; j < DVS; j += 4) {
+        for (int j = 0; j < 32; j += 4) {
             float4 v = src ? *reinterpret_cast<const float4 *>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
             S[j] = v.x; S[j + 1] = v.y; S[j + 2] = v.z; S[j + 3] = v.w;
         }
@@ -144,6 +157,8 @@ __global__ void __launch_bounds__(128, 1) prefill_tc_kernel(const __grid_constan
         issue_loads(0);
         issued = 1;
     }
+    // prep-phase thread map: channel group u (8 channels), row block rb (4 rows)
+    const int pu = tid >> 4, prb = tid & 15, pc0 = 8 * pu, pkb = pu >> 3, pcc = pu & 7;
 
     for (int ci = 0; ci < n_chunks; ++ci) {
         const int n = min(C, sq.len - ci * C);
@@ -151,48 +166,53 @@ __global__ void __launch_bounds__(128, 1) prefill_tc_kernel(const __grid_constan
         ok = tc::bar_wait(&tma_bar[ci & 1], (ci >> 1) & 1);
         if (!__syncthreads_and(ok)) { ok = false; break; }
         landed = ci + 1;
-        // ---- B. beta, cumsum of g, per-channel scalars, Sm = Diag(e^m) S ---
-        if (tid < C) bet[tid] = tid < n ? p.beta[(int64_t)(sq.tok0 + ci * C + tid) * H + h] : 0.f;
-        {
-            const int c = tid;
-            float b = 0.f, m = 0.f, b0 = 0.f;
-#pragma unroll 8
-            for (int r = 0; r < C; ++r) {
-                const float gv = r < n ? Gs[r * D + c] : 0.f;
-                b += gv;
-                Gs[r * D + c] = b;
-                if (r == 0) b0 = b;
-                if (r == C / 2 - 1) m = b;
-            }
-            mC[c] = m;
-            const float em = expf(m);
-            eM[c] = em;
-            eC[c] = expf(b - m);
-            gC[c] = expf(b);
-            if (b0 - m > RANGE_LIMIT || m - b > RANGE_LIMIT) record_status(KDA_ERR_RANGE);
+        // ---- B. b = cumsum(g) in log2 units: local 4 rows, then a 16-lane scan
+        float b[4][8];
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-                uint4 u;
-                u.x = pack_bf16(S[8 * cc + 0] * em, S[8 * cc + 1] * em);
-                u.y = pack_bf16(S[8 * cc + 2] * em, S[8 * cc + 3] * em);
-                u.z = pack_bf16(S[8 * cc + 4] * em, S[8 * cc + 5] * em);
-                u.w = pack_bf16(S[8 * cc + 6] * em, S[8 * cc + 7] * em);
-                *reinterpret_cast<uint4 *>(sm + OP_SM + tc::sw128(c, cc)) = u;
+        for (int i = 0; i < 4; ++i) {
+            const int r = 4 * prb + i;
+            const float4 x0 = *reinterpret_cast<const float4 *>(Gs + r * D + pc0);
+            const float4 x1 = *reinterpret_cast<const float4 *>(Gs + r * D + pc0 + 4);
+            const float sc = r < n ? LOG2E : 0.f;
+            b[i][0] = x0.x * sc; b[i][1] = x0.y * sc; b[i][2] = x0.z * sc; b[i][3] = x0.w * sc;
+            b[i][4] = x1.x * sc; b[i][5] = x1.y * sc; b[i][6] = x1.z * sc; b[i][7] = x1.w * sc;
+        }
+#pragma unroll
+        for (int i = 1; i < 4; ++i)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) b[i][e] += b[i - 1][e];
+        float m2[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float tot = b[3][e];
+            float incl = tot;
+#pragma unroll
+            for (int off = 1; off < 16; off <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, incl, off, 16);
+                if (prb >= off) incl += y;
+            }
+            const float ex = incl - tot;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) b[i][e] += ex;
+            m2[e] = __shfl_sync(0xffffffffu, b[3][e], 7, 16);        // row 31
+            const float bc = __shfl_sync(0xffffffffu, b[3][e], 15, 16);  // row 63
+            const float b0 = __shfl_sync(0xffffffffu, b[0][e], 0, 16);   // row 0
+            if (prb == 0) {
+                const int c = pc0 + e;
+                eM[c] = tc::ex2(m2[e]);
+                eC[c] = tc::ex2(bc - m2[e]);
+                gC[c] = tc::ex2(bc);
+                if (b0 - m2[e] > RANGE_LIMIT2 || m2[e] - bc > RANGE_LIMIT2) record_status(KDA_ERR_RANGE);
             }
         }
-        __syncthreads();
-        // ---- C. scaled bf16 operands Qh, Ka, Kb -----------------------------
-#pragma unroll 2
-        for (int j = 0; j < 8; ++j) {
-            const int unit = tid + NT * j;
-            const int r = unit >> 4, u = unit & 15, kb = u >> 3, cc = u & 7;
-            const uint32_t so = kb * 8192 + tc::sw128(r, cc);
+        if (tid < C) bet[tid] = tid < n ? p.beta[(int64_t)(sq.tok0 + ci * C + tid) * H + h] : 0.f;
+        // ---- C. scaled bf16 operands Qh = q 2^(b-m), Ka = k 2^(b-m), Kb = k 2^(m-b)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = 4 * prb + i;
+            const uint32_t so = pkb * 8192 + tc::sw128(r, pcc);
             const uint4 qraw = *reinterpret_cast<const uint4 *>(sm + STG_Q + so);
             const uint4 kraw = *reinterpret_cast<const uint4 *>(sm + STG_K + so);
-            const int c0 = kb * 64 + cc * 8;
-            const float4 b_lo = *reinterpret_cast<const float4 *>(Gs + r * D + c0);
-            const float4 b_hi = *reinterpret_cast<const float4 *>(Gs + r * D + c0 + 4);
-            const float bv[8] = {b_lo.x, b_lo.y, b_lo.z, b_lo.w, b_hi.x, b_hi.y, b_hi.z, b_hi.w};
             const uint32_t qw[4] = {qraw.x, qraw.y, qraw.z, qraw.w};
             const uint32_t kw[4] = {kraw.x, kraw.y, kraw.z, kraw.w};
             uint32_t oq[4], oa[4], ob[4];
@@ -200,19 +220,27 @@ __global__ void __launch_bounds__(128, 1) prefill_tc_kernel(const __grid_constan
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float2 qf = unpack_bf16(qw[e]), kf = unpack_bf16(kw[e]);
-                const float m0 = mC[c0 + 2 * e], m1 = mC[c0 + 2 * e + 1];
-                const float e10 = expf(bv[2 * e] - m0), e11 = expf(bv[2 * e + 1] - m1);
-                const float e20 = expf(m0 - bv[2 * e]), e21 = expf(m1 - bv[2 * e + 1]);
+                const float d0 = b[i][2 * e] - m2[2 * e], d1 = b[i][2 * e + 1] - m2[2 * e + 1];
+                const float e10 = tc::ex2(d0), e11 = tc::ex2(d1);
+                const float e20 = tc::ex2(-d0), e21 = tc::ex2(-d1);
                 oq[e] = live ? pack_bf16(qf.x * e10, qf.y * e11) : 0u;
                 oa[e] = live ? pack_bf16(kf.x * e10, kf.y * e11) : 0u;
                 ob[e] = live ? pack_bf16(kf.x * e20, kf.y * e21) : 0u;
             }
-            *reinterpret_cast<uint4 *>(sm + OP_AK + kb * 16384 + tc::sw128(r, cc)) =
+            *reinterpret_cast<uint4 *>(sm + OP_AK + pkb * 16384 + tc::sw128(r, pcc)) =
                 make_uint4(oq[0], oq[1], oq[2], oq[3]);
-            *reinterpret_cast<uint4 *>(sm + OP_AK + kb * 16384 + tc::sw128(64 + r, cc)) =
+            *reinterpret_cast<uint4 *>(sm + OP_AK + pkb * 16384 + tc::sw128(64 + r, pcc)) =
                 make_uint4(oa[0], oa[1], oa[2], oa[3]);
-            *reinterpret_cast<uint4 *>(sm + OP_KB + kb * 8192 + tc::sw128(r, cc)) =
+            *reinterpret_cast<uint4 *>(sm + OP_KB + pkb * 8192 + tc::sw128(r, pcc)) =
                 make_uint4(ob[0], ob[1], ob[2], ob[3]);
+        }
+        __syncthreads();   // eM visible
+        // ---- Sm = Diag(e^m) S_0 (bf16 operand of the chain products) ---------
+        {
+            const float em = eM[c_own];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+                *reinterpret_cast<uint4 *>(sm + OP_SM + tc::sw128(c_own, 4 * wh + q4)) = pack8(S + 8 * q4, em);
         }
         tc::fence_async_smem();
         __syncthreads();
@@ -236,38 +264,35 @@ __global__ void __launch_bounds__(128, 1) prefill_tc_kernel(const __grid_constan
         tc::fence_after_sync();
         // ---- E. A_qk (masked, bf16 operand) and L = Diag(beta) A_kk (fp32) --
         {
-            const int r = tid & 63;
             float a[32];
+            tc::tmem_ld32(tbase + tlane + COL_A + 32 * wh, a);
+            tc::tmem_ld_wait();
+            if (wq < 2) {
+                const int r = 32 * wq + lane;
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                tc::tmem_ld32(tbase + tlane + COL_A + 32 * half, a);
-                tc::tmem_ld_wait();
-                if (warp < 2) {
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint32_t w[4];
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int jj = 32 * half + 8 * q4 + 2 * e;
-                            w[e] = pack_bf16(jj <= r ? a[8 * q4 + 2 * e] : 0.f,
-                                             jj + 1 <= r ? a[8 * q4 + 2 * e + 1] : 0.f);
-                        }
-                        *reinterpret_cast<uint4 *>(sm + OP_AQK + tc::sw128(r, 4 * half + q4)) =
-                            make_uint4(w[0], w[1], w[2], w[3]);
+                    for (int e = 0; e < 4; ++e) {
+                        const int jj = 32 * wh + 8 * q4 + 2 * e;
+                        w[e] = pack_bf16(jj <= r ? a[8 * q4 + 2 * e] : 0.f, jj + 1 <= r ? a[8 * q4 + 2 * e + 1] : 0.f);
                     }
-                } else {
-                    const float br = bet[r];
+                    *reinterpret_cast<uint4 *>(sm + OP_AQK + tc::sw128(r, 4 * wh + q4)) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            } else {
+                const int r = 32 * (wq - 2) + lane;
+                const float br = bet[r];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int jj = 32 * half + e;
-                        Ls[r * 65 + jj] = jj < r ? br * a[e] : 0.f;
-                    }
+                for (int e = 0; e < 32; ++e) {
+                    const int jj = 32 * wh + e;
+                    Ls[r * 65 + jj] = jj < r ? br * a[e] : 0.f;
                 }
             }
         }
         __syncthreads();
-        // ---- F. X = (I + L)^{-1}, blocked by 16; T = X Diag(beta) -----------
-        // F1: the four 16x16 diagonal blocks, one column per thread (64 threads)
+        // ---- F. X = (I + L)^{-1}: 16x16 diagonal blocks by forward substitution
+        // (fp32), off-diagonal blocks X[R][Cb] = -X[R][R] sum_J L[R][J] X[J][Cb]
+        // by distance R - Cb on tf32 mma.sync; T = X Diag(beta) -> bf16 -------
         if (tid < 64) {
             const int blk = tid >> 4, c = tid & 15, base = 16 * blk;
             float x[16];
@@ -278,50 +303,29 @@ __global__ void __launch_bounds__(128, 1) prefill_tc_kernel(const __grid_constan
                 for (int i = 0; i < r; ++i) acc = fmaf(-Ls[(base + r) * 65 + base + i], x[i], acc);
                 x[r] = acc;
             }
-            // X overwrites L inside the diagonal block (L there is no longer needed
-            // by other threads: each thread reads only its own block's rows)
             __syncwarp();
 #pragma unroll
             for (int r = 0; r < 16; ++r) Ls[(base + r) * 65 + base + c] = x[r];
         }
         __syncthreads();
-        // F2: off-diagonal blocks by distance d = R - Cb = 1, 2, 3:
-        //   X[R][Cb] = -X[R][R] * sum_{Cb <= J < R} L[R][J] X[J][Cb]
-        // L stays in Ls (off-diagonal blocks), the diagonal blocks of Ls now
-        // hold X[b][b]; the six off-diagonal X blocks and the partial sums Y
-        // live in the OP_WK region, which is free until step H writes Wk.
-        float *Xo = reinterpret_cast<float *>(sm + OP_WK);   // 6 blocks of 16x16
-        float *Y = Xo + 6 * 256;                               // up to 3 blocks
-        auto xslot = [](int dist, int bi) { return (dist == 1 ? 0 : dist == 2 ? 3 : 5) + bi; };
 #pragma unroll 1
         for (int dist = 1; dist < 4; ++dist) {
-            const int nb = 4 - dist;                 // blocks at this distance
-            for (int e = tid; e < nb * 256; e += NT) {
-                const int bi = e >> 8, a = (e >> 4) & 15, bcol = e & 15;
-                const int R = bi + dist, Cb = bi;
-                float acc = 0.f;
-                for (int J = Cb; J < R; ++J) {
-                    const float *xj = J == Cb ? Ls + (16 * J) * 65 + 16 * Cb : Xo + xslot(J - Cb, Cb) * 256;
-                    const int xs = J == Cb ? 65 : 16;
-#pragma unroll
-                    for (int l = 0; l < 16; ++l)
-                        acc = fmaf(Ls[(16 * R + a) * 65 + 16 * J + l], xj[l * xs + bcol], acc);
+            if (warp < 4 - dist) {
+                const int cb = warp, R = cb + dist;
+                float pacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                for (int J = cb; J < R; ++J) {
+                    const float *xj = J == cb ? Ls + (16 * J) * 65 + 16 * cb : Xo + xslot(J - cb, cb) * 256;
+                    tc::mma16x16(pacc, Ls + (16 * R) * 65 + 16 * J, 65, xj, J == cb ? 65 : 16);
                 }
-                Y[e] = acc;
-            }
-            __syncthreads();
-            for (int e = tid; e < nb * 256; e += NT) {
-                const int bi = e >> 8, a = (e >> 4) & 15, bcol = e & 15;
-                const int R = bi + dist;
-                float acc = 0.f;
-#pragma unroll
-                for (int l = 0; l < 16; ++l)
-                    acc = fmaf(Ls[(16 * R + a) * 65 + 16 * R + l], Y[(bi << 8) + (l << 4) + bcol], acc);
-                Xo[xslot(dist, bi) * 256 + a * 16 + bcol] = -acc;
+                float *yw = Yw + warp * 256;
+                tc::store16x16(yw, 16, pacc, 1.f);
+                __syncwarp();
+                float pr[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                tc::mma16x16(pr, Ls + (16 * R) * 65 + 16 * R, 65, yw, 16);
+                tc::store16x16(Xo + xslot(dist, cb) * 256, 16, pr, -1.f);
             }
             __syncthreads();
         }
-        // T[r][c] = X[r][c] beta_c (zero above the diagonal) -> bf16 slab
         for (int e = tid; e < 64 * 8; e += NT) {
             const int r = e >> 3, cc = e & 7;
             uint32_t w[4];
@@ -333,7 +337,7 @@ __global__ void __launch_bounds__(128, 1) prefill_tc_kernel(const __grid_constan
                     const int c = 8 * cc + 2 * q + t2;
                     const int R = r >> 4, Cb = c >> 4;
                     float x = 0.f;
-                    if (R == Cb) x = c <= r ? Ls[r * 65 + c] : 0.f;
+                    if (R == Cb) x = Ls[r * 65 + c];
                     else if (R > Cb) x = Xo[xslot(R - Cb, Cb) * 256 + (r & 15) * 16 + (c & 15)];
                     x2[t2] = x * bet[c];
                 }
@@ -365,18 +369,17 @@ __global__ void __launch_bounds__(128, 1) prefill_tc_kernel(const __grid_constan
         tc::fence_after_sync();
         // ---- H. Wk -> bf16 operand (M=64 layout: lanes 32w..32w+15 = rows 16w..) ---
         {
-            const int r = 16 * warp + (lane & 15);
+            const int r = 16 * wq + (lane & 15);
             float a[32];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                tc::tmem_ld32(tbase + tlane + COL_WK + 32 * q, a);
+            for (int q = 0; q < 2; ++q) {
+                tc::tmem_ld32(tbase + tlane + COL_WK + 64 * wh + 32 * q, a);
                 tc::tmem_ld_wait();
                 if (lane < 16) {
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4)
-                        *reinterpret_cast<uint4 *>(sm + OP_WK + (q >> 1) * 8192 + tc::sw128(r, 4 * (q & 1) + q4)) =
-                            make_uint4(pack_bf16(a[8 * q4], a[8 * q4 + 1]), pack_bf16(a[8 * q4 + 2], a[8 * q4 + 3]),
-                                       pack_bf16(a[8 * q4 + 4], a[8 * q4 + 5]), pack_bf16(a[8 * q4 + 6], a[8 * q4 + 7]));
+                        *reinterpret_cast<uint4 *>(sm + OP_WK + wh * 8192 + tc::sw128(r, 4 * q + q4)) =
+                            pack8(a + 8 * q4, 1.f);
                 }
             }
         }
@@ -404,19 +407,14 @@ __global__ void __launch_bounds__(128, 1) prefill_tc_kernel(const __grid_constan
         tc::fence_after_sync();
         // ---- J. W -> bf16 operand ------------------------------------------------
         {
-            const int r = 16 * warp + (lane & 15);
+            const int r = 16 * wq + (lane & 15);
             float a[32];
+            tc::tmem_ld32(tbase + tlane + COL_W + 32 * wh, a);
+            tc::tmem_ld_wait();
+            if (lane < 16) {
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                tc::tmem_ld32(tbase + tlane + COL_W + 32 * q, a);
-                tc::tmem_ld_wait();
-                if (lane < 16) {
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4)
-                        *reinterpret_cast<uint4 *>(sm + OP_W + tc::sw128(r, 4 * q + q4)) =
-                            make_uint4(pack_bf16(a[8 * q4], a[8 * q4 + 1]), pack_bf16(a[8 * q4 + 2], a[8 * q4 + 3]),
-                                       pack_bf16(a[8 * q4 + 4], a[8 * q4 + 5]), pack_bf16(a[8 * q4 + 6], a[8 * q4 + 7]));
-                }
+                for (int q4 = 0; q4 < 4; ++q4)
+                    *reinterpret_cast<uint4 *>(sm + OP_W + tc::sw128(r, 4 * wh + q4)) = pack8(a + 8 * q4, 1.f);
             }
         }
         tc::fence_async_smem();
@@ -443,36 +441,25 @@ __global__ void __launch_bounds__(128, 1) prefill_tc_kernel(const __grid_constan
         tc::fence_after_sync();
         // ---- L. outputs, state update, snapshot ---------------------------------
         {
-            const int r = 16 * warp + (lane & 15);
             float a[32];
-            __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(p.o);
+            const int r = 16 * wq + (lane & 15);
+            tc::tmem_ld32(tbase + tlane + COL_O + 32 * wh, a);
+            tc::tmem_ld_wait();
+            if (lane < 16 && r < n) {
+                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) +
+                                                       ((int64_t)(sq.tok0 + ci * C + r) * H + h) * D + j0 + 32 * wh);
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                tc::tmem_ld32(tbase + tlane + COL_O + 32 * q, a);
-                tc::tmem_ld_wait();
-                if (lane < 16 && r < n) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(
-                        og + ((int64_t)(sq.tok0 + ci * C + r) * H + h) * D + j0 + 32 * q);
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4)
-                        dst[q4] = make_uint4(pack_bf16(p.scale * a[8 * q4], p.scale * a[8 * q4 + 1]),
-                                             pack_bf16(p.scale * a[8 * q4 + 2], p.scale * a[8 * q4 + 3]),
-                                             pack_bf16(p.scale * a[8 * q4 + 4], p.scale * a[8 * q4 + 5]),
-                                             pack_bf16(p.scale * a[8 * q4 + 6], p.scale * a[8 * q4 + 7]));
-                }
+                for (int q4 = 0; q4 < 4; ++q4) dst[q4] = pack8(a + 8 * q4, p.scale);
             }
-            const float g_c = gC[tid], e_c = eC[tid];
+            const float g_c = gC[c_own], e_c = eC[c_own];
+            tc::tmem_ld32(tbase + tlane + COL_S + 32 * wh, a);
+            tc::tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                tc::tmem_ld32(tbase + tlane + COL_S + 32 * q, a);
-                tc::tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) S[32 * q + e] = fmaf(g_c, S[32 * q + e], e_c * a[e]);
-            }
+            for (int e = 0; e < 32; ++e) S[e] = fmaf(g_c, S[e], e_c * a[e]);
             if (p.snap_interval > 0 && (sq.start_pos + (int64_t)ci * C + n) % p.snap_interval == 0) {
-                float *dst = p.snapshots + ((snap_row * H + h) * D + tid) * (int64_t)D + j0;
+                float *dst = p.snapshots + ((snap_row * H + h) * D + c_own) * (int64_t)D + j0 + 32 * wh;
 #pragma unroll
-                for (int j = 0; j < DVS; j += 4)
+                for (int j = 0; j < 32; j += 4)
                     *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
                 ++snap_row;
             }
@@ -482,9 +469,9 @@ __global__ void __launch_bounds__(128, 1) prefill_tc_kernel(const __grid_constan
     }
 
     if (ok && p.state_out) {
-        float *dst = p.state_out + (((int64_t)s * H + h) * D + tid) * (int64_t)D + j0;
+        float *dst = p.state_out + (((int64_t)s * H + h) * D + c_own) * (int64_t)D + j0 + 32 * wh;
 #pragma unroll
-        for (int j = 0; j < DVS; j += 4)
+        for (int j = 0; j < 32; j += 4)
             *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
     }
     // teardown: on an early exit, let loads already in flight land before the

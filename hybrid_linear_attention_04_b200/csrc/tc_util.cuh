@@ -159,5 +159,55 @@ __device__ __forceinline__ void tma_load3(void *smem_dst, const CUtensorMap *m, 
         : "memory");
 }
 
+// ---- small warp-level helpers ----------------------------------------------------
+// 2^x (hardware approximation, relative error ~2^-22; inputs here are bounded)
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+// D[16x8] += A[16x8] B[8x8], tf32 inputs, fp32 accumulate (warp-wide).
+// Fragments (g = lane/4, t = lane%4): a = A[g][t], A[g+8][t], A[g][t+4], A[g+8][t+4];
+// b = B[t][g], B[t+4][g]; d = D[g][2t], D[g][2t+1], D[g+8][2t], D[g+8][2t+1].
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// P[16x16] += A[16x16] B[16x16]; A, B fp32 in shared memory with row strides sa, sb.
+// Result fragments: p[nt] covers columns 8nt..8nt+7 in the d layout above.
+__device__ __forceinline__ void mma16x16(float (&p)[2][4], const float *A, int sa, const float *B, int sb) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+        const uint32_t a[4] = {to_tf32(A[g * sa + 8 * kk + t]), to_tf32(A[(g + 8) * sa + 8 * kk + t]),
+                               to_tf32(A[g * sa + 8 * kk + t + 4]), to_tf32(A[(g + 8) * sa + 8 * kk + t + 4])};
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const uint32_t b[2] = {to_tf32(B[(8 * kk + t) * sb + 8 * nt + g]),
+                                   to_tf32(B[(8 * kk + t + 4) * sb + 8 * nt + g])};
+            mma_tf32(p[nt], a, b);
+        }
+    }
+}
+// store P (fragments) scaled by `s` into a 16x16 fp32 block with row stride ld
+__device__ __forceinline__ void store16x16(float *Pm, int ld, const float (&p)[2][4], float s) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        Pm[g * ld + 8 * nt + 2 * t] = s * p[nt][0];
+        Pm[g * ld + 8 * nt + 2 * t + 1] = s * p[nt][1];
+        Pm[(g + 8) * ld + 8 * nt + 2 * t] = s * p[nt][2];
+        Pm[(g + 8) * ld + 8 * nt + 2 * t + 1] = s * p[nt][3];
+    }
+}
+
 }  // namespace tc
 }  // namespace kda
