@@ -334,6 +334,12 @@ void kda_internal_force_prefill_path(int32_t path) { g_prefill_path.store(path);
 
 }  // extern "C"
 
+#ifdef KDA_PHASE_TIMING
+extern "C" int kda_internal_phase_clock(long long *out) {
+    return (int)cudaMemcpyFromSymbol(out, kda::g_phase_clock, sizeof(kda::g_phase_clock));
+}
+#endif
+
 // ------------------------------------------------ failure-injection hook ----
 namespace kda {
 __device__ int g_never_set;

@@ -13,13 +13,15 @@
 //   tcgen05  [Qh; Ka] Kb^T -> TMEM (M=128: A_qk rows 0-63, A_kk rows 64-127)
 //   CUDA     T = (I + Diag(beta) A_kk)^{-1} Diag(beta) by blocked forward
 //   cores    substitution in fp32 (16x16 diagonal blocks, then merges)
-//   tcgen05  Wk = T Ka, U = T V                      (M=64)
-//            W = U - Wk Sm, O = Qh Sm                (M=64; Sm = Diag(e^m) S_0)
+//   tcgen05  (same round as A) R' = Ka Sm, O = Qh Sm  (M=64; Sm = Diag(e^m) S_0)
+//   CUDA     R = V - R' (bf16), concurrently with the solve
+//   tcgen05  W = T R                                 (M=64)
 //            O += A_qk W, D = Kb^T W                 (M=64 / M=128)
 //   CUDA     o = scale O (bf16 store); S_C = Diag(Gamma_C) S_0 + Diag(e^(b_C-m)) D
 //   cores    with the fp32 master state held in registers (thread = d_k row).
 // Identities used: Q.Gamma = Qh.e^m and K.Gamma = Ka.e^m, so (Q.Gamma) S_0 =
-// Qh Sm and (K.Gamma) S_0 = Ka Sm; K.exp(b_C-b) = Kb.e^(b_C-m) row-wise.
+// Qh Sm and (K.Gamma) S_0 = Ka Sm; K.exp(b_C-b) = Kb.e^(b_C-m) row-wise; and
+// W = T (V - (K.Gamma) S_0) = T R.
 // A chunk whose per-channel decay from its middle exceeds 80 nats in either
 // direction is reported through the status word (KDA_ERR_RANGE).
 #pragma once
@@ -30,6 +32,14 @@
 
 namespace kda {
 
+#ifdef KDA_PHASE_TIMING
+__device__ long long g_phase_clock[64][16];
+#define KDA_MARK(ci, k) \
+    do { if (threadIdx.x == 0 && blockIdx.x == 0 && (ci) < 64) g_phase_clock[(ci)][(k)] = clock64(); } while (0)
+#else
+#define KDA_MARK(ci, k) do { } while (0)
+#endif
+
 struct TcParams {
     CUtensorMap tm_q, tm_k, tm_v, tm_g;
     PrefillParams p;
@@ -38,24 +48,27 @@ struct TcParams {
 namespace tcp {
 constexpr int C = 64, D = 128, DVS = 64, NT = 256;
 // shared memory map (bytes from a 1024-aligned base)
-constexpr uint32_t STG_Q = 0;          // q   [64 tok x 128 ch] bf16: 2 slabs of 64 rows
-constexpr uint32_t STG_K = 16384;      // k   same
-constexpr uint32_t STG_V = 32768;      // v   slice, 2 buffers of 1 slab [64 tok x 64]
+constexpr uint32_t STG_Q = 0;          // q  [64 tok x 128 ch] bf16: 2 slabs of 64 rows
+constexpr uint32_t STG_K = 16384;      // k  same
+constexpr uint32_t STG_V = 32768;      // v  slice, 2 buffers of 1 slab [64 tok x 64]
 constexpr uint32_t OP_AK = 49152;      // [Qh; Ka]: 2 slabs of 128 rows (channels 0-63, 64-127)
-constexpr uint32_t OP_KB = 81920;      // Kb: 2 slabs of 64 rows
-constexpr uint32_t OP_T = 98304;       // T  [64 x 64]
-constexpr uint32_t OP_WK = 106496;     // Wk [64 tok x 128 ch]: 2 slabs; solve scratch before that
+constexpr uint32_t OP_KB = 81920;      // [Kb; Sm^T]: 2 slabs (channels 0-63, 64-127) of 128 rows:
+                                       // rows 0-63 Kb (tokens), rows 64-127 Sm^T (d_v columns)
+constexpr uint32_t OP_T = 114688;      // T  [64 x 64]
 constexpr uint32_t OP_AQK = 122880;    // A_qk masked [64 x 64]
-constexpr uint32_t OP_W = 131072;      // W  [64 tok x 64 dv]
-constexpr uint32_t OP_SM = 139264;     // Sm [128 ch x 64 dv]: 1 slab of 128 rows
-constexpr uint32_t STG_G = 155648;     // g, fp32 [64][128]
-constexpr uint32_t SOLVE = 188416;     // fp32 [64][65]: L off the diagonal, X on it
-constexpr uint32_t VEC = SOLVE + 64 * 65 * 4;  // eM, eC, gC [128] + bet [64]
+constexpr uint32_t OP_RW = 131072;     // R = V - Ka Sm, then W [64 tok x 64 dv]
+constexpr uint32_t STG_G = 139264;     // g, fp32 [64][128]
+constexpr uint32_t SOLVE = 172032;     // fp32 [64][65]: L off the diagonal blocks, X on them
+constexpr uint32_t XO = SOLVE + 64 * 65 * 4;   // 6 off-diagonal X blocks + 3 scratch blocks (16x16 fp32)
+constexpr uint32_t TOT = XO + 9 * 1024;        // per-warp row-block totals of b [8][128]
+constexpr uint32_t VEC = TOT + 8 * 128 * 4;    // eM, eC, gC [128] + beta [64]
 constexpr uint32_t BARS = VEC + (3 * 128 + 64) * 4;
-constexpr uint32_t SMEM_USED = BARS + 32;
+constexpr uint32_t SMEM_USED = BARS + 48;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
 // TMEM columns
-constexpr uint32_t COL_A = 0, COL_WK = 64, COL_W = 192, COL_O = 256, COL_S = 320, TMEM_COLS = 512;
+// round 1 writes [A_qk | O ; A_kk | R'] into columns 0-127 (rows 0-63 | 64-127);
+// W = T R lands in COL_W (M=64), D = Kb^T W in COL_S
+constexpr uint32_t COL_A = 0, COL_O = 64, COL_W = 128, COL_S = 192, TMEM_COLS = 256;
 constexpr uint32_t CHUNK_TX = 16384 + 16384 + 32768 + 8192;   // bytes per chunk of loads
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RANGE_LIMIT2 = 80.f * LOG2E;    // 80 nats, in log2 units
@@ -84,13 +97,15 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
     const uint32_t sbase = tc::smem_u32(sm);
     float *Gs = reinterpret_cast<float *>(sm + STG_G);
     float *Ls = reinterpret_cast<float *>(sm + SOLVE);
+    float *Xo = reinterpret_cast<float *>(sm + XO);     // 6 blocks 16x16
+    float *Yw = Xo + 6 * 256;                             // 3 per-warp 16x16 blocks
+    float *Tot = reinterpret_cast<float *>(sm + TOT);
     float *eM = reinterpret_cast<float *>(sm + VEC);
     float *eC = eM + 128, *gC = eM + 256, *bet = eM + 384;
-    float *Xo = reinterpret_cast<float *>(sm + OP_WK);     // 6 blocks 16x16 (solve only)
-    float *Yw = Xo + 6 * 256;                                // 3 per-warp 16x16 blocks
     uint64_t *tma_bar = reinterpret_cast<uint64_t *>(sm + BARS);   // [2]
-    uint64_t *mma_bar = tma_bar + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_bar + 1);
+    uint64_t *mma_bar = tma_bar + 2;       // rounds 2 and 3
+    uint64_t *bar_a = tma_bar + 3;         // round 1: [Qh; Ka] [Kb; Sm^T]^T
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tma_bar + 5);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3, wh = warp >> 2;          // TMEM sub-partition, column half
@@ -107,6 +122,7 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
         tc::bar_init(&tma_bar[0], 1);
         tc::bar_init(&tma_bar[1], 1);
         tc::bar_init(mma_bar, 1);
+        tc::bar_init(bar_a, 1);
         tc::bar_init_fence();
         tc::tma_prefetch_desc(&P.tm_q);
         tc::tma_prefetch_desc(&P.tm_k);
@@ -157,255 +173,278 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
         issue_loads(0);
         issued = 1;
     }
-    // prep-phase thread map: channel group u (8 channels), row block rb (4 rows)
-    const int pu = tid >> 4, prb = tid & 15, pc0 = 8 * pu, pkb = pu >> 3, pcc = pu & 7;
+    // smem matrix descriptors (start-address field advanced by 16-byte units)
+    const uint64_t dAK = tc::desc_k(sbase + OP_AK, 0), dKB = tc::desc_k(sbase + OP_KB, 0);
+    const uint64_t dT = tc::desc_k(sbase + OP_T, 0), dAQK = tc::desc_k(sbase + OP_AQK, 0);
+    const uint64_t dRW = tc::desc_mn(sbase + OP_RW, 0, 8192);
+    const uint64_t dKBmn = tc::desc_mn(sbase + OP_KB, 0, 16384);
+    // T's blocks above the diagonal are always zero: clear the whole T tile once
+    // (the diagonal and lower blocks are rewritten every chunk)
+    for (int e = tid; e < 64 * 8; e += NT)
+        *reinterpret_cast<uint4 *>(sm + OP_T + 16 * e) = make_uint4(0u, 0u, 0u, 0u);
+    // prep map: warp w owns rows 8w..8w+7, lane l owns channels 4l..4l+3
+    const int pkb = lane >> 4, pchk = (lane & 15) >> 1, phf = (lane & 1) * 8;
 
     for (int ci = 0; ci < n_chunks; ++ci) {
         const int n = min(C, sq.len - ci * C);
+        KDA_MARK(ci, 0);
         // ---- A. this chunk's operands have landed --------------------------
         ok = tc::bar_wait(&tma_bar[ci & 1], (ci >> 1) & 1);
         if (!__syncthreads_and(ok)) { ok = false; break; }
         landed = ci + 1;
-        // ---- B. b = cumsum(g) in log2 units: local 4 rows, then a 16-lane scan
-        float b[4][8];
+        KDA_MARK(ci, 1);
+        // ---- B. b = cumsum(g) over the chunk, in log2 units -------------------
+        float b[8][4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int r = 4 * prb + i;
-            const float4 x0 = *reinterpret_cast<const float4 *>(Gs + r * D + pc0);
-            const float4 x1 = *reinterpret_cast<const float4 *>(Gs + r * D + pc0 + 4);
+        for (int i = 0; i < 8; ++i) {
+            const int r = 8 * warp + i;
+            const float4 x = *reinterpret_cast<const float4 *>(Gs + r * D + 4 * lane);
             const float sc = r < n ? LOG2E : 0.f;
-            b[i][0] = x0.x * sc; b[i][1] = x0.y * sc; b[i][2] = x0.z * sc; b[i][3] = x0.w * sc;
-            b[i][4] = x1.x * sc; b[i][5] = x1.y * sc; b[i][6] = x1.z * sc; b[i][7] = x1.w * sc;
+            b[i][0] = x.x * sc; b[i][1] = x.y * sc; b[i][2] = x.z * sc; b[i][3] = x.w * sc;
         }
 #pragma unroll
-        for (int i = 1; i < 4; ++i)
+        for (int i = 1; i < 8; ++i)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) b[i][e] += b[i - 1][e];
-        float m2[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const float tot = b[3][e];
-            float incl = tot;
-#pragma unroll
-            for (int off = 1; off < 16; off <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, incl, off, 16);
-                if (prb >= off) incl += y;
-            }
-            const float ex = incl - tot;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) b[i][e] += ex;
-            m2[e] = __shfl_sync(0xffffffffu, b[3][e], 7, 16);        // row 31
-            const float bc = __shfl_sync(0xffffffffu, b[3][e], 15, 16);  // row 63
-            const float b0 = __shfl_sync(0xffffffffu, b[0][e], 0, 16);   // row 0
-            if (prb == 0) {
-                const int c = pc0 + e;
-                eM[c] = tc::ex2(m2[e]);
-                eC[c] = tc::ex2(bc - m2[e]);
-                gC[c] = tc::ex2(bc);
-                if (b0 - m2[e] > RANGE_LIMIT2 || m2[e] - bc > RANGE_LIMIT2) record_status(KDA_ERR_RANGE);
-            }
-        }
+            for (int e = 0; e < 4; ++e) b[i][e] += b[i - 1][e];
+        *reinterpret_cast<float4 *>(Tot + warp * 128 + 4 * lane) = make_float4(b[7][0], b[7][1], b[7][2], b[7][3]);
         if (tid < C) bet[tid] = tid < n ? p.beta[(int64_t)(sq.tok0 + ci * C + tid) * H + h] : 0.f;
+        __syncthreads();
+        float m2[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+            float off[4] = {0.f, 0.f, 0.f, 0.f}, bc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int w2 = 0; w2 < 8; ++w2) {
+                const float4 t = *reinterpret_cast<const float4 *>(Tot + w2 * 128 + 4 * lane);
+                const float tv[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    if (w2 < warp) off[e] += tv[e];
+                    if (w2 < 4) m2[e] += tv[e];     // b at row 31
+                    bc[e] += tv[e];                 // b at row 63
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) b[i][e] += off[e];
+            if (warp == 0) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int c = 4 * lane + e;
+                    eM[c] = tc::ex2(m2[e]);
+                    eC[c] = tc::ex2(bc[e] - m2[e]);
+                    gC[c] = tc::ex2(bc[e]);
+                    // b <= 0, so row 0 is at most -m above the reference
+                    if (-m2[e] > RANGE_LIMIT2 || m2[e] - bc[e] > RANGE_LIMIT2) record_status(KDA_ERR_RANGE);
+                }
+            }
+        }
         // ---- C. scaled bf16 operands Qh = q 2^(b-m), Ka = k 2^(b-m), Kb = k 2^(m-b)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int r = 4 * prb + i;
-            const uint32_t so = pkb * 8192 + tc::sw128(r, pcc);
-            const uint4 qraw = *reinterpret_cast<const uint4 *>(sm + STG_Q + so);
-            const uint4 kraw = *reinterpret_cast<const uint4 *>(sm + STG_K + so);
-            const uint32_t qw[4] = {qraw.x, qraw.y, qraw.z, qraw.w};
-            const uint32_t kw[4] = {kraw.x, kraw.y, kraw.z, kraw.w};
-            uint32_t oq[4], oa[4], ob[4];
-            const bool live = r < n;
+        for (int i = 0; i < 8; ++i) {
+            const int r = 8 * warp + i;
+            const uint32_t so = pkb * 8192 + tc::sw128(r, pchk) + phf;
+            const uint2 qv = *reinterpret_cast<const uint2 *>(sm + STG_Q + so);
+            const uint2 kv = *reinterpret_cast<const uint2 *>(sm + STG_K + so);
+            const float2 q01 = unpack_bf16(qv.x), q23 = unpack_bf16(qv.y);
+            const float2 k01 = unpack_bf16(kv.x), k23 = unpack_bf16(kv.y);
+            float e1[4], e2[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float2 qf = unpack_bf16(qw[e]), kf = unpack_bf16(kw[e]);
-                const float d0 = b[i][2 * e] - m2[2 * e], d1 = b[i][2 * e + 1] - m2[2 * e + 1];
-                const float e10 = tc::ex2(d0), e11 = tc::ex2(d1);
-                const float e20 = tc::ex2(-d0), e21 = tc::ex2(-d1);
-                oq[e] = live ? pack_bf16(qf.x * e10, qf.y * e11) : 0u;
-                oa[e] = live ? pack_bf16(kf.x * e10, kf.y * e11) : 0u;
-                ob[e] = live ? pack_bf16(kf.x * e20, kf.y * e21) : 0u;
+                const float d = b[i][e] - m2[e];
+                e1[e] = tc::ex2(d);
+                e2[e] = tc::ex2(-d);
             }
-            *reinterpret_cast<uint4 *>(sm + OP_AK + pkb * 16384 + tc::sw128(r, pcc)) =
-                make_uint4(oq[0], oq[1], oq[2], oq[3]);
-            *reinterpret_cast<uint4 *>(sm + OP_AK + pkb * 16384 + tc::sw128(64 + r, pcc)) =
-                make_uint4(oa[0], oa[1], oa[2], oa[3]);
-            *reinterpret_cast<uint4 *>(sm + OP_KB + pkb * 8192 + tc::sw128(r, pcc)) =
-                make_uint4(ob[0], ob[1], ob[2], ob[3]);
+            const bool live = r < n;
+            const uint2 oq = live ? make_uint2(pack_bf16(q01.x * e1[0], q01.y * e1[1]), pack_bf16(q23.x * e1[2], q23.y * e1[3]))
+                                  : make_uint2(0u, 0u);
+            const uint2 oa = live ? make_uint2(pack_bf16(k01.x * e1[0], k01.y * e1[1]), pack_bf16(k23.x * e1[2], k23.y * e1[3]))
+                                  : make_uint2(0u, 0u);
+            const uint2 ob = live ? make_uint2(pack_bf16(k01.x * e2[0], k01.y * e2[1]), pack_bf16(k23.x * e2[2], k23.y * e2[3]))
+                                  : make_uint2(0u, 0u);
+            *reinterpret_cast<uint2 *>(sm + OP_AK + pkb * 16384 + tc::sw128(r, pchk) + phf) = oq;
+            *reinterpret_cast<uint2 *>(sm + OP_AK + pkb * 16384 + tc::sw128(64 + r, pchk) + phf) = oa;
+            *reinterpret_cast<uint2 *>(sm + OP_KB + pkb * 16384 + tc::sw128(r, pchk) + phf) = ob;
         }
         __syncthreads();   // eM visible
-        // ---- Sm = Diag(e^m) S_0 (bf16 operand of the chain products) ---------
+        KDA_MARK(ci, 2);
+        // ---- Sm^T = (Diag(e^m) S_0)^T (bf16, K-major B operand of round 1) ----
         {
             const float em = eM[c_own];
+            __nv_bfloat16 *st = reinterpret_cast<__nv_bfloat16 *>(sm + OP_KB + (c_own >> 6) * 16384);
+            const int cch = (c_own & 63) >> 3, cin = c_own & 7;
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-                *reinterpret_cast<uint4 *>(sm + OP_SM + tc::sw128(c_own, 4 * wh + q4)) = pack8(S + 8 * q4, em);
+            for (int j = 0; j < 32; ++j) {
+                const int row = 64 + 32 * wh + j;
+                st[(tc::sw128(row, cch) >> 1) + cin] = __float2bfloat16_rn(S[j] * em);
+            }
         }
         tc::fence_async_smem();
         __syncthreads();
-        // ---- D. next chunk's loads; A = [Qh; Ka] Kb^T ------------------------
+        KDA_MARK(ci, 3);
+        // ---- D. round 1: A = [Qh; Ka] Kb^T; R' = Ka Sm; O = Qh Sm; then the next
+        // chunk's loads (descriptors advance by 16-byte units in their low bits)
         if (tid == 0) {
+            tc::fence_after_sync();
+            constexpr uint32_t id_a = tc::idesc_bf16(128, 128, false, false);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                tc::mma_bf16(tbase + COL_A, dAK + (k >> 2) * 1024 + (k & 3) * 2, dKB + (k >> 2) * 1024 + (k & 3) * 2,
+                             id_a, k > 0);
+            tc::mma_commit(bar_a);
             if (ci + 1 < n_chunks) {
                 issue_loads(ci + 1);
                 issued = ci + 2;
             }
-            tc::fence_after_sync();
-            constexpr uint32_t id = tc::idesc_bf16(128, 64, false, false);
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                tc::mma_bf16(tbase + COL_A, tc::desc_k(sbase + OP_AK + (k >> 2) * 16384, 16 * (k & 3)),
-                             tc::desc_k(sbase + OP_KB + (k >> 2) * 8192, 16 * (k & 3)), id, k > 0);
-            tc::mma_commit(mma_bar);
         }
-        ok = tc::bar_wait(mma_bar, mma_phase);
-        mma_phase ^= 1;
-        if (!__syncthreads_and(ok)) { ok = false; break; }
+        // a timed-out wait is acted on at the block-wide vote after phase E
+        ok = tc::bar_wait(bar_a, (uint32_t)(ci & 1));
         tc::fence_after_sync();
-        // ---- E. A_qk (masked, bf16 operand) and L = Diag(beta) A_kk (fp32) --
-        {
-            float a[32];
-            tc::tmem_ld32(tbase + tlane + COL_A + 32 * wh, a);
-            tc::tmem_ld_wait();
-            if (wq < 2) {
-                const int r = 32 * wq + lane;
+        KDA_MARK(ci, 4);
+        if (warp < 4) {
+            // ---- E1. A_qk (masked bf16 operand), L = Diag(beta) A_kk, then the
+            // solve X = (I + L)^{-1} and T = X Diag(beta) (warps 0-3) ----------
+            {
+                const int r = 32 * (warp & 1) + lane;
+                float a[32];
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    uint32_t w[4];
+                for (int half = 0; half < 2; ++half) {
+                    tc::tmem_ld32(tbase + tlane + COL_A + 32 * half, a);
+                    tc::tmem_ld_wait();
+                    if (warp < 2) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int jj = 32 * wh + 8 * q4 + 2 * e;
-                        w[e] = pack_bf16(jj <= r ? a[8 * q4 + 2 * e] : 0.f, jj + 1 <= r ? a[8 * q4 + 2 * e + 1] : 0.f);
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int jj = 32 * half + 8 * q4 + 2 * e;
+                                w[e] = pack_bf16(jj <= r ? a[8 * q4 + 2 * e] : 0.f,
+                                                 jj + 1 <= r ? a[8 * q4 + 2 * e + 1] : 0.f);
+                            }
+                            *reinterpret_cast<uint4 *>(sm + OP_AQK + tc::sw128(r, 4 * half + q4)) =
+                                make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    } else {
+                        const float br = bet[r];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int jj = 32 * half + e;
+                            Ls[r * 65 + jj] = jj < r ? br * a[e] : 0.f;
+                        }
                     }
-                    *reinterpret_cast<uint4 *>(sm + OP_AQK + tc::sw128(r, 4 * wh + q4)) = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-            } else {
-                const int r = 32 * (wq - 2) + lane;
-                const float br = bet[r];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int jj = 32 * wh + e;
-                    Ls[r * 65 + jj] = jj < r ? br * a[e] : 0.f;
                 }
             }
-        }
-        __syncthreads();
-        // ---- F. X = (I + L)^{-1}: 16x16 diagonal blocks by forward substitution
-        // (fp32), off-diagonal blocks X[R][Cb] = -X[R][R] sum_J L[R][J] X[J][Cb]
-        // by distance R - Cb on tf32 mma.sync; T = X Diag(beta) -> bf16 -------
-        if (tid < 64) {
-            const int blk = tid >> 4, c = tid & 15, base = 16 * blk;
-            float x[16];
+            tc::named_sync(1, 128);
+            KDA_MARK(ci, 10);
+            // 16x16 diagonal blocks by forward substitution, one column per thread
+            if (tid < 64) {
+                const int blk = tid >> 4, c = tid & 15, base = 16 * blk;
+                float x[16];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float acc = r == c ? 1.f : 0.f;
+                for (int r = 0; r < 16; ++r) {
+                    float a0 = r == c ? 1.f : 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                    const float *lr = Ls + (base + r) * 65 + base;
 #pragma unroll
-                for (int i = 0; i < r; ++i) acc = fmaf(-Ls[(base + r) * 65 + base + i], x[i], acc);
-                x[r] = acc;
-            }
-            __syncwarp();
-#pragma unroll
-            for (int r = 0; r < 16; ++r) Ls[(base + r) * 65 + base + c] = x[r];
-        }
-        __syncthreads();
-#pragma unroll 1
-        for (int dist = 1; dist < 4; ++dist) {
-            if (warp < 4 - dist) {
-                const int cb = warp, R = cb + dist;
-                float pacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                for (int J = cb; J < R; ++J) {
-                    const float *xj = J == cb ? Ls + (16 * J) * 65 + 16 * cb : Xo + xslot(J - cb, cb) * 256;
-                    tc::mma16x16(pacc, Ls + (16 * R) * 65 + 16 * J, 65, xj, J == cb ? 65 : 16);
+                    for (int i = 0; i < r; ++i) {
+                        const float t = lr[i] * x[i];
+                        if ((i & 3) == 0) a0 -= t;
+                        else if ((i & 3) == 1) a1 -= t;
+                        else if ((i & 3) == 2) a2 -= t;
+                        else a3 -= t;
+                    }
+                    x[r] = (a0 + a1) + (a2 + a3);
                 }
-                float *yw = Yw + warp * 256;
-                tc::store16x16(yw, 16, pacc, 1.f);
                 __syncwarp();
-                float pr[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                tc::mma16x16(pr, Ls + (16 * R) * 65 + 16 * R, 65, yw, 16);
-                tc::store16x16(Xo + xslot(dist, cb) * 256, 16, pr, -1.f);
-            }
-            __syncthreads();
-        }
-        for (int e = tid; e < 64 * 8; e += NT) {
-            const int r = e >> 3, cc = e & 7;
-            uint32_t w[4];
+                const float bc = bet[base + c];
+                __nv_bfloat16 *tt = reinterpret_cast<__nv_bfloat16 *>(sm + OP_T);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                float x2[2];
-#pragma unroll
-                for (int t2 = 0; t2 < 2; ++t2) {
-                    const int c = 8 * cc + 2 * q + t2;
-                    const int R = r >> 4, Cb = c >> 4;
-                    float x = 0.f;
-                    if (R == Cb) x = Ls[r * 65 + c];
-                    else if (R > Cb) x = Xo[xslot(R - Cb, Cb) * 256 + (r & 15) * 16 + (c & 15)];
-                    x2[t2] = x * bet[c];
+                for (int r = 0; r < 16; ++r) {
+                    Ls[(base + r) * 65 + base + c] = x[r];
+                    const int rr = base + r, cc = base + c;
+                    tt[(tc::sw128(rr, cc >> 3) >> 1) + (cc & 7)] = __float2bfloat16_rn(x[r] * bc);
                 }
-                w[q] = pack_bf16(x2[0], x2[1]);
             }
-            *reinterpret_cast<uint4 *>(sm + OP_T + tc::sw128(r, cc)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        tc::fence_async_smem();
-        tc::fence_before_sync();
-        __syncthreads();
-        // ---- G. Wk = T Ka, U = T V --------------------------------------------
-        if (tid == 0) {
-            tc::fence_after_sync();
-            constexpr uint32_t id_wk = tc::idesc_bf16(64, 128, false, true);
-            constexpr uint32_t id_u = tc::idesc_bf16(64, 64, false, true);
+            tc::named_sync(1, 128);
+            KDA_MARK(ci, 11);
+            // off-diagonal blocks by distance: X[R][Cb] = -X[R][R] sum_J L[R][J] X[J][Cb]
+#pragma unroll 1
+            for (int dist = 1; dist < 4; ++dist) {
+                if (warp < 4 - dist) {
+                    const int cb = warp, R = cb + dist;
+                    float pacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                    for (int J = cb; J < R; ++J) {
+                        const float *xj = J == cb ? Ls + (16 * J) * 65 + 16 * cb : Xo + xslot(J - cb, cb) * 256;
+                        tc::mma16x16(pacc, Ls + (16 * R) * 65 + 16 * J, 65, xj, J == cb ? 65 : 16);
+                    }
+                    float *yw = Yw + warp * 256;
+                    tc::store16x16(yw, 16, pacc, 1.f);
+                    __syncwarp();
+                    float pr[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                    tc::mma16x16(pr, Ls + (16 * R) * 65 + 16 * R, 65, yw, 16);
+                    tc::store16x16(Xo + xslot(dist, cb) * 256, 16, pr, -1.f);
+                    // T[16R + row][16cb + col] = -pr * beta[col] (bf16 pairs)
+                    const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                tc::mma_bf16(tbase + COL_WK, tc::desc_k(sbase + OP_T, 16 * k),
-                             tc::desc_mn(sbase + OP_AK + 64 * 128, 16 * k, 16384), id_wk, k > 0);
+                    for (int nt = 0; nt < 2; ++nt) {
+                        const int col = 16 * cb + 8 * nt + 2 * t;
+                        const float b0 = -bet[col], b1 = -bet[col + 1];
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                tc::mma_bf16(tbase + COL_W, tc::desc_k(sbase + OP_T, 16 * k),
-                             tc::desc_mn(sbase + STG_V + (ci & 1) * 8192, 16 * k, 8192), id_u, k > 0);
-            tc::mma_commit(mma_bar);
-        }
-        ok = tc::bar_wait(mma_bar, mma_phase);
-        mma_phase ^= 1;
-        if (!__syncthreads_and(ok)) { ok = false; break; }
-        tc::fence_after_sync();
-        // ---- H. Wk -> bf16 operand (M=64 layout: lanes 32w..32w+15 = rows 16w..) ---
-        {
-            const int r = 16 * wq + (lane & 15);
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const int row = 16 * R + g + 8 * hh;
+                            *reinterpret_cast<uint32_t *>(sm + OP_T + tc::sw128(row, col >> 3) + 2 * (col & 7)) =
+                                pack_bf16(pr[nt][2 * hh] * b0, pr[nt][2 * hh + 1] * b1);
+                        }
+                    }
+                }
+                tc::named_sync(1, 128);
+                KDA_MARK(ci, 11 + dist);
+            }
+        } else if (warp >= 6) {
+            // ---- E2. R = V - Ka Sm (bf16 operand): R' is rows 64-127 (TMEM lanes
+            // 64-127, sub-partitions 2 and 3) of columns COL_O..COL_O+63; warps 6
+            // and 7 own those sub-partitions ---------------------------------------
+            const int r = 32 * (wq - 2) + lane;
+            const uint8_t *vs = sm + STG_V + (ci & 1) * 8192;
             float a[32];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                tc::tmem_ld32(tbase + tlane + COL_WK + 64 * wh + 32 * q, a);
+            for (int half = 0; half < 2; ++half) {
+                tc::tmem_ld32(tbase + tlane + COL_O + 32 * half, a);
                 tc::tmem_ld_wait();
-                if (lane < 16) {
+                {
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4)
-                        *reinterpret_cast<uint4 *>(sm + OP_WK + wh * 8192 + tc::sw128(r, 4 * q + q4)) =
-                            pack8(a + 8 * q4, 1.f);
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const uint32_t off = tc::sw128(r, 4 * half + q4);
+                        const uint4 vv = *reinterpret_cast<const uint4 *>(vs + off);
+                        const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 vf = unpack_bf16(vw[e]);
+                            w[e] = pack_bf16(vf.x - a[8 * q4 + 2 * e], vf.y - a[8 * q4 + 2 * e + 1]);
+                        }
+                        *reinterpret_cast<uint4 *>(sm + OP_RW + off) = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
                 }
             }
         }
         tc::fence_async_smem();
         tc::fence_before_sync();
-        __syncthreads();
-        // ---- I. W = U - Wk Sm ; O = Qh Sm ---------------------------------------
+        if (!__syncthreads_and(ok)) { ok = false; break; }
+        KDA_MARK(ci, 5);
+        // ---- F. round 2: W = T R ----------------------------------------------------
         if (tid == 0) {
             tc::fence_after_sync();
-            constexpr uint32_t id_w = tc::idesc_bf16(64, 64, false, true, /*a_neg=*/true);
-            constexpr uint32_t id_o = tc::idesc_bf16(64, 64, false, true);
+            constexpr uint32_t id_w = tc::idesc_bf16(64, 64, false, true);
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-                tc::mma_bf16(tbase + COL_W, tc::desc_k(sbase + OP_WK + (k >> 2) * 8192, 16 * (k & 3)),
-                             tc::desc_mn(sbase + OP_SM, 16 * k, 8192), id_w, 1);
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                tc::mma_bf16(tbase + COL_O, tc::desc_k(sbase + OP_AK + (k >> 2) * 16384, 16 * (k & 3)),
-                             tc::desc_mn(sbase + OP_SM, 16 * k, 8192), id_o, k > 0);
+            for (int k = 0; k < 4; ++k) tc::mma_bf16(tbase + COL_W, dT + 2 * k, dRW + 128 * k, id_w, k > 0);
             tc::mma_commit(mma_bar);
         }
         ok = tc::bar_wait(mma_bar, mma_phase);
         mma_phase ^= 1;
         if (!__syncthreads_and(ok)) { ok = false; break; }
         tc::fence_after_sync();
-        // ---- J. W -> bf16 operand ------------------------------------------------
+        KDA_MARK(ci, 6);
+        // ---- G. W -> bf16 operand (replaces R, which round 2 consumed) ----------------
         {
             const int r = 16 * wq + (lane & 15);
             float a[32];
@@ -414,38 +453,41 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
             if (lane < 16) {
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4)
-                    *reinterpret_cast<uint4 *>(sm + OP_W + tc::sw128(r, 4 * wh + q4)) = pack8(a + 8 * q4, 1.f);
+                    *reinterpret_cast<uint4 *>(sm + OP_RW + tc::sw128(r, 4 * wh + q4)) = pack8(a + 8 * q4, 1.f);
             }
         }
         tc::fence_async_smem();
         tc::fence_before_sync();
         __syncthreads();
-        // ---- K. O += A_qk W ; D = Kb^T W -----------------------------------------
+        KDA_MARK(ci, 7);
+        // ---- H. round 3: O += A_qk W ; D = Kb^T W ---------------------------------------
         if (tid == 0) {
             tc::fence_after_sync();
-            constexpr uint32_t id_o = tc::idesc_bf16(64, 64, false, true);
+            // O += A_qk W as an M=128 MMA (O1 came from the M=128 round 1): its A rows
+            // 64-127 are the W tile that follows A_qk in shared memory, and land in
+            // TMEM lanes 64-127 of COL_O, which are not read afterwards
+            constexpr uint32_t id_o = tc::idesc_bf16(128, 64, false, true);
             constexpr uint32_t id_s = tc::idesc_bf16(128, 64, true, true);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                tc::mma_bf16(tbase + COL_O, tc::desc_k(sbase + OP_AQK, 16 * k),
-                             tc::desc_mn(sbase + OP_W, 16 * k, 8192), id_o, 1);
+            for (int k = 0; k < 4; ++k) tc::mma_bf16(tbase + COL_O, dAQK + 2 * k, dRW + 128 * k, id_o, 1);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                tc::mma_bf16(tbase + COL_S, tc::desc_mn(sbase + OP_KB, 16 * k, 8192),
-                             tc::desc_mn(sbase + OP_W, 16 * k, 8192), id_s, k > 0);
+            for (int k = 0; k < 4; ++k) tc::mma_bf16(tbase + COL_S, dKBmn + 128 * k, dRW + 128 * k, id_s, k > 0);
             tc::mma_commit(mma_bar);
         }
         ok = tc::bar_wait(mma_bar, mma_phase);
         mma_phase ^= 1;
         if (!__syncthreads_and(ok)) { ok = false; break; }
         tc::fence_after_sync();
-        // ---- L. outputs, state update, snapshot ---------------------------------
+        KDA_MARK(ci, 8);
+        // ---- I. outputs, state update, snapshot -------------------------------------------
         {
             float a[32];
-            const int r = 16 * wq + (lane & 15);
-            tc::tmem_ld32(tbase + tlane + COL_O + 32 * wh, a);
-            tc::tmem_ld_wait();
-            if (lane < 16 && r < n) {
+            const int r = 32 * wq + lane;          // O row in the M=128 layout (warps 0,1,4,5)
+            if (wq < 2) {
+                tc::tmem_ld32(tbase + tlane + COL_O + 32 * wh, a);
+                tc::tmem_ld_wait();
+            }
+            if (wq < 2 && r < n) {
                 uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) +
                                                        ((int64_t)(sq.tok0 + ci * C + r) * H + h) * D + j0 + 32 * wh);
 #pragma unroll
@@ -466,6 +508,7 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
         }
         tc::fence_before_sync();
         __syncthreads();
+        KDA_MARK(ci, 9);
     }
 
     if (ok && p.state_out) {

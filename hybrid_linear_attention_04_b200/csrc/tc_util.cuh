@@ -160,6 +160,10 @@ __device__ __forceinline__ void tma_load3(void *smem_dst, const CUtensorMap *m, 
 }
 
 // ---- small warp-level helpers ----------------------------------------------------
+// barrier among `nthreads` threads (whole warps) using hardware barrier `id` (1..15)
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 // 2^x (hardware approximation, relative error ~2^-22; inputs here are bounded)
 __device__ __forceinline__ float ex2(float x) {
     float y;
@@ -182,17 +186,19 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 // P[16x16] += A[16x16] B[16x16]; A, B fp32 in shared memory with row strides sa, sb.
+// The fp32 bits are passed as tf32 operands (the MMA reads the top 19 bits).
 // Result fragments: p[nt] covers columns 8nt..8nt+7 in the d layout above.
 __device__ __forceinline__ void mma16x16(float (&p)[2][4], const float *A, int sa, const float *B, int sb) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int kk = 0; kk < 2; ++kk) {
-        const uint32_t a[4] = {to_tf32(A[g * sa + 8 * kk + t]), to_tf32(A[(g + 8) * sa + 8 * kk + t]),
-                               to_tf32(A[g * sa + 8 * kk + t + 4]), to_tf32(A[(g + 8) * sa + 8 * kk + t + 4])};
+        const uint32_t a[4] = {__float_as_uint(A[g * sa + 8 * kk + t]), __float_as_uint(A[(g + 8) * sa + 8 * kk + t]),
+                               __float_as_uint(A[g * sa + 8 * kk + t + 4]),
+                               __float_as_uint(A[(g + 8) * sa + 8 * kk + t + 4])};
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-            const uint32_t b[2] = {to_tf32(B[(8 * kk + t) * sb + 8 * nt + g]),
-                                   to_tf32(B[(8 * kk + t + 4) * sb + 8 * nt + g])};
+            const uint32_t b[2] = {__float_as_uint(B[(8 * kk + t) * sb + 8 * nt + g]),
+                                   __float_as_uint(B[(8 * kk + t + 4) * sb + 8 * nt + g])};
             mma_tf32(p[nt], a, b);
         }
     }
