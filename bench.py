@@ -60,77 +60,93 @@ def load_peaks():
     return {**FALLBACK, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def kernel_source_hash():
+def _src_hash(files):
     h = hashlib.sha256()
-    for f in sorted((ROOT / "hybrid_linear_attention_04_b200" / "csrc").glob("*")):
-        h.update(f.read_bytes())
+    for f in files:
+        h.update((ROOT / "hybrid_linear_attention_04_b200" / "csrc" / f).read_bytes())
     return h.hexdigest()[:16]
 
 
-def ncu_traffic():
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources (else None)."""
+def ncu_traffic(kernel, read_units, write_units):
+    """DRAM bytes per launch (read + write) of `kernel` scaled from the committed
+    ncu capture by the units this launch processes, or None when the capture is
+    missing or was taken on other kernel sources."""
     p = ROOT / "profiles" / "dram_traffic.json"
     if not p.exists():
-        return {}
+        return None
     d = json.loads(p.read_text())
-    if d.get("csrc_hash") != kernel_source_hash():
-        return {}
-    return d.get("kernels", {})
+    k = d.get("kernels", {}).get(kernel)
+    if not k or _src_hash(d["sources"][kernel]) != k["src_hash"]:
+        return None
+    return int(k["read"] / k["read_units"] * read_units + k["write"] / k["write_units"] * write_units)
 
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples SM clock, max clock, power and clock-event reasons through NVML
+    every ~5 ms in a background thread while the timed region runs (read-only;
+    no setting of the GPU is changed)."""
 
-    def __init__(self, index):
-        self.index = index
-        self.proc = None
-        self.path = Path(f"/tmp/kda_clocks_{os.getpid()}.csv")
+    def __init__(self, dev):
+        self.dev = dev
+        self.samples = []
+        self.thread = None
+        self.stop = False
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            pr = torch.cuda.get_device_properties(self.dev)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            idx = int(vis.split(",")[self.dev.index or 0]) if vis and vis.split(",")[0].isdigit() else (self.dev.index or 0)
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(idx)
+
+    def _run(self):
+        nv, h = self.nv, self.h
+        names = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                 "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                 "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                 "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap,
+                 "hw_power_brake": nv.nvmlClocksEventReasonHwPowerBrakeSlowdown}
+        self.sm_max = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self.stop:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                self.samples.append((sm, pw, [n for n, b in names.items() if rs & b]))
+            except Exception:
+                pass
+            time.sleep(0.005)
 
     def __enter__(self):
+        import threading
         try:
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
-                stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            self.nv, self.h = self._handle()
+        except Exception:
+            return self
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+        while not self.samples and self.thread.is_alive():
+            time.sleep(0.001)
         return self
 
     def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.f.close()
+        self.stop = True
+        if self.thread is not None:
+            self.thread.join(timeout=5)
 
     def summary(self):
-        if self.proc is None or not self.path.exists():
+        if not self.samples:
             return None
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.path.read_text().splitlines():
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() in ("active", "1"):
-                    reasons.add(n)
-        self.path.unlink(missing_ok=True)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        sm = [x[0] for x in self.samples]
+        reasons = sorted({r for x in self.samples for r in x[2]})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": getattr(self, "sm_max", None),
+                "reasons": reasons, "samples": len(sm),
+                "power_w_max": round(max(x[1] for x in self.samples), 1)}
 
 
 # ----------------------------------------------------------------------------
@@ -284,7 +300,7 @@ def run_ours(args):
         dist.barrier()
     torch.cuda.synchronize(dev)
     launches0 = K.kda_launch_count()
-    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+    with ClockSampler(dev) as clk:
         t_start.record(stream)
         for s in range(args.steps):
             step(evs[s])
@@ -336,7 +352,6 @@ def run_ours(args):
             "verify": (wl.n_tok * H, "state-steps/s", verify_bytes(N_SEQ, wl.n_tok)),
             "commit": (wl.n_commit, "states/s", commit_bytes(wl.n_commit)),
         }
-        traffic = ncu_traffic()
         for name, ms in zip(comps, comp_ms):
             n_units, unit, byts = units[name]
             gbs = byts / (ms * 1e-3) / 1e9
@@ -347,9 +362,11 @@ def run_ours(args):
         comp["prefill"]["algorithmic_flops"] = pf
         comp["prefill"]["tc_frac"] = round(pf / (comp_ms[0] * 1e-3) / (peaks["bf16_tflops"] * 1e12), 4)
         dom = max(comps, key=lambda c: comp[c]["ms"])
-        kname = {"prefill": "prefill", "decode": "decode_kernel", "verify": "verify_kernel",
+        kname = {"prefill": "prefill_tc_kernel", "decode": "decode_kernel", "verify": "verify_kernel",
                  "commit": "snapshot_kernel"}[dom]
-        tr = traffic.get(kname)
+        tr_units = {"prefill": (PREFILL_T * H, PREFILL_T * H), "decode": (N_SEQ * H, N_SEQ * H),
+                    "verify": (N_SEQ * H, wl.n_tok * H), "commit": (wl.n_commit, wl.n_commit)}[dom]
+        tr = ncu_traffic(kname, *tr_units)
         roof = {"bound": "hbm", "kernel": kname, "achieved": comp[dom]["achieved_gbs"],
                 "peak": hbm, "unit": "GB/s", "frac": comp[dom]["hbm_frac"],
                 "traffic": tr, "peak_source": peaks["source"]}
@@ -388,6 +405,96 @@ def run_ours(args):
         dist.barrier()
         dist.destroy_process_group()
     return result
+
+
+def time_calls(fn, steps, warmup, dev):
+    """Average ms per call of fn() over `steps` calls after `warmup`, CUDA events."""
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    return a.elapsed_time(b) / steps
+
+
+def run_workload(args):
+    """Single-workload timing lines (tiny fp32, ragged batch, 1M-token segments)
+    used for the design notes; the default run is the serving step."""
+    from hybrid_linear_attention_04_b200 import build as kbuild
+    kbuild.build()
+    from hybrid_linear_attention_04_b200 import kda as K
+    dev = torch.device("cuda", 0)
+    peaks = load_peaks()
+    wl = synth.WORKLOADS
+    out = {"impl": "ours", "workload": args.workload, "steps": args.steps, "warmup": args.warmup}
+    if args.workload == "tiny":
+        c = wl["tiny_fp32"]
+        x = synth.token_inputs(c["seed"], c["T"], c["H"], c["d"], c["d"], io="fp32")
+        xd = {k: v.to(dev) for k, v in x.items()}
+        o = torch.empty_like(xd["v"])
+        so = torch.empty((1, c["H"], c["d"], c["d"]), device=dev)
+        cu = np.array([0, c["T"]], dtype=np.int32)
+        ms = time_calls(lambda: K.kda_prefill(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], cu, o,
+                                              state_out=so, chunk=c["chunk"]), args.steps, args.warmup, dev)
+        out.update({"unit": "us/call", "value": ms * 1e3, "tokens": c["T"]})
+    elif args.workload == "ragged":
+        c = wl["ragged_prefix_32"]
+        plan = synth.ragged_plan(c["seed"], c["n_seq"], c["mu"], c["sigma"], c["lo"], c["hi"],
+                                 c["prefix"], c["n_resume"], c["snap"])
+        lens, start = plan["lens"], plan["start_pos"]
+        cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+        T = int(cu[-1])
+        x = synth.token_inputs(c["seed"], T, H, D, D, io="bf16")
+        xd = {k: v.to(dev) for k, v in x.items()}
+        del x
+        s0 = synth.states(c["seed"], c["n_seq"], H, D, D, std=0.1).to(dev)
+        o = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+        so = torch.empty_like(s0)
+        offs, _ = K.kda_snapshot_plan(cu, start, c["snap"])
+        sn = torch.empty((int(offs[-1]), H, D, D), device=dev)
+        ms = time_calls(lambda: K.kda_prefill(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], cu, o,
+                                              state_out=so, state_in=s0, start_pos=start,
+                                              snap_interval=c["snap"], snapshots=sn, chunk=C),
+                        args.steps, args.warmup, dev)
+        byts = T * H * (3 * D * 2 + D * 2 + D * 4 + 4) + (int(offs[-1]) + 2 * c["n_seq"]) * H * D * D * 4
+        out.update({"unit": "tok/s", "value": T / (ms * 1e-3), "ms": ms, "tokens": T,
+                    "algorithmic_bytes": byts, "hbm_frac": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]})
+    elif args.workload == "long":
+        c = wl["long_1m"]
+        seg, n_seg = c["segment"], c["T"] // c["segment"]
+        # two distinct seeded segments alternate (identical work per call; the
+        # host draws 2 of the 16 segments to keep set-up short)
+        segs = []
+        for i in range(2):
+            x = synth.token_inputs(c["seed"], seg, H, D, D, io="bf16", t0=i * seg)
+            segs.append({k: v.to(dev) for k, v in x.items()})
+            del x
+        o = torch.empty((seg, H, D), dtype=torch.bfloat16, device=dev)
+        st = [torch.zeros((1, H, D, D), device=dev) for _ in range(2)]
+        n_snap = seg // c["snap"]
+        sn = torch.empty((n_snap, H, D, D), device=dev)
+        cu = np.array([0, seg], dtype=np.int32)
+
+        def one_pass():
+            for i in range(n_seg):
+                xd = segs[i % 2]
+                K.kda_prefill(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], cu, o,
+                              state_out=st[(i + 1) % 2], state_in=st[i % 2] if i else None,
+                              start_pos=[i * seg], snap_interval=c["snap"], snapshots=sn, chunk=C)
+        ms = time_calls(one_pass, max(1, args.steps // 5), 1, dev)
+        T = c["T"]
+        byts = T * H * (3 * D * 2 + D * 2 + D * 4 + 4) + (T // c["snap"] + 2 * n_seg) * H * D * D * 4
+        out.update({"unit": "tok/s", "value": T / (ms * 1e-3), "ms": ms, "tokens": T,
+                    "algorithmic_bytes": byts, "hbm_frac": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]})
+    st_ = K.kda_check_device_status()
+    if st_ != 0:
+        raise RuntimeError(K.kda_status_string(st_))
+    print(json.dumps(out), flush=True)
 
 
 def run_reference(args):
@@ -431,10 +538,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=2048)
     ap.add_argument("--ref-tokens", type=int, default=512)
+    ap.add_argument("--workload", choices=["serving", "tiny", "ragged", "long"], default="serving")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload != "serving":
+        run_workload(args)
     else:
         run_ours(args)
 

@@ -183,8 +183,9 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
 // Verify: tokens are processed in batches of kTokBatch staged in shared memory.
 constexpr int kTokBatch = 8;
 
+// two CTAs per SM (register cap) keep enough state loads and stores in flight
 template <int D, typename TIO>
-__global__ void __launch_bounds__(DecodeShape<D>::NT)
+__global__ void __launch_bounds__(DecodeShape<D>::NT, 2)
 verify_kernel(const __grid_constant__ DecodeParams p) {
     using Sh = DecodeShape<D>;
     __shared__ TokVec<D> tv[kTokBatch];
