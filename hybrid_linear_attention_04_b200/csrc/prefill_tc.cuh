@@ -11,17 +11,17 @@
 //            so that Qh Kb^T = A_qk and Ka Kb^T = A_kk with every exponent
 //            inside the chunk bounded by half the chunk's decay range.
 //   tcgen05  [Qh; Ka] Kb^T -> TMEM (M=128: A_qk rows 0-63, A_kk rows 64-127)
-//   CUDA     T = (I + Diag(beta) A_kk)^{-1} Diag(beta) by blocked forward
-//   cores    substitution in fp32 (16x16 diagonal blocks, then merges)
-//   tcgen05  (same round as A) R' = Ka Sm, O = Qh Sm  (M=64; Sm = Diag(e^m) S_0)
-//   CUDA     R = V - R' (bf16), concurrently with the solve
-//   tcgen05  W = T R                                 (M=64)
-//            O += A_qk W, D = Kb^T W                 (M=64 / M=128)
+//   tcgen05  (same MMAs as A) R' = Ka Sm, O = Qh Sm  (Sm = Diag(e^m) S_0, stored
+//            transposed under Kb so one N=128 round yields all four blocks)
+//   CUDA     L = Diag(beta) A_kk; inverses of its 16x16 diagonal blocks (fp32);
+//   cores    R = V - R' (fp32); then W = (I + L)^{-1} Diag(beta) R by block
+//            forward substitution on tf32 mma.sync, 8 d_v columns per warp
+//   tcgen05  O += A_qk W, D = Kb^T W                 (M=128)
 //   CUDA     o = scale O (bf16 store); S_C = Diag(Gamma_C) S_0 + Diag(e^(b_C-m)) D
 //   cores    with the fp32 master state held in registers (thread = d_k row).
 // Identities used: Q.Gamma = Qh.e^m and K.Gamma = Ka.e^m, so (Q.Gamma) S_0 =
 // Qh Sm and (K.Gamma) S_0 = Ka Sm; K.exp(b_C-b) = Kb.e^(b_C-m) row-wise; and
-// W = T (V - (K.Gamma) S_0) = T R.
+// W = (I + Diag(beta) A_kk)^{-1} Diag(beta) (V - (K.Gamma) S_0).
 // A chunk whose per-channel decay from its middle exceeds 80 nats in either
 // direction is reported through the status word (KDA_ERR_RANGE).
 #pragma once
@@ -54,21 +54,21 @@ constexpr uint32_t STG_V = 32768;      // v  slice, 2 buffers of 1 slab [64 tok 
 constexpr uint32_t OP_AK = 49152;      // [Qh; Ka]: 2 slabs of 128 rows (channels 0-63, 64-127)
 constexpr uint32_t OP_KB = 81920;      // [Kb; Sm^T]: 2 slabs (channels 0-63, 64-127) of 128 rows:
                                        // rows 0-63 Kb (tokens), rows 64-127 Sm^T (d_v columns)
-constexpr uint32_t OP_T = 114688;      // T  [64 x 64]
-constexpr uint32_t OP_AQK = 122880;    // A_qk masked [64 x 64]
-constexpr uint32_t OP_RW = 131072;     // R = V - Ka Sm, then W [64 tok x 64 dv]
-constexpr uint32_t STG_G = 139264;     // g, fp32 [64][128]
-constexpr uint32_t SOLVE = 172032;     // fp32 [64][65]: L off the diagonal blocks, X on them
-constexpr uint32_t XO = SOLVE + 64 * 65 * 4;   // 6 off-diagonal X blocks + 3 scratch blocks (16x16 fp32)
-constexpr uint32_t TOT = XO + 9 * 1024;        // per-warp row-block totals of b [8][128]
+constexpr uint32_t OP_AQK = 114688;    // A_qk masked [64 x 64] (followed by OP_W: see round 3)
+constexpr uint32_t OP_W = 122880;      // W [64 tok x 64 dv] bf16
+constexpr uint32_t STG_G = 131072;     // g, fp32 [64][128]
+constexpr uint32_t SOLVE = 163840;     // fp32 [64][65]: L = Diag(beta) A_kk, inverse on diagonal blocks
+constexpr uint32_t RF = SOLVE + 64 * 65 * 4;   // R = V - Ka Sm, fp32 [64][68]
+constexpr uint32_t LB = RF + 64 * 68 * 4;      // bf16 [64][72]: L off the diagonal blocks, X on them
+constexpr uint32_t WSC = LB + 64 * 72 * 2;     // per-warp Y / W columns, bf16 [8 warps][8][72]
+constexpr uint32_t TOT = WSC + 8 * 8 * 72 * 2; // per-warp row-block totals of b [8][128]
 constexpr uint32_t VEC = TOT + 8 * 128 * 4;    // eM, eC, gC [128] + beta [64]
 constexpr uint32_t BARS = VEC + (3 * 128 + 64) * 4;
 constexpr uint32_t SMEM_USED = BARS + 48;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
-// TMEM columns
-// round 1 writes [A_qk | O ; A_kk | R'] into columns 0-127 (rows 0-63 | 64-127);
-// W = T R lands in COL_W (M=64), D = Kb^T W in COL_S
-constexpr uint32_t COL_A = 0, COL_O = 64, COL_W = 128, COL_S = 192, TMEM_COLS = 256;
+// TMEM columns: round 1 writes [A_qk | O ; A_kk | R'] into columns 0-127 (rows
+// 0-63 | 64-127); D = Kb^T W lands in COL_S
+constexpr uint32_t COL_A = 0, COL_O = 64, COL_S = 128, TMEM_COLS = 256;
 constexpr uint32_t CHUNK_TX = 16384 + 16384 + 32768 + 8192;   // bytes per chunk of loads
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RANGE_LIMIT2 = 80.f * LOG2E;    // 80 nats, in log2 units
@@ -97,8 +97,9 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
     const uint32_t sbase = tc::smem_u32(sm);
     float *Gs = reinterpret_cast<float *>(sm + STG_G);
     float *Ls = reinterpret_cast<float *>(sm + SOLVE);
-    float *Xo = reinterpret_cast<float *>(sm + XO);     // 6 blocks 16x16
-    float *Yw = Xo + 6 * 256;                             // 3 per-warp 16x16 blocks
+    float *Rf = reinterpret_cast<float *>(sm + RF);
+    __nv_bfloat16 *Lb = reinterpret_cast<__nv_bfloat16 *>(sm + LB);
+    __nv_bfloat16 *Wsc = reinterpret_cast<__nv_bfloat16 *>(sm + WSC);
     float *Tot = reinterpret_cast<float *>(sm + TOT);
     float *eM = reinterpret_cast<float *>(sm + VEC);
     float *eC = eM + 128, *gC = eM + 256, *bet = eM + 384;
@@ -175,13 +176,9 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
     }
     // smem matrix descriptors (start-address field advanced by 16-byte units)
     const uint64_t dAK = tc::desc_k(sbase + OP_AK, 0), dKB = tc::desc_k(sbase + OP_KB, 0);
-    const uint64_t dT = tc::desc_k(sbase + OP_T, 0), dAQK = tc::desc_k(sbase + OP_AQK, 0);
-    const uint64_t dRW = tc::desc_mn(sbase + OP_RW, 0, 8192);
+    const uint64_t dAQK = tc::desc_k(sbase + OP_AQK, 0);
+    const uint64_t dW = tc::desc_mn(sbase + OP_W, 0, 8192);
     const uint64_t dKBmn = tc::desc_mn(sbase + OP_KB, 0, 16384);
-    // T's blocks above the diagonal are always zero: clear the whole T tile once
-    // (the diagonal and lower blocks are rewritten every chunk)
-    for (int e = tid; e < 64 * 8; e += NT)
-        *reinterpret_cast<uint4 *>(sm + OP_T + 16 * e) = make_uint4(0u, 0u, 0u, 0u);
     // prep map: warp w owns rows 8w..8w+7, lane l owns channels 4l..4l+3
     const int pkb = lane >> 4, pchk = (lane & 15) >> 1, phf = (lane & 1) * 8;
 
@@ -301,108 +298,74 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
         ok = tc::bar_wait(bar_a, (uint32_t)(ci & 1));
         tc::fence_after_sync();
         KDA_MARK(ci, 4);
-        if (warp < 4) {
-            // ---- E1. A_qk (masked bf16 operand), L = Diag(beta) A_kk, then the
-            // solve X = (I + L)^{-1} and T = X Diag(beta) (warps 0-3) ----------
-            {
-                const int r = 32 * (warp & 1) + lane;
-                float a[32];
+        // ---- E. warps 0,1: A_qk (masked bf16 operand). Warps 2,3: L = Diag(beta)
+        // A_kk (fp32), then the inverses X of its four 16x16 diagonal blocks by
+        // forward substitution (each warp owns two blocks: no block-wide sync).
+        // Warps 6,7: R = V - Ka Sm (fp32) from TMEM lanes 64-127 (their sub-partitions).
+        if (warp < 2) {
+            const int r = 32 * warp + lane;
+            float a[32];
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    tc::tmem_ld32(tbase + tlane + COL_A + 32 * half, a);
-                    tc::tmem_ld_wait();
-                    if (warp < 2) {
+            for (int half = 0; half < 2; ++half) {
+                tc::tmem_ld32(tbase + tlane + COL_A + 32 * half, a);
+                tc::tmem_ld_wait();
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            uint32_t w[4];
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint32_t w[4];
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int jj = 32 * half + 8 * q4 + 2 * e;
-                                w[e] = pack_bf16(jj <= r ? a[8 * q4 + 2 * e] : 0.f,
-                                                 jj + 1 <= r ? a[8 * q4 + 2 * e + 1] : 0.f);
-                            }
-                            *reinterpret_cast<uint4 *>(sm + OP_AQK + tc::sw128(r, 4 * half + q4)) =
-                                make_uint4(w[0], w[1], w[2], w[3]);
-                        }
-                    } else {
-                        const float br = bet[r];
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const int jj = 32 * half + e;
-                            Ls[r * 65 + jj] = jj < r ? br * a[e] : 0.f;
-                        }
+                    for (int e = 0; e < 4; ++e) {
+                        const int jj = 32 * half + 8 * q4 + 2 * e;
+                        w[e] = pack_bf16(jj <= r ? a[8 * q4 + 2 * e] : 0.f, jj + 1 <= r ? a[8 * q4 + 2 * e + 1] : 0.f);
                     }
+                    *reinterpret_cast<uint4 *>(sm + OP_AQK + tc::sw128(r, 4 * half + q4)) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
-            tc::named_sync(1, 128);
-            KDA_MARK(ci, 10);
-            // 16x16 diagonal blocks by forward substitution, one column per thread
-            if (tid < 64) {
-                const int blk = tid >> 4, c = tid & 15, base = 16 * blk;
-                float x[16];
+        } else if (warp < 4) {
+            const int r = 32 * (warp - 2) + lane;
+            const float br = bet[r];
+            float a[32];
 #pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    float a0 = r == c ? 1.f : 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-                    const float *lr = Ls + (base + r) * 65 + base;
+            for (int half = 0; half < 2; ++half) {
+                tc::tmem_ld32(tbase + tlane + COL_A + 32 * half, a);
+                tc::tmem_ld_wait();
+                // bf16 L for the forward substitution (16-byte stores: conflict-free
+                // with the 144-byte row pitch); fp32 L only on the diagonal block,
+                // which the inversion below reads
+                const int dblk = r & ~15;
 #pragma unroll
-                    for (int i = 0; i < r; ++i) {
-                        const float t = lr[i] * x[i];
-                        if ((i & 3) == 0) a0 -= t;
-                        else if ((i & 3) == 1) a1 -= t;
-                        else if ((i & 3) == 2) a2 -= t;
-                        else a3 -= t;
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    float l[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int jj = 32 * half + 8 * q4 + e;
+                        l[e] = jj < r ? br * a[8 * q4 + e] : 0.f;
+                        if (jj >= dblk && jj < dblk + 16) Ls[r * 65 + jj] = l[e];
                     }
-                    x[r] = (a0 + a1) + (a2 + a3);
-                }
-                __syncwarp();
-                const float bc = bet[base + c];
-                __nv_bfloat16 *tt = reinterpret_cast<__nv_bfloat16 *>(sm + OP_T);
-#pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    Ls[(base + r) * 65 + base + c] = x[r];
-                    const int rr = base + r, cc = base + c;
-                    tt[(tc::sw128(rr, cc >> 3) >> 1) + (cc & 7)] = __float2bfloat16_rn(x[r] * bc);
+                    *reinterpret_cast<uint4 *>(Lb + r * 72 + 32 * half + 8 * q4) = pack8(l, 1.f);
                 }
             }
-            tc::named_sync(1, 128);
-            KDA_MARK(ci, 11);
-            // off-diagonal blocks by distance: X[R][Cb] = -X[R][R] sum_J L[R][J] X[J][Cb]
-#pragma unroll 1
-            for (int dist = 1; dist < 4; ++dist) {
-                if (warp < 4 - dist) {
-                    const int cb = warp, R = cb + dist;
-                    float pacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                    for (int J = cb; J < R; ++J) {
-                        const float *xj = J == cb ? Ls + (16 * J) * 65 + 16 * cb : Xo + xslot(J - cb, cb) * 256;
-                        tc::mma16x16(pacc, Ls + (16 * R) * 65 + 16 * J, 65, xj, J == cb ? 65 : 16);
-                    }
-                    float *yw = Yw + warp * 256;
-                    tc::store16x16(yw, 16, pacc, 1.f);
-                    __syncwarp();
-                    float pr[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                    tc::mma16x16(pr, Ls + (16 * R) * 65 + 16 * R, 65, yw, 16);
-                    tc::store16x16(Xo + xslot(dist, cb) * 256, 16, pr, -1.f);
-                    // T[16R + row][16cb + col] = -pr * beta[col] (bf16 pairs)
-                    const int g = lane >> 2, t = lane & 3;
+            __syncwarp();
+            // diagonal block 2*(warp-2) + lane/16, column lane%16
+            const int base = 16 * (2 * (warp - 2) + (lane >> 4)), c = lane & 15;
+            float x[16];
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        const int col = 16 * cb + 8 * nt + 2 * t;
-                        const float b0 = -bet[col], b1 = -bet[col + 1];
+            for (int rr = 0; rr < 16; ++rr) {
+                float a0 = rr == c ? 1.f : 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                const float *lr = Ls + (base + rr) * 65 + base;
 #pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            const int row = 16 * R + g + 8 * hh;
-                            *reinterpret_cast<uint32_t *>(sm + OP_T + tc::sw128(row, col >> 3) + 2 * (col & 7)) =
-                                pack_bf16(pr[nt][2 * hh] * b0, pr[nt][2 * hh + 1] * b1);
-                        }
-                    }
+                for (int i = 0; i < rr; ++i) {
+                    const float t = lr[i] * x[i];
+                    if ((i & 3) == 0) a0 -= t;
+                    else if ((i & 3) == 1) a1 -= t;
+                    else if ((i & 3) == 2) a2 -= t;
+                    else a3 -= t;
                 }
-                tc::named_sync(1, 128);
-                KDA_MARK(ci, 11 + dist);
+                x[rr] = (a0 + a1) + (a2 + a3);
             }
+            __syncwarp();
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) Lb[(base + rr) * 72 + base + c] = __float2bfloat16_rn(x[rr]);
         } else if (warp >= 6) {
-            // ---- E2. R = V - Ka Sm (bf16 operand): R' is rows 64-127 (TMEM lanes
-            // 64-127, sub-partitions 2 and 3) of columns COL_O..COL_O+63; warps 6
-            // and 7 own those sub-partitions ---------------------------------------
             const int r = 32 * (wq - 2) + lane;
             const uint8_t *vs = sm + STG_V + (ci & 1) * 8192;
             float a[32];
@@ -410,20 +373,20 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
             for (int half = 0; half < 2; ++half) {
                 tc::tmem_ld32(tbase + tlane + COL_O + 32 * half, a);
                 tc::tmem_ld_wait();
-                {
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const uint32_t off = tc::sw128(r, 4 * half + q4);
-                        const uint4 vv = *reinterpret_cast<const uint4 *>(vs + off);
-                        const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
-                        uint32_t w[4];
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const uint4 vv = *reinterpret_cast<const uint4 *>(vs + tc::sw128(r, 4 * half + q4));
+                    const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
+                    float rr[8];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 vf = unpack_bf16(vw[e]);
-                            w[e] = pack_bf16(vf.x - a[8 * q4 + 2 * e], vf.y - a[8 * q4 + 2 * e + 1]);
-                        }
-                        *reinterpret_cast<uint4 *>(sm + OP_RW + off) = make_uint4(w[0], w[1], w[2], w[3]);
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 vf = unpack_bf16(vw[e]);
+                        rr[2 * e] = vf.x - a[8 * q4 + 2 * e];
+                        rr[2 * e + 1] = vf.y - a[8 * q4 + 2 * e + 1];
                     }
+                    float *dst = Rf + r * 68 + 32 * half + 8 * q4;
+                    *reinterpret_cast<float4 *>(dst) = make_float4(rr[0], rr[1], rr[2], rr[3]);
+                    *reinterpret_cast<float4 *>(dst + 4) = make_float4(rr[4], rr[5], rr[6], rr[7]);
                 }
             }
         }
@@ -431,29 +394,70 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
         tc::fence_before_sync();
         if (!__syncthreads_and(ok)) { ok = false; break; }
         KDA_MARK(ci, 5);
-        // ---- F. round 2: W = T R ----------------------------------------------------
-        if (tid == 0) {
-            tc::fence_after_sync();
-            constexpr uint32_t id_w = tc::idesc_bf16(64, 64, false, true);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) tc::mma_bf16(tbase + COL_W, dT + 2 * k, dRW + 128 * k, id_w, k > 0);
-            tc::mma_commit(mma_bar);
-        }
-        ok = tc::bar_wait(mma_bar, mma_phase);
-        mma_phase ^= 1;
-        if (!__syncthreads_and(ok)) { ok = false; break; }
-        tc::fence_after_sync();
-        KDA_MARK(ci, 6);
-        // ---- G. W -> bf16 operand (replaces R, which round 2 consumed) ----------------
+        // ---- F. W = (I + L)^{-1} Diag(beta) R by block forward substitution on bf16
+        // mma.sync (fp32 accumulate): W_R = X_RR (beta R_R - sum_{J<R} L_RJ W_J).
+        // Warp w owns the eight d_v columns 8w..8w+7, so the four block rows need
+        // only warp syncs. Y and W columns are kept transposed (ws[col][row], bf16)
+        // so that B fragments are 32-bit pairs along k.
         {
-            const int r = 16 * wq + (lane & 15);
-            float a[32];
-            tc::tmem_ld32(tbase + tlane + COL_W + 32 * wh, a);
-            tc::tmem_ld_wait();
-            if (lane < 16) {
+            const int g = lane >> 2, t = lane & 3, c0 = 8 * warp;
+            __nv_bfloat16 *ws = Wsc + warp * 8 * 72;                // [8 cols][72]
+            KDA_MARK(ci, 14);
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    *reinterpret_cast<uint4 *>(sm + OP_RW + tc::sw128(r, 4 * wh + q4)) = pack8(a + 8 * q4, 1.f);
+            for (int R = 0; R < 4; ++R) {
+                const int r0 = 16 * R + g, r1 = r0 + 8;
+                float y[4];
+                {
+                    const float2 v0 = *reinterpret_cast<const float2 *>(Rf + r0 * 68 + c0 + 2 * t);
+                    const float2 v1 = *reinterpret_cast<const float2 *>(Rf + r1 * 68 + c0 + 2 * t);
+                    const float b0 = bet[r0], b1 = bet[r1];
+                    y[0] = b0 * v0.x; y[1] = b0 * v0.y; y[2] = b1 * v1.x; y[3] = b1 * v1.y;
+                }
+                float part[3][4];
+#pragma unroll
+                for (int J = 0; J < R; ++J) {
+                    const int kc = 16 * J + 2 * t;
+                    const uint32_t a[4] = {*reinterpret_cast<const uint32_t *>(Lb + r0 * 72 + kc),
+                                           *reinterpret_cast<const uint32_t *>(Lb + r1 * 72 + kc),
+                                           *reinterpret_cast<const uint32_t *>(Lb + r0 * 72 + kc + 8),
+                                           *reinterpret_cast<const uint32_t *>(Lb + r1 * 72 + kc + 8)};
+                    const uint32_t b[2] = {*reinterpret_cast<const uint32_t *>(ws + g * 72 + kc),
+                                           *reinterpret_cast<const uint32_t *>(ws + g * 72 + kc + 8)};
+                    float (&pp)[4] = part[J];
+                    pp[0] = pp[1] = pp[2] = pp[3] = 0.f;
+                    tc::mma_bf16_16816(pp, a, b);
+                }
+#pragma unroll
+                for (int J = 0; J < R; ++J) {
+                    y[0] -= part[J][0]; y[1] -= part[J][1]; y[2] -= part[J][2]; y[3] -= part[J][3];
+                }
+                // Y (rows of block R) -> ws, then W_R = X_RR Y
+                ws[(2 * t) * 72 + r0] = __float2bfloat16_rn(y[0]);
+                ws[(2 * t + 1) * 72 + r0] = __float2bfloat16_rn(y[1]);
+                ws[(2 * t) * 72 + r1] = __float2bfloat16_rn(y[2]);
+                ws[(2 * t + 1) * 72 + r1] = __float2bfloat16_rn(y[3]);
+                __syncwarp();
+                float w[4] = {0.f, 0.f, 0.f, 0.f};
+                {
+                    const int kc = 16 * R + 2 * t;
+                    const uint32_t a[4] = {*reinterpret_cast<const uint32_t *>(Lb + r0 * 72 + kc),
+                                           *reinterpret_cast<const uint32_t *>(Lb + r1 * 72 + kc),
+                                           *reinterpret_cast<const uint32_t *>(Lb + r0 * 72 + kc + 8),
+                                           *reinterpret_cast<const uint32_t *>(Lb + r1 * 72 + kc + 8)};
+                    const uint32_t b[2] = {*reinterpret_cast<const uint32_t *>(ws + g * 72 + kc),
+                                           *reinterpret_cast<const uint32_t *>(ws + g * 72 + kc + 8)};
+                    tc::mma_bf16_16816(w, a, b);
+                }
+                __syncwarp();
+                ws[(2 * t) * 72 + r0] = __float2bfloat16_rn(w[0]);
+                ws[(2 * t + 1) * 72 + r0] = __float2bfloat16_rn(w[1]);
+                ws[(2 * t) * 72 + r1] = __float2bfloat16_rn(w[2]);
+                ws[(2 * t + 1) * 72 + r1] = __float2bfloat16_rn(w[3]);
+                // bf16 W for round 3: columns c0 + 2t, c0 + 2t + 1 lie in 16-byte chunk `warp`
+                *reinterpret_cast<uint32_t *>(sm + OP_W + tc::sw128(r0, warp) + 4 * t) = pack_bf16(w[0], w[1]);
+                *reinterpret_cast<uint32_t *>(sm + OP_W + tc::sw128(r1, warp) + 4 * t) = pack_bf16(w[2], w[3]);
+                __syncwarp();
+                KDA_MARK(ci, 10 + R);
             }
         }
         tc::fence_async_smem();
@@ -469,9 +473,9 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
             constexpr uint32_t id_o = tc::idesc_bf16(128, 64, false, true);
             constexpr uint32_t id_s = tc::idesc_bf16(128, 64, true, true);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) tc::mma_bf16(tbase + COL_O, dAQK + 2 * k, dRW + 128 * k, id_o, 1);
+            for (int k = 0; k < 4; ++k) tc::mma_bf16(tbase + COL_O, dAQK + 2 * k, dW + 128 * k, id_o, 1);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) tc::mma_bf16(tbase + COL_S, dKBmn + 128 * k, dRW + 128 * k, id_s, k > 0);
+            for (int k = 0; k < 4; ++k) tc::mma_bf16(tbase + COL_S, dKBmn + 128 * k, dW + 128 * k, id_s, k > 0);
             tc::mma_commit(mma_bar);
         }
         ok = tc::bar_wait(mma_bar, mma_phase);

@@ -185,6 +185,17 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
+// D[16x8] += A[16x16] B[16x8], bf16 inputs (pairs packed in 32-bit registers),
+// fp32 accumulate. a = (A[g][2t..2t+1]), (A[g+8][2t..]), (A[g][2t+8..]), (A[g+8][2t+8..]);
+// b = (B[2t..2t+1][g]), (B[2t+8..2t+9][g]); d as for the tf32 shape.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
 // P[16x16] += A[16x16] B[16x16]; A, B fp32 in shared memory with row strides sa, sb.
 // The fp32 bits are passed as tf32 operands (the MMA reads the top 19 bits).
 // Result fragments: p[nt] covers columns 8nt..8nt+7 in the d layout above.
