@@ -179,6 +179,7 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
     const uint64_t dAQK = tc::desc_k(sbase + OP_AQK, 0);
     const uint64_t dW = tc::desc_mn(sbase + OP_W, 0, 8192);
     const uint64_t dKBmn = tc::desc_mn(sbase + OP_KB, 0, 16384);
+    float bnext = (tid < C && tid < sq.len) ? p.beta[(int64_t)(sq.tok0 + tid) * H + h] : 0.f;
     // prep map: warp w owns rows 8w..8w+7, lane l owns channels 4l..4l+3
     const int pkb = lane >> 4, pchk = (lane & 15) >> 1, phf = (lane & 1) * 8;
 
@@ -204,7 +205,12 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
 #pragma unroll
             for (int e = 0; e < 4; ++e) b[i][e] += b[i - 1][e];
         *reinterpret_cast<float4 *>(Tot + warp * 128 + 4 * lane) = make_float4(b[7][0], b[7][1], b[7][2], b[7][3]);
-        if (tid < C) bet[tid] = tid < n ? p.beta[(int64_t)(sq.tok0 + ci * C + tid) * H + h] : 0.f;
+        // beta of this chunk was fetched one chunk ahead (a strided global load)
+        if (tid < C) {
+            bet[tid] = bnext;
+            const int nn = min(C, sq.len - (ci + 1) * C);
+            bnext = (ci + 1 < n_chunks && tid < nn) ? p.beta[(int64_t)(sq.tok0 + (ci + 1) * C + tid) * H + h] : 0.f;
+        }
         __syncthreads();
         float m2[4] = {0.f, 0.f, 0.f, 0.f};
         {
@@ -236,6 +242,7 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
                 }
             }
         }
+        KDA_MARK(ci, 15);
         // ---- C. scaled bf16 operands Qh = q 2^(b-m), Ka = k 2^(b-m), Kb = k 2^(m-b)
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
