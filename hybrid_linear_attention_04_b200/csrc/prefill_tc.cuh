@@ -105,7 +105,8 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
     float *eC = eM + 128, *gC = eM + 256, *bet = eM + 384;
     uint64_t *tma_bar = reinterpret_cast<uint64_t *>(sm + BARS);   // [2]
     uint64_t *mma_bar = tma_bar + 2;       // rounds 2 and 3
-    uint64_t *bar_a = tma_bar + 3;         // round 1: [Qh; Ka] [Kb; Sm^T]^T
+    uint64_t *bar_a = tma_bar + 3;         // round 1a: [Qh; Ka] Kb^T
+    uint64_t *bar_b = tma_bar + 4;         // round 1b: [Qh; Ka] Sm
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tma_bar + 5);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -124,6 +125,7 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
         tc::bar_init(&tma_bar[1], 1);
         tc::bar_init(mma_bar, 1);
         tc::bar_init(bar_a, 1);
+        tc::bar_init(bar_b, 1);
         tc::bar_init_fence();
         tc::tma_prefetch_desc(&P.tm_q);
         tc::tma_prefetch_desc(&P.tm_k);
@@ -270,9 +272,21 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
             *reinterpret_cast<uint2 *>(sm + OP_AK + pkb * 16384 + tc::sw128(64 + r, pchk) + phf) = oa;
             *reinterpret_cast<uint2 *>(sm + OP_KB + pkb * 16384 + tc::sw128(r, pchk) + phf) = ob;
         }
-        __syncthreads();   // eM visible
+        tc::fence_async_smem();
+        __syncthreads();   // operands and eM visible
         KDA_MARK(ci, 2);
-        // ---- Sm^T = (Diag(e^m) S_0)^T (bf16, K-major B operand of round 1) ----
+        // ---- D1. round 1a: A = [Qh; Ka] Kb^T (independent of the state), issued
+        // before Sm^T is written so that the L extraction can start earlier
+        if (tid == 0) {
+            tc::fence_after_sync();
+            constexpr uint32_t id_a = tc::idesc_bf16(128, 64, false, false);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                tc::mma_bf16(tbase + COL_A, dAK + (k >> 2) * 1024 + (k & 3) * 2, dKB + (k >> 2) * 1024 + (k & 3) * 2,
+                             id_a, k > 0);
+            tc::mma_commit(bar_a);
+        }
+        // ---- Sm^T = (Diag(e^m) S_0)^T (bf16, K-major B operand of round 1b) ----
         {
             const float em = eM[c_own];
             __nv_bfloat16 *st = reinterpret_cast<__nv_bfloat16 *>(sm + OP_KB + (c_own >> 6) * 16384);
@@ -286,23 +300,23 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
         tc::fence_async_smem();
         __syncthreads();
         KDA_MARK(ci, 3);
-        // ---- D. round 1: A = [Qh; Ka] Kb^T; R' = Ka Sm; O = Qh Sm; then the next
-        // chunk's loads (descriptors advance by 16-byte units in their low bits)
+        // ---- D2. round 1b: [R'; O] = [Qh; Ka] Sm; then the next chunk's loads ----
         if (tid == 0) {
             tc::fence_after_sync();
-            constexpr uint32_t id_a = tc::idesc_bf16(128, 128, false, false);
+            constexpr uint32_t id_b = tc::idesc_bf16(128, 64, false, false);
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-                tc::mma_bf16(tbase + COL_A, dAK + (k >> 2) * 1024 + (k & 3) * 2, dKB + (k >> 2) * 1024 + (k & 3) * 2,
-                             id_a, k > 0);
-            tc::mma_commit(bar_a);
+                tc::mma_bf16(tbase + COL_O, dAK + (k >> 2) * 1024 + (k & 3) * 2,
+                             dKB + (k >> 2) * 1024 + 512 + (k & 3) * 2, id_b, k > 0);
+            tc::mma_commit(bar_b);
             if (ci + 1 < n_chunks) {
                 issue_loads(ci + 1);
                 issued = ci + 2;
             }
         }
-        // a timed-out wait is acted on at the block-wide vote after phase E
-        ok = tc::bar_wait(bar_a, (uint32_t)(ci & 1));
+        // warps 0-3 need A (round 1a), warps 6-7 need R' (round 1b); a timed-out
+        // wait is acted on at the block-wide vote after phase E
+        ok = tc::bar_wait(warp < 4 ? bar_a : bar_b, (uint32_t)(ci & 1));
         tc::fence_after_sync();
         KDA_MARK(ci, 4);
         // ---- E. warps 0,1: A_qk (masked bf16 operand). Warps 2,3: L = Diag(beta)
