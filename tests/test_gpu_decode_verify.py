@@ -154,3 +154,25 @@ def test_snapshot_copies_bit_exact_and_checks_range(cuda_device):
     bad = torch.tensor([10], dtype=torch.int64, device=cuda_device)
     K.kda_snapshot(bad, di[:1], src, dst)
     assert K.kda_check_device_status() == 7
+
+
+def test_verify_more_sequences_than_one_launch(cuda_device):
+    """1030 sequences: the library splits the batch into launches of at most
+    KDA_SEQS_PER_LAUNCH sequences; outputs and per-token states match the oracle."""
+    H, d, n_seq = 2, 64, 1030
+    x, cu, pool, slots = _verify_case(500, n_seq, H, d, "bf16", lo=1, hi=3)
+    dv = {k: v.to(cuda_device) for k, v in x.items()}
+    pool_d = pool.to(cuda_device)
+    T = int(cu[-1])
+    ts = torch.empty((T, H, d, d), dtype=torch.float32, device=cuda_device)
+    o = torch.empty_like(dv["v"])
+    K.kda_verify(dv["q"], dv["k"], dv["v"], dv["g"], dv["beta"], cu, slots.to(cuda_device), pool_d,
+                 ts, o)
+    assert K.kda_check_device_status() == 0
+    o_got, ts_got = to_np(o), ts.cpu().numpy()
+    for s in range(0, n_seq, 7):
+        a, b = int(cu[s]), int(cu[s + 1])
+        oo, _, sn = native.oracle_sequence(x["q"][a:b], x["k"][a:b], x["v"][a:b], x["g"][a:b],
+                                           x["beta"][a:b], pool[int(slots[s])], None, 0, 1)
+        assert blockwise_err(o_got[a:b], oo, (2,)) <= TOL_BF16, s
+        assert blockwise_err(ts_got[a:b], sn, (2, 3)) <= TOL_BF16, s

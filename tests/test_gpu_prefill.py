@@ -129,3 +129,42 @@ def test_segment_handoff_equals_one_shot(cuda_device, path):
     assert torch.equal(torch.cat(outs), o)
     assert torch.equal(state, sout)
     assert torch.equal(torch.cat(sn_all), snaps[:int(offs[-1])])
+
+
+def test_more_sequences_than_one_launch(cuda_device, path):
+    """1030 sequences (more than KDA_SEQS_PER_LAUNCH) split into several launches,
+    including zero-length ones, with snapshots and initial states."""
+    n_seq, H, d = 1030, 2, 128
+    lens = synth.randint(31, "lens", n_seq, 0, 140)
+    x, dev, cu = packed_inputs(31, lens, H, d, "bf16", cuda_device)
+    start = [64 * m for m in synth.randint(31, "resume", n_seq, 0, 3)]
+    s0 = synth.states(31, n_seq, H, d, d, std=0.1)
+    o, sout, snaps, offs = run_prefill(dev, cu, H, d, 64, "bf16", start, s0.to(cuda_device), 128,
+                                       cuda_device)
+    check(o, sout, snaps, offs, oracle_prefill(x, cu, start, s0, 128), "bf16")
+
+
+def test_gate_outside_tensor_core_range_is_reported(cuda_device):
+    """A chunk whose per-channel decay from its middle exceeds the tensor-core
+    path's range (here 96 nats) is reported as KDA_ERR_RANGE; the CUDA-core path
+    has no such limit and matches the oracle on the same input."""
+    H, d, T = 2, 128, 64
+    x = synth.token_inputs(41, T, H, d, d, io="bf16")
+    x["g"][:, 0, 5] = -3.0                       # one channel of head 0: 3 nats per token
+    dev = {k: v.to(cuda_device) for k, v in x.items()}
+    cu = np.array([0, T], dtype=np.int32)
+    o = torch.empty_like(dev["v"])
+    K.lib().kda_internal_force_prefill_path(0)
+    K.kda_prefill(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], cu, o, chunk=64)
+    assert K.kda_check_device_status() == 7
+    K.lib().kda_internal_force_prefill_path(1)
+    try:
+        sout = torch.empty((1, H, d, d), device=cuda_device)
+        K.kda_prefill(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], cu, o, state_out=sout,
+                      chunk=64)
+        assert K.kda_check_device_status() == 0
+    finally:
+        K.lib().kda_internal_force_prefill_path(0)
+    o_ref, s_ref, _ = oracle_prefill(x, cu)
+    assert blockwise_err(to_np(o), o_ref, (2,)) <= tol_for("bf16")
+    assert blockwise_err(to_np(sout), s_ref, (2, 3)) <= tol_for("bf16")
