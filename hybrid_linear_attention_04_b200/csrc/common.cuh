@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "kda.h"
 
 namespace kda {
@@ -14,6 +16,20 @@ __device__ unsigned int g_status;
 
 __device__ __forceinline__ void record_status(unsigned int code) {
     atomicCAS(&g_status, 0u, code);
+}
+
+// Raise a kernel's dynamic shared-memory limit on the current device once.
+// The attribute is per device, so a process that drives several GPUs keeps one
+// bit per device ordinal in `done` (ordinals >= 64 set it on every call).
+inline bool set_smem_limit_once(const void *fn, int bytes, std::atomic<unsigned long long> &done) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return true;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return false;
+    done.fetch_or(bit, std::memory_order_release);
+    return true;
 }
 
 // Element type traits for the q/k/v/o arrays.

@@ -85,14 +85,10 @@ static kda_status dispatch_decode(int D, DecodeParams &p, int n_blocks, cudaStre
 template <int D, int C, typename TIO>
 static kda_status launch_simt(const PrefillParams &p, cudaStream_t st) {
     using Sh = SimtShape<D, C>;
-    static bool attr_done = false;
-    if (!attr_done) {
-        if (cudaFuncSetAttribute(prefill_simt_kernel<D, C, TIO>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)Sh::smem_bytes) != cudaSuccess)
-            return KDA_ERR_CUDA;
-        attr_done = true;
-    }
+    static std::atomic<unsigned long long> attr_done{0};
+    if (!set_smem_limit_once((const void *)prefill_simt_kernel<D, C, TIO>, (int)Sh::smem_bytes,
+                             attr_done))
+        return KDA_ERR_CUDA;
     if (!launch_gate()) return KDA_ERR_CUDA;
     prefill_simt_kernel<D, C, TIO><<<p.n_items, Sh::NT, Sh::smem_bytes, st>>>(p);
     return last_launch_status();

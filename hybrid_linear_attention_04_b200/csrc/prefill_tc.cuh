@@ -593,13 +593,9 @@ inline kda_status launch_prefill_tc(PrefillParams &p, const kda_dims &d, int64_t
         return KDA_ERR_CUDA;
     P.p = p;
     P.p.n_items = p.n_seq * H * 2;
-    static bool attr_done = false;
-    if (!attr_done) {
-        if (cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)tcp::SMEM_BYTES) != cudaSuccess)
-            return KDA_ERR_CUDA;
-        attr_done = true;
-    }
+    static std::atomic<unsigned long long> attr_done{0};
+    if (!set_smem_limit_once((const void *)prefill_tc_kernel, (int)tcp::SMEM_BYTES, attr_done))
+        return KDA_ERR_CUDA;
     if (!gate()) return KDA_ERR_CUDA;
     prefill_tc_kernel<<<P.p.n_items, tcp::NT, tcp::SMEM_BYTES, st>>>(P);
     cudaError_t e = cudaGetLastError();
