@@ -177,7 +177,7 @@ def commit_bytes(n):
 class Workload:
     """The serving-step workload, resident on one device."""
 
-    def __init__(self, dev):
+    def __init__(self, dev, prefill_path="split"):
         from hybrid_linear_attention_04_b200 import kda as K
         self.K = K
         self.dev = dev
@@ -190,6 +190,11 @@ class Workload:
         self.p_o = torch.empty((PREFILL_T, H, D), dtype=torch.bfloat16, device=dev)
         self.p_sout = torch.empty((1, H, D, D), device=dev)
         self.p_snaps = torch.empty((self.n_snap, H, D, D), device=dev)
+        # "split": two launches through a workspace; "fused": one launch, no workspace
+        self.p_ws = None
+        if prefill_path == "split":
+            nbytes = K.kda_prefill_workspace_size(self.p["q"], self.p["v"], self.cu, C)
+            self.p_ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
         # decode + verify
         self.pool = synth.states(1002, N_SEQ, H, D, D, std=0.1).to(dev)
         self.slots = torch.arange(N_SEQ, dtype=torch.int32, device=dev)
@@ -217,7 +222,8 @@ class Workload:
     def prefill(self):
         K, p = self.K, self.p
         K.kda_prefill(p["q"], p["k"], p["v"], p["g"], p["beta"], self.cu, self.p_o,
-                      state_out=self.p_sout, snap_interval=SNAP, snapshots=self.p_snaps, chunk=C)
+                      state_out=self.p_sout, snap_interval=SNAP, snapshots=self.p_snaps, chunk=C,
+                      workspace=self.p_ws)
 
     def decode(self):
         d = self.d
@@ -275,7 +281,7 @@ def run_ours(args):
     if dist is not None:
         dist.barrier()
     from hybrid_linear_attention_04_b200 import kda as K
-    wl = Workload(dev)
+    wl = Workload(dev, args.prefill_path)
     stream = torch.cuda.current_stream(dev)
     comps = ["prefill", "decode", "verify", "commit"]
     fns = [wl.prefill, wl.decode, wl.verify, wl.commit]
@@ -361,12 +367,17 @@ def run_ours(args):
         pf = prefill_flops(PREFILL_T)
         comp["prefill"]["algorithmic_flops"] = pf
         comp["prefill"]["tc_frac"] = round(pf / (comp_ms[0] * 1e-3) / (peaks["bf16_tflops"] * 1e12), 4)
+        comp["prefill"]["path"] = args.prefill_path
         dom = max(comps, key=lambda c: comp[c]["ms"])
-        kname = {"prefill": "prefill_tc_kernel", "decode": "decode_kernel", "verify": "verify_kernel",
-                 "commit": "snapshot_kernel"}[dom]
+        pk = ["prefill_prep_kernel", "prefill_chain_kernel"] if args.prefill_path == "split" \
+            else ["prefill_tc_kernel"]
+        knames = {"prefill": pk, "decode": ["decode_kernel"], "verify": ["verify_kernel"],
+                  "commit": ["snapshot_kernel"]}[dom]
+        kname = "+".join(knames)
         tr_units = {"prefill": (PREFILL_T * H, PREFILL_T * H), "decode": (N_SEQ * H, N_SEQ * H),
                     "verify": (N_SEQ * H, wl.n_tok * H), "commit": (wl.n_commit, wl.n_commit)}[dom]
-        tr = ncu_traffic(kname, *tr_units)
+        trs = [ncu_traffic(k, *tr_units) for k in knames]
+        tr = None if any(t is None for t in trs) else sum(trs)
         roof = {"bound": "hbm", "kernel": kname, "achieved": comp[dom]["achieved_gbs"],
                 "peak": hbm, "unit": "GB/s", "frac": comp[dom]["hbm_frac"],
                 "traffic": tr, "peak_source": peaks["source"]}
@@ -431,7 +442,14 @@ def run_workload(args):
     dev = torch.device("cuda", 0)
     peaks = load_peaks()
     wl = synth.WORKLOADS
-    out = {"impl": "ours", "workload": args.workload, "steps": args.steps, "warmup": args.warmup}
+    out = {"impl": "ours", "workload": args.workload, "steps": args.steps, "warmup": args.warmup,
+           "prefill_path": args.prefill_path}
+
+    def workspace(xd, cu):
+        if args.prefill_path != "split":
+            return None
+        n = K.kda_prefill_workspace_size(xd["q"], xd["v"], cu, C)
+        return torch.empty(n, dtype=torch.uint8, device=dev) if n else None
     if args.workload == "tiny":
         c = wl["tiny_fp32"]
         x = synth.token_inputs(c["seed"], c["T"], c["H"], c["d"], c["d"], io="fp32")
@@ -440,7 +458,8 @@ def run_workload(args):
         so = torch.empty((1, c["H"], c["d"], c["d"]), device=dev)
         cu = np.array([0, c["T"]], dtype=np.int32)
         ms = time_calls(lambda: K.kda_prefill(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], cu, o,
-                                              state_out=so, chunk=c["chunk"]), args.steps, args.warmup, dev)
+                                              state_out=so, chunk=c["chunk"], workspace=None),
+                        args.steps, args.warmup, dev)
         out.update({"unit": "us/call", "value": ms * 1e3, "tokens": c["T"]})
     elif args.workload == "ragged":
         c = wl["ragged_prefix_32"]
@@ -457,9 +476,11 @@ def run_workload(args):
         so = torch.empty_like(s0)
         offs, _ = K.kda_snapshot_plan(cu, start, c["snap"])
         sn = torch.empty((int(offs[-1]), H, D, D), device=dev)
+        ws = workspace(xd, cu)
         ms = time_calls(lambda: K.kda_prefill(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], cu, o,
                                               state_out=so, state_in=s0, start_pos=start,
-                                              snap_interval=c["snap"], snapshots=sn, chunk=C),
+                                              snap_interval=c["snap"], snapshots=sn, chunk=C,
+                                              workspace=ws),
                         args.steps, args.warmup, dev)
         byts = T * H * (3 * D * 2 + D * 2 + D * 4 + 4) + (int(offs[-1]) + 2 * c["n_seq"]) * H * D * D * 4
         out.update({"unit": "tok/s", "value": T / (ms * 1e-3), "ms": ms, "tokens": T,
@@ -479,13 +500,15 @@ def run_workload(args):
         n_snap = seg // c["snap"]
         sn = torch.empty((n_snap, H, D, D), device=dev)
         cu = np.array([0, seg], dtype=np.int32)
+        ws = workspace(segs[0], cu)
 
         def one_pass():
             for i in range(n_seg):
                 xd = segs[i % 2]
                 K.kda_prefill(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], cu, o,
                               state_out=st[(i + 1) % 2], state_in=st[i % 2] if i else None,
-                              start_pos=[i * seg], snap_interval=c["snap"], snapshots=sn, chunk=C)
+                              start_pos=[i * seg], snap_interval=c["snap"], snapshots=sn, chunk=C,
+                              workspace=ws)
         ms = time_calls(one_pass, max(1, args.steps // 5), 1, dev)
         T = c["T"]
         byts = T * H * (3 * D * 2 + D * 2 + D * 4 + 4) + (T // c["snap"] + 2 * n_seg) * H * D * D * 4
@@ -539,6 +562,9 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=2048)
     ap.add_argument("--ref-tokens", type=int, default=512)
     ap.add_argument("--workload", choices=["serving", "tiny", "ragged", "long"], default="serving")
+    ap.add_argument("--prefill-path", choices=["split", "fused"], default="split",
+                    help="tensor-core prefill in two launches through a workspace (split) or in "
+                         "one launch without one (fused)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
     if args.impl == "reference":

@@ -18,7 +18,8 @@ __device__ __forceinline__ void record_status(unsigned int code) {
     atomicCAS(&g_status, 0u, code);
 }
 
-// Raise a kernel's dynamic shared-memory limit on the current device once.
+// Raise a kernel's dynamic shared-memory limit (and prefer the largest shared
+// memory carveout) on the current device once.
 // The attribute is per device, so a process that drives several GPUs keeps one
 // bit per device ordinal in `done` (ordinals >= 64 set it on every call).
 inline bool set_smem_limit_once(const void *fn, int bytes, std::atomic<unsigned long long> &done) {
@@ -26,7 +27,9 @@ inline bool set_smem_limit_once(const void *fn, int bytes, std::atomic<unsigned 
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
     const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
     if (bit && (done.load(std::memory_order_acquire) & bit)) return true;
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
+        cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
         return false;
     done.fetch_or(bit, std::memory_order_release);
     return true;

@@ -15,6 +15,7 @@
 #include "decode.cuh"
 #include "prefill_simt.cuh"
 #include "prefill_tc.cuh"
+#include "prefill_split.cuh"
 #include "snapshot.cuh"
 
 namespace kda {
@@ -120,7 +121,7 @@ const char *kda_status_string(kda_status s) {
     case KDA_ERR_INVALID: return "KDA_ERR_INVALID: invalid argument";
     case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: unsupported dimensions";
     case KDA_ERR_ALIGN: return "KDA_ERR_ALIGN: device pointer not 16-byte aligned";
-    case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE: reserved";
+    case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE: workspace smaller than kda_prefill_workspace_size";
     case KDA_ERR_CUDA: return "KDA_ERR_CUDA: CUDA call or launch failed";
     case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: device wait ran out of iterations";
     case KDA_ERR_RANGE: return "KDA_ERR_RANGE: device-side range check failed";
@@ -158,11 +159,32 @@ kda_status kda_snapshot_plan(int32_t n_seq, const int32_t *cu, const int64_t *st
     return KDA_OK;
 }
 
+kda_status kda_prefill_workspace_size(const kda_dims *dims, int32_t n_seq, const int32_t *cu,
+                                      size_t *bytes) {
+    if (!bytes) return KDA_ERR_INVALID;
+    *bytes = 0;
+    kda_status st = check_dims(dims, true);
+    if (st != KDA_OK) return st;
+    if (n_seq < 0) return KDA_ERR_INVALID;
+    if (n_seq == 0) return KDA_OK;
+    if (!cu || cu[0] != 0) return KDA_ERR_INVALID;
+    for (int s = 0; s < n_seq; ++s)
+        if (cu[s + 1] < cu[s]) return KDA_ERR_INVALID;
+    if (!tc_prefill_supported(*dims)) return KDA_OK;   // the CUDA-core path uses none
+    size_t need = 0;
+    for (int g0 = 0; g0 < n_seq; g0 += kPrefillSeqs) {
+        const int ng = std::min(kPrefillSeqs, n_seq - g0);
+        need = std::max(need, split_group_bytes((int64_t)cu[g0 + ng] - cu[g0], ng, dims->H));
+    }
+    *bytes = need;
+    return KDA_OK;
+}
+
 kda_status kda_prefill(const kda_dims *dims, int32_t n_seq, const int32_t *cu,
                        const int64_t *start_pos, const void *q, const void *k, const void *v,
                        const float *g, const float *beta, const float *state_in,
                        float *state_out, void *o, int32_t snap_interval, float *snapshots,
-                       kda_stream_t stream) {
+                       void *workspace, size_t workspace_bytes, kda_stream_t stream) {
     kda_status st = check_dims(dims, true);
     if (st != KDA_OK) return st;
     if (n_seq < 0 || snap_interval < 0) return KDA_ERR_INVALID;
@@ -180,7 +202,7 @@ kda_status kda_prefill(const kda_dims *dims, int32_t n_seq, const int32_t *cu,
     const int64_t T = cu[n_seq];
     if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID;
     if (offs[n_seq] > 0 && !snapshots) return KDA_ERR_INVALID;
-    const void *ptrs[] = {q, k, v, g, beta, state_in, state_out, o, snapshots};
+    const void *ptrs[] = {q, k, v, g, beta, state_in, state_out, o, snapshots, workspace};
     for (const void *ptr : ptrs)
         if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
 
@@ -193,6 +215,13 @@ kda_status kda_prefill(const kda_dims *dims, int32_t n_seq, const int32_t *cu,
 
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     const bool tc = g_prefill_path.load() == 0 && tc_prefill_supported(*dims);
+    const bool split = tc && workspace != nullptr;
+    if (split) {
+        size_t need = 0;
+        st = kda_prefill_workspace_size(dims, n_seq, cu, &need);
+        if (st != KDA_OK) return st;
+        if (workspace_bytes < need) return KDA_ERR_WORKSPACE;
+    }
     static thread_local PrefillParams p;  // ~27 KB: keep it off the stack
     for (int g0 = 0; g0 < n_seq; g0 += kPrefillSeqs) {
         const int ng = std::min(kPrefillSeqs, n_seq - g0);
@@ -212,7 +241,9 @@ kda_status kda_prefill(const kda_dims *dims, int32_t n_seq, const int32_t *cu,
             p.seq[i].start_pos = start_pos ? start_pos[s] : 0;
             p.seq[i].snap_off = offs[s];
         }
-        if (tc) {
+        if (split) {
+            st = launch_prefill_split(p, *dims, T, cu[g0], cu[g0 + ng], workspace, cs, launch_gate);
+        } else if (tc) {
             st = launch_prefill_tc(p, *dims, T, cs, launch_gate);
         } else {
             p.n_items = ng * H * (D / SimtShape<32, 16>::DVS);

@@ -1,0 +1,697 @@
+// KDA chunked prefill in two launches (d_k = d_v = 128, chunk 64, bf16 q/k/v/o,
+// fp32 state), for callers that provide a workspace. The chunk form is the one in
+// prefill_common.cuh; the scaled operands are those of prefill_tc.cuh (Qh, Ka, Kb
+// around a per-channel reference m at the chunk middle, Sm = Diag(e^m) S_0).
+//
+// With T = (I + Diag(beta) A_kk)^{-1} (unit lower triangular), W' = T Diag(beta) Ka
+// and U = T Diag(beta) V, the chunk update becomes
+//     W   = U - W' Sm
+//     O   = scale (Qh Sm + A_qk W)
+//     S_C = Diag(Gamma_C) S_0 + Diag(e^(b_C - m)) Kb^T W
+// so everything except two small products per chunk is independent of S_0:
+//
+//   prep   one CTA per (chunk, head), all chunks of all sequences at once:
+//          cumsum, scaled operands, A = [Qh; Ka] Kb^T (tcgen05), T by block forward
+//          substitution (mma.sync), [W' | U] = T [beta Ka | beta V] (tcgen05). Writes
+//          one packet per (chunk, head) to the workspace, laid out as the shared
+//          memory images the chain kernel feeds to its MMAs.
+//   chain  one CTA per (sequence, head, 64-column d_v slice): per chunk, one bulk
+//          copy of the packet (three chunks in flight), then
+//            round 1  [Qh; W'] Sm          -> TMEM (M=128: rows 0-63 O, 64-127 W'Sm)
+//            W = U - W'Sm (bf16)
+//            round 2  O += A_qk W,  D = Kb^T W
+//          and the fp32 state update in registers.
+#pragma once
+#include <cudaTypedefs.h>
+
+#include "prefill_common.cuh"
+#include "tc_util.cuh"
+
+namespace kda {
+
+namespace spl {
+constexpr int C = 64, D = 128;
+// ---- workspace packet of one (chunk, head); every image is 128B-swizzled slabs
+constexpr uint32_t PK_QW = 0;         // [Qh; W']: 2 slabs (channels 0-63, 64-127) x 128 rows
+constexpr uint32_t PK_KB = 32768;     // Kb: 2 slabs x 64 token rows
+constexpr uint32_t PK_AQK = 49152;    // A_qk masked (i <= r), 1 slab x 64 rows
+constexpr uint32_t PK_VEC = 57344;    // eM, eC, gC: fp32 [3][128] (1536 B, slot of 2048)
+constexpr uint32_t PK_U = 59392;      // U: 2 slabs (d_v 0-63, 64-127) x 64 token rows
+constexpr uint32_t PACKET = PK_U + 16384;   // 75776 bytes
+// ---- prep kernel shared memory
+constexpr uint32_t P_QK = 0;          // 2 slabs x 128 rows: q -> Qh (rows 0-63), k -> Ka -> beta Ka
+constexpr uint32_t P_V = 32768;       // v: 2 slabs x 64 rows -> beta V in place
+constexpr uint32_t P_KB = 49152;      // Kb: 2 slabs x 64 rows
+constexpr uint32_t P_TI = 65536;      // T (bf16): 1 slab x 64 rows
+constexpr uint32_t P_G = 73728;       // g fp32 [64][128]; once the operands are built, the solve
+                                      // scratch: Ls, Lb, Wsc below
+constexpr uint32_t P_LS = P_G;                    // fp32 [64][17]: L on its diagonal 16x16 blocks
+constexpr uint32_t P_LB = P_LS + 64 * 17 * 4;     // bf16 [64][72]: L, and X on the diagonal blocks
+constexpr uint32_t P_WSC = P_LB + 64 * 72 * 2;    // bf16 [8 warps][8][72]
+constexpr uint32_t P_TOT = P_G + 32768;           // fp32 [8][128] row-block totals of b
+constexpr uint32_t P_VEC = P_TOT + 4096;          // eM, eC, gC [128], beta [64]
+constexpr uint32_t P_BARS = P_VEC + (3 * 128 + 64) * 4;
+constexpr uint32_t P_SMEM = P_BARS + 32 + 1024;   // + slack for 1024-byte alignment
+constexpr uint32_t P_TX = 16384 * 3 + 32768;      // q, k, v, g bytes per chunk
+constexpr uint32_t P_COL_A = 0, P_COL_W = 0, P_COL_U = 128, P_TMEM = 256;
+// ---- chain kernel shared memory
+constexpr uint32_t STAGE = PK_U + 8192;           // a packet without the other d_v slice of U
+constexpr int NSTAGE = 3;
+constexpr uint32_t S_U = PK_U;                    // U slice inside a stage
+constexpr uint32_t C_SM = NSTAGE * STAGE;         // Sm (bf16): MN-major B, 128 d_k rows x 64 d_v
+constexpr uint32_t C_W = C_SM + 16384;            // W (bf16): MN-major B, 64 token rows x 64 d_v
+constexpr uint32_t C_BARS = C_W + 8192;
+constexpr uint32_t C_SMEM = C_BARS + 64 + 1024;
+constexpr uint32_t C_COL_R1 = 0, C_COL_D = 64, C_TMEM = 128;
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float RANGE_LIMIT2 = 80.f * LOG2E;      // 80 nats, in log2 units
+static_assert(P_WSC + 8 * 8 * 72 * 2 <= P_TOT, "solve scratch overlaps");
+static_assert(STAGE % 1024 == 0 && PACKET % 16 == 0, "packet alignment");
+}  // namespace spl
+
+// Packet row of chunk c of sequence i (launch-local index): ((tok0 - tok_first) >> 6) + i + c.
+// Sequences' ranges are disjoint and increasing, and every index is below
+// ((tok_end - tok_first) >> 6) + n_seq.
+struct PrepParams {
+    CUtensorMap tm_q, tm_k, tm_v, tm_g;
+    const float *beta;
+    uint8_t *ws;
+    int32_t H, n_seq, tok_first, n_packets;
+    int32_t tok0[kPrefillSeqs];
+    int32_t len[kPrefillSeqs];
+};
+
+struct ChainParams {
+    PrefillParams p;
+    const uint8_t *ws;
+    int32_t tok_first;
+};
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+__device__ __forceinline__ uint32_t bf16x2(float a, float b) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+__device__ __forceinline__ float2 bf16x2_unpack(uint32_t u) {
+    return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&u));
+}
+__device__ __forceinline__ uint4 bf16x8(const float *a, float s) {
+    return make_uint4(bf16x2(s * a[0], s * a[1]), bf16x2(s * a[2], s * a[3]), bf16x2(s * a[4], s * a[5]),
+                      bf16x2(s * a[6], s * a[7]));
+}
+
+// ============================================================================ prep
+__global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_constant__ PrepParams P) {
+    using namespace spl;
+    const int H = P.H;
+    const int h = blockIdx.x % H;
+    const int pk = blockIdx.x / H;
+    // owner sequence: the last one whose first packet is <= pk
+    auto first_packet = [&](int i) { return ((P.tok0[i] - P.tok_first) >> 6) + i; };
+    int lo = 0, hi = P.n_seq - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (first_packet(mid) <= pk) lo = mid; else hi = mid - 1;
+    }
+    const int c = pk - first_packet(lo);
+    const int len = P.len[lo];
+    if (c < 0 || c * C >= len) return;       // an unused packet row (block-uniform)
+    const int n = min(C, len - c * C);
+    const int z = P.tok0[lo] + c * C;
+    uint8_t *pkt = P.ws + ((int64_t)pk * H + h) * PACKET;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = align1024(smem_raw);
+    const uint32_t sbase = tc::smem_u32(sm);
+    float *Gs = reinterpret_cast<float *>(sm + P_G);
+    float *Ls = reinterpret_cast<float *>(sm + P_LS);
+    __nv_bfloat16 *Lb = reinterpret_cast<__nv_bfloat16 *>(sm + P_LB);
+    __nv_bfloat16 *Wsc = reinterpret_cast<__nv_bfloat16 *>(sm + P_WSC);
+    float *Tot = reinterpret_cast<float *>(sm + P_TOT);
+    float *eM = reinterpret_cast<float *>(sm + P_VEC);
+    float *eC = eM + 128, *gC = eM + 256, *bet = eM + 384;
+    uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + P_BARS);
+    uint64_t *bar_a = bar_ld + 1, *bar_w = bar_ld + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_ld + 3);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wq = warp & 3;
+    if (tid == 0) {
+        tc::bar_init(bar_ld, 1);
+        tc::bar_init(bar_a, 1);
+        tc::bar_init(bar_w, 1);
+        tc::bar_init_fence();
+        tc::bar_expect_tx(bar_ld, P_TX);
+        tc::tma_load3(sm + P_QK, &P.tm_q, 0, h, z, bar_ld);
+        tc::tma_load3(sm + P_QK + 16384, &P.tm_q, 64, h, z, bar_ld);
+        tc::tma_load3(sm + P_QK + 8192, &P.tm_k, 0, h, z, bar_ld);
+        tc::tma_load3(sm + P_QK + 16384 + 8192, &P.tm_k, 64, h, z, bar_ld);
+        tc::tma_load3(sm + P_V, &P.tm_v, 0, h, z, bar_ld);
+        tc::tma_load3(sm + P_V + 8192, &P.tm_v, 64, h, z, bar_ld);
+        tc::tma_load3(sm + P_G, &P.tm_g, 0, h, z, bar_ld);
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(tmem_slot, P_TMEM);
+        tc::tmem_relinquish();
+    }
+    if (tid < C) bet[tid] = tid < n ? P.beta[(int64_t)(z + tid) * H + h] : 0.f;
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = *tmem_slot;
+    const uint32_t tlane = (uint32_t)(32 * wq) << 16;
+    bool ok = true, stored = false;
+
+    do {
+        ok = tc::bar_wait(bar_ld, 0);
+        if (!__syncthreads_and(ok)) { ok = false; break; }
+        // ---- b = cumsum(g) (log2 units): warp w rows 8w..8w+7, lane channels 4l..4l+3
+        float b[8][4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int r = 8 * warp + i;
+            const float4 x = *reinterpret_cast<const float4 *>(Gs + r * D + 4 * lane);
+            const float sc = r < n ? LOG2E : 0.f;
+            b[i][0] = x.x * sc; b[i][1] = x.y * sc; b[i][2] = x.z * sc; b[i][3] = x.w * sc;
+        }
+#pragma unroll
+        for (int i = 1; i < 8; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) b[i][e] += b[i - 1][e];
+        *reinterpret_cast<float4 *>(Tot + warp * 128 + 4 * lane) = make_float4(b[7][0], b[7][1], b[7][2], b[7][3]);
+        __syncthreads();
+        float m2[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+            float off[4] = {0.f, 0.f, 0.f, 0.f}, bc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int w2 = 0; w2 < 8; ++w2) {
+                const float4 t = *reinterpret_cast<const float4 *>(Tot + w2 * 128 + 4 * lane);
+                const float tv[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    if (w2 < warp) off[e] += tv[e];
+                    if (w2 < 4) m2[e] += tv[e];     // b at row 31
+                    bc[e] += tv[e];                 // b at row 63 (= row n-1)
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) b[i][e] += off[e];
+            if (warp == 0) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int ch = 4 * lane + e;
+                    eM[ch] = tc::ex2(m2[e]);
+                    eC[ch] = tc::ex2(bc[e] - m2[e]);
+                    gC[ch] = tc::ex2(bc[e]);
+                    if (-m2[e] > RANGE_LIMIT2 || m2[e] - bc[e] > RANGE_LIMIT2) record_status(KDA_ERR_RANGE);
+                }
+            }
+        }
+        // ---- Qh = q 2^(b-m), Ka = k 2^(b-m) in place; Kb = k 2^(m-b); beta V in place
+        {
+            const int pkb = lane >> 4, pchk = (lane & 15) >> 1, phf = (lane & 1) * 8;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int r = 8 * warp + i;
+                const uint32_t so = tc::sw128(r, pchk) + phf;
+                uint8_t *qp = sm + P_QK + pkb * 16384 + so;
+                uint8_t *kp = sm + P_QK + pkb * 16384 + 8192 + so;
+                uint8_t *vp = sm + P_V + pkb * 8192 + so;
+                const uint2 qv = *reinterpret_cast<const uint2 *>(qp);
+                const uint2 kv = *reinterpret_cast<const uint2 *>(kp);
+                const uint2 vv = *reinterpret_cast<const uint2 *>(vp);
+                const float2 q01 = bf16x2_unpack(qv.x), q23 = bf16x2_unpack(qv.y);
+                const float2 k01 = bf16x2_unpack(kv.x), k23 = bf16x2_unpack(kv.y);
+                const float2 v01 = bf16x2_unpack(vv.x), v23 = bf16x2_unpack(vv.y);
+                float e1[4], e2[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float d = b[i][e] - m2[e];
+                    e1[e] = tc::ex2(d);
+                    e2[e] = tc::ex2(-d);
+                }
+                const bool live = r < n;
+                const float br = bet[r];
+                *reinterpret_cast<uint2 *>(qp) =
+                    live ? make_uint2(bf16x2(q01.x * e1[0], q01.y * e1[1]), bf16x2(q23.x * e1[2], q23.y * e1[3]))
+                         : make_uint2(0u, 0u);
+                *reinterpret_cast<uint2 *>(kp) =
+                    live ? make_uint2(bf16x2(k01.x * e1[0], k01.y * e1[1]), bf16x2(k23.x * e1[2], k23.y * e1[3]))
+                         : make_uint2(0u, 0u);
+                *reinterpret_cast<uint2 *>(sm + P_KB + pkb * 8192 + so) =
+                    live ? make_uint2(bf16x2(k01.x * e2[0], k01.y * e2[1]), bf16x2(k23.x * e2[2], k23.y * e2[3]))
+                         : make_uint2(0u, 0u);
+                *reinterpret_cast<uint2 *>(vp) =
+                    make_uint2(bf16x2(br * v01.x, br * v01.y), bf16x2(br * v23.x, br * v23.y));
+            }
+        }
+        tc::fence_async_smem();
+        __syncthreads();
+        // ---- A = [Qh; Ka] Kb^T (M=128: A_qk rows 0-63, A_kk rows 64-127); Qh and Kb
+        // go to the packet as they are
+        if (tid == 0) {
+            tc::fence_after_sync();
+            constexpr uint32_t id_a = tc::idesc_bf16(128, 64, false, false);
+            const uint64_t dQK = tc::desc_k(sbase + P_QK, 0), dKB = tc::desc_k(sbase + P_KB, 0);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                tc::mma_bf16(tbase + P_COL_A, dQK + (k >> 2) * 1024 + (k & 3) * 2, dKB + (k >> 2) * 512 + (k & 3) * 2,
+                             id_a, k > 0);
+            tc::mma_commit(bar_a);
+        } else if (tid == 32) {
+            tc::bulk_store(pkt + PK_QW, sm + P_QK, 8192);
+            tc::bulk_store(pkt + PK_QW + 16384, sm + P_QK + 16384, 8192);
+            tc::bulk_store(pkt + PK_KB, sm + P_KB, 16384);
+            tc::bulk_commit();
+            stored = true;
+        }
+        if (tid < 96)
+            reinterpret_cast<float4 *>(pkt + PK_VEC)[tid] = reinterpret_cast<const float4 *>(eM)[tid];
+        ok = tc::bar_wait(bar_a, 0);
+        tc::fence_after_sync();
+        if (warp < 2) {
+            // A_qk, masked to i <= r, straight into the packet image
+            const int r = 32 * warp + lane;
+            float a[32];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                tc::tmem_ld32(tbase + tlane + P_COL_A + 32 * half, a);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int jj = 32 * half + 8 * q4 + 2 * e;
+                        w[e] = bf16x2(jj <= r ? a[8 * q4 + 2 * e] : 0.f, jj + 1 <= r ? a[8 * q4 + 2 * e + 1] : 0.f);
+                    }
+                    *reinterpret_cast<uint4 *>(pkt + PK_AQK + tc::sw128(r, 4 * half + q4)) =
+                        make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+        } else if (warp < 4) {
+            // L = Diag(beta) A_kk strictly below the diagonal: bf16 everywhere, fp32 on
+            // the diagonal blocks; then the inverses X of the four diagonal blocks
+            const int r = 32 * (warp - 2) + lane;
+            const float br = bet[r];
+            const int dblk = r & ~15;
+            float a[32];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                tc::tmem_ld32(tbase + tlane + P_COL_A + 32 * half, a);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    float l[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int jj = 32 * half + 8 * q4 + e;
+                        l[e] = jj < r ? br * a[8 * q4 + e] : 0.f;
+                        if (jj >= dblk && jj < dblk + 16) Ls[r * 17 + (jj - dblk)] = l[e];
+                    }
+                    *reinterpret_cast<uint4 *>(Lb + r * 72 + 32 * half + 8 * q4) = bf16x8(l, 1.f);
+                }
+            }
+            __syncwarp();
+            const int base = 16 * (2 * (warp - 2) + (lane >> 4)), cc = lane & 15;
+            float x[16];
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) {
+                float a0 = rr == cc ? 1.f : 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                const float *lr = Ls + (base + rr) * 17;
+#pragma unroll
+                for (int i = 0; i < rr; ++i) {
+                    const float t = lr[i] * x[i];
+                    if ((i & 3) == 0) a0 -= t;
+                    else if ((i & 3) == 1) a1 -= t;
+                    else if ((i & 3) == 2) a2 -= t;
+                    else a3 -= t;
+                }
+                x[rr] = (a0 + a1) + (a2 + a3);
+            }
+            __syncwarp();
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) Lb[(base + rr) * 72 + base + cc] = __float2bfloat16_rn(x[rr]);
+        } else {
+            // beta Ka in place (rows 64-127 of both slabs; A has been read)
+            const int t = tid - 128;
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+                const int idx = t + 128 * it;
+                const int slab = idx >> 9, row = (idx >> 3) & 63, chunk = idx & 7;
+                uint4 *p4 = reinterpret_cast<uint4 *>(sm + P_QK + slab * 16384 + (64 + row) * 128 + chunk * 16);
+                const uint4 u = *p4;
+                const float br = bet[row];
+                const float2 x0 = bf16x2_unpack(u.x), x1 = bf16x2_unpack(u.y), x2 = bf16x2_unpack(u.z),
+                             x3 = bf16x2_unpack(u.w);
+                *p4 = make_uint4(bf16x2(br * x0.x, br * x0.y), bf16x2(br * x1.x, br * x1.y),
+                                 bf16x2(br * x2.x, br * x2.y), bf16x2(br * x3.x, br * x3.y));
+            }
+        }
+        tc::fence_async_smem();
+        tc::fence_before_sync();
+        if (!__syncthreads_and(ok)) { ok = false; break; }
+        // ---- T = (I + L)^{-1} by block forward substitution on bf16 mma.sync (fp32
+        // accumulate): T_R = X_RR (E_R - sum_{J<R} L_RJ T_J), E = identity. Warp w
+        // owns columns 8w..8w+7.
+        {
+            const int g = lane >> 2, t = lane & 3, c0 = 8 * warp;
+            __nv_bfloat16 *ws = Wsc + warp * 8 * 72;
+#pragma unroll
+            for (int R = 0; R < 4; ++R) {
+                const int r0 = 16 * R + g, r1 = r0 + 8;
+                float y[4] = {r0 == c0 + 2 * t ? 1.f : 0.f, r0 == c0 + 2 * t + 1 ? 1.f : 0.f,
+                              r1 == c0 + 2 * t ? 1.f : 0.f, r1 == c0 + 2 * t + 1 ? 1.f : 0.f};
+                float part[3][4];
+#pragma unroll
+                for (int J = 0; J < R; ++J) {
+                    const int kc = 16 * J + 2 * t;
+                    const uint32_t a[4] = {*reinterpret_cast<const uint32_t *>(Lb + r0 * 72 + kc),
+                                           *reinterpret_cast<const uint32_t *>(Lb + r1 * 72 + kc),
+                                           *reinterpret_cast<const uint32_t *>(Lb + r0 * 72 + kc + 8),
+                                           *reinterpret_cast<const uint32_t *>(Lb + r1 * 72 + kc + 8)};
+                    const uint32_t bb[2] = {*reinterpret_cast<const uint32_t *>(ws + g * 72 + kc),
+                                            *reinterpret_cast<const uint32_t *>(ws + g * 72 + kc + 8)};
+                    float (&pp)[4] = part[J];
+                    pp[0] = pp[1] = pp[2] = pp[3] = 0.f;
+                    tc::mma_bf16_16816(pp, a, bb);
+                }
+#pragma unroll
+                for (int J = 0; J < R; ++J) {
+                    y[0] -= part[J][0]; y[1] -= part[J][1]; y[2] -= part[J][2]; y[3] -= part[J][3];
+                }
+                ws[(2 * t) * 72 + r0] = __float2bfloat16_rn(y[0]);
+                ws[(2 * t + 1) * 72 + r0] = __float2bfloat16_rn(y[1]);
+                ws[(2 * t) * 72 + r1] = __float2bfloat16_rn(y[2]);
+                ws[(2 * t + 1) * 72 + r1] = __float2bfloat16_rn(y[3]);
+                __syncwarp();
+                float w[4] = {0.f, 0.f, 0.f, 0.f};
+                {
+                    const int kc = 16 * R + 2 * t;
+                    const uint32_t a[4] = {*reinterpret_cast<const uint32_t *>(Lb + r0 * 72 + kc),
+                                           *reinterpret_cast<const uint32_t *>(Lb + r1 * 72 + kc),
+                                           *reinterpret_cast<const uint32_t *>(Lb + r0 * 72 + kc + 8),
+                                           *reinterpret_cast<const uint32_t *>(Lb + r1 * 72 + kc + 8)};
+                    const uint32_t bb[2] = {*reinterpret_cast<const uint32_t *>(ws + g * 72 + kc),
+                                            *reinterpret_cast<const uint32_t *>(ws + g * 72 + kc + 8)};
+                    tc::mma_bf16_16816(w, a, bb);
+                }
+                __syncwarp();
+                ws[(2 * t) * 72 + r0] = __float2bfloat16_rn(w[0]);
+                ws[(2 * t + 1) * 72 + r0] = __float2bfloat16_rn(w[1]);
+                ws[(2 * t) * 72 + r1] = __float2bfloat16_rn(w[2]);
+                ws[(2 * t + 1) * 72 + r1] = __float2bfloat16_rn(w[3]);
+                // T (bf16, K-major A operand): columns c0 + 2t, c0 + 2t + 1 are in 16-byte chunk `warp`
+                *reinterpret_cast<uint32_t *>(sm + P_TI + tc::sw128(r0, warp) + 4 * t) = bf16x2(w[0], w[1]);
+                *reinterpret_cast<uint32_t *>(sm + P_TI + tc::sw128(r1, warp) + 4 * t) = bf16x2(w[2], w[3]);
+                __syncwarp();
+            }
+        }
+        tc::fence_async_smem();
+        tc::fence_before_sync();
+        __syncthreads();
+        // ---- [W' | U] = T [beta Ka | beta V]  (M=64: row r in TMEM lane (r % 16) + 32 (r / 16))
+        if (tid == 0) {
+            tc::fence_after_sync();
+            constexpr uint32_t id_w = tc::idesc_bf16(64, 128, false, true);
+            const uint64_t dT = tc::desc_k(sbase + P_TI, 0);
+            const uint64_t dBK = tc::desc_mn(sbase + P_QK + 8192, 0, 16384);
+            const uint64_t dBV = tc::desc_mn(sbase + P_V, 0, 8192);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) tc::mma_bf16(tbase + P_COL_W, dT + 2 * k, dBK + 128 * k, id_w, k > 0);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) tc::mma_bf16(tbase + P_COL_U, dT + 2 * k, dBV + 128 * k, id_w, k > 0);
+            tc::mma_commit(bar_w);
+        }
+        ok = tc::bar_wait(bar_w, 0);
+        tc::fence_after_sync();
+        {
+            // warp (wq, wh): rows 16 wq .. 16 wq + 15 (lanes 0-15), columns 64 wh .. 64 wh + 63
+            const int wh = warp >> 2, r = 16 * wq + lane;
+            float a[32];
+#pragma unroll
+            for (int mat = 0; mat < 2; ++mat) {
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    tc::tmem_ld32(tbase + tlane + (mat ? P_COL_U : P_COL_W) + 64 * wh + 32 * hh, a);
+                    tc::tmem_ld_wait();
+                    if (lane < 16) {
+                        uint8_t *dst = mat ? pkt + PK_U + wh * 8192 : pkt + PK_QW + wh * 16384 + 8192;
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4)
+                            *reinterpret_cast<uint4 *>(dst + tc::sw128(r, 4 * hh + q4)) = bf16x8(a + 8 * q4, 1.f);
+                    }
+                }
+            }
+        }
+    } while (0);
+
+    if (!ok && tid == 0) tc::bar_wait(bar_ld, 0, 1u << 16);   // loads still in flight land first
+    if (stored) tc::bulk_wait_read_all();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, P_TMEM);
+}
+
+// =========================================================================== chain
+__global__ void __launch_bounds__(256, 1) prefill_chain_kernel(const __grid_constant__ ChainParams CP) {
+    using namespace spl;
+    const PrefillParams &p = CP.p;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = align1024(smem_raw);
+    const uint32_t sbase = tc::smem_u32(sm);
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + C_BARS);   // [NSTAGE]
+    uint64_t *bar_r1 = full + NSTAGE, *bar_r2 = full + NSTAGE + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(full + NSTAGE + 2);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wq = warp & 3, wh = warp >> 2;
+    const int H = p.H;
+    const int item = blockIdx.x;
+    const int rank = item / (H * 2);
+    const int h = (item >> 1) % H;
+    const int half = item & 1, j0 = 64 * half;
+    const int s = p.order[rank];
+    const PrefillSeq sq = p.seq[s];
+    const int n_chunks = (sq.len + C - 1) / C;
+    const int64_t pk0 = ((sq.tok0 - CP.tok_first) >> 6) + s;
+
+    if (tid == 0) {
+        for (int i = 0; i < NSTAGE + 2; ++i) tc::bar_init(&full[i], 1);
+        tc::bar_init_fence();
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(tmem_slot, C_TMEM);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = *tmem_slot;
+    const uint32_t tlane = (uint32_t)(32 * wq) << 16;
+
+    // fp32 master state: thread owns d_k row c_own, columns [32 wh, 32 wh + 32) of the slice
+    const int c_own = tid & 127;
+    float S[32];
+    {
+        const float *src =
+            p.state_in ? p.state_in + (((int64_t)s * H + h) * D + c_own) * D + j0 + 32 * wh : nullptr;
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+            float4 v = src ? *reinterpret_cast<const float4 *>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            S[j] = v.x; S[j + 1] = v.y; S[j + 2] = v.z; S[j + 3] = v.w;
+        }
+    }
+
+    auto issue_loads = [&](int ci) {
+        uint8_t *stg = sm + (ci % NSTAGE) * STAGE;
+        const uint8_t *pkt = CP.ws + ((pk0 + ci) * H + h) * PACKET;
+        uint64_t *bar = &full[ci % NSTAGE];
+        tc::bar_expect_tx(bar, STAGE);
+        tc::bulk_load(stg, pkt, PK_U, bar);
+        tc::bulk_load(stg + S_U, pkt + PK_U + half * 8192, 8192, bar);
+    };
+    int issued = 0, landed = 0;
+    if (tid == 0)
+        for (; issued < NSTAGE - 1 && issued < n_chunks; ++issued) issue_loads(issued);
+
+    const uint64_t dSM = tc::desc_mn(sbase + C_SM, 0, 16384);
+    const uint64_t dW = tc::desc_mn(sbase + C_W, 0, 8192);
+    bool ok = true;
+    int64_t snap_row = sq.snap_off;
+
+    for (int ci = 0; ci < n_chunks; ++ci) {
+        const int n = min(C, sq.len - ci * C);
+        const int st = ci % NSTAGE;
+        uint8_t *stg = sm + st * STAGE;
+        const uint32_t sstg = sbase + st * STAGE;
+        const float *eM = reinterpret_cast<const float *>(stg + PK_VEC);
+        const float *eC = eM + 128, *gC = eM + 256;
+        ok = tc::bar_wait(&full[st], (uint32_t)((ci / NSTAGE) & 1));
+        if (!__syncthreads_and(ok)) { ok = false; break; }
+        landed = ci + 1;
+        // ---- Sm = Diag(e^m) S_0 (bf16, MN-major: row = d_k channel, 64 d_v columns)
+        {
+            const float em = eM[c_own];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+                *reinterpret_cast<uint4 *>(sm + C_SM + tc::sw128(c_own, 4 * wh + q4)) = bf16x8(S + 8 * q4, em);
+        }
+        tc::fence_async_smem();
+        __syncthreads();
+        // ---- round 1: [Qh; W'] Sm; then the loads of chunk ci + NSTAGE - 1
+        if (tid == 0) {
+            tc::fence_after_sync();
+            constexpr uint32_t id1 = tc::idesc_bf16(128, 64, false, true);
+            const uint64_t dQW = tc::desc_k(sstg + PK_QW, 0);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                tc::mma_bf16(tbase + C_COL_R1, dQW + (k >> 2) * 1024 + (k & 3) * 2, dSM + 128 * k, id1, k > 0);
+            tc::mma_commit(bar_r1);
+            if (issued < n_chunks) {
+                issue_loads(issued);
+                ++issued;
+            }
+        }
+        // ---- W = U - W' Sm (warps on TMEM lanes 64-127: token rows)
+        if (wq >= 2) {
+            ok = tc::bar_wait(bar_r1, (uint32_t)(ci & 1));
+            tc::fence_after_sync();
+            const int r = 32 * (wq - 2) + lane;
+            float a[32];
+            tc::tmem_ld32(tbase + tlane + C_COL_R1 + 32 * wh, a);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const uint32_t off = tc::sw128(r, 4 * wh + q4);
+                const uint4 u = *reinterpret_cast<const uint4 *>(stg + S_U + off);
+                const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+                float w[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 uf = bf16x2_unpack(uw[e]);
+                    w[2 * e] = uf.x - a[8 * q4 + 2 * e];
+                    w[2 * e + 1] = uf.y - a[8 * q4 + 2 * e + 1];
+                }
+                *reinterpret_cast<uint4 *>(sm + C_W + off) = bf16x8(w, 1.f);
+            }
+        }
+        tc::fence_async_smem();
+        tc::fence_before_sync();
+        if (!__syncthreads_and(ok)) { ok = false; break; }
+        // ---- round 2: O += A_qk W (M=128; A rows 64-127 are the bytes after A_qk and land
+        // in TMEM lanes 64-127, which are not read again), D = Kb^T W
+        if (tid == 0) {
+            tc::fence_after_sync();
+            constexpr uint32_t id_o = tc::idesc_bf16(128, 64, false, true);
+            constexpr uint32_t id_d = tc::idesc_bf16(128, 64, true, true);
+            const uint64_t dAQK = tc::desc_k(sstg + PK_AQK, 0);
+            const uint64_t dKB = tc::desc_mn(sstg + PK_KB, 0, 8192);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) tc::mma_bf16(tbase + C_COL_R1, dAQK + 2 * k, dW + 128 * k, id_o, 1);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) tc::mma_bf16(tbase + C_COL_D, dKB + 128 * k, dW + 128 * k, id_d, k > 0);
+            tc::mma_commit(bar_r2);
+        }
+        ok = tc::bar_wait(bar_r2, (uint32_t)(ci & 1));
+        if (!__syncthreads_and(ok)) { ok = false; break; }
+        tc::fence_after_sync();
+        // ---- outputs, state update, snapshot
+        {
+            float a[32];
+            const int r = 32 * wq + lane;
+            if (wq < 2) {
+                tc::tmem_ld32(tbase + tlane + C_COL_R1 + 32 * wh, a);
+                tc::tmem_ld_wait();
+                if (r < n) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) +
+                                                           ((int64_t)(sq.tok0 + ci * C + r) * H + h) * D + j0 + 32 * wh);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) dst[q4] = bf16x8(a + 8 * q4, p.scale);
+                }
+            }
+            const float g_c = gC[c_own], e_c = eC[c_own];
+            tc::tmem_ld32(tbase + tlane + C_COL_D + 32 * wh, a);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) S[e] = fmaf(g_c, S[e], e_c * a[e]);
+            if (p.snap_interval > 0 && (sq.start_pos + (int64_t)ci * C + n) % p.snap_interval == 0) {
+                float *dst = p.snapshots + ((snap_row * H + h) * D + c_own) * (int64_t)D + j0 + 32 * wh;
+#pragma unroll
+                for (int j = 0; j < 32; j += 4)
+                    *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+                ++snap_row;
+            }
+        }
+        tc::fence_before_sync();
+        __syncthreads();
+    }
+
+    if (ok && p.state_out) {
+        float *dst = p.state_out + (((int64_t)s * H + h) * D + c_own) * (int64_t)D + j0 + 32 * wh;
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+    }
+    if (tid == 0 && !ok) {
+        for (int c2 = landed; c2 < issued; ++c2)
+            tc::bar_wait(&full[c2 % NSTAGE], (uint32_t)((c2 / NSTAGE) & 1), 1u << 16);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, C_TMEM);
+}
+
+// ---------------------------------------------------------------------------- host
+// Workspace bytes of one launch group: packets for ((tokens >> 6) + sequences) rows x H heads.
+inline size_t split_group_bytes(int64_t group_tokens, int n_seq, int H) {
+    return (size_t)((group_tokens >> 6) + n_seq) * (size_t)H * spl::PACKET;
+}
+
+template <typename Gate>
+inline kda_status launch_prefill_split(PrefillParams &p, const kda_dims &d, int64_t T, int32_t tok_first,
+                                       int32_t tok_end, void *ws, cudaStream_t st, Gate gate) {
+    using namespace spl;
+    static thread_local PrepParams PP;
+    static thread_local ChainParams CPm;
+    const int H = d.H;
+    const int64_t n_packets = ((int64_t)(tok_end - tok_first) >> 6) + p.n_seq;
+    if (n_packets * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    if (!encode_map(&PP.tm_q, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, T, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_map(&PP.tm_k, p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, T, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_map(&PP.tm_v, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, T, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_map(&PP.tm_g, p.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, T, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return KDA_ERR_CUDA;
+    PP.beta = p.beta;
+    PP.ws = static_cast<uint8_t *>(ws);
+    PP.H = H;
+    PP.n_seq = p.n_seq;
+    PP.tok_first = tok_first;
+    PP.n_packets = (int32_t)n_packets;
+    for (int i = 0; i < p.n_seq; ++i) {
+        PP.tok0[i] = p.seq[i].tok0;
+        PP.len[i] = p.seq[i].len;
+    }
+    CPm.p = p;
+    CPm.p.n_items = p.n_seq * H * 2;
+    CPm.ws = static_cast<const uint8_t *>(ws);
+    CPm.tok_first = tok_first;
+    static std::atomic<unsigned long long> prep_attr{0}, chain_attr{0};
+    if (!set_smem_limit_once((const void *)prefill_prep_kernel, (int)P_SMEM, prep_attr) ||
+        !set_smem_limit_once((const void *)prefill_chain_kernel, (int)C_SMEM, chain_attr))
+        return KDA_ERR_CUDA;
+    if (n_packets > 0) {
+        if (!gate()) return KDA_ERR_CUDA;
+        prefill_prep_kernel<<<(unsigned)(n_packets * H), 256, P_SMEM, st>>>(PP);
+        if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    if (!gate()) return KDA_ERR_CUDA;
+    prefill_chain_kernel<<<CPm.p.n_items, 256, C_SMEM, st>>>(CPm);
+    return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // namespace kda

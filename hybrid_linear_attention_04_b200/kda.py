@@ -40,7 +40,9 @@ _I32, _I64 = ctypes.c_int32, ctypes.c_int64
 
 _SIGNATURES = {
     "kda_snapshot_plan": (_I32, [_I32, _P, _P, _I32, _P, _P]),
-    "kda_prefill": (_I32, [_P, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P]),
+    "kda_prefill_workspace_size": (_I32, [_P, _I32, _P, _P]),
+    "kda_prefill": (_I32, [_P, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P,
+                           ctypes.c_size_t, _P]),
     "kda_decode": (_I32, [_P, _I32, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P]),
     "kda_verify": (_I32, [_P, _I32, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P]),
     "kda_snapshot": (_I32, [_I32, _P, _P, _P, _I64, _P, _I64, _I32, _I32, _I32, _P]),
@@ -138,16 +140,39 @@ def kda_snapshot_plan(cu_seqlens, start_pos=None, snap_interval=0):
     return offs, pos
 
 
+def kda_prefill_workspace_size(q, v, cu_seqlens, chunk=64) -> int:
+    """Workspace bytes kda_prefill can use for these shapes (see include/kda.h)."""
+    cu = _host_array(cu_seqlens, np.int32)
+    dims = _dims(q, v, chunk)
+    n = ctypes.c_size_t(0)
+    _check(lib().kda_prefill_workspace_size(ctypes.byref(dims), len(cu) - 1, _hptr(cu),
+                                            ctypes.byref(n)), "kda_prefill_workspace_size")
+    return int(n.value)
+
+
 def kda_prefill(q, k, v, g, beta, cu_seqlens, o, state_out=None, state_in=None, start_pos=None,
-                snap_interval=0, snapshots=None, chunk=64, scale=0.0, stream=None):
-    """Packed variable-length chunked prefill (see include/kda.h)."""
+                snap_interval=0, snapshots=None, chunk=64, scale=0.0, stream=None,
+                workspace="auto"):
+    """Packed variable-length chunked prefill (see include/kda.h).
+
+    ``workspace``: a device uint8 tensor of at least kda_prefill_workspace_size
+    bytes, ``None`` for the single-launch kernel without scratch memory, or
+    ``"auto"`` to allocate one of the required size on q's device (through
+    PyTorch's allocator) for this call.
+    """
     cu = _host_array(cu_seqlens, np.int32)
     sp = _host_array(start_pos, np.int64)
     dims = _dims(q, v, chunk, scale)
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise KDAError(1, f"workspace must be a tensor, None or 'auto', not {workspace!r}")
+        nbytes = kda_prefill_workspace_size(q, v, cu, chunk)
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device) if nbytes else None
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().kda_prefill(ctypes.byref(dims), len(cu) - 1, _hptr(cu), _hptr(sp), _dptr(q),
                              _dptr(k), _dptr(v), _dptr(g), _dptr(beta), _dptr(state_in),
                              _dptr(state_out), _dptr(o), int(snap_interval), _dptr(snapshots),
-                             _stream(stream)), "kda_prefill")
+                             _dptr(workspace), ws_bytes, _stream(stream)), "kda_prefill")
 
 
 def kda_decode(q, k, v, g, beta, slots, state_pool, o, scale=0.0, stream=None):

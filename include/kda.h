@@ -24,6 +24,7 @@
  *  - Pointers suffixed _h are host memory read during the call only. All other
  *    pointers are device memory owned by the caller; the library allocates no
  *    memory and keeps no state between calls except a device status word.
+ *    Scratch memory, where a call can use it, is a caller-provided workspace.
  *  - Every device pointer must be 16-byte aligned (KDA_ERR_ALIGN otherwise).
  *  - Calls are asynchronous on `stream`: argument errors return synchronously
  *    before anything is launched; device-side range errors and bounded-wait
@@ -48,7 +49,7 @@ typedef enum {
     KDA_ERR_INVALID = 1,     /* bad argument: null pointer, negative size, bad cu_seqlens ... */
     KDA_ERR_UNSUPPORTED = 2, /* dimensions outside the compiled set (see kda_dims) */
     KDA_ERR_ALIGN = 3,       /* a device pointer is not 16-byte aligned */
-    KDA_ERR_WORKSPACE = 4,   /* reserved */
+    KDA_ERR_WORKSPACE = 4,   /* workspace smaller than kda_prefill_workspace_size reports */
     KDA_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
     KDA_ERR_TIMEOUT = 6,     /* a device-side wait ran out of iterations (device status) */
     KDA_ERR_RANGE = 7        /* device-side check failed: a slot or index out of range, or a
@@ -91,6 +92,19 @@ kda_status kda_snapshot_plan(int32_t n_seq, const int32_t *cu_seqlens_h,
                              int64_t *snap_offsets_h, int64_t *snap_pos_h);
 
 /*
+ * kda_prefill_workspace_size — bytes of device workspace that kda_prefill can
+ * use for these dimensions and sequence lengths (host only, no GPU). 0 when the
+ * dimensions run on the CUDA-core path, which uses none. For the tensor-core
+ * dimensions (dk = dv = 128, chunk 64, bf16) it is, over each launch group of
+ * at most KDA_SEQS_PER_LAUNCH sequences, the largest
+ * (floor(group tokens / 64) + group sequences) * H * 75776.
+ * Errors: KDA_ERR_INVALID (null `bytes` or cu_seqlens_h, bad cu_seqlens_h),
+ * KDA_ERR_UNSUPPORTED as kda_prefill.
+ */
+kda_status kda_prefill_workspace_size(const kda_dims *dims, int32_t n_seq,
+                                      const int32_t *cu_seqlens_h, size_t *bytes);
+
+/*
  * kda_prefill — packed variable-length chunked prefill (Kimi K3 technical FAQ,
  * "What is KDA": parallel within a chunk, recurrent across chunks; the
  * chunk-form algebra is derived from the recurrence in the library's design
@@ -106,8 +120,17 @@ kda_status kda_snapshot_plan(int32_t n_seq, const int32_t *cu_seqlens_h,
  *               every start_pos must be a multiple of dims->chunk.
  *   snapshots [kda_snapshot_plan total, H, dk, dv] (required when any
  *               snapshot is due): fp32 states, rows as kda_snapshot_plan says.
+ *   workspace (nullable), workspace_bytes: device scratch, 16-byte aligned,
+ *               owned by the caller and not read back by it. With a workspace
+ *               the tensor-core dimensions run in two launches per group (all
+ *               chunks' state-independent work in parallel, then the
+ *               recurrence across chunks); with NULL they run in one launch
+ *               that keeps every intermediate on chip. Results agree to
+ *               rounding, not bit for bit, between the two. The workspace must
+ *               not be used by other work until the call's kernels finish.
  * A zero-length sequence writes state_out = state_in and no snapshots.
- * Errors (before launch): KDA_ERR_INVALID, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGN.
+ * Errors (before launch): KDA_ERR_INVALID, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGN,
+ * KDA_ERR_WORKSPACE (non-null workspace below kda_prefill_workspace_size).
  * Device status KDA_ERR_RANGE: a chunk whose per-channel decay exceeds the
  * tensor-core path's range (sum of g over one chunk below -170 in some channel;
  * the outputs of that chunk are then not reliable).
@@ -116,7 +139,8 @@ kda_status kda_prefill(const kda_dims *dims, int32_t n_seq, const int32_t *cu_se
                        const int64_t *start_pos_h, const void *q, const void *k,
                        const void *v, const float *g, const float *beta,
                        const float *state_in, float *state_out, void *o,
-                       int32_t snap_interval, float *snapshots, kda_stream_t stream);
+                       int32_t snap_interval, float *snapshots, void *workspace,
+                       size_t workspace_bytes, kda_stream_t stream);
 
 /*
  * kda_decode — one token per sequence against a pool of live states (the

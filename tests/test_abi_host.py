@@ -91,14 +91,14 @@ def _dims(H=4, d=128, chunk=64, io=0, scale=0.0):
     return K.kda_dims(H, d, d, chunk, io, scale)
 
 
-def _prefill(dims, cu, start=None, snap=0, ptr=A, snapshots=A, n_seq=None):
+def _prefill(dims, cu, start=None, snap=0, ptr=A, snapshots=A, n_seq=None, ws=None, ws_bytes=0):
     cu = np.asarray(cu, dtype=np.int32)
     sp = None if start is None else np.asarray(start, dtype=np.int64)
     L = K.lib()
     return L.kda_prefill(ctypes.byref(dims), len(cu) - 1 if n_seq is None else n_seq,
                          cu.ctypes.data_as(ctypes.c_void_p),
                          None if sp is None else sp.ctypes.data_as(ctypes.c_void_p),
-                         ptr, A, A, A, A, None, A, A, snap, snapshots, None)
+                         ptr, A, A, A, A, None, A, A, snap, snapshots, ws, ws_bytes, None)
 
 
 def test_prefill_validation():
@@ -117,6 +117,39 @@ def test_prefill_validation():
     assert _prefill(_dims(), [0, 64], ptr=MIS) == 3            # misaligned q
     assert _prefill(_dims(), [0, 64], ptr=None) == 1           # null q
     assert _prefill(_dims(), [0], n_seq=0) == 0                # nothing to do
+    need = _workspace_size(_dims(), [0, 64])
+    assert _prefill(_dims(), [0, 64], ws=A, ws_bytes=need - 16) == 4   # workspace too small
+    assert _prefill(_dims(), [0, 64], ws=MIS, ws_bytes=need) == 3      # misaligned workspace
+
+
+def _workspace_size(dims, cu, n_seq=None):
+    cu = np.asarray(cu, dtype=np.int32)
+    n = ctypes.c_size_t(12345)
+    st = K.lib().kda_prefill_workspace_size(ctypes.byref(dims), len(cu) - 1 if n_seq is None else n_seq,
+                                            cu.ctypes.data_as(ctypes.c_void_p), ctypes.byref(n))
+    return n.value if st == 0 else -st
+
+
+def test_prefill_workspace_size():
+    """One packet of 75776 bytes per (64-token chunk row, head); chunk rows of a
+    launch group are (group tokens >> 6) + group sequences, so that every
+    sequence's ragged chunks get rows of their own."""
+    P = 75776
+    assert _workspace_size(_dims(H=4), [0, 64]) == (1 + 1) * 4 * P
+    assert _workspace_size(_dims(H=2), [0, 1, 65, 200]) == ((200 >> 6) + 3) * 2 * P
+    assert _workspace_size(_dims(H=1), [0], n_seq=0) == 0
+    # more sequences than one launch: the largest group decides
+    cu = np.arange(0, 64 * 1030 + 1, 64)
+    assert _workspace_size(_dims(H=1), cu) == (1024 + 1024) * P
+    # dimensions of the CUDA-core path use none
+    assert _workspace_size(_dims(d=64, chunk=32), [0, 640]) == 0
+    assert _workspace_size(_dims(io=1), [0, 640]) == 0
+    # errors
+    assert _workspace_size(_dims(), [0, 64, 10]) == -1
+    assert _workspace_size(_dims(d=96), [0, 64]) == -2
+    assert K.lib().kda_prefill_workspace_size(ctypes.byref(_dims()), 1,
+                                              np.array([0, 64], np.int32).ctypes.data_as(ctypes.c_void_p),
+                                              None) == 1
 
 
 def test_decode_verify_snapshot_validation():

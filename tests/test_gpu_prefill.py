@@ -1,7 +1,8 @@
 """GPU parity of kda_prefill against the fp64 oracle (token recurrence), through
 the C ABI: packed ragged batches, initial states, start positions and
-block-boundary snapshots (vLLM day-0 blog, "Kimi Delta Attention"), on both
-prefill paths (tensor-core and CUDA-core) where the dims allow.
+block-boundary snapshots (vLLM day-0 blog, "Kimi Delta Attention"), on all three
+prefill paths (tensor cores in two launches or one, CUDA cores) where the dims
+allow.
 """
 from __future__ import annotations
 
@@ -16,10 +17,19 @@ from kda_cases import blockwise_err, oracle_prefill, packed_inputs, to_np, tol_f
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(params=["auto", "simt"])
+# prefill paths: "split" (tensor cores, two launches through a workspace), "fused"
+# (tensor cores, one launch, no workspace), "simt" (CUDA cores); dimensions the
+# tensor-core kernels do not cover run on the CUDA cores under every setting.
+_WS = {"split": "auto", "fused": None, "simt": "auto"}
+_mode = {"ws": "auto"}
+
+
+@pytest.fixture(params=["split", "fused", "simt"])
 def path(request):
     K.lib().kda_internal_force_prefill_path(1 if request.param == "simt" else 0)
+    _mode["ws"] = _WS[request.param]
     yield request.param
+    _mode["ws"] = "auto"
     K.lib().kda_internal_force_prefill_path(0)
 
 
@@ -33,7 +43,8 @@ def run_prefill(dev, cu, H, d, chunk, io, start=None, s0=None, snap=0, device=No
     # sentinel-filled snapshot pool with one spare row: only planned rows change
     snaps = torch.full((n_snap + 1, H, d, d), float("nan"), device=device)
     K.kda_prefill(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], cu, o, state_out=sout,
-                  state_in=s0, start_pos=start, snap_interval=snap, snapshots=snaps, chunk=chunk)
+                  state_in=s0, start_pos=start, snap_interval=snap, snapshots=snaps, chunk=chunk,
+                  workspace=_mode["ws"])
     assert K.kda_check_device_status() == 0
     return o, sout, snaps, offs
 
@@ -144,10 +155,12 @@ def test_more_sequences_than_one_launch(cuda_device, path):
     check(o, sout, snaps, offs, oracle_prefill(x, cu, start, s0, 128), "bf16")
 
 
-def test_gate_outside_tensor_core_range_is_reported(cuda_device):
+@pytest.mark.parametrize("ws", ["auto", None])
+def test_gate_outside_tensor_core_range_is_reported(cuda_device, ws):
     """A chunk whose per-channel decay from its middle exceeds the tensor-core
-    path's range (here 96 nats) is reported as KDA_ERR_RANGE; the CUDA-core path
-    has no such limit and matches the oracle on the same input."""
+    path's range (here 96 nats) is reported as KDA_ERR_RANGE by both tensor-core
+    kernels; the CUDA-core path has no such limit and matches the oracle on the
+    same input."""
     H, d, T = 2, 128, 64
     x = synth.token_inputs(41, T, H, d, d, io="bf16")
     x["g"][:, 0, 5] = -3.0                       # one channel of head 0: 3 nats per token
@@ -155,7 +168,7 @@ def test_gate_outside_tensor_core_range_is_reported(cuda_device):
     cu = np.array([0, T], dtype=np.int32)
     o = torch.empty_like(dev["v"])
     K.lib().kda_internal_force_prefill_path(0)
-    K.kda_prefill(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], cu, o, chunk=64)
+    K.kda_prefill(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], cu, o, chunk=64, workspace=ws)
     assert K.kda_check_device_status() == 7
     K.lib().kda_internal_force_prefill_path(1)
     try:

@@ -30,7 +30,7 @@ pytestmark = pytest.mark.gpu
 H, D, C = 64, 128, 64
 
 
-def _prefill(dev_in, cu, start=None, s0=None, snap=0, device=None):
+def _prefill(dev_in, cu, start=None, s0=None, snap=0, device=None, workspace="auto"):
     n_seq = len(cu) - 1
     T = int(cu[-1])
     o = torch.empty((T, H, D), dtype=torch.bfloat16, device=device)
@@ -39,22 +39,28 @@ def _prefill(dev_in, cu, start=None, s0=None, snap=0, device=None):
     snaps = torch.full((int(offs[-1]) + 1, H, D, D), float("nan"), device=device)
     K.kda_prefill(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["g"], dev_in["beta"], cu, o,
                   state_out=sout, state_in=s0, start_pos=start, snap_interval=snap, snapshots=snaps,
-                  chunk=C)
+                  chunk=C, workspace=workspace)
     assert K.kda_check_device_status() == 0
     assert torch.isnan(snaps[-1]).all()
     assert not torch.isnan(snaps[:-1]).any()
     return o, sout, snaps[:-1], offs, pos
 
 
-def test_prefill_8k_all_heads(cuda_device):
+_ORACLE_8K = {}
+
+
+@pytest.mark.parametrize("workspace", ["auto", None], ids=["split", "fused"])
+def test_prefill_8k_all_heads(cuda_device, workspace):
     T, snap = 8192, 256
     x = synth.token_inputs(1001, T, H, D, D, io="bf16")
     dev = {k: v.to(cuda_device) for k, v in x.items()}
     cu = np.array([0, T], dtype=np.int32)
-    o, sout, snaps, offs, pos = _prefill(dev, cu, snap=snap, device=cuda_device)
+    o, sout, snaps, offs, pos = _prefill(dev, cu, snap=snap, device=cuda_device, workspace=workspace)
     assert pos.tolist() == list(range(256, 8193, 256))
-    o_ref, s_ref, sn_ref = native.oracle_sequence(x["q"], x["k"], x["v"], x["g"], x["beta"],
-                                                  None, None, 0, snap, out_dtype=np.float32)
+    if not _ORACLE_8K:
+        _ORACLE_8K["ref"] = native.oracle_sequence(x["q"], x["k"], x["v"], x["g"], x["beta"],
+                                                   None, None, 0, snap, out_dtype=np.float32)
+    o_ref, s_ref, sn_ref = _ORACLE_8K["ref"]
     assert blockwise_err(to_np(o), o_ref, (0, 2)) <= TOL_BF16
     assert blockwise_err(to_np(sout[0]), s_ref, (1, 2)) <= TOL_BF16
     assert blockwise_err(snaps.cpu().numpy(), sn_ref, (2, 3)) <= TOL_BF16
