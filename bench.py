@@ -177,17 +177,18 @@ def commit_bytes(n):
 class Workload:
     """The serving-step workload, resident on one device."""
 
-    def __init__(self, dev, prefill_path="split"):
+    def __init__(self, dev, prefill_path="split", T=PREFILL_T, n_seq=N_SEQ):
         from hybrid_linear_attention_04_b200 import kda as K
         self.K = K
         self.dev = dev
-        x = synth.token_inputs(1001, PREFILL_T, H, D, D, io="bf16")
+        self.T, self.n_seq = T, n_seq
+        x = synth.token_inputs(1001, T, H, D, D, io="bf16")
         self.host_prefill = x
         self.p = {k: v.to(dev) for k, v in x.items()}
-        self.cu = np.array([0, PREFILL_T], dtype=np.int32)
+        self.cu = np.array([0, T], dtype=np.int32)
         offs, _ = K.kda_snapshot_plan(self.cu, None, SNAP)
         self.n_snap = int(offs[-1])
-        self.p_o = torch.empty((PREFILL_T, H, D), dtype=torch.bfloat16, device=dev)
+        self.p_o = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
         self.p_sout = torch.empty((1, H, D, D), device=dev)
         self.p_snaps = torch.empty((self.n_snap, H, D, D), device=dev)
         # "split": two launches through a workspace; "fused": one launch, no workspace
@@ -196,21 +197,21 @@ class Workload:
             nbytes = K.kda_prefill_workspace_size(self.p["q"], self.p["v"], self.cu, C)
             self.p_ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
         # decode + verify
-        self.pool = synth.states(1002, N_SEQ, H, D, D, std=0.1).to(dev)
-        self.slots = torch.arange(N_SEQ, dtype=torch.int32, device=dev)
-        y = synth.token_inputs(1002, N_SEQ, H, D, D, io="bf16")
+        self.pool = synth.states(1002, n_seq, H, D, D, std=0.1).to(dev)
+        self.slots = torch.arange(n_seq, dtype=torch.int32, device=dev)
+        y = synth.token_inputs(1002, n_seq, H, D, D, io="bf16")
         self.d = {k: v.to(dev) for k, v in y.items()}
-        self.d_o = torch.empty((N_SEQ, H, D), dtype=torch.bfloat16, device=dev)
-        lens = synth.draft_lengths(1002, N_SEQ, 1, 8)
+        self.d_o = torch.empty((n_seq, H, D), dtype=torch.bfloat16, device=dev)
+        lens = synth.draft_lengths(1002, n_seq, 1, 8)
         self.cu_draft = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
         self.n_tok = int(self.cu_draft[-1])
-        z = synth.token_inputs(1002, self.n_tok, H, D, D, io="bf16", t0=N_SEQ)
+        z = synth.token_inputs(1002, self.n_tok, H, D, D, io="bf16", t0=n_seq)
         self.v = {k: v.to(dev) for k, v in z.items()}
         self.v_o = torch.empty((self.n_tok, H, D), dtype=torch.bfloat16, device=dev)
         self.ts = torch.empty((self.n_tok, H, D, D), device=dev)
-        acc = synth.randint(1002, "misc", N_SEQ, 0, 8)
+        acc = synth.randint(1002, "misc", n_seq, 0, 8)
         src, dst = [], []
-        for s in range(N_SEQ):
+        for s in range(n_seq):
             a = min(acc[s], lens[s])
             if a > 0:
                 src.append(int(self.cu_draft[s]) + a - 1)
@@ -281,7 +282,7 @@ def run_ours(args):
     if dist is not None:
         dist.barrier()
     from hybrid_linear_attention_04_b200 import kda as K
-    wl = Workload(dev, args.prefill_path)
+    wl = Workload(dev, args.prefill_path, args.prefill_tokens, args.decode_seqs)
     stream = torch.cuda.current_stream(dev)
     comps = ["prefill", "decode", "verify", "commit"]
     fns = [wl.prefill, wl.decode, wl.verify, wl.commit]
@@ -353,9 +354,9 @@ def run_ours(args):
         hbm = peaks["hbm_gbs"]
         comp = {}
         units = {
-            "prefill": (PREFILL_T, "tok/s", prefill_bytes(PREFILL_T, 1, wl.n_snap, False)),
-            "decode": (N_SEQ * H, "state-steps/s", decode_bytes(N_SEQ)),
-            "verify": (wl.n_tok * H, "state-steps/s", verify_bytes(N_SEQ, wl.n_tok)),
+            "prefill": (wl.T, "tok/s", prefill_bytes(wl.T, 1, wl.n_snap, False)),
+            "decode": (wl.n_seq * H, "state-steps/s", decode_bytes(wl.n_seq)),
+            "verify": (wl.n_tok * H, "state-steps/s", verify_bytes(wl.n_seq, wl.n_tok)),
             "commit": (wl.n_commit, "states/s", commit_bytes(wl.n_commit)),
         }
         for name, ms in zip(comps, comp_ms):
@@ -364,7 +365,7 @@ def run_ours(args):
             comp[name] = {"ms": round(ms, 4), "value": world * n_units / (ms * 1e-3), "unit": unit,
                           "algorithmic_bytes": byts, "achieved_gbs": round(gbs, 1),
                           "hbm_frac": round(gbs / hbm, 4)}
-        pf = prefill_flops(PREFILL_T)
+        pf = prefill_flops(wl.T)
         comp["prefill"]["algorithmic_flops"] = pf
         comp["prefill"]["tc_frac"] = round(pf / (comp_ms[0] * 1e-3) / (peaks["bf16_tflops"] * 1e12), 4)
         comp["prefill"]["path"] = args.prefill_path
@@ -374,8 +375,8 @@ def run_ours(args):
         knames = {"prefill": pk, "decode": ["decode_kernel"], "verify": ["verify_kernel"],
                   "commit": ["snapshot_kernel"]}[dom]
         kname = "+".join(knames)
-        tr_units = {"prefill": (PREFILL_T * H, PREFILL_T * H), "decode": (N_SEQ * H, N_SEQ * H),
-                    "verify": (N_SEQ * H, wl.n_tok * H), "commit": (wl.n_commit, wl.n_commit)}[dom]
+        tr_units = {"prefill": (wl.T * H, wl.T * H), "decode": (wl.n_seq * H, wl.n_seq * H),
+                    "verify": (wl.n_seq * H, wl.n_tok * H), "commit": (wl.n_commit, wl.n_commit)}[dom]
         trs = [ncu_traffic(k, *tr_units) for k in knames]
         tr = None if any(t is None for t in trs) else sum(trs)
         roof = {"bound": "hbm", "kernel": kname, "achieved": comp[dom]["achieved_gbs"],
@@ -391,21 +392,21 @@ def run_ours(args):
         clocks = clk.summary()
         result = {
             "metric": METRIC,
-            "value": world * PREFILL_T / (comp_ms[0] * 1e-3),
+            "value": world * wl.T / (comp_ms[0] * 1e-3),
             "unit": "tok/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(total_ms / args.steps, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "prefill 8192 tok x 64 heads (d=128, chunk 64, snapshots /256)"
-                                   " + decode/verify/commit 512 seq x 64 heads (drafts 1..8)",
-                       "global_batch": world * (1 + N_SEQ), "seq_len": PREFILL_T,
+            "config": {"workload": f"prefill {wl.T} tok x 64 heads (d=128, chunk 64, snapshots /256)"
+                                   f" + decode/verify/commit {wl.n_seq} seq x 64 heads (drafts 1..8)",
+                       "global_batch": world * (1 + wl.n_seq), "seq_len": wl.T,
                        "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (no flush)"},
             "components": comp,
             "roofline": roof,
             "cpu_baseline": cpu,
-            "e2e": {"value": world * PREFILL_T / (e2e_ms * 1e-3), "unit": "tok/s",
+            "e2e": {"value": world * wl.T / (e2e_ms * 1e-3), "unit": "tok/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "scope": "prefill call with pinned-host inputs and outputs"},
             "gpu_launches": launches,
@@ -562,6 +563,10 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=2048)
     ap.add_argument("--ref-tokens", type=int, default=512)
     ap.add_argument("--workload", choices=["serving", "tiny", "ragged", "long"], default="serving")
+    ap.add_argument("--prefill-tokens", type=int, default=PREFILL_T,
+                    help="prefill length of the serving step (smaller only for profiler captures)")
+    ap.add_argument("--decode-seqs", type=int, default=N_SEQ,
+                    help="decode/verify sequences of the serving step (smaller only for profiler captures)")
     ap.add_argument("--prefill-path", choices=["split", "fused"], default="split",
                     help="tensor-core prefill in two launches through a workspace (split) or in "
                          "one launch without one (fused)")

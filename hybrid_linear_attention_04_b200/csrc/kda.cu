@@ -242,7 +242,8 @@ kda_status kda_prefill(const kda_dims *dims, int32_t n_seq, const int32_t *cu,
             p.seq[i].snap_off = offs[s];
         }
         if (split) {
-            st = launch_prefill_split(p, *dims, T, cu[g0], cu[g0 + ng], workspace, cs, launch_gate);
+            st = launch_prefill_split(p, *dims, T, cu[g0], cu[g0 + ng], offs[n_seq], workspace, cs,
+                                      launch_gate);
         } else if (tc) {
             st = launch_prefill_tc(p, *dims, T, cs, launch_gate);
         } else {
@@ -364,6 +365,9 @@ void kda_internal_force_prefill_path(int32_t path) { g_prefill_path.store(path);
 #ifdef KDA_PHASE_TIMING
 extern "C" int kda_internal_phase_clock(long long *out) {
     return (int)cudaMemcpyFromSymbol(out, kda::g_phase_clock, sizeof(kda::g_phase_clock));
+}
+extern "C" int kda_internal_prep_clock(long long *out) {
+    return (int)cudaMemcpyFromSymbol(out, kda::g_prep_clock, sizeof(kda::g_prep_clock));
 }
 #endif
 

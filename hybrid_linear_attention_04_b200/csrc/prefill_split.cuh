@@ -29,6 +29,21 @@
 
 namespace kda {
 
+#ifdef KDA_PHASE_TIMING
+#define KDA_CMARK_T(t, ci, k) \
+    do { if (threadIdx.x == (t) && blockIdx.x == 0 && (ci) < 64) g_phase_clock[(ci)][(k)] = clock64(); } while (0)
+#else
+#define KDA_CMARK_T(t, ci, k) do { } while (0)
+#endif
+#define KDA_CMARK(ci, k) KDA_CMARK_T(64, ci, k)
+#ifdef KDA_PHASE_TIMING
+__device__ long long g_prep_clock[16][16];
+#define KDA_PMARK(k) \
+    do { if (threadIdx.x == 64 && blockIdx.x >= 4096 && blockIdx.x < 4112) g_prep_clock[blockIdx.x - 4096][(k)] = clock64(); } while (0)
+#else
+#define KDA_PMARK(k) do { } while (0)
+#endif
+
 namespace spl {
 constexpr int C = 64, D = 128;
 // ---- workspace packet of one (chunk, head); every image is 128B-swizzled slabs
@@ -55,18 +70,29 @@ constexpr uint32_t P_SMEM = P_BARS + 32 + 1024;   // + slack for 1024-byte align
 constexpr uint32_t P_TX = 16384 * 3 + 32768;      // q, k, v, g bytes per chunk
 constexpr uint32_t P_COL_A = 0, P_COL_W = 0, P_COL_U = 128, P_TMEM = 256;
 // ---- chain kernel shared memory
-constexpr uint32_t STAGE = PK_U + 8192;           // a packet without the other d_v slice of U
+constexpr uint32_t STAGE = PK_U;                  // the packet head ([Qh; W'], Kb, A_qk, vectors)
 constexpr int NSTAGE = 3;
-constexpr uint32_t S_U = PK_U;                    // U slice inside a stage
 constexpr uint32_t C_SM = NSTAGE * STAGE;         // Sm (bf16): MN-major B, 128 d_k rows x 64 d_v
 constexpr uint32_t C_W = C_SM + 16384;            // W (bf16): MN-major B, 64 token rows x 64 d_v
-constexpr uint32_t C_BARS = C_W + 8192;
+constexpr uint32_t C_O = C_W + 8192;              // O staging for a tiled store: 64 tokens x 64 d_v bf16
+constexpr uint32_t C_SN = C_O + 8192;             // snapshot staging: 64 d_k rows x 64 d_v fp32 as two
+                                                  // 128B-swizzled boxes of 32 columns
+constexpr uint32_t C_BARS = C_SN + 16384;
 constexpr uint32_t C_SMEM = C_BARS + 64 + 1024;
-constexpr uint32_t C_COL_R1 = 0, C_COL_D = 64, C_TMEM = 128;
+// TMEM: round 1 / O of chunk c in columns 64 (c % 2) .. +63 (O is read during chunk c + 1),
+// D = Kb^T W in 128 .. 191
+constexpr uint32_t C_COL_R1 = 0, C_COL_D = 128, C_TMEM = 256;
+// U in the packet, in the order the chain's W threads read it: 16-byte piece q4 (8 d_v
+// columns) of column group wg (32 columns) of d_v half hf for token row r is at
+// PK_U + ((hf * 2 + wg) * 4 + q4) * 1024 + 16 r, so a warp's 32 rows are 512 contiguous bytes
+__host__ __device__ constexpr uint32_t u_piece(int hf, int wg, int q4, int r) {
+    return PK_U + (uint32_t)(((hf * 2 + wg) * 4 + q4) * 1024 + 16 * r);
+}
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RANGE_LIMIT2 = 80.f * LOG2E;      // 80 nats, in log2 units
 static_assert(P_WSC + 8 * 8 * 72 * 2 <= P_TOT, "solve scratch overlaps");
-static_assert(STAGE % 1024 == 0 && PACKET % 16 == 0, "packet alignment");
+static_assert(STAGE % 1024 == 0 && PACKET % 16 == 0 && C_O % 1024 == 0 && C_SN % 1024 == 0, "alignment");
+static_assert(C_SMEM <= 232448, "chain shared memory");
 }  // namespace spl
 
 // Packet row of chunk c of sequence i (launch-local index): ((tok0 - tok_first) >> 6) + i + c.
@@ -82,9 +108,12 @@ struct PrepParams {
 };
 
 struct ChainParams {
+    CUtensorMap tm_o;        // o [T, H, 128] bf16, boxes of 64 d_v x 1 head x 64 tokens, 128B swizzle
+    CUtensorMap tm_snap;     // snapshots as [rows, 128] fp32, boxes of 32 x 64, 128B swizzle
     PrefillParams p;
     const uint8_t *ws;
     int32_t tok_first;
+    int32_t snap_tma;        // 1: snapshot rows fit the 32-bit box coordinates of tm_snap
 };
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
@@ -163,10 +192,12 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
     const uint32_t tbase = *tmem_slot;
     const uint32_t tlane = (uint32_t)(32 * wq) << 16;
     bool ok = true, stored = false;
+    KDA_PMARK(0);
 
     do {
         ok = tc::bar_wait(bar_ld, 0);
         if (!__syncthreads_and(ok)) { ok = false; break; }
+        KDA_PMARK(1);
         // ---- b = cumsum(g) (log2 units): warp w rows 8w..8w+7, lane channels 4l..4l+3
         float b[8][4];
 #pragma unroll
@@ -211,6 +242,7 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
                 }
             }
         }
+        KDA_PMARK(10);
         // ---- Qh = q 2^(b-m), Ka = k 2^(b-m) in place; Kb = k 2^(m-b); beta V in place
         {
             const int pkb = lane >> 4, pchk = (lane & 15) >> 1, phf = (lane & 1) * 8;
@@ -251,6 +283,7 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
         }
         tc::fence_async_smem();
         __syncthreads();
+        KDA_PMARK(2);
         // ---- A = [Qh; Ka] Kb^T (M=128: A_qk rows 0-63, A_kk rows 64-127); Qh and Kb
         // go to the packet as they are
         if (tid == 0) {
@@ -273,6 +306,7 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
             reinterpret_cast<float4 *>(pkt + PK_VEC)[tid] = reinterpret_cast<const float4 *>(eM)[tid];
         ok = tc::bar_wait(bar_a, 0);
         tc::fence_after_sync();
+        KDA_PMARK(3);
         if (warp < 2) {
             // A_qk, masked to i <= r, straight into the packet image
             const int r = 32 * warp + lane;
@@ -355,6 +389,7 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
         tc::fence_async_smem();
         tc::fence_before_sync();
         if (!__syncthreads_and(ok)) { ok = false; break; }
+        KDA_PMARK(4);
         // ---- T = (I + L)^{-1} by block forward substitution on bf16 mma.sync (fp32
         // accumulate): T_R = X_RR (E_R - sum_{J<R} L_RJ T_J), E = identity. Warp w
         // owns columns 8w..8w+7.
@@ -414,6 +449,7 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
         tc::fence_async_smem();
         tc::fence_before_sync();
         __syncthreads();
+        KDA_PMARK(5);
         // ---- [W' | U] = T [beta Ka | beta V]  (M=64: row r in TMEM lane (r % 16) + 32 (r / 16))
         if (tid == 0) {
             tc::fence_after_sync();
@@ -429,8 +465,11 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
         }
         ok = tc::bar_wait(bar_w, 0);
         tc::fence_after_sync();
+        KDA_PMARK(6);
         {
-            // warp (wq, wh): rows 16 wq .. 16 wq + 15 (lanes 0-15), columns 64 wh .. 64 wh + 63
+            // warp (wq, wh): rows 16 wq .. 16 wq + 15 (lanes 0-15), columns 64 wh .. 64 wh + 63.
+            // The images are staged in the solve scratch (free since T was built): W' slabs at
+            // P_G, P_G + 8192; U (in the chain's read order) at P_G + 16384; then bulk-stored.
             const int wh = warp >> 2, r = 16 * wq + lane;
             float a[32];
 #pragma unroll
@@ -440,20 +479,33 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
                     tc::tmem_ld32(tbase + tlane + (mat ? P_COL_U : P_COL_W) + 64 * wh + 32 * hh, a);
                     tc::tmem_ld_wait();
                     if (lane < 16) {
-                        uint8_t *dst = mat ? pkt + PK_U + wh * 8192 : pkt + PK_QW + wh * 16384 + 8192;
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4)
-                            *reinterpret_cast<uint4 *>(dst + tc::sw128(r, 4 * hh + q4)) = bf16x8(a + 8 * q4, 1.f);
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const uint32_t off = mat ? P_G + u_piece(wh, hh, q4, r) - PK_U + 16384
+                                                     : P_G + wh * 8192 + tc::sw128(r, 4 * hh + q4);
+                            *reinterpret_cast<uint4 *>(sm + off) = bf16x8(a + 8 * q4, 1.f);
+                        }
                     }
                 }
             }
         }
+        tc::fence_async_smem();
+        __syncthreads();
+        KDA_PMARK(7);
+        if (tid == 32) {
+            tc::bulk_store(pkt + PK_QW + 8192, sm + P_G, 8192);
+            tc::bulk_store(pkt + PK_QW + 16384 + 8192, sm + P_G + 8192, 8192);
+            tc::bulk_store(pkt + PK_U, sm + P_G + 16384, 16384);
+            tc::bulk_commit();
+        }
     } while (0);
 
+    KDA_PMARK(8);
     if (!ok && tid == 0) tc::bar_wait(bar_ld, 0, 1u << 16);   // loads still in flight land first
     if (stored) tc::bulk_wait_read_all();
     tc::fence_before_sync();
     __syncthreads();
+    KDA_PMARK(9);
     if (warp == 0) tc::tmem_dealloc(tbase, P_TMEM);
 }
 
@@ -465,11 +517,12 @@ __global__ void __launch_bounds__(256, 1) prefill_chain_kernel(const __grid_cons
     uint8_t *sm = align1024(smem_raw);
     const uint32_t sbase = tc::smem_u32(sm);
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + C_BARS);   // [NSTAGE]
-    uint64_t *bar_r1 = full + NSTAGE, *bar_r2 = full + NSTAGE + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(full + NSTAGE + 2);
+    uint64_t *bar_r1 = full + NSTAGE, *bar_d = full + NSTAGE + 1, *bar_o = full + NSTAGE + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(full + NSTAGE + 3);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3, wh = warp >> 2;
+    const bool wwarp = wq >= 2;                   // TMEM lanes 64-127: W rows; else O rows
     const int H = p.H;
     const int item = blockIdx.x;
     const int rank = item / (H * 2);
@@ -479,10 +532,13 @@ __global__ void __launch_bounds__(256, 1) prefill_chain_kernel(const __grid_cons
     const PrefillSeq sq = p.seq[s];
     const int n_chunks = (sq.len + C - 1) / C;
     const int64_t pk0 = ((sq.tok0 - CP.tok_first) >> 6) + s;
+    auto packet = [&](int ci) { return CP.ws + ((pk0 + ci) * H + h) * PACKET; };
 
     if (tid == 0) {
-        for (int i = 0; i < NSTAGE + 2; ++i) tc::bar_init(&full[i], 1);
+        for (int i = 0; i < NSTAGE + 3; ++i) tc::bar_init(&full[i], 1);
         tc::bar_init_fence();
+        tc::tma_prefetch_desc(&CP.tm_o);
+        if (p.snap_interval > 0 && CP.snap_tma) tc::tma_prefetch_desc(&CP.tm_snap);
     }
     if (warp == 0) {
         tc::tmem_alloc(tmem_slot, C_TMEM);
@@ -508,68 +564,109 @@ __global__ void __launch_bounds__(256, 1) prefill_chain_kernel(const __grid_cons
     }
 
     auto issue_loads = [&](int ci) {
-        uint8_t *stg = sm + (ci % NSTAGE) * STAGE;
-        const uint8_t *pkt = CP.ws + ((pk0 + ci) * H + h) * PACKET;
         uint64_t *bar = &full[ci % NSTAGE];
         tc::bar_expect_tx(bar, STAGE);
-        tc::bulk_load(stg, pkt, PK_U, bar);
-        tc::bulk_load(stg + S_U, pkt + PK_U + half * 8192, 8192, bar);
+        tc::bulk_load(sm + (ci % NSTAGE) * STAGE, packet(ci), STAGE, bar);
     };
     int issued = 0, landed = 0;
     if (tid == 0)
         for (; issued < NSTAGE - 1 && issued < n_chunks; ++issued) issue_loads(issued);
+    // U rows of a chunk for the W threads (token row r_w, columns 32 wh .. +31 of the slice),
+    // read from the workspace one chunk ahead
+    const int r_w = 32 * (wq - 2) + lane;
+    uint4 u[4];
+    auto load_u = [&](int ci) {
+        const uint8_t *pkt = packet(ci);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+            u[q4] = *reinterpret_cast<const uint4 *>(pkt + u_piece(half, wh, q4, r_w));
+    };
+    if (wwarp && n_chunks > 0) load_u(0);
 
     const uint64_t dSM = tc::desc_mn(sbase + C_SM, 0, 16384);
     const uint64_t dW = tc::desc_mn(sbase + C_W, 0, 8192);
     bool ok = true;
-    int64_t snap_row = sq.snap_off;
+    // Sm = Diag(e^m) S (bf16, MN-major: row = d_k channel, 64 d_v columns) for the chunk
+    // whose packet sits in stage `st`
+    auto write_sm = [&](int st) {
+        const float em = reinterpret_cast<const float *>(sm + st * STAGE + PK_VEC)[c_own];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+            *reinterpret_cast<uint4 *>(sm + C_SM + tc::sw128(c_own, 4 * wh + q4)) = bf16x8(S + 8 * q4, em);
+    };
+    if (n_chunks > 0) {
+        ok = tc::bar_wait(&full[0], 0);
+        if (ok) write_sm(0);
+        tc::fence_async_smem();
+        ok = __syncthreads_and(ok);
+        landed = 1;
+    }
 
-    for (int ci = 0; ci < n_chunks; ++ci) {
+    // Snapshots: the state after a due chunk is written during the next two chunks through
+    // the staging tile and tiled stores: d_k rows 0-63 (held by the O warps) during the
+    // first, rows 64-127 (W warps, from the copy Ss) during the second. Threads 32 and 64
+    // issue the stores and wait for their reads before the staging is written again.
+    float Ss[32];
+    int64_t next_snap = p.snap_interval > 0 ? (sq.start_pos / p.snap_interval + 1) * p.snap_interval : -1;
+    int64_t snap_row = sq.snap_off;
+    int64_t snap_pend = -1;               // snapshot row with a half still to be written
+    int snap_half = 0;                    // which half goes out during this chunk
+    bool stores_pending = false;          // thread 32 / 64: tiled stores issued, reads not waited for
+    auto direct_snapshot = [&](int64_t row, const float *src) {
+        float *dst = p.snapshots + ((row * H + h) * D + c_own) * (int64_t)D + j0 + 32 * wh;
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4 *>(dst + j) = make_float4(src[j], src[j + 1], src[j + 2], src[j + 3]);
+    };
+    auto stage_snapshot = [&](const float *src) {
+        uint8_t *box = sm + C_SN + wh * 8192;
+        const int r = c_own & 63;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4 *>(box + tc::sw128(r, q)) =
+                make_float4(src[4 * q], src[4 * q + 1], src[4 * q + 2], src[4 * q + 3]);
+    };
+    auto store_snapshot_half = [&](int64_t row, int hf) {
+        const int y = (int)((row * H + h) * D + 64 * hf);
+        tc::tma_store2(&CP.tm_snap, sm + C_SN, j0, y);
+        tc::tma_store2(&CP.tm_snap, sm + C_SN + 8192, j0 + 32, y);
+    };
+
+    for (int ci = 0; ok && ci < n_chunks; ++ci) {
         const int n = min(C, sq.len - ci * C);
         const int st = ci % NSTAGE;
         uint8_t *stg = sm + st * STAGE;
         const uint32_t sstg = sbase + st * STAGE;
-        const float *eM = reinterpret_cast<const float *>(stg + PK_VEC);
-        const float *eC = eM + 128, *gC = eM + 256;
-        ok = tc::bar_wait(&full[st], (uint32_t)((ci / NSTAGE) & 1));
-        if (!__syncthreads_and(ok)) { ok = false; break; }
-        landed = ci + 1;
-        // ---- Sm = Diag(e^m) S_0 (bf16, MN-major: row = d_k channel, 64 d_v columns)
-        {
-            const float em = eM[c_own];
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-                *reinterpret_cast<uint4 *>(sm + C_SM + tc::sw128(c_own, 4 * wh + q4)) = bf16x8(S + 8 * q4, em);
-        }
-        tc::fence_async_smem();
-        __syncthreads();
-        // ---- round 1: [Qh; W'] Sm; then the loads of chunk ci + NSTAGE - 1
+        const uint32_t col_r1 = C_COL_R1 + 64 * (ci & 1);
+        const float *eC = reinterpret_cast<const float *>(stg + PK_VEC) + 128, *gC = eC + 128;
+        KDA_CMARK(ci, 0);
+        // ---- round 1: [Qh; W'] Sm -> rows 0-63 O, rows 64-127 W'Sm; then the loads of
+        // chunk ci + NSTAGE - 1 (its stage was released at the end of chunk ci - 1)
         if (tid == 0) {
             tc::fence_after_sync();
             constexpr uint32_t id1 = tc::idesc_bf16(128, 64, false, true);
             const uint64_t dQW = tc::desc_k(sstg + PK_QW, 0);
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-                tc::mma_bf16(tbase + C_COL_R1, dQW + (k >> 2) * 1024 + (k & 3) * 2, dSM + 128 * k, id1, k > 0);
+                tc::mma_bf16(tbase + col_r1, dQW + (k >> 2) * 1024 + (k & 3) * 2, dSM + 128 * k, id1, k > 0);
             tc::mma_commit(bar_r1);
             if (issued < n_chunks) {
                 issue_loads(issued);
                 ++issued;
             }
         }
-        // ---- W = U - W' Sm (warps on TMEM lanes 64-127: token rows)
-        if (wq >= 2) {
+        float ov[32];          // O of chunk ci - 1 (O warps)
+        if (wwarp) {
+            // ---- W = U - W' Sm (token rows in TMEM lanes 64-127)
             ok = tc::bar_wait(bar_r1, (uint32_t)(ci & 1));
             tc::fence_after_sync();
-            const int r = 32 * (wq - 2) + lane;
+            KDA_CMARK(ci, 1);
             float a[32];
-            tc::tmem_ld32(tbase + tlane + C_COL_R1 + 32 * wh, a);
+            tc::tmem_ld32(tbase + tlane + col_r1 + 32 * wh, a);
             tc::tmem_ld_wait();
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
-                const uint32_t off = tc::sw128(r, 4 * wh + q4);
-                const uint4 u = *reinterpret_cast<const uint4 *>(stg + S_U + off);
-                const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+                const uint32_t uw[4] = {u[q4].x, u[q4].y, u[q4].z, u[q4].w};
                 float w[8];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -577,14 +674,26 @@ __global__ void __launch_bounds__(256, 1) prefill_chain_kernel(const __grid_cons
                     w[2 * e] = uf.x - a[8 * q4 + 2 * e];
                     w[2 * e + 1] = uf.y - a[8 * q4 + 2 * e + 1];
                 }
-                *reinterpret_cast<uint4 *>(sm + C_W + off) = bf16x8(w, 1.f);
+                *reinterpret_cast<uint4 *>(sm + C_W + tc::sw128(r_w, 4 * wh + q4)) = bf16x8(w, 1.f);
             }
+            tc::fence_async_smem();
+        } else if (ci > 0) {
+            // O of chunk ci - 1: its MMAs were committed before this chunk's barrier below, so
+            // the phase awaited is bar_o's latest
+            ok = tc::bar_wait(bar_o, (uint32_t)((ci - 1) & 1));
+            tc::fence_after_sync();
+            tc::tmem_ld32(tbase + tlane + C_COL_R1 + 64 * ((ci - 1) & 1) + 32 * wh, ov);
+            tc::tmem_ld_wait();
         }
-        tc::fence_async_smem();
+        if (stores_pending) {                 // staging tiles may be written after the barrier
+            tc::bulk_wait_read_all();
+            stores_pending = false;
+        }
         tc::fence_before_sync();
-        if (!__syncthreads_and(ok)) { ok = false; break; }
-        // ---- round 2: O += A_qk W (M=128; A rows 64-127 are the bytes after A_qk and land
-        // in TMEM lanes 64-127, which are not read again), D = Kb^T W
+        __syncthreads();
+        KDA_CMARK(ci, 2);
+        // ---- round 2: D = Kb^T W (commit bar_d), then O += A_qk W (M=128; A rows 64-127 are
+        // the bytes after A_qk and land in TMEM lanes 64-127, not read again; commit bar_o)
         if (tid == 0) {
             tc::fence_after_sync();
             constexpr uint32_t id_o = tc::idesc_bf16(128, 64, false, true);
@@ -592,43 +701,116 @@ __global__ void __launch_bounds__(256, 1) prefill_chain_kernel(const __grid_cons
             const uint64_t dAQK = tc::desc_k(sstg + PK_AQK, 0);
             const uint64_t dKB = tc::desc_mn(sstg + PK_KB, 0, 8192);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) tc::mma_bf16(tbase + C_COL_R1, dAQK + 2 * k, dW + 128 * k, id_o, 1);
-#pragma unroll
             for (int k = 0; k < 4; ++k) tc::mma_bf16(tbase + C_COL_D, dKB + 128 * k, dW + 128 * k, id_d, k > 0);
-            tc::mma_commit(bar_r2);
-        }
-        ok = tc::bar_wait(bar_r2, (uint32_t)(ci & 1));
-        if (!__syncthreads_and(ok)) { ok = false; break; }
-        tc::fence_after_sync();
-        // ---- outputs, state update, snapshot
-        {
-            float a[32];
-            const int r = 32 * wq + lane;
-            if (wq < 2) {
-                tc::tmem_ld32(tbase + tlane + C_COL_R1 + 32 * wh, a);
-                tc::tmem_ld_wait();
-                if (r < n) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) +
-                                                           ((int64_t)(sq.tok0 + ci * C + r) * H + h) * D + j0 + 32 * wh);
+            tc::mma_commit(bar_d);
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) dst[q4] = bf16x8(a + 8 * q4, p.scale);
+            for (int k = 0; k < 4; ++k) tc::mma_bf16(tbase + col_r1, dAQK + 2 * k, dW + 128 * k, id_o, 1);
+            tc::mma_commit(bar_o);
+        }
+        // ---- while this chunk's MMAs run: outputs of chunk ci - 1 and half of a pending
+        // snapshot go through the staging tiles
+        if (!wwarp) {
+            const int pn = min(C, sq.len - (ci - 1) * C);
+            const int r = 32 * wq + lane;
+            const bool tiled = ci > 0 && pn == C;
+            if (ci > 0 && !tiled && r < pn) {
+                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) +
+                                                       ((int64_t)(sq.tok0 + (ci - 1) * C + r) * H + h) * D + j0 + 32 * wh);
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) dst[q4] = bf16x8(ov + 8 * q4, p.scale);
+            }
+            if (tiled) {
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4)
+                    *reinterpret_cast<uint4 *>(sm + C_O + tc::sw128(r, 4 * wh + q4)) = bf16x8(ov + 8 * q4, p.scale);
+            }
+            const bool snap = snap_pend >= 0 && snap_half == 0;
+            if (snap) stage_snapshot(S);
+            if (tiled || snap) {
+                tc::fence_async_smem();
+                tc::named_sync(1, 128);
+                if (tid == 32) {
+                    if (tiled) tc::tma_store3(&CP.tm_o, sm + C_O, j0, h, sq.tok0 + (ci - 1) * C);
+                    if (snap) store_snapshot_half(snap_pend, 0);
+                    tc::bulk_commit();
+                    stores_pending = true;
                 }
             }
+        } else if (snap_pend >= 0 && snap_half == 1) {
+            stage_snapshot(Ss);
+            tc::fence_async_smem();
+            tc::named_sync(2, 128);
+            if (tid == 64) {
+                store_snapshot_half(snap_pend, 1);
+                tc::bulk_commit();
+                stores_pending = true;
+            }
+        }
+        if (snap_pend >= 0) {                 // the same bookkeeping in every thread
+            if (snap_half == 0) snap_half = 1;
+            else snap_pend = -1;
+        }
+        // ---- state update, then Sm of the next chunk
+        {
+            bool okd = tc::bar_wait(bar_d, (uint32_t)(ci & 1));
+            tc::fence_after_sync();
+            KDA_CMARK(ci, 3);
+            float a[32];
             const float g_c = gC[c_own], e_c = eC[c_own];
             tc::tmem_ld32(tbase + tlane + C_COL_D + 32 * wh, a);
             tc::tmem_ld_wait();
+            KDA_CMARK(ci, 4);
 #pragma unroll
             for (int e = 0; e < 32; ++e) S[e] = fmaf(g_c, S[e], e_c * a[e]);
-            if (p.snap_interval > 0 && (sq.start_pos + (int64_t)ci * C + n) % p.snap_interval == 0) {
-                float *dst = p.snapshots + ((snap_row * H + h) * D + c_own) * (int64_t)D + j0 + 32 * wh;
+            KDA_CMARK(ci, 5);
+            if (ci + 1 < n_chunks) {
+                okd = okd && tc::bar_wait(&full[(ci + 1) % NSTAGE], (uint32_t)(((ci + 1) / NSTAGE) & 1));
+                KDA_CMARK(ci, 6);
+                if (okd) write_sm((ci + 1) % NSTAGE);
+                tc::fence_async_smem();
+                if (wwarp) load_u(ci + 1);
+            }
+            KDA_CMARK(ci, 7);
+            if (sq.start_pos + (int64_t)ci * C + n == next_snap) {
+                next_snap += p.snap_interval;
+                // a snapshot due at consecutive chunks: the W rows of the previous one go out now
+                if (wwarp && snap_pend >= 0) direct_snapshot(snap_pend, Ss);
+                if (CP.snap_tma) {
+                    snap_pend = snap_row;
+                    snap_half = 0;
 #pragma unroll
-                for (int j = 0; j < 32; j += 4)
-                    *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+                    for (int e = 0; e < 32; ++e) Ss[e] = S[e];
+                } else {
+                    direct_snapshot(snap_row, S);
+                }
                 ++snap_row;
             }
+            ok = ok && okd;
         }
         tc::fence_before_sync();
-        __syncthreads();
+        ok = __syncthreads_and(ok);
+        if (ok) landed = ci + 2 < n_chunks ? ci + 2 : n_chunks;
+        KDA_CMARK(ci, 9);
+    }
+    if (ok && n_chunks > 0) {
+        // outputs of the last chunk; snapshot halves still pending
+        if (!wwarp) {
+            float a[32];
+            ok = tc::bar_wait(bar_o, (uint32_t)((n_chunks - 1) & 1));
+            tc::fence_after_sync();
+            tc::tmem_ld32(tbase + tlane + C_COL_R1 + 64 * ((n_chunks - 1) & 1) + 32 * wh, a);
+            tc::tmem_ld_wait();
+            const int r = 32 * wq + lane;
+            if (r < min(C, sq.len - (n_chunks - 1) * C)) {
+                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) +
+                                                       ((int64_t)(sq.tok0 + (n_chunks - 1) * C + r) * H + h) * D + j0 + 32 * wh);
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) dst[q4] = bf16x8(a + 8 * q4, p.scale);
+            }
+            if (snap_pend >= 0 && snap_half == 0) direct_snapshot(snap_pend, S);
+        } else if (snap_pend >= 0) {
+            direct_snapshot(snap_pend, Ss);
+        }
     }
 
     if (ok && p.state_out) {
@@ -641,6 +823,7 @@ __global__ void __launch_bounds__(256, 1) prefill_chain_kernel(const __grid_cons
         for (int c2 = landed; c2 < issued; ++c2)
             tc::bar_wait(&full[c2 % NSTAGE], (uint32_t)((c2 / NSTAGE) & 1), 1u << 16);
     }
+    if (stores_pending) tc::bulk_wait_read_all();     // staging must outlive the stores' reads
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tbase, C_TMEM);
@@ -652,9 +835,23 @@ inline size_t split_group_bytes(int64_t group_tokens, int n_seq, int H) {
     return (size_t)((group_tokens >> 6) + n_seq) * (size_t)H * spl::PACKET;
 }
 
+// snapshots viewed as [rows, 128] fp32, boxes of 32 columns x 64 rows (128B swizzle)
+inline bool encode_snap_map(CUtensorMap *m, float *base, int64_t rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {128 * sizeof(float)};
+    cuuint32_t box[2] = {32, 64};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <typename Gate>
 inline kda_status launch_prefill_split(PrefillParams &p, const kda_dims &d, int64_t T, int32_t tok_first,
-                                       int32_t tok_end, void *ws, cudaStream_t st, Gate gate) {
+                                       int32_t tok_end, int64_t n_snap_total, void *ws, cudaStream_t st,
+                                       Gate gate) {
     using namespace spl;
     static thread_local PrepParams PP;
     static thread_local ChainParams CPm;
@@ -680,6 +877,11 @@ inline kda_status launch_prefill_split(PrefillParams &p, const kda_dims &d, int6
     CPm.p.n_items = p.n_seq * H * 2;
     CPm.ws = static_cast<const uint8_t *>(ws);
     CPm.tok_first = tok_first;
+    if (!encode_map(&CPm.tm_o, p.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, T, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return KDA_ERR_CUDA;
+    const int64_t snap_rows = n_snap_total * H * D;
+    CPm.snap_tma = p.snapshots && n_snap_total > 0 && snap_rows < 0x7fffffffLL;
+    if (CPm.snap_tma && !encode_snap_map(&CPm.tm_snap, p.snapshots, snap_rows)) return KDA_ERR_CUDA;
     static std::atomic<unsigned long long> prep_attr{0}, chain_attr{0};
     if (!set_smem_limit_once((const void *)prefill_prep_kernel, (int)P_SMEM, prep_attr) ||
         !set_smem_limit_once((const void *)prefill_chain_kernel, (int)C_SMEM, chain_attr))

@@ -159,6 +159,21 @@ __device__ __forceinline__ void tma_load3(void *smem_dst, const CUtensorMap *m, 
         : "memory");
 }
 
+// tiled stores from this CTA's shared memory, tracked by the issuing thread's bulk groups
+// (coordinates are never negative here; x * element size is a multiple of 16 bytes)
+__device__ __forceinline__ void tma_store3(const CUtensorMap *m, const void *smem_src, int x, int y, int z) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_store2(const CUtensorMap *m, const void *smem_src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+                 : "memory");
+}
+
 // ---- untiled bulk copies (addresses 16-byte aligned, size a multiple of 16) ---------
 // global -> this CTA's shared memory, completing on `bar`
 __device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint32_t bytes, uint64_t *bar) {
