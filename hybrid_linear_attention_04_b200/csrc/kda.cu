@@ -109,6 +109,11 @@ static kda_status dispatch_simt(int D, int C, const PrefillParams &p, cudaStream
 // Forced path selection for tests: 0 = automatic, 1 = CUDA-core path only.
 static std::atomic<int> g_prefill_path{0};
 
+// Scratch of kda_prefill_noalloc: a fixed module-level device array, so that call needs
+// neither an allocation nor a caller buffer. Its size bounds the workspaces it can serve.
+constexpr size_t kNoallocScratchBytes = size_t(64) << 20;
+__device__ __align__(1024) uint8_t g_noalloc_scratch[kNoallocScratchBytes];
+
 }  // namespace kda
 
 using namespace kda;
@@ -255,6 +260,25 @@ kda_status kda_prefill(const kda_dims *dims, int32_t n_seq, const int32_t *cu,
     }
     return KDA_OK;
 }
+
+kda_status kda_prefill_noalloc(const kda_dims *dims, int32_t n_seq, const int32_t *cu,
+                               const int64_t *start_pos, const void *q, const void *k,
+                               const void *v, const float *g, const float *beta,
+                               const float *state_in, float *state_out, void *o,
+                               int32_t snap_interval, float *snapshots, kda_stream_t stream) {
+    size_t need = 0;
+    kda_status st = kda_prefill_workspace_size(dims, n_seq, cu, &need);
+    if (st != KDA_OK) return st;
+    void *scratch = nullptr;
+    if (need > 0 && need <= kNoallocScratchBytes) {
+        cudaError_t e = cudaGetSymbolAddress(&scratch, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return kda_prefill(dims, n_seq, cu, start_pos, q, k, v, g, beta, state_in, state_out, o,
+                       snap_interval, snapshots, scratch, scratch ? kNoallocScratchBytes : 0, stream);
+}
+
+size_t kda_prefill_noalloc_capacity(void) { return kNoallocScratchBytes; }
 
 kda_status kda_decode(const kda_dims *dims, int32_t n_seq, const void *q, const void *k,
                       const void *v, const float *g, const float *beta, const int32_t *slots,

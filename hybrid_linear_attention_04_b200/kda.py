@@ -43,6 +43,8 @@ _SIGNATURES = {
     "kda_prefill_workspace_size": (_I32, [_P, _I32, _P, _P]),
     "kda_prefill": (_I32, [_P, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P,
                            ctypes.c_size_t, _P]),
+    "kda_prefill_noalloc": (_I32, [_P, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P]),
+    "kda_prefill_noalloc_capacity": (ctypes.c_size_t, []),
     "kda_decode": (_I32, [_P, _I32, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P]),
     "kda_verify": (_I32, [_P, _I32, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P]),
     "kda_snapshot": (_I32, [_I32, _P, _P, _P, _I64, _P, _I64, _I32, _I32, _I32, _P]),
@@ -173,6 +175,24 @@ def kda_prefill(q, k, v, g, beta, cu_seqlens, o, state_out=None, state_in=None, 
                              _dptr(k), _dptr(v), _dptr(g), _dptr(beta), _dptr(state_in),
                              _dptr(state_out), _dptr(o), int(snap_interval), _dptr(snapshots),
                              _dptr(workspace), ws_bytes, _stream(stream)), "kda_prefill")
+
+
+def kda_prefill_noalloc(q, k, v, g, beta, cu_seqlens, o, state_out=None, state_in=None,
+                        start_pos=None, snap_interval=0, snapshots=None, chunk=64, scale=0.0,
+                        stream=None):
+    """kda_prefill on the library's fixed device scratch: no allocation (see include/kda.h)."""
+    cu = _host_array(cu_seqlens, np.int32)
+    sp = _host_array(start_pos, np.int64)
+    dims = _dims(q, v, chunk, scale)
+    _check(lib().kda_prefill_noalloc(ctypes.byref(dims), len(cu) - 1, _hptr(cu), _hptr(sp),
+                                     _dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(beta),
+                                     _dptr(state_in), _dptr(state_out), _dptr(o),
+                                     int(snap_interval), _dptr(snapshots), _stream(stream)),
+           "kda_prefill_noalloc")
+
+
+def kda_prefill_noalloc_capacity() -> int:
+    return int(lib().kda_prefill_noalloc_capacity())
 
 
 def kda_decode(q, k, v, g, beta, slots, state_pool, o, scale=0.0, stream=None):

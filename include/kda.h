@@ -143,6 +143,25 @@ kda_status kda_prefill(const kda_dims *dims, int32_t n_seq, const int32_t *cu_se
                        size_t workspace_bytes, kda_stream_t stream);
 
 /*
+ * kda_prefill_noalloc — kda_prefill without a caller workspace and without any
+ * allocation: the two-launch path uses the library's fixed device scratch of
+ * kda_prefill_noalloc_capacity() bytes (a module-level array, resident from the
+ * library's first use on a device) whenever kda_prefill_workspace_size fits in
+ * it, and the single-launch path otherwise. Arguments, layouts and errors as
+ * kda_prefill. The scratch is shared by all calls on a device: calls that may
+ * run concurrently (different streams, threads or processes sharing a context)
+ * must be ordered by the caller, e.g. issued on one stream.
+ */
+kda_status kda_prefill_noalloc(const kda_dims *dims, int32_t n_seq, const int32_t *cu_seqlens_h,
+                               const int64_t *start_pos_h, const void *q, const void *k,
+                               const void *v, const float *g, const float *beta,
+                               const float *state_in, float *state_out, void *o,
+                               int32_t snap_interval, float *snapshots, kda_stream_t stream);
+
+/* Bytes of the fixed scratch kda_prefill_noalloc uses (64 MiB). */
+size_t kda_prefill_noalloc_capacity(void);
+
+/*
  * kda_decode — one token per sequence against a pool of live states (the
  * recurrence above for a single t), updating each state in place with one
  * read and one write of it.
