@@ -92,8 +92,12 @@ def test_larger_than_scratch_runs_single_launch(cuda_device):
     assert K.kda_launch_count() - n0 == 1
     ref = oracle_prefill(x, cu, None, None, 256)
     tol = tol_for("bf16")
-    assert blockwise_err(to_np(got[0]), ref[0], (2,)) <= tol
+    # outputs normwise per head over all tokens (as for the 8192-token workload): from a
+    # zero state the first tokens' output rows are tiny, and a per-row ratio would measure
+    # bf16 rounding against a near-zero norm
+    assert blockwise_err(to_np(got[0]), ref[0], (0, 2)) <= tol
     assert blockwise_err(to_np(got[1]), ref[1], (2, 3)) <= tol
+    assert blockwise_err(got[2].cpu().numpy(), ref[2], (2, 3)) <= tol
     again = _run(K.kda_prefill, x, dev, cu, H, d, None, None, 256, workspace=None)
     for a, b in zip(got, again):
         assert torch.equal(a, b)
