@@ -185,7 +185,9 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
         tc::tmem_alloc(tmem_slot, P_TMEM);
         tc::tmem_relinquish();
     }
-    if (tid < C) bet[tid] = tid < n ? P.beta[(int64_t)(z + tid) * H + h] : 0.f;
+    // beta (a strided load): issued now, stored once the TMA loads have landed, so the two
+    // latencies overlap
+    const float bv = (tid < C && tid < n) ? P.beta[(int64_t)(z + tid) * H + h] : 0.f;
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -196,6 +198,7 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
 
     do {
         ok = tc::bar_wait(bar_ld, 0);
+        if (tid < C) bet[tid] = bv;
         if (!__syncthreads_and(ok)) { ok = false; break; }
         KDA_PMARK(1);
         // ---- b = cumsum(g) (log2 units): warp w rows 8w..8w+7, lane channels 4l..4l+3
