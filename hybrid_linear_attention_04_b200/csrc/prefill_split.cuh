@@ -63,6 +63,7 @@ constexpr uint32_t P_G = 73728;       // g fp32 [64][128]; once the operands are
 constexpr uint32_t P_LS = P_G;                    // fp32 [64][17]: L on its diagonal 16x16 blocks
 constexpr uint32_t P_LB = P_LS + 64 * 17 * 4;     // bf16 [64][72]: L, and X on the diagonal blocks
 constexpr uint32_t P_WSC = P_LB + 64 * 72 * 2;    // bf16 [8 warps][8][72]
+constexpr uint32_t P_AQK = P_G + 23552;           // A_qk staging (1 slab x 64 rows), 1024-aligned
 constexpr uint32_t P_TOT = P_G + 32768;           // fp32 [8][128] row-block totals of b
 constexpr uint32_t P_VEC = P_TOT + 4096;          // eM, eC, gC [128], beta [64]
 constexpr uint32_t P_BARS = P_VEC + (3 * 128 + 64) * 4;
@@ -90,7 +91,8 @@ __host__ __device__ constexpr uint32_t u_piece(int hf, int wg, int q4, int r) {
 }
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RANGE_LIMIT2 = 80.f * LOG2E;      // 80 nats, in log2 units
-static_assert(P_WSC + 8 * 8 * 72 * 2 <= P_TOT, "solve scratch overlaps");
+static_assert(P_WSC + 8 * 8 * 72 * 2 <= P_AQK && P_AQK + 8192 <= P_TOT && P_AQK % 1024 == 0,
+              "solve scratch overlaps");
 static_assert(STAGE % 1024 == 0 && PACKET % 16 == 0 && C_O % 1024 == 0 && C_SN % 1024 == 0, "alignment");
 static_assert(C_SMEM <= 232448, "chain shared memory");
 }  // namespace spl
@@ -311,7 +313,7 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
         tc::fence_after_sync();
         KDA_PMARK(3);
         if (warp < 2) {
-            // A_qk, masked to i <= r, straight into the packet image
+            // A_qk, masked to i <= r, into its staging image (bulk-stored after this phase)
             const int r = 32 * warp + lane;
             float a[32];
 #pragma unroll
@@ -326,7 +328,7 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
                         const int jj = 32 * half + 8 * q4 + 2 * e;
                         w[e] = bf16x2(jj <= r ? a[8 * q4 + 2 * e] : 0.f, jj + 1 <= r ? a[8 * q4 + 2 * e + 1] : 0.f);
                     }
-                    *reinterpret_cast<uint4 *>(pkt + PK_AQK + tc::sw128(r, 4 * half + q4)) =
+                    *reinterpret_cast<uint4 *>(sm + P_AQK + tc::sw128(r, 4 * half + q4)) =
                         make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
@@ -393,6 +395,11 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
         tc::fence_before_sync();
         if (!__syncthreads_and(ok)) { ok = false; break; }
         KDA_PMARK(4);
+        if (tid == 32) {
+            tc::bulk_store(pkt + PK_AQK, sm + P_AQK, 8192);
+            tc::bulk_commit();
+            stored = true;
+        }
         // ---- T = (I + L)^{-1} by block forward substitution on bf16 mma.sync (fp32
         // accumulate): T_R = X_RR (E_R - sum_{J<R} L_RJ T_J), E = identity. Warp w
         // owns columns 8w..8w+7.
@@ -449,6 +456,10 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
                 __syncwarp();
             }
         }
+        if (tid == 32 && stored) {            // A_qk, Qh, Kb read out: the staging area is reused below
+            tc::bulk_wait_read_all();
+            stored = false;
+        }
         tc::fence_async_smem();
         tc::fence_before_sync();
         __syncthreads();
@@ -500,6 +511,7 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
             tc::bulk_store(pkt + PK_QW + 16384 + 8192, sm + P_G + 8192, 8192);
             tc::bulk_store(pkt + PK_U, sm + P_G + 16384, 16384);
             tc::bulk_commit();
+            stored = true;
         }
     } while (0);
 

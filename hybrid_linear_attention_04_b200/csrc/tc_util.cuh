@@ -134,9 +134,23 @@ __device__ __forceinline__ bool bar_try_wait(uint64_t *bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// non-blocking test of the phase with the given parity
+__device__ __forceinline__ bool bar_test(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 // Bounded wait: gives up after `limit` polls (each try_wait itself blocks for
-// a hardware-chosen interval), records KDA_ERR_TIMEOUT and returns false.
+// a hardware-chosen interval), records KDA_ERR_TIMEOUT and returns false. A phase
+// that has already completed is seen by one non-blocking test.
 __device__ __forceinline__ bool bar_wait(uint64_t *bar, uint32_t parity, uint32_t limit = 1u << 22) {
+    if (bar_test(bar, parity)) return true;
     for (uint32_t i = 0; i < limit; ++i) {
         if (bar_try_wait(bar, parity)) return true;
         if (i > 64) __nanosleep(64);
