@@ -12,7 +12,7 @@
 //
 //   prep   one CTA per (chunk, head), all chunks of all sequences at once:
 //          cumsum, scaled operands, A = [Qh; Ka] Kb^T (tcgen05), T by block forward
-//          substitution (mma.sync), [W' | U] = T [beta Ka | beta V] (tcgen05). Writes
+//          substitution (mma.sync), [W' | U] = (T Diag(beta)) [Ka | V] (tcgen05). Writes
 //          one packet per (chunk, head) to the workspace, laid out as the shared
 //          memory images the chain kernel feeds to its MMAs.
 //   chain  one CTA per (sequence, head, 64-column d_v slice): per chunk, one bulk
@@ -54,8 +54,8 @@ constexpr uint32_t PK_VEC = 57344;    // eM, eC, gC: fp32 [3][128] (1536 B, slot
 constexpr uint32_t PK_U = 59392;      // U: 2 slabs (d_v 0-63, 64-127) x 64 token rows
 constexpr uint32_t PACKET = PK_U + 16384;   // 75776 bytes
 // ---- prep kernel shared memory
-constexpr uint32_t P_QK = 0;          // 2 slabs x 128 rows: q -> Qh (rows 0-63), k -> Ka -> beta Ka
-constexpr uint32_t P_V = 32768;       // v: 2 slabs x 64 rows -> beta V in place
+constexpr uint32_t P_QK = 0;          // 2 slabs x 128 rows: q -> Qh (rows 0-63), k -> Ka (rows 64-127)
+constexpr uint32_t P_V = 32768;       // v: 2 slabs x 64 rows
 constexpr uint32_t P_KB = 49152;      // Kb: 2 slabs x 64 rows
 constexpr uint32_t P_TI = 65536;      // T (bf16): 1 slab x 64 rows
 constexpr uint32_t P_G = 73728;       // g fp32 [64][128]; once the operands are built, the solve
@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
             }
         }
         KDA_PMARK(10);
-        // ---- Qh = q 2^(b-m), Ka = k 2^(b-m) in place; Kb = k 2^(m-b); beta V in place
+        // ---- Qh = q 2^(b-m), Ka = k 2^(b-m) in place; Kb = k 2^(m-b)
         {
             const int pkb = lane >> 4, pchk = (lane & 15) >> 1, phf = (lane & 1) * 8;
 #pragma unroll
@@ -257,13 +257,10 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
                 const uint32_t so = tc::sw128(r, pchk) + phf;
                 uint8_t *qp = sm + P_QK + pkb * 16384 + so;
                 uint8_t *kp = sm + P_QK + pkb * 16384 + 8192 + so;
-                uint8_t *vp = sm + P_V + pkb * 8192 + so;
                 const uint2 qv = *reinterpret_cast<const uint2 *>(qp);
                 const uint2 kv = *reinterpret_cast<const uint2 *>(kp);
-                const uint2 vv = *reinterpret_cast<const uint2 *>(vp);
                 const float2 q01 = bf16x2_unpack(qv.x), q23 = bf16x2_unpack(qv.y);
                 const float2 k01 = bf16x2_unpack(kv.x), k23 = bf16x2_unpack(kv.y);
-                const float2 v01 = bf16x2_unpack(vv.x), v23 = bf16x2_unpack(vv.y);
                 float e1[4], e2[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -272,7 +269,6 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
                     e2[e] = tc::ex2(-d);
                 }
                 const bool live = r < n;
-                const float br = bet[r];
                 *reinterpret_cast<uint2 *>(qp) =
                     live ? make_uint2(bf16x2(q01.x * e1[0], q01.y * e1[1]), bf16x2(q23.x * e1[2], q23.y * e1[3]))
                          : make_uint2(0u, 0u);
@@ -282,8 +278,6 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
                 *reinterpret_cast<uint2 *>(sm + P_KB + pkb * 8192 + so) =
                     live ? make_uint2(bf16x2(k01.x * e2[0], k01.y * e2[1]), bf16x2(k23.x * e2[2], k23.y * e2[3]))
                          : make_uint2(0u, 0u);
-                *reinterpret_cast<uint2 *>(vp) =
-                    make_uint2(bf16x2(br * v01.x, br * v01.y), bf16x2(br * v23.x, br * v23.y));
             }
         }
         tc::fence_async_smem();
@@ -375,21 +369,6 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
             __syncwarp();
 #pragma unroll
             for (int rr = 0; rr < 16; ++rr) Lb[(base + rr) * 72 + base + cc] = __float2bfloat16_rn(x[rr]);
-        } else {
-            // beta Ka in place (rows 64-127 of both slabs; A has been read)
-            const int t = tid - 128;
-#pragma unroll
-            for (int it = 0; it < 8; ++it) {
-                const int idx = t + 128 * it;
-                const int slab = idx >> 9, row = (idx >> 3) & 63, chunk = idx & 7;
-                uint4 *p4 = reinterpret_cast<uint4 *>(sm + P_QK + slab * 16384 + (64 + row) * 128 + chunk * 16);
-                const uint4 u = *p4;
-                const float br = bet[row];
-                const float2 x0 = bf16x2_unpack(u.x), x1 = bf16x2_unpack(u.y), x2 = bf16x2_unpack(u.z),
-                             x3 = bf16x2_unpack(u.w);
-                *p4 = make_uint4(bf16x2(br * x0.x, br * x0.y), bf16x2(br * x1.x, br * x1.y),
-                                 bf16x2(br * x2.x, br * x2.y), bf16x2(br * x3.x, br * x3.y));
-            }
         }
         tc::fence_async_smem();
         tc::fence_before_sync();
@@ -450,9 +429,11 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
                 ws[(2 * t + 1) * 72 + r0] = __float2bfloat16_rn(w[1]);
                 ws[(2 * t) * 72 + r1] = __float2bfloat16_rn(w[2]);
                 ws[(2 * t + 1) * 72 + r1] = __float2bfloat16_rn(w[3]);
-                // T (bf16, K-major A operand): columns c0 + 2t, c0 + 2t + 1 are in 16-byte chunk `warp`
-                *reinterpret_cast<uint32_t *>(sm + P_TI + tc::sw128(r0, warp) + 4 * t) = bf16x2(w[0], w[1]);
-                *reinterpret_cast<uint32_t *>(sm + P_TI + tc::sw128(r1, warp) + 4 * t) = bf16x2(w[2], w[3]);
+                // T Diag(beta) (bf16, K-major A operand of the next MMAs: W' = T Diag(beta) Ka,
+                // U = T Diag(beta) V); columns c0 + 2t, c0 + 2t + 1 are in 16-byte chunk `warp`
+                const float b0 = bet[c0 + 2 * t], b1 = bet[c0 + 2 * t + 1];
+                *reinterpret_cast<uint32_t *>(sm + P_TI + tc::sw128(r0, warp) + 4 * t) = bf16x2(w[0] * b0, w[1] * b1);
+                *reinterpret_cast<uint32_t *>(sm + P_TI + tc::sw128(r1, warp) + 4 * t) = bf16x2(w[2] * b0, w[3] * b1);
                 __syncwarp();
             }
         }
@@ -464,7 +445,7 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
         tc::fence_before_sync();
         __syncthreads();
         KDA_PMARK(5);
-        // ---- [W' | U] = T [beta Ka | beta V]  (M=64: row r in TMEM lane (r % 16) + 32 (r / 16))
+        // ---- [W' | U] = (T Diag(beta)) [Ka | V]  (M=64: row r in TMEM lane (r % 16) + 32 (r / 16))
         if (tid == 0) {
             tc::fence_after_sync();
             constexpr uint32_t id_w = tc::idesc_bf16(64, 128, false, true);
