@@ -16,11 +16,13 @@
 //          one packet per (chunk, head) to the workspace, laid out as the shared
 //          memory images the chain kernel feeds to its MMAs.
 //   chain  one CTA per (sequence, head, 64-column d_v slice): per chunk, one bulk
-//          copy of the packet (three chunks in flight), then
+//          copy of the packet head (three chunks in flight; U is read into registers
+//          a chunk ahead), then
 //            round 1  [Qh; W'] Sm          -> TMEM (M=128: rows 0-63 O, 64-127 W'Sm)
 //            W = U - W'Sm (bf16)
-//            round 2  O += A_qk W,  D = Kb^T W
-//          and the fp32 state update in registers.
+//            round 2  D = Kb^T W, then O += A_qk W (separate commits)
+//          the fp32 state update in registers and Sm of the next chunk. O and snapshots
+//          leave during the following chunks through staging tiles and tiled TMA stores.
 #pragma once
 #include <cudaTypedefs.h>
 
