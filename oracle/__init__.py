@@ -13,6 +13,9 @@ Contents
                   snapshot rule, and the chunked (WY/UT) form derived from it.
   exact.py      : the definition as an explicit product of rational matrices,
                   in exact arithmetic (fractions.Fraction), for T <= 8.
+  frontend.py   : the q/k front-end (short causal depthwise convolution with a
+                  carried conv state, Swish, L2 normalisation), for the next row
+                  of the path; pinned in tests/test_frontend_oracle.py.
 
 Source of the definition: Kimi K3 technical FAQ (runpod.io), "What is KDA, and
 why does a serving engineer care?" (delta-rule recurrence, per-channel forget
