@@ -16,6 +16,9 @@ Contents
   frontend.py   : the q/k front-end (short causal depthwise convolution with a
                   carried conv state, Swish, L2 normalisation), for the next row
                   of the path; pinned in tests/test_frontend_oracle.py.
+  segments.py   : affine state maps of token segments and their composition (the
+                  algebra of splitting one sequence across workers); pinned in
+                  tests/test_segment_maps.py.
 
 Source of the definition: Kimi K3 technical FAQ (runpod.io), "What is KDA, and
 why does a serving engineer care?" (delta-rule recurrence, per-channel forget
