@@ -180,3 +180,16 @@ def test_decode_verify_snapshot_validation():
 def test_no_launch_issued_by_host_tests():
     # the validation failures above must not have launched anything
     assert K.kda_launch_count() == 0
+
+
+def test_binding_workspace_argument():
+    """The binding's workspace argument: a wrong kind raises before any CUDA call, and
+    its size query matches the C function for tensors of the prefill's shape."""
+    import torch
+    q = torch.zeros((200, 4, 128), dtype=torch.bfloat16)
+    cu = [0, 70, 200]
+    with pytest.raises(K.KDAError) as e:
+        K.kda_prefill(q, q, q, q.float(), q[..., 0].float(), cu, q, workspace="bogus")
+    assert e.value.status == 1
+    assert K.kda_prefill_workspace_size(q, q, cu) == ((200 >> 6) + 2) * 4 * 75776
+    assert K.kda_prefill_workspace_size(q.float(), q.float(), cu) == 0     # fp32 I/O: CUDA-core path
