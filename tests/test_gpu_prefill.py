@@ -84,6 +84,21 @@ def test_ragged_with_state_and_snapshots(cuda_device, path, d, chunk, io):
     check(o, sout, snaps, offs, oracle_prefill(x, cu, start, s0, snap), io)
 
 
+def test_snapshot_after_every_chunk(cuda_device, path):
+    """snap_interval == chunk: a snapshot is due at every chunk boundary, the case in
+    which the two-launch chain writes part of each snapshot directly rather than
+    through its staging tile."""
+    lens = [200, 64, 130, 1]
+    H, d, C = 2, 128, 64
+    x, dev, cu = packed_inputs(91, lens, H, d, "bf16", cuda_device)
+    start = [0, 64, 128, 192]
+    s0 = synth.states(92, len(lens), H, d, d, std=0.1)
+    o, sout, snaps, offs = run_prefill(dev, cu, H, d, C, "bf16", start, s0.to(cuda_device), C,
+                                       cuda_device)
+    assert int(offs[-1]) == 3 + 1 + 2 + 0
+    check(o, sout, snaps, offs, oracle_prefill(x, cu, start, s0, C), "bf16")
+
+
 def test_zero_length_sequence_passes_state_through(cuda_device, path):
     H, d = 2, 128
     x, dev, cu = packed_inputs(9, [0, 70, 0], H, d, "bf16", cuda_device)
