@@ -193,3 +193,26 @@ def test_binding_workspace_argument():
     assert e.value.status == 1
     assert K.kda_prefill_workspace_size(q, q, cu) == ((200 >> 6) + 2) * 4 * 75776
     assert K.kda_prefill_workspace_size(q.float(), q.float(), cu) == 0     # fp32 I/O: CUDA-core path
+
+
+def test_workspace_rows_are_disjoint_and_within_the_reported_size():
+    """Both prefill kernels place chunk c of sequence i (of a launch group whose first
+    token is tok_first) at packet row ((tok0_i - tok_first) >> 6) + i + c. For random
+    ragged batches those rows never collide and stay below the rows that
+    kda_prefill_workspace_size reports for the group."""
+    rng = np.random.default_rng(5)
+    for trial in range(200):
+        n = int(rng.integers(1, 40))
+        lens = rng.integers(0, 400, size=n)
+        lens[rng.random(n) < 0.2] = 0
+        cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+        H = int(rng.integers(1, 5))
+        rows = set()
+        for i in range(n):
+            first = ((int(cu[i]) - 0) >> 6) + i
+            for c in range((int(lens[i]) + 63) // 64):
+                assert first + c not in rows
+                rows.add(first + c)
+        size = _workspace_size(_dims(H=H), cu)
+        assert size % (H * 75776) == 0
+        assert all(r < size // (H * 75776) for r in rows)
