@@ -7,7 +7,12 @@ A step is one pass of the whole hot path over one batch of synthetic input:
   3. kda_verify   - 1..8 draft tokens per sequence (seeded uniform), writing the
                     state after every token;
   4. kda_snapshot - commit the state of each sequence's last accepted token
-                    (seeded acceptance) into its live slot.
+                    (seeded acceptance) into its live slot;
+  5. kda_verify_commit - the same speculative step with the commit fused in: the
+                    verify batch above, accepted as in 4, is replayed into the live
+                    state, then the next 1..8 draft tokens run with outputs only.
+The tiny fp32 workload, the 32-sequence ragged batch and the 1M-token segmented
+prefill are timed in the same run, each on its own, under "components".
 Inputs are seeded (synth.py) and resident in HBM before timing; every input set
 is larger than the 126 MB L2 (prefill 0.94 GB, decode 2.1 GB, verify 12 GB), so
 no L2 flush is needed between steps.
@@ -174,6 +179,13 @@ def commit_bytes(n):
     return n * H * D * D * 4 * 2
 
 
+def verify_commit_bytes(n_seq, n_written, n_replayed, n_tok):
+    """State read once per sequence and written once where a commit happened; replayed
+    tokens' k, v (bf16), g, beta; drafted tokens' q, k, v, o (bf16), g, beta."""
+    return (n_seq + n_written) * H * D * D * 4 + n_replayed * H * (2 * D * 2 + D * 4 + 4) \
+        + n_tok * H * (4 * D * 2 + D * 4 + 4)
+
+
 class Workload:
     """The serving-step workload, resident on one device."""
 
@@ -219,6 +231,17 @@ class Workload:
         self.c_src = torch.tensor(src, dtype=torch.int64, device=dev)
         self.c_dst = torch.tensor(dst, dtype=torch.int64, device=dev)
         self.n_commit = len(src)
+        # verify with the previous step's commit fused in: the previous batch is the
+        # verify batch above with the same seeded acceptance; this step's drafts are the
+        # next 1..8 tokens per sequence of the same streams
+        self.vc_acc = [min(acc[s], lens[s]) for s in range(n_seq)]
+        self.vc_acc_d = torch.tensor(self.vc_acc, dtype=torch.int32, device=dev)
+        lens2 = synth.draft_lengths(1002, n_seq, 1, 8, start=n_seq)
+        self.vc_cu = np.concatenate([[0], np.cumsum(lens2)]).astype(np.int32)
+        self.vc_tok = int(self.vc_cu[-1])
+        z2 = synth.token_inputs(1002, self.vc_tok, H, D, D, io="bf16", t0=n_seq + self.n_tok)
+        self.vc = {k: v.to(dev) for k, v in z2.items()}
+        self.vc_o = torch.empty((self.vc_tok, H, D), dtype=torch.bfloat16, device=dev)
 
     def prefill(self):
         K, p = self.K, self.p
@@ -237,6 +260,11 @@ class Workload:
 
     def commit(self):
         self.K.kda_snapshot(self.c_src, self.c_dst, self.ts, self.pool)
+
+    def verify_commit(self):
+        c = self.vc
+        self.K.kda_verify_commit(self.v, self.vc_acc_d, self.cu_draft, c["q"], c["k"], c["v"],
+                                 c["g"], c["beta"], self.vc_cu, self.slots, self.pool, self.vc_o)
 
 
 def dist_setup(n_gpus):
@@ -284,8 +312,8 @@ def run_ours(args):
     from hybrid_linear_attention_04_b200 import kda as K
     wl = Workload(dev, args.prefill_path, args.prefill_tokens, args.decode_seqs)
     stream = torch.cuda.current_stream(dev)
-    comps = ["prefill", "decode", "verify", "commit"]
-    fns = [wl.prefill, wl.decode, wl.verify, wl.commit]
+    comps = ["prefill", "decode", "verify", "commit", "verify_commit"]
+    fns = [wl.prefill, wl.decode, wl.verify, wl.commit, wl.verify_commit]
 
     def step(ev=None):
         for i, f in enumerate(fns):
@@ -348,9 +376,23 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(dist, [e0.elapsed_time(e1) / args.steps], dev)[0]
 
+    # the other workloads, each timed on its own (CUDA events over `steps` calls)
+    peaks = load_peaks()
+    extra = {}
+    if not args.serving_only:
+        del wl.p_ws, wl.ts
+        torch.cuda.empty_cache()
+        extra["tiny"] = bench_tiny(K, dev, args.steps, args.warmup)
+        extra["ragged"] = bench_ragged(K, dev, args.steps, args.warmup, peaks)
+        torch.cuda.empty_cache()
+        extra["long"] = bench_long(K, dev, max(3, args.steps // 4), args.warmup, peaks)
+        torch.cuda.empty_cache()
+        for name in extra:
+            key = "ms"
+            extra[name][key] = max_over_ranks(dist, [extra[name][key]], dev)[0]
+
     result = None
     if rank == 0:
-        peaks = load_peaks()
         hbm = peaks["hbm_gbs"]
         comp = {}
         units = {
@@ -358,6 +400,9 @@ def run_ours(args):
             "decode": (wl.n_seq * H, "state-steps/s", decode_bytes(wl.n_seq)),
             "verify": (wl.n_tok * H, "state-steps/s", verify_bytes(wl.n_seq, wl.n_tok)),
             "commit": (wl.n_commit, "states/s", commit_bytes(wl.n_commit)),
+            "verify_commit": ((sum(wl.vc_acc) + wl.vc_tok) * H, "state-steps/s",
+                              verify_commit_bytes(wl.n_seq, sum(1 for a in wl.vc_acc if a > 0),
+                                                  sum(wl.vc_acc), wl.vc_tok)),
         }
         for name, ms in zip(comps, comp_ms):
             n_units, unit, byts = units[name]
@@ -369,14 +414,19 @@ def run_ours(args):
         comp["prefill"]["algorithmic_flops"] = pf
         comp["prefill"]["tc_frac"] = round(pf / (comp_ms[0] * 1e-3) / (peaks["bf16_tflops"] * 1e12), 4)
         comp["prefill"]["path"] = args.prefill_path
+        for name, e in extra.items():
+            if "tokens" in e:
+                e["value"] = world * e["tokens"] / (e["ms"] * 1e-3)
+            comp[name] = e
         dom = max(comps, key=lambda c: comp[c]["ms"])
         pk = ["prefill_prep_kernel", "prefill_chain_kernel"] if args.prefill_path == "split" \
             else ["prefill_tc_kernel"]
         knames = {"prefill": pk, "decode": ["decode_kernel"], "verify": ["verify_kernel"],
-                  "commit": ["snapshot_kernel"]}[dom]
+                  "commit": ["snapshot_kernel"], "verify_commit": ["verify_commit_kernel"]}[dom]
         kname = "+".join(knames)
         tr_units = {"prefill": (wl.T * H, wl.T * H), "decode": (wl.n_seq * H, wl.n_seq * H),
-                    "verify": (wl.n_seq * H, wl.n_tok * H), "commit": (wl.n_commit, wl.n_commit)}[dom]
+                    "verify": (wl.n_seq * H, wl.n_tok * H), "commit": (wl.n_commit, wl.n_commit),
+                    "verify_commit": (wl.n_seq * H, wl.n_seq * H)}[dom]
         trs = [ncu_traffic(k, *tr_units) for k in knames]
         tr = None if any(t is None for t in trs) else sum(trs)
         roof = {"bound": "hbm", "kernel": kname, "achieved": comp[dom]["achieved_gbs"],
@@ -417,6 +467,132 @@ def run_ours(args):
         dist.barrier()
         dist.destroy_process_group()
     return result
+
+
+def prefill_bytes_general(T, n_seq, n_snap, n_state_in, io_bytes=2, d=D, heads=H):
+    """Algorithmic bytes of one prefill call: q, k, v, o in the I/O type, g fp32, beta,
+    snapshots, final states and the initial states read."""
+    per_tok = heads * (4 * d * io_bytes + d * 4 + 4)
+    return T * per_tok + (n_snap + n_seq + n_state_in) * heads * d * d * 4
+
+
+def bench_tiny(K, dev, steps, warmup):
+    """The tiny all-fp32 workload: B=1, H=2, T=64, d=32, chunk 16 (CUDA-core path)."""
+    c = synth.WORKLOADS["tiny_fp32"]
+    x = synth.token_inputs(c["seed"], c["T"], c["H"], c["d"], c["d"], io="fp32")
+    xd = {k: v.to(dev) for k, v in x.items()}
+    o = torch.empty_like(xd["v"])
+    so = torch.empty((1, c["H"], c["d"], c["d"]), device=dev)
+    cu = np.array([0, c["T"]], dtype=np.int32)
+    n0 = K.kda_launch_count()
+    K.kda_prefill(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], cu, o, state_out=so,
+                  chunk=c["chunk"], workspace=None)
+    launches = K.kda_launch_count() - n0
+    ms = time_calls(lambda: K.kda_prefill(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], cu, o,
+                                          state_out=so, chunk=c["chunk"], workspace=None),
+                    steps, warmup, dev)
+    byts = prefill_bytes_general(c["T"], 1, 0, 0, io_bytes=4, d=c["d"], heads=c["H"])
+    return {"ms": round(ms, 5), "value": round(ms * 1e3, 2), "unit": "us/call",
+            "tok_per_s": c["T"] / (ms * 1e-3), "algorithmic_bytes": byts,
+            "bound": "launch latency", "launches_per_call": launches,
+            "workload": "B=1, H=2, T=64, d=32, chunk 16, fp32 throughout, zero initial state"}
+
+
+def bench_ragged(K, dev, steps, warmup, peaks):
+    """The ragged packed prefill with prefix reuse: 32 sequences, lognormal lengths,
+    half of them resuming from the GPU's own snapshot of a shared 16384-token prefix."""
+    c = synth.WORKLOADS["ragged_prefix_32"]
+    plan = synth.ragged_plan(c["seed"], c["n_seq"], c["mu"], c["sigma"], c["lo"], c["hi"],
+                             c["prefix"], c["n_resume"], c["snap"])
+    lens, start = plan["lens"], plan["start_pos"]
+    n_seq, snap, P = len(lens), c["snap"], c["prefix"]
+    # the shared prefix, prefilled once (untimed), gives the resumers' initial states
+    xp = synth.token_inputs_device(c["seed"] + 1, P, H, D, D, io="bf16", device=dev)
+    cup = np.array([0, P], dtype=np.int32)
+    po = torch.empty((P, H, D), dtype=torch.bfloat16, device=dev)
+    psn = torch.empty((P // snap, H, D, D), device=dev)
+    K.kda_prefill(xp["q"], xp["k"], xp["v"], xp["g"], xp["beta"], cup, po, snap_interval=snap,
+                  snapshots=psn, chunk=C)
+    s0 = torch.zeros((n_seq, H, D, D), device=dev)
+    res = plan["resumers"]
+    K.kda_snapshot(torch.tensor([plan["resume_block"][s] - 1 for s in res], dtype=torch.int64,
+                                device=dev),
+                   torch.tensor(res, dtype=torch.int64, device=dev), psn, s0)
+    del xp, po, psn
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(cu[-1])
+    xd = synth.token_inputs_device(c["seed"], T, H, D, D, io="bf16", device=dev)
+    o = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+    so = torch.empty_like(s0)
+    offs, _ = K.kda_snapshot_plan(cu, start, snap)
+    sn = torch.empty((int(offs[-1]), H, D, D), device=dev)
+    ws = torch.empty(K.kda_prefill_workspace_size(xd["q"], xd["v"], cu, C), dtype=torch.uint8,
+                     device=dev)
+
+    def call():
+        K.kda_prefill(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], cu, o, state_out=so,
+                      state_in=s0, start_pos=start, snap_interval=snap, snapshots=sn, chunk=C,
+                      workspace=ws)
+    n0 = K.kda_launch_count()
+    call()
+    launches = K.kda_launch_count() - n0
+    ms = time_calls(call, steps, warmup, dev)
+    byts = prefill_bytes_general(T, n_seq, int(offs[-1]), n_seq)
+    flops = prefill_flops(T)
+    st = K.kda_check_device_status()
+    if st != 0:
+        raise RuntimeError(f"ragged workload: device status {K.kda_status_string(st)}")
+    return {"ms": round(ms, 4), "value": T / (ms * 1e-3), "unit": "tok/s", "tokens": T,
+            "algorithmic_bytes": byts, "achieved_gbs": round(byts / (ms * 1e-3) / 1e9, 1),
+            "hbm_frac": round(byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+            "algorithmic_flops": flops,
+            "tc_frac": round(flops / (ms * 1e-3) / (peaks["bf16_tflops"] * 1e12), 4),
+            "launches_per_call": launches, "path": "split",
+            "workload": f"{n_seq} sequences ({T} tokens) x 64 heads, lognormal(ln 4096, 1) "
+                        f"lengths clipped to [512, 65536], {len(res)} resuming from snapshots "
+                        f"of a shared {P}-token prefix, snapshots /{snap}"}
+
+
+def bench_long(K, dev, steps, warmup, peaks):
+    """The long-context prefill: 1,048,576 tokens as 16 calls of 65,536 with the state
+    handed across calls and snapshots every 4096 tokens; one pass = 16 calls."""
+    c = synth.WORKLOADS["long_1m"]
+    seg, n_seg, snap = c["segment"], c["T"] // c["segment"], c["snap"]
+    segs = [synth.token_inputs_device(c["seed"], seg, H, D, D, io="bf16", t0=i * seg, device=dev)
+            for i in range(n_seg)]
+    o = torch.empty((seg, H, D), dtype=torch.bfloat16, device=dev)
+    st = [torch.empty((1, H, D, D), device=dev) for _ in range(2)]
+    sn = torch.empty((c["T"] // snap, H, D, D), device=dev)
+    cu = np.array([0, seg], dtype=np.int32)
+    ws = torch.empty(K.kda_prefill_workspace_size(segs[0]["q"], segs[0]["v"], cu, C),
+                     dtype=torch.uint8, device=dev)
+    per = seg // snap
+
+    def one_pass():
+        for i in range(n_seg):
+            xd = segs[i]
+            K.kda_prefill(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], cu, o,
+                          state_out=st[(i + 1) % 2], state_in=st[i % 2] if i else None,
+                          start_pos=[i * seg], snap_interval=snap, snapshots=sn[i * per:(i + 1) * per],
+                          chunk=C, workspace=ws)
+    n0 = K.kda_launch_count()
+    one_pass()
+    launches = K.kda_launch_count() - n0
+    ms = time_calls(one_pass, steps, warmup, dev)
+    T = c["T"]
+    byts = prefill_bytes_general(T, n_seg, T // snap, n_seg - 1)
+    flops = prefill_flops(T)
+    stt = K.kda_check_device_status()
+    if stt != 0:
+        raise RuntimeError(f"long workload: device status {K.kda_status_string(stt)}")
+    return {"ms": round(ms, 3), "value": T / (ms * 1e-3), "unit": "tok/s", "tokens": T,
+            "algorithmic_bytes": byts, "achieved_gbs": round(byts / (ms * 1e-3) / 1e9, 1),
+            "hbm_frac": round(byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+            "algorithmic_flops": flops,
+            "tc_frac": round(flops / (ms * 1e-3) / (peaks["bf16_tflops"] * 1e12), 4),
+            "launches_per_pass": launches, "path": "split",
+            "workload": "1,048,576 tokens x 64 heads as 16 calls of 65,536 (state handed "
+                        "across calls), snapshots /4096; one pass = 16 calls"}
 
 
 def time_calls(fn, steps, warmup, dev):
@@ -567,6 +743,8 @@ def main():
                     help="prefill length of the serving step (smaller only for profiler captures)")
     ap.add_argument("--decode-seqs", type=int, default=N_SEQ,
                     help="decode/verify sequences of the serving step (smaller only for profiler captures)")
+    ap.add_argument("--serving-only", action="store_true",
+                    help="time the serving step only (skip the tiny, ragged and 1M-token workloads)")
     ap.add_argument("--prefill-path", choices=["split", "fused"], default="split",
                     help="tensor-core prefill in two launches through a workspace (split) or in "
                          "one launch without one (fused)")

@@ -18,21 +18,43 @@ __device__ __forceinline__ void record_status(unsigned int code) {
     atomicCAS(&g_status, 0u, code);
 }
 
+// Text behind the most recent KDA_ERR_CUDA (static storage), read by kda_last_cuda_error.
+inline std::atomic<const char *> &last_error_text() {
+    static std::atomic<const char *> text{"no error"};
+    return text;
+}
+// Record a failed CUDA call (or another failure reported as KDA_ERR_CUDA) and return it.
+inline kda_status fail_cuda(cudaError_t e) {
+    last_error_text().store(cudaGetErrorString(e));
+    return KDA_ERR_CUDA;
+}
+inline kda_status fail_text(const char *msg) {
+    last_error_text().store(msg);
+    return KDA_ERR_CUDA;
+}
+// Status of the launch just issued.
+inline kda_status launch_result() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? KDA_OK : fail_cuda(e);
+}
+
 // Raise a kernel's dynamic shared-memory limit (and prefer the largest shared
 // memory carveout) on the current device once.
 // The attribute is per device, so a process that drives several GPUs keeps one
 // bit per device ordinal in `done` (ordinals >= 64 set it on every call).
-inline bool set_smem_limit_once(const void *fn, int bytes, std::atomic<unsigned long long> &done) {
+inline kda_status set_smem_limit_once(const void *fn, int bytes, std::atomic<unsigned long long> &done) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail_cuda(e);
     const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
-    if (bit && (done.load(std::memory_order_acquire) & bit)) return true;
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
-        cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
-        return false;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return KDA_OK;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return fail_cuda(e);
     done.fetch_or(bit, std::memory_order_release);
-    return true;
+    return KDA_OK;
 }
 
 // Element type traits for the q/k/v/o arrays.

@@ -55,20 +55,27 @@ template <int D> struct __align__(16) TokVec {
 };
 static_assert(sizeof(TokVec<128>) % 16 == 0 && sizeof(TokVec<32>) % 16 == 0, "TokVec padding");
 
+// Stage the vectors of token row `row` (= token * H + head); q may be null (a token
+// whose output is not needed). D threads (or fewer, looping) fill the vectors.
 template <int D, typename TIO>
-__device__ __forceinline__ void load_token(TokVec<D> &tv, const DecodeParams &p, int64_t row) {
-    // row = token * H + head; D threads (or fewer, looping) fill the vectors.
-    const TIO *q = static_cast<const TIO *>(p.q) + row * D;
-    const TIO *k = static_cast<const TIO *>(p.k) + row * D;
-    const TIO *v = static_cast<const TIO *>(p.v) + row * D;
-    const float *g = p.g + row * D;
+__device__ __forceinline__ void load_vectors(TokVec<D> &tv, const void *q_, const void *k_, const void *v_,
+                                             const float *g_, const float *beta, int64_t row) {
+    const TIO *q = q_ ? static_cast<const TIO *>(q_) + row * D : nullptr;
+    const TIO *k = static_cast<const TIO *>(k_) + row * D;
+    const TIO *v = static_cast<const TIO *>(v_) + row * D;
+    const float *g = g_ + row * D;
     for (int i = threadIdx.x; i < D; i += blockDim.x) {
         tv.k[i] = IO<TIO>::ld(k + i);
-        tv.q[i] = IO<TIO>::ld(q + i);
+        tv.q[i] = q ? IO<TIO>::ld(q + i) : 0.f;
         tv.v[i] = IO<TIO>::ld(v + i);
         tv.a[i] = expf(g[i]);
     }
-    if (threadIdx.x == 0) tv.beta = p.beta[row];
+    if (threadIdx.x == 0) tv.beta = beta[row];
+}
+
+template <int D, typename TIO>
+__device__ __forceinline__ void load_token(TokVec<D> &tv, const DecodeParams &p, int64_t row) {
+    load_vectors<D, TIO>(tv, p.q, p.k, p.v, p.g, p.beta, row);
 }
 
 // k . q for a staged token, by one warp, fixed reduction order.
@@ -84,8 +91,10 @@ __device__ __forceinline__ void token_kq(TokVec<D> &tv) {
 }
 
 // One recurrence step on the register-resident state. red: [NW][2][D] scratch
-// in shared memory; the caller separates reuses of `red` by a barrier.
-template <int D>
+// in shared memory; the caller separates reuses of `red` by a barrier. With
+// OUT = false the output read (y and o) is skipped; the state arithmetic is the
+// same instruction for instruction, so both forms give bit-identical states.
+template <int D, bool OUT = true>
 __device__ __forceinline__ float4 kda_step(float4 (&st)[DecodeShape<D>::R], const TokVec<D> &tv,
                                            float *red, float scale) {
     using Sh = DecodeShape<D>;
@@ -95,14 +104,17 @@ __device__ __forceinline__ float4 kda_step(float4 (&st)[DecodeShape<D>::R], cons
 #pragma unroll
     for (int m = 0; m < Sh::R; ++m) {
         const int r = rs + Sh::RS * m;
-        const float a = tv.a[r], kr = tv.k[r], qr = tv.q[r];
+        const float a = tv.a[r], kr = tv.k[r];
         float4 s = st[m];
         s.x *= a; s.y *= a; s.z *= a; s.w *= a;
         st[m] = s;
         x.x = fmaf(kr, s.x, x.x); x.y = fmaf(kr, s.y, x.y);
         x.z = fmaf(kr, s.z, x.z); x.w = fmaf(kr, s.w, x.w);
-        y.x = fmaf(qr, s.x, y.x); y.y = fmaf(qr, s.y, y.y);
-        y.z = fmaf(qr, s.z, y.z); y.w = fmaf(qr, s.w, y.w);
+        if (OUT) {
+            const float qr = tv.q[r];
+            y.x = fmaf(qr, s.x, y.x); y.y = fmaf(qr, s.y, y.y);
+            y.z = fmaf(qr, s.z, y.z); y.w = fmaf(qr, s.w, y.w);
+        }
     }
 #pragma unroll
     for (int off = Sh::CG; off < 32; off <<= 1) {
@@ -110,23 +122,27 @@ __device__ __forceinline__ float4 kda_step(float4 (&st)[DecodeShape<D>::R], cons
         x.y += __shfl_xor_sync(0xffffffffu, x.y, off);
         x.z += __shfl_xor_sync(0xffffffffu, x.z, off);
         x.w += __shfl_xor_sync(0xffffffffu, x.w, off);
-        y.x += __shfl_xor_sync(0xffffffffu, y.x, off);
-        y.y += __shfl_xor_sync(0xffffffffu, y.y, off);
-        y.z += __shfl_xor_sync(0xffffffffu, y.z, off);
-        y.w += __shfl_xor_sync(0xffffffffu, y.w, off);
+        if (OUT) {
+            y.x += __shfl_xor_sync(0xffffffffu, y.x, off);
+            y.y += __shfl_xor_sync(0xffffffffu, y.y, off);
+            y.z += __shfl_xor_sync(0xffffffffu, y.z, off);
+            y.w += __shfl_xor_sync(0xffffffffu, y.w, off);
+        }
     }
     if (lane < Sh::CG) {
         *reinterpret_cast<float4 *>(red + (warp * 2 + 0) * D + cg * 4) = x;
-        *reinterpret_cast<float4 *>(red + (warp * 2 + 1) * D + cg * 4) = y;
+        if (OUT) *reinterpret_cast<float4 *>(red + (warp * 2 + 1) * D + cg * 4) = y;
     }
     __syncthreads();
     float4 X = make_float4(0.f, 0.f, 0.f, 0.f), Y = X;
 #pragma unroll
     for (int w = 0; w < Sh::NW; ++w) {
         float4 a = *reinterpret_cast<const float4 *>(red + (w * 2 + 0) * D + cg * 4);
-        float4 b = *reinterpret_cast<const float4 *>(red + (w * 2 + 1) * D + cg * 4);
         X.x += a.x; X.y += a.y; X.z += a.z; X.w += a.w;
-        Y.x += b.x; Y.y += b.y; Y.z += b.z; Y.w += b.w;
+        if (OUT) {
+            float4 b = *reinterpret_cast<const float4 *>(red + (w * 2 + 1) * D + cg * 4);
+            Y.x += b.x; Y.y += b.y; Y.z += b.z; Y.w += b.w;
+        }
     }
     const float4 vv = *reinterpret_cast<const float4 *>(tv.v + cg * 4);
     float4 wv;
@@ -140,9 +156,11 @@ __device__ __forceinline__ float4 kda_step(float4 (&st)[DecodeShape<D>::R], cons
         s.z = fmaf(kr, wv.z, s.z); s.w = fmaf(kr, wv.w, s.w);
         st[m] = s;
     }
-    float4 o;
-    o.x = scale * fmaf(tv.kq, wv.x, Y.x); o.y = scale * fmaf(tv.kq, wv.y, Y.y);
-    o.z = scale * fmaf(tv.kq, wv.z, Y.z); o.w = scale * fmaf(tv.kq, wv.w, Y.w);
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (OUT) {
+        o.x = scale * fmaf(tv.kq, wv.x, Y.x); o.y = scale * fmaf(tv.kq, wv.y, Y.y);
+        o.z = scale * fmaf(tv.kq, wv.z, Y.z); o.w = scale * fmaf(tv.kq, wv.w, Y.w);
+    }
     return o;
 }
 
@@ -222,6 +240,110 @@ verify_kernel(const __grid_constant__ DecodeParams p) {
 #pragma unroll
             for (int m = 0; m < Sh::R; ++m)
                 st_stream(dst + (int64_t)(rs + Sh::RS * m) * D + cg * 4, st[m]);
+            if (rs == 0) IO<TIO>::st4(static_cast<TIO *>(p.o) + row * D + cg * 4, o);
+        }
+    }
+}
+
+}  // namespace kda
+
+namespace kda {
+
+// ---------------------------------------------------------------- verify + commit
+// One speculative step with the previous step's commit fused in: the live state is
+// read once, the previous step's first n_accept tokens are replayed into it (state
+// only), it is written back once, and this step's draft tokens run from it with
+// outputs only. No per-token state is written.
+struct CommitParams {
+    const void *k, *v;          // the previous step's tokens (packed like verify's)
+    const float *g, *beta;
+    const int32_t *n_accept;    // [n_seq] leading tokens of the previous batch to commit
+    const int64_t *pos;         // [n_seq] tokens absorbed by the live state (snapshots only)
+    const int64_t *snap_row;    // [n_seq] snapshot row for a boundary crossed, or < 0
+    float *snapshots;
+    int64_t n_snap_rows;
+    int32_t snap_interval;
+    int64_t tok_base;                     // absolute offset of tok0[0] in the previous batch
+    int32_t tok0[kMaxSeqsPerLaunch + 1];  // previous batch offsets (relative)
+};
+
+struct VerifyCommitParams {
+    DecodeParams p;   // this step: q, k, v, g, beta, o, tok0/tok_base, slots, pool (in/out)
+    CommitParams c;
+};
+
+template <int D, typename TIO>
+__global__ void __launch_bounds__(DecodeShape<D>::NT, 2)
+verify_commit_kernel(const __grid_constant__ VerifyCommitParams P) {
+    using Sh = DecodeShape<D>;
+    const DecodeParams &p = P.p;
+    const CommitParams &c = P.c;
+    __shared__ TokVec<D> tv[kTokBatch];
+    __shared__ __align__(16) float red[2][Sh::NW * 2 * D];
+    const int s = blockIdx.x / p.H, h = blockIdx.x % p.H;
+    const int32_t slot = p.slots[s];
+    const int m_prev = c.tok0[s + 1] - c.tok0[s];
+    const int32_t na = c.n_accept[s];
+    int64_t srow = -1, jsnap = -1;          // snapshot row, and the replayed token after which it falls
+    if (c.snap_interval > 0 && c.snap_row != nullptr && c.snap_row[s] >= 0) {
+        srow = c.snap_row[s];
+        const int64_t p0 = c.pos[s];
+        jsnap = (p0 / c.snap_interval + 1) * c.snap_interval - p0 - 1;
+    }
+    if (slot < 0 || slot >= p.n_slots || na < 0 || na > m_prev || srow >= c.n_snap_rows) {
+        if (threadIdx.x == 0) record_status(KDA_ERR_RANGE);
+        return;
+    }
+    const int t = threadIdx.x, cg = t % Sh::CG, rs = t / Sh::CG, warp = t >> 5;
+    float *S = p.pool + ((int64_t)slot * p.H + h) * (int64_t)D * D;
+    float4 st[Sh::R];
+#pragma unroll
+    for (int m = 0; m < Sh::R; ++m) {
+        const float *src = S + (int64_t)(rs + Sh::RS * m) * D + cg * 4;
+        asm volatile("ld.global.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
+                     : "=f"(st[m].x), "=f"(st[m].y), "=f"(st[m].z), "=f"(st[m].w)
+                     : "l"(src));
+    }
+    int parity = 0;
+    // 1. commit: replay the accepted prefix of the previous batch (state only)
+    const int64_t prev_first = c.tok_base + c.tok0[s];
+    for (int j0 = 0; j0 < na; j0 += kTokBatch) {
+        const int nb = min(kTokBatch, na - j0);
+        __syncthreads();
+        for (int j = 0; j < nb; ++j)
+            load_vectors<D, TIO>(tv[j], nullptr, c.k, c.v, c.g, c.beta, (prev_first + j0 + j) * p.H + h);
+        __syncthreads();
+        for (int j = 0; j < nb; ++j) {
+            kda_step<D, false>(st, tv[j], red[parity], 0.f);
+            parity ^= 1;
+            if (j0 + j == jsnap) {
+                float *dst = c.snapshots + (srow * p.H + h) * (int64_t)D * D;
+#pragma unroll
+                for (int m = 0; m < Sh::R; ++m) st_stream(dst + (int64_t)(rs + Sh::RS * m) * D + cg * 4, st[m]);
+            }
+        }
+    }
+    if (na > 0) {
+#pragma unroll
+        for (int m = 0; m < Sh::R; ++m) st_stream(S + (int64_t)(rs + Sh::RS * m) * D + cg * 4, st[m]);
+    }
+    // 2. verify this step's tokens from the committed state: outputs only
+    const int n_tok = p.tok0[s + 1] - p.tok0[s];
+    const int64_t tok_first = p.tok_base + p.tok0[s];
+    for (int j0 = 0; j0 < n_tok; j0 += kTokBatch) {
+        const int nb = min(kTokBatch, n_tok - j0);
+        __syncthreads();
+        for (int j = 0; j < nb; ++j)
+            load_token<D, TIO>(tv[j], p, (tok_first + j0 + j) * p.H + h);
+        __syncthreads();
+        if (warp < nb) token_kq<D>(tv[warp]);
+        for (int j = Sh::NW; j < nb; ++j)
+            if (warp == 0) token_kq<D>(tv[j]);
+        __syncthreads();
+        for (int j = 0; j < nb; ++j) {
+            const float4 o = kda_step<D>(st, tv[j], red[parity], p.scale);
+            parity ^= 1;
+            const int64_t row = (tok_first + j0 + j) * p.H + h;
             if (rs == 0) IO<TIO>::st4(static_cast<TIO *>(p.o) + row * D + cg * 4, o);
         }
     }

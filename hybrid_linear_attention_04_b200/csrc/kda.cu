@@ -22,27 +22,24 @@ namespace kda {
 
 static std::atomic<int64_t> g_launches{0};
 static std::atomic<int32_t> g_fail_next{0};
-static std::atomic<int> g_last_cuda_error{0};
 
-static kda_status cuda_fail(cudaError_t e) {
-    g_last_cuda_error.store((int)e);
-    return KDA_ERR_CUDA;
-}
+static kda_status cuda_fail(cudaError_t e) { return fail_cuda(e); }
 
-// Count a launch, or simulate a failed one (failure-injection hook).
+// Count a launch, or simulate a failed one (failure-injection hook; the caller then
+// reports KDA_ERR_CUDA, whose text says the launch was not issued).
 static bool launch_gate() {
     int32_t n = g_fail_next.load();
     while (n > 0) {
-        if (g_fail_next.compare_exchange_weak(n, n - 1)) return false;
+        if (g_fail_next.compare_exchange_weak(n, n - 1)) {
+            fail_text("launch not issued (failure injection)");
+            return false;
+        }
     }
     g_launches.fetch_add(1);
     return true;
 }
 
-static kda_status last_launch_status() {
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? KDA_OK : cuda_fail(e);
-}
+static kda_status last_launch_status() { return launch_result(); }
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -82,14 +79,26 @@ static kda_status dispatch_decode(int D, DecodeParams &p, int n_blocks, cudaStre
     return KDA_ERR_UNSUPPORTED;
 }
 
+template <typename TIO>
+static kda_status dispatch_verify_commit(int D, VerifyCommitParams &P, int n_blocks, cudaStream_t st) {
+    if (D != 32 && D != 64 && D != 128) return KDA_ERR_UNSUPPORTED;
+    if (!launch_gate()) return KDA_ERR_CUDA;
+    switch (D) {
+    case 32: verify_commit_kernel<32, TIO><<<n_blocks, DecodeShape<32>::NT, 0, st>>>(P); break;
+    case 64: verify_commit_kernel<64, TIO><<<n_blocks, DecodeShape<64>::NT, 0, st>>>(P); break;
+    default: verify_commit_kernel<128, TIO><<<n_blocks, DecodeShape<128>::NT, 0, st>>>(P); break;
+    }
+    return last_launch_status();
+}
+
 // --------------------------------------------------------------- prefill ----
 template <int D, int C, typename TIO>
 static kda_status launch_simt(const PrefillParams &p, cudaStream_t st) {
     using Sh = SimtShape<D, C>;
     static std::atomic<unsigned long long> attr_done{0};
-    if (!set_smem_limit_once((const void *)prefill_simt_kernel<D, C, TIO>, (int)Sh::smem_bytes,
-                             attr_done))
-        return KDA_ERR_CUDA;
+    const kda_status st_attr = set_smem_limit_once((const void *)prefill_simt_kernel<D, C, TIO>,
+                                                   (int)Sh::smem_bytes, attr_done);
+    if (st_attr != KDA_OK) return st_attr;
     if (!launch_gate()) return KDA_ERR_CUDA;
     prefill_simt_kernel<D, C, TIO><<<p.n_items, Sh::NT, Sh::smem_bytes, st>>>(p);
     return last_launch_status();
@@ -112,6 +121,7 @@ static std::atomic<int> g_prefill_path{0};
 // Scratch of kda_prefill_noalloc: a fixed module-level device array, so that call needs
 // neither an allocation nor a caller buffer. Its size bounds the workspaces it can serve.
 constexpr size_t kNoallocScratchBytes = size_t(64) << 20;
+constexpr int kMaxDevices = 64;     // devices whose scratch address is cached
 __device__ __align__(1024) uint8_t g_noalloc_scratch[kNoallocScratchBytes];
 
 }  // namespace kda
@@ -271,8 +281,18 @@ kda_status kda_prefill_noalloc(const kda_dims *dims, int32_t n_seq, const int32_
     if (st != KDA_OK) return st;
     void *scratch = nullptr;
     if (need > 0 && need <= kNoallocScratchBytes) {
-        cudaError_t e = cudaGetSymbolAddress(&scratch, g_noalloc_scratch);
+        // the array's device address on the current device, looked up on the first call
+        // that needs it there (host code only sees a stand-in for the symbol)
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
         if (e != cudaSuccess) return cuda_fail(e);
+        static std::atomic<void *> addr[kMaxDevices];
+        scratch = dev < kMaxDevices ? addr[dev].load(std::memory_order_acquire) : nullptr;
+        if (!scratch) {
+            e = cudaGetSymbolAddress(&scratch, g_noalloc_scratch);
+            if (e != cudaSuccess) return cuda_fail(e);
+            if (dev < kMaxDevices) addr[dev].store(scratch, std::memory_order_release);
+        }
     }
     return kda_prefill(dims, n_seq, cu, start_pos, q, k, v, g, beta, state_in, state_out, o,
                        snap_interval, snapshots, scratch, scratch ? kNoallocScratchBytes : 0, stream);
@@ -337,6 +357,56 @@ kda_status kda_verify(const kda_dims *dims, int32_t n_seq, const int32_t *cu_dra
     return KDA_OK;
 }
 
+kda_status kda_verify_commit(const kda_dims *dims, int32_t n_seq, const int32_t *cu_prev,
+                             const void *k_prev, const void *v_prev, const float *g_prev,
+                             const float *beta_prev, const int32_t *n_accept, const int64_t *pos,
+                             int32_t snap_interval, const int64_t *snap_row, float *snapshots,
+                             int64_t n_snap_rows, const int32_t *cu_draft, const void *q,
+                             const void *k, const void *v, const float *g, const float *beta,
+                             const int32_t *slots, int32_t n_slots, float *pool, void *o,
+                             kda_stream_t stream) {
+    kda_status st = check_dims(dims, false);
+    if (st != KDA_OK) return st;
+    if (n_seq < 0 || n_slots < 0 || snap_interval < 0 || n_snap_rows < 0) return KDA_ERR_INVALID;
+    if (n_seq == 0) return KDA_OK;
+    if (!cu_prev || !cu_draft || cu_prev[0] != 0 || cu_draft[0] != 0) return KDA_ERR_INVALID;
+    for (int s = 0; s < n_seq; ++s)
+        if (cu_prev[s + 1] < cu_prev[s] || cu_draft[s + 1] < cu_draft[s]) return KDA_ERR_INVALID;
+    const int64_t Tp = cu_prev[n_seq], T = cu_draft[n_seq];
+    if (!slots || !pool || !n_accept) return KDA_ERR_INVALID;
+    if (Tp > 0 && (!k_prev || !v_prev || !g_prev || !beta_prev)) return KDA_ERR_INVALID;
+    if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID;
+    if (snap_interval > 0 && snap_row && (!pos || !snapshots)) return KDA_ERR_INVALID;
+    const void *ptrs[] = {k_prev, v_prev, g_prev, beta_prev, n_accept, pos, snap_row, snapshots,
+                          q, k, v, g, beta, slots, pool, o};
+    for (const void *ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    static thread_local VerifyCommitParams P;
+    for (int g0 = 0; g0 < n_seq; g0 += kMaxSeqsPerLaunch) {
+        const int ng = std::min(kMaxSeqsPerLaunch, n_seq - g0);
+        std::memset(&P, 0, sizeof(P));
+        DecodeParams &p = P.p;
+        p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.slots = slots + g0;
+        p.pool = pool; p.o = o;
+        p.n_seq = ng; p.H = dims->H; p.n_slots = n_slots; p.scale = eff_scale(dims);
+        p.tok_base = cu_draft[g0];
+        for (int i = 0; i <= ng; ++i) p.tok0[i] = cu_draft[g0 + i] - cu_draft[g0];
+        CommitParams &c = P.c;
+        c.k = k_prev; c.v = v_prev; c.g = g_prev; c.beta = beta_prev;
+        c.n_accept = n_accept + g0;
+        c.pos = pos ? pos + g0 : nullptr;
+        c.snap_row = (snap_interval > 0 && snap_row) ? snap_row + g0 : nullptr;
+        c.snapshots = snapshots; c.n_snap_rows = n_snap_rows; c.snap_interval = snap_interval;
+        c.tok_base = cu_prev[g0];
+        for (int i = 0; i <= ng; ++i) c.tok0[i] = cu_prev[g0 + i] - cu_prev[g0];
+        st = dims->io == KDA_IO_BF16 ? dispatch_verify_commit<__nv_bfloat16>(dims->dk, P, ng * dims->H, cs)
+                                     : dispatch_verify_commit<float>(dims->dk, P, ng * dims->H, cs);
+        if (st != KDA_OK) return st;
+    }
+    return KDA_OK;
+}
+
 kda_status kda_snapshot(int32_t n, const int64_t *src_idx, const int64_t *dst_idx,
                         const float *src, int64_t n_src, float *dst, int64_t n_dst, int32_t H,
                         int32_t dk, int32_t dv, kda_stream_t stream) {
@@ -358,7 +428,8 @@ kda_status kda_snapshot(int32_t n, const int64_t *src_idx, const int64_t *dst_id
         p.dst_idx = dst_idx + i0;
         if (!launch_gate()) return KDA_ERR_CUDA;
         snapshot_kernel<<<dim3(per_copy, ni), 256, 0, cs>>>(p);
-        if (last_launch_status() != KDA_OK) return KDA_ERR_CUDA;
+        const kda_status st = last_launch_status();
+        if (st != KDA_OK) return st;
     }
     return KDA_OK;
 }
@@ -377,7 +448,7 @@ kda_status kda_check_device_status(kda_stream_t stream) {
 }
 
 const char *kda_last_cuda_error(void) {
-    return cudaGetErrorString(static_cast<cudaError_t>(g_last_cuda_error.load()));
+    return last_error_text().load();
 }
 
 // Forces the CUDA-core prefill path (1) or restores automatic selection (0).
@@ -385,15 +456,6 @@ const char *kda_last_cuda_error(void) {
 void kda_internal_force_prefill_path(int32_t path) { g_prefill_path.store(path); }
 
 }  // extern "C"
-
-#ifdef KDA_PHASE_TIMING
-extern "C" int kda_internal_phase_clock(long long *out) {
-    return (int)cudaMemcpyFromSymbol(out, kda::g_phase_clock, sizeof(kda::g_phase_clock));
-}
-extern "C" int kda_internal_prep_clock(long long *out) {
-    return (int)cudaMemcpyFromSymbol(out, kda::g_prep_clock, sizeof(kda::g_prep_clock));
-}
-#endif
 
 // ------------------------------------------------ failure-injection hook ----
 namespace kda {

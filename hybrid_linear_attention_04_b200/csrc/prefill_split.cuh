@@ -11,7 +11,8 @@
 // so everything except two small products per chunk is independent of S_0:
 //
 //   prep   one CTA per (chunk, head), all chunks of all sequences at once:
-//          cumsum, scaled operands, A = [Qh; Ka] Kb^T (tcgen05), T by block forward
+//          cumsum, scaled operands, A = [Qh; Ka] Kb^T (tcgen05; each scaled operand split
+//          into bf16 high and low parts, three products, so A is fp32-accurate), T by block forward
 //          substitution (mma.sync), [W' | U] = (T Diag(beta)) [Ka | V] (tcgen05). Writes
 //          one packet per (chunk, head) to the workspace, laid out as the shared
 //          memory images the chain kernel feeds to its MMAs.
@@ -31,21 +32,6 @@
 
 namespace kda {
 
-#ifdef KDA_PHASE_TIMING
-#define KDA_CMARK_T(t, ci, k) \
-    do { if (threadIdx.x == (t) && blockIdx.x == 0 && (ci) < 64) g_phase_clock[(ci)][(k)] = clock64(); } while (0)
-#else
-#define KDA_CMARK_T(t, ci, k) do { } while (0)
-#endif
-#define KDA_CMARK(ci, k) KDA_CMARK_T(64, ci, k)
-#ifdef KDA_PHASE_TIMING
-__device__ long long g_prep_clock[16][16];
-#define KDA_PMARK(k) \
-    do { if (threadIdx.x == 64 && blockIdx.x >= 4096 && blockIdx.x < 4112) g_prep_clock[blockIdx.x - 4096][(k)] = clock64(); } while (0)
-#else
-#define KDA_PMARK(k) do { } while (0)
-#endif
-
 namespace spl {
 constexpr int C = 64, D = 128;
 // ---- workspace packet of one (chunk, head); every image is 128B-swizzled slabs
@@ -57,7 +43,8 @@ constexpr uint32_t PK_U = 59392;      // U: 2 slabs (d_v 0-63, 64-127) x 64 toke
 constexpr uint32_t PACKET = PK_U + 16384;   // 75776 bytes
 // ---- prep kernel shared memory
 constexpr uint32_t P_QK = 0;          // 2 slabs x 128 rows: q -> Qh (rows 0-63), k -> Ka (rows 64-127)
-constexpr uint32_t P_V = 32768;       // v: 2 slabs x 64 rows
+constexpr uint32_t P_V = 32768;       // v: 2 slabs x 64 rows (loaded once MMA A has finished: until
+                                      // then slab 0 of the low parts below lives here)
 constexpr uint32_t P_KB = 49152;      // Kb: 2 slabs x 64 rows
 constexpr uint32_t P_TI = 65536;      // T (bf16): 1 slab x 64 rows
 constexpr uint32_t P_G = 73728;       // g fp32 [64][128]; once the operands are built, the solve
@@ -69,8 +56,15 @@ constexpr uint32_t P_AQK = P_G + 23552;           // A_qk staging (1 slab x 64 r
 constexpr uint32_t P_TOT = P_G + 32768;           // fp32 [8][128] row-block totals of b
 constexpr uint32_t P_VEC = P_TOT + 4096;          // eM, eC, gC [128], beta [64]
 constexpr uint32_t P_BARS = P_VEC + (3 * 128 + 64) * 4;
-constexpr uint32_t P_SMEM = P_BARS + 32 + 1024;   // + slack for 1024-byte alignment
-constexpr uint32_t P_TX = 16384 * 3 + 32768;      // q, k, v, g bytes per chunk
+constexpr uint32_t P_SMEM = P_BARS + 48 + 1024;   // + slack for 1024-byte alignment
+constexpr uint32_t P_TX = 16384 * 2 + 32768;      // q, k, g bytes per chunk
+constexpr uint32_t P_TX_V = 16384;                // v bytes per chunk
+// Low bf16 parts of the scaled operands (x - bf16(x), rounded to bf16), live from the
+// operand pass until MMA A completes, in memory that is free during that window:
+// [Qh_lo; Ka_lo] slab 0 over v's buffer, slab 1 and Kb_lo over T and g (g is in registers)
+constexpr uint32_t P_LO0 = P_V;                   // [Qh_lo; Ka_lo] channels 0-63, 128 rows
+constexpr uint32_t P_LO1 = P_TI;                  // [Qh_lo; Ka_lo] channels 64-127, 128 rows
+constexpr uint32_t P_KBLO = P_TI + 16384;         // Kb_lo: 2 slabs x 64 rows
 constexpr uint32_t P_COL_A = 0, P_COL_W = 0, P_COL_U = 128, P_TMEM = 256;
 // ---- chain kernel shared memory
 constexpr uint32_t STAGE = PK_U;                  // the packet head ([Qh; W'], Kb, A_qk, vectors)
@@ -95,6 +89,9 @@ constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RANGE_LIMIT2 = 80.f * LOG2E;      // 80 nats, in log2 units
 static_assert(P_WSC + 8 * 8 * 72 * 2 <= P_AQK && P_AQK + 8192 <= P_TOT && P_AQK % 1024 == 0,
               "solve scratch overlaps");
+static_assert(P_KBLO + 16384 <= P_TOT && P_LO1 % 1024 == 0 && P_KBLO % 1024 == 0,
+              "low parts overlap live data");
+static_assert(2 * (P_SMEM + 1024) <= 233472, "two prep CTAs per SM");
 static_assert(STAGE % 1024 == 0 && PACKET % 16 == 0 && C_O % 1024 == 0 && C_SN % 1024 == 0, "alignment");
 static_assert(C_SMEM <= 232448, "chain shared memory");
 }  // namespace spl
@@ -129,6 +126,17 @@ __device__ __forceinline__ uint32_t bf16x2(float a, float b) {
 }
 __device__ __forceinline__ float2 bf16x2_unpack(uint32_t u) {
     return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&u));
+}
+// a, b -> (bf16 pair hi, bf16 pair lo) with hi + lo = (a, b) to about 2^-17 relative:
+// the operands of a three-term bf16 product hi*hi' + lo*hi' + hi*lo' that is accurate to
+// fp32 level although the tensor cores take bf16
+__device__ __forceinline__ void bf16x2_split(float a, float b, uint32_t &hi, uint32_t &lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    // the residuals are exact in fp32; they are truncated to bf16 (their upper halves,
+    // one byte permute instead of a second conversion): error below 2^-17 of a, b
+    const float ra = a - __uint_as_float(hi << 16), rb = b - __uint_as_float(hi & 0xffff0000u);
+    lo = __byte_perm(__float_as_uint(ra), __float_as_uint(rb), 0x7632);
 }
 __device__ __forceinline__ uint4 bf16x8(const float *a, float s) {
     return make_uint4(bf16x2(s * a[0], s * a[1]), bf16x2(s * a[2], s * a[3]), bf16x2(s * a[4], s * a[5]),
@@ -166,8 +174,8 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
     float *eM = reinterpret_cast<float *>(sm + P_VEC);
     float *eC = eM + 128, *gC = eM + 256, *bet = eM + 384;
     uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + P_BARS);
-    uint64_t *bar_a = bar_ld + 1, *bar_w = bar_ld + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_ld + 3);
+    uint64_t *bar_a = bar_ld + 1, *bar_w = bar_ld + 2, *bar_v = bar_ld + 3;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_ld + 4);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3;
@@ -175,14 +183,13 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
         tc::bar_init(bar_ld, 1);
         tc::bar_init(bar_a, 1);
         tc::bar_init(bar_w, 1);
+        tc::bar_init(bar_v, 1);
         tc::bar_init_fence();
         tc::bar_expect_tx(bar_ld, P_TX);
         tc::tma_load3(sm + P_QK, &P.tm_q, 0, h, z, bar_ld);
         tc::tma_load3(sm + P_QK + 16384, &P.tm_q, 64, h, z, bar_ld);
         tc::tma_load3(sm + P_QK + 8192, &P.tm_k, 0, h, z, bar_ld);
         tc::tma_load3(sm + P_QK + 16384 + 8192, &P.tm_k, 64, h, z, bar_ld);
-        tc::tma_load3(sm + P_V, &P.tm_v, 0, h, z, bar_ld);
-        tc::tma_load3(sm + P_V + 8192, &P.tm_v, 64, h, z, bar_ld);
         tc::tma_load3(sm + P_G, &P.tm_g, 0, h, z, bar_ld);
     }
     if (warp == 0) {
@@ -197,14 +204,12 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
     tc::fence_after_sync();
     const uint32_t tbase = *tmem_slot;
     const uint32_t tlane = (uint32_t)(32 * wq) << 16;
-    bool ok = true, stored = false;
-    KDA_PMARK(0);
+    bool ok = true, stored = false, v_issued = false;
 
     do {
         ok = tc::bar_wait(bar_ld, 0);
         if (tid < C) bet[tid] = bv;
         if (!__syncthreads_and(ok)) { ok = false; break; }
-        KDA_PMARK(1);
         // ---- b = cumsum(g) (log2 units): warp w rows 8w..8w+7, lane channels 4l..4l+3
         float b[8][4];
 #pragma unroll
@@ -249,7 +254,6 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
                 }
             }
         }
-        KDA_PMARK(10);
         // ---- Qh = q 2^(b-m), Ka = k 2^(b-m) in place; Kb = k 2^(m-b)
         {
             const int pkb = lane >> 4, pchk = (lane & 15) >> 1, phf = (lane & 1) * 8;
@@ -270,31 +274,48 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
                     e1[e] = tc::ex2(d);
                     e2[e] = tc::ex2(-d);
                 }
-                const bool live = r < n;
-                *reinterpret_cast<uint2 *>(qp) =
-                    live ? make_uint2(bf16x2(q01.x * e1[0], q01.y * e1[1]), bf16x2(q23.x * e1[2], q23.y * e1[3]))
-                         : make_uint2(0u, 0u);
-                *reinterpret_cast<uint2 *>(kp) =
-                    live ? make_uint2(bf16x2(k01.x * e1[0], k01.y * e1[1]), bf16x2(k23.x * e1[2], k23.y * e1[3]))
-                         : make_uint2(0u, 0u);
-                *reinterpret_cast<uint2 *>(sm + P_KB + pkb * 8192 + so) =
-                    live ? make_uint2(bf16x2(k01.x * e2[0], k01.y * e2[1]), bf16x2(k23.x * e2[2], k23.y * e2[3]))
-                         : make_uint2(0u, 0u);
+                // high parts in place of q and k (and Kb), low parts in the P_LO* slabs
+                uint2 qh = make_uint2(0u, 0u), ql = qh, ah = qh, al = qh, bh = qh, bl = qh;
+                if (r < n) {
+                    bf16x2_split(q01.x * e1[0], q01.y * e1[1], qh.x, ql.x);
+                    bf16x2_split(q23.x * e1[2], q23.y * e1[3], qh.y, ql.y);
+                    bf16x2_split(k01.x * e1[0], k01.y * e1[1], ah.x, al.x);
+                    bf16x2_split(k23.x * e1[2], k23.y * e1[3], ah.y, al.y);
+                    bf16x2_split(k01.x * e2[0], k01.y * e2[1], bh.x, bl.x);
+                    bf16x2_split(k23.x * e2[2], k23.y * e2[3], bh.y, bl.y);
+                }
+                uint8_t *lo = sm + (pkb ? P_LO1 : P_LO0) + so;
+                *reinterpret_cast<uint2 *>(qp) = qh;
+                *reinterpret_cast<uint2 *>(kp) = ah;
+                *reinterpret_cast<uint2 *>(lo) = ql;
+                *reinterpret_cast<uint2 *>(lo + 8192) = al;
+                *reinterpret_cast<uint2 *>(sm + P_KB + pkb * 8192 + so) = bh;
+                *reinterpret_cast<uint2 *>(sm + P_KBLO + pkb * 8192 + so) = bl;
             }
         }
         tc::fence_async_smem();
         __syncthreads();
-        KDA_PMARK(2);
-        // ---- A = [Qh; Ka] Kb^T (M=128: A_qk rows 0-63, A_kk rows 64-127); Qh and Kb
-        // go to the packet as they are
+        // ---- A = [Qh; Ka] Kb^T (M=128: A_qk rows 0-63, A_kk rows 64-127) to fp32 accuracy as
+        // hi hi' + lo hi' + hi lo' (the lo lo' term is below fp32 rounding); Qh and Kb (high
+        // parts) go to the packet as they are
         if (tid == 0) {
             tc::fence_after_sync();
             constexpr uint32_t id_a = tc::idesc_bf16(128, 64, false, false);
             const uint64_t dQK = tc::desc_k(sbase + P_QK, 0), dKB = tc::desc_k(sbase + P_KB, 0);
+            const uint64_t dQKlo = tc::desc_k(sbase + P_LO0, 0), dKBlo = tc::desc_k(sbase + P_KBLO, 0);
+            constexpr uint32_t lo_slab = (P_LO1 - P_LO0) >> 4;
 #pragma unroll
             for (int k = 0; k < 8; ++k)
                 tc::mma_bf16(tbase + P_COL_A, dQK + (k >> 2) * 1024 + (k & 3) * 2, dKB + (k >> 2) * 512 + (k & 3) * 2,
                              id_a, k > 0);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                tc::mma_bf16(tbase + P_COL_A, dQKlo + (k >> 2) * lo_slab + (k & 3) * 2,
+                             dKB + (k >> 2) * 512 + (k & 3) * 2, id_a, 1);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                tc::mma_bf16(tbase + P_COL_A, dQK + (k >> 2) * 1024 + (k & 3) * 2,
+                             dKBlo + (k >> 2) * 512 + (k & 3) * 2, id_a, 1);
             tc::mma_commit(bar_a);
         } else if (tid == 32) {
             tc::bulk_store(pkt + PK_QW, sm + P_QK, 8192);
@@ -307,7 +328,13 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
             reinterpret_cast<float4 *>(pkt + PK_VEC)[tid] = reinterpret_cast<const float4 *>(eM)[tid];
         ok = tc::bar_wait(bar_a, 0);
         tc::fence_after_sync();
-        KDA_PMARK(3);
+        if (tid == 0 && ok) {
+            // the low parts are dead: v goes into its buffer (needed by the last MMAs only)
+            tc::bar_expect_tx(bar_v, P_TX_V);
+            tc::tma_load3(sm + P_V, &P.tm_v, 0, h, z, bar_v);
+            tc::tma_load3(sm + P_V + 8192, &P.tm_v, 64, h, z, bar_v);
+            v_issued = true;
+        }
         if (warp < 2) {
             // A_qk, masked to i <= r, into its staging image (bulk-stored after this phase)
             const int r = 32 * warp + lane;
@@ -375,7 +402,6 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
         tc::fence_async_smem();
         tc::fence_before_sync();
         if (!__syncthreads_and(ok)) { ok = false; break; }
-        KDA_PMARK(4);
         if (tid == 32) {
             tc::bulk_store(pkt + PK_AQK, sm + P_AQK, 8192);
             tc::bulk_commit();
@@ -443,10 +469,10 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
             tc::bulk_wait_read_all();
             stored = false;
         }
+        if (tid == 0) ok = tc::bar_wait(bar_v, 0);    // v has landed (the MMAs below read it)
         tc::fence_async_smem();
         tc::fence_before_sync();
-        __syncthreads();
-        KDA_PMARK(5);
+        if (!__syncthreads_and(ok)) { ok = false; break; }
         // ---- [W' | U] = (T Diag(beta)) [Ka | V]  (M=64: row r in TMEM lane (r % 16) + 32 (r / 16))
         if (tid == 0) {
             tc::fence_after_sync();
@@ -462,7 +488,6 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
         }
         ok = tc::bar_wait(bar_w, 0);
         tc::fence_after_sync();
-        KDA_PMARK(6);
         {
             // warp (wq, wh): rows 16 wq .. 16 wq + 15 (lanes 0-15), columns 64 wh .. 64 wh + 63.
             // The images are staged in the solve scratch (free since T was built): W' slabs at
@@ -488,7 +513,6 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
         }
         tc::fence_async_smem();
         __syncthreads();
-        KDA_PMARK(7);
         if (tid == 32) {
             tc::bulk_store(pkt + PK_QW + 8192, sm + P_G, 8192);
             tc::bulk_store(pkt + PK_QW + 16384 + 8192, sm + P_G + 8192, 8192);
@@ -498,12 +522,13 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
         }
     } while (0);
 
-    KDA_PMARK(8);
-    if (!ok && tid == 0) tc::bar_wait(bar_ld, 0, 1u << 16);   // loads still in flight land first
+    if (!ok && tid == 0) {                              // loads still in flight land first
+        tc::bar_wait(bar_ld, 0, 1u << 16);
+        if (v_issued) tc::bar_wait(bar_v, 0, 1u << 16);
+    }
     if (stored) tc::bulk_wait_read_all();
     tc::fence_before_sync();
     __syncthreads();
-    KDA_PMARK(9);
     if (warp == 0) tc::tmem_dealloc(tbase, P_TMEM);
 }
 
@@ -637,7 +662,6 @@ __global__ void __launch_bounds__(256, 1) prefill_chain_kernel(const __grid_cons
         const uint32_t sstg = sbase + st * STAGE;
         const uint32_t col_r1 = C_COL_R1 + 64 * (ci & 1);
         const float *eC = reinterpret_cast<const float *>(stg + PK_VEC) + 128, *gC = eC + 128;
-        KDA_CMARK(ci, 0);
         // ---- round 1: [Qh; W'] Sm -> rows 0-63 O, rows 64-127 W'Sm; then the loads of
         // chunk ci + NSTAGE - 1 (its stage was released at the end of chunk ci - 1)
         if (tid == 0) {
@@ -658,7 +682,6 @@ __global__ void __launch_bounds__(256, 1) prefill_chain_kernel(const __grid_cons
             // ---- W = U - W' Sm (token rows in TMEM lanes 64-127)
             ok = tc::bar_wait(bar_r1, (uint32_t)(ci & 1));
             tc::fence_after_sync();
-            KDA_CMARK(ci, 1);
             float a[32];
             tc::tmem_ld32(tbase + tlane + col_r1 + 32 * wh, a);
             tc::tmem_ld_wait();
@@ -689,7 +712,6 @@ __global__ void __launch_bounds__(256, 1) prefill_chain_kernel(const __grid_cons
         }
         tc::fence_before_sync();
         __syncthreads();
-        KDA_CMARK(ci, 2);
         // ---- round 2: D = Kb^T W (commit bar_d), then O += A_qk W (M=128; A rows 64-127 are
         // the bytes after A_qk and land in TMEM lanes 64-127, not read again; commit bar_o)
         if (tid == 0) {
@@ -752,23 +774,18 @@ __global__ void __launch_bounds__(256, 1) prefill_chain_kernel(const __grid_cons
         {
             bool okd = tc::bar_wait(bar_d, (uint32_t)(ci & 1));
             tc::fence_after_sync();
-            KDA_CMARK(ci, 3);
             float a[32];
             const float g_c = gC[c_own], e_c = eC[c_own];
             tc::tmem_ld32(tbase + tlane + C_COL_D + 32 * wh, a);
             tc::tmem_ld_wait();
-            KDA_CMARK(ci, 4);
 #pragma unroll
             for (int e = 0; e < 32; ++e) S[e] = fmaf(g_c, S[e], e_c * a[e]);
-            KDA_CMARK(ci, 5);
             if (ci + 1 < n_chunks) {
                 okd = okd && tc::bar_wait(&full[(ci + 1) % NSTAGE], (uint32_t)(((ci + 1) / NSTAGE) & 1));
-                KDA_CMARK(ci, 6);
                 if (okd) write_sm((ci + 1) % NSTAGE);
                 tc::fence_async_smem();
                 if (wwarp) load_u(ci + 1);
             }
-            KDA_CMARK(ci, 7);
             if (sq.start_pos + (int64_t)ci * C + n == next_snap) {
                 next_snap += p.snap_interval;
                 // a snapshot due at consecutive chunks: the W rows of the previous one go out now
@@ -788,7 +805,6 @@ __global__ void __launch_bounds__(256, 1) prefill_chain_kernel(const __grid_cons
         tc::fence_before_sync();
         ok = __syncthreads_and(ok);
         if (ok) landed = ci + 2 < n_chunks ? ci + 2 : n_chunks;
-        KDA_CMARK(ci, 9);
     }
     if (ok && n_chunks > 0) {
         // outputs of the last chunk; snapshot halves still pending
@@ -860,7 +876,7 @@ inline kda_status launch_prefill_split(PrefillParams &p, const kda_dims &d, int6
         !encode_map(&PP.tm_k, p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, T, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_map(&PP.tm_v, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, T, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_map(&PP.tm_g, p.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, T, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return KDA_ERR_CUDA;
+        return fail_text("cuTensorMapEncodeTiled failed for q, k, v or g");
     PP.beta = p.beta;
     PP.ws = static_cast<uint8_t *>(ws);
     PP.H = H;
@@ -876,22 +892,24 @@ inline kda_status launch_prefill_split(PrefillParams &p, const kda_dims &d, int6
     CPm.ws = static_cast<const uint8_t *>(ws);
     CPm.tok_first = tok_first;
     if (!encode_map(&CPm.tm_o, p.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, T, 64, CU_TENSOR_MAP_SWIZZLE_128B))
-        return KDA_ERR_CUDA;
+        return fail_text("cuTensorMapEncodeTiled failed for o");
     const int64_t snap_rows = n_snap_total * H * D;
     CPm.snap_tma = p.snapshots && n_snap_total > 0 && snap_rows < 0x7fffffffLL;
-    if (CPm.snap_tma && !encode_snap_map(&CPm.tm_snap, p.snapshots, snap_rows)) return KDA_ERR_CUDA;
+    if (CPm.snap_tma && !encode_snap_map(&CPm.tm_snap, p.snapshots, snap_rows))
+        return fail_text("cuTensorMapEncodeTiled failed for the snapshots");
     static std::atomic<unsigned long long> prep_attr{0}, chain_attr{0};
-    if (!set_smem_limit_once((const void *)prefill_prep_kernel, (int)P_SMEM, prep_attr) ||
-        !set_smem_limit_once((const void *)prefill_chain_kernel, (int)C_SMEM, chain_attr))
-        return KDA_ERR_CUDA;
+    kda_status r = set_smem_limit_once((const void *)prefill_prep_kernel, (int)P_SMEM, prep_attr);
+    if (r == KDA_OK) r = set_smem_limit_once((const void *)prefill_chain_kernel, (int)C_SMEM, chain_attr);
+    if (r != KDA_OK) return r;
     if (n_packets > 0) {
         if (!gate()) return KDA_ERR_CUDA;
         prefill_prep_kernel<<<(unsigned)(n_packets * H), 256, P_SMEM, st>>>(PP);
-        if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+        r = launch_result();
+        if (r != KDA_OK) return r;
     }
     if (!gate()) return KDA_ERR_CUDA;
     prefill_chain_kernel<<<CPm.p.n_items, 256, C_SMEM, st>>>(CPm);
-    return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    return launch_result();
 }
 
 }  // namespace kda

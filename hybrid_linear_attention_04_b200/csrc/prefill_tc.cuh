@@ -1,7 +1,7 @@
 // KDA chunked prefill on the tcgen05 tensor cores (d_k = d_v = 128, chunk 64,
 // bf16 q/k/v/o, fp32 state). The chunk form is the one in prefill_common.cuh.
 //
-// One CTA (128 threads) walks the chunks of one (sequence, head, 64-column
+// One CTA (256 threads) walks the chunks of one (sequence, head, 64-column
 // d_v slice); d_v columns are independent, so two CTAs per head run in
 // parallel. Per chunk:
 //   TMA      q, k (bf16, 128B-swizzled slabs), g (fp32) and the v slice; the
@@ -10,12 +10,14 @@
 //   cores    Qh = q.exp(b-m), Ka = k.exp(b-m), Kb = k.exp(m-b) (bf16 operands),
 //            so that Qh Kb^T = A_qk and Ka Kb^T = A_kk with every exponent
 //            inside the chunk bounded by half the chunk's decay range.
-//   tcgen05  [Qh; Ka] Kb^T -> TMEM (M=128: A_qk rows 0-63, A_kk rows 64-127)
+//   tcgen05  [Qh; Ka] Kb^T -> TMEM (M=128: A_qk rows 0-63, A_kk rows 64-127), each
+//            scaled operand split into bf16 high and low parts (three products, so A
+//            is fp32-accurate)
 //   tcgen05  (same MMAs as A) R' = Ka Sm, O = Qh Sm  (Sm = Diag(e^m) S_0, stored
 //            transposed under Kb so one N=128 round yields all four blocks)
 //   CUDA     L = Diag(beta) A_kk; inverses of its 16x16 diagonal blocks (fp32);
 //   cores    R = V - R' (fp32); then W = (I + L)^{-1} Diag(beta) R by block
-//            forward substitution on tf32 mma.sync, 8 d_v columns per warp
+//            forward substitution on bf16 mma.sync, 8 d_v columns per warp
 //   tcgen05  O += A_qk W, D = Kb^T W                 (M=128)
 //   CUDA     o = scale O (bf16 store); S_C = Diag(Gamma_C) S_0 + Diag(e^(b_C-m)) D
 //   cores    with the fp32 master state held in registers (thread = d_k row).
@@ -31,14 +33,6 @@
 #include "tc_util.cuh"
 
 namespace kda {
-
-#ifdef KDA_PHASE_TIMING
-__device__ long long g_phase_clock[64][16];
-#define KDA_MARK(ci, k) \
-    do { if (threadIdx.x == 0 && blockIdx.x == 0 && (ci) < 64) g_phase_clock[(ci)][(k)] = clock64(); } while (0)
-#else
-#define KDA_MARK(ci, k) do { } while (0)
-#endif
 
 struct TcParams {
     CUtensorMap tm_q, tm_k, tm_v, tm_g;
@@ -62,6 +56,12 @@ constexpr uint32_t RF = SOLVE + 64 * 65 * 4;   // R = V - Ka Sm, fp32 [64][68]
 constexpr uint32_t LB = RF + 64 * 68 * 4;      // bf16 [64][72]: L off the diagonal blocks, X on them
 constexpr uint32_t WSC = LB + 64 * 72 * 2;     // per-warp Y / W columns, bf16 [8 warps][8][72]
 constexpr uint32_t TOT = WSC + 8 * 8 * 72 * 2; // per-warp row-block totals of b [8][128]
+// Low bf16 parts of the scaled operands (x - bf16(x), rounded to bf16), live from the
+// operand pass until round 1a completes, over the solve scratch (free in that window)
+constexpr uint32_t LO_AK0 = SOLVE;             // [Qh_lo; Ka_lo] channels 0-63, 128 rows
+constexpr uint32_t LO_AK1 = SOLVE + 16384;     // [Qh_lo; Ka_lo] channels 64-127, 128 rows
+constexpr uint32_t LO_KB = SOLVE + 32768;      // Kb_lo: 2 slabs x 64 rows
+static_assert(LO_KB + 16384 <= TOT && SOLVE % 1024 == 0, "low parts overlap live data");
 constexpr uint32_t VEC = TOT + 8 * 128 * 4;    // eM, eC, gC [128] + beta [64]
 constexpr uint32_t BARS = VEC + (3 * 128 + 64) * 4;
 constexpr uint32_t SMEM_USED = BARS + 48;
@@ -80,6 +80,15 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 }
 __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
     return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&u));
+}
+// a, b -> bf16 pairs hi and lo with hi + lo = (a, b) to about 2^-17 relative
+__device__ __forceinline__ void split_bf16(float a, float b, uint32_t &hi, uint32_t &lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    // the residuals are exact in fp32; they are truncated to bf16 (their upper halves,
+    // one byte permute instead of a second conversion): error below 2^-17 of a, b
+    const float ra = a - __uint_as_float(hi << 16), rb = b - __uint_as_float(hi & 0xffff0000u);
+    lo = __byte_perm(__float_as_uint(ra), __float_as_uint(rb), 0x7632);
 }
 __device__ __forceinline__ uint4 pack8(const float *a, float s) {
     return make_uint4(pack_bf16(s * a[0], s * a[1]), pack_bf16(s * a[2], s * a[3]),
@@ -187,12 +196,10 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
 
     for (int ci = 0; ci < n_chunks; ++ci) {
         const int n = min(C, sq.len - ci * C);
-        KDA_MARK(ci, 0);
         // ---- A. this chunk's operands have landed --------------------------
         ok = tc::bar_wait(&tma_bar[ci & 1], (ci >> 1) & 1);
         if (!__syncthreads_and(ok)) { ok = false; break; }
         landed = ci + 1;
-        KDA_MARK(ci, 1);
         // ---- B. b = cumsum(g) over the chunk, in log2 units -------------------
         float b[8][4];
 #pragma unroll
@@ -244,7 +251,6 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
                 }
             }
         }
-        KDA_MARK(ci, 15);
         // ---- C. scaled bf16 operands Qh = q 2^(b-m), Ka = k 2^(b-m), Kb = k 2^(m-b)
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -261,29 +267,46 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
                 e1[e] = tc::ex2(d);
                 e2[e] = tc::ex2(-d);
             }
-            const bool live = r < n;
-            const uint2 oq = live ? make_uint2(pack_bf16(q01.x * e1[0], q01.y * e1[1]), pack_bf16(q23.x * e1[2], q23.y * e1[3]))
-                                  : make_uint2(0u, 0u);
-            const uint2 oa = live ? make_uint2(pack_bf16(k01.x * e1[0], k01.y * e1[1]), pack_bf16(k23.x * e1[2], k23.y * e1[3]))
-                                  : make_uint2(0u, 0u);
-            const uint2 ob = live ? make_uint2(pack_bf16(k01.x * e2[0], k01.y * e2[1]), pack_bf16(k23.x * e2[2], k23.y * e2[3]))
-                                  : make_uint2(0u, 0u);
-            *reinterpret_cast<uint2 *>(sm + OP_AK + pkb * 16384 + tc::sw128(r, pchk) + phf) = oq;
-            *reinterpret_cast<uint2 *>(sm + OP_AK + pkb * 16384 + tc::sw128(64 + r, pchk) + phf) = oa;
-            *reinterpret_cast<uint2 *>(sm + OP_KB + pkb * 16384 + tc::sw128(r, pchk) + phf) = ob;
+            // high parts (the MMA operands) and low parts (for the fp32-accurate A)
+            uint2 oq = make_uint2(0u, 0u), lq = oq, oa = oq, la = oq, ob = oq, lb = oq;
+            if (r < n) {
+                split_bf16(q01.x * e1[0], q01.y * e1[1], oq.x, lq.x);
+                split_bf16(q23.x * e1[2], q23.y * e1[3], oq.y, lq.y);
+                split_bf16(k01.x * e1[0], k01.y * e1[1], oa.x, la.x);
+                split_bf16(k23.x * e1[2], k23.y * e1[3], oa.y, la.y);
+                split_bf16(k01.x * e2[0], k01.y * e2[1], ob.x, lb.x);
+                split_bf16(k23.x * e2[2], k23.y * e2[3], ob.y, lb.y);
+            }
+            const uint32_t sr = tc::sw128(r, pchk) + phf, sr64 = tc::sw128(64 + r, pchk) + phf;
+            const uint32_t lo_ak = pkb ? LO_AK1 : LO_AK0;
+            *reinterpret_cast<uint2 *>(sm + OP_AK + pkb * 16384 + sr) = oq;
+            *reinterpret_cast<uint2 *>(sm + OP_AK + pkb * 16384 + sr64) = oa;
+            *reinterpret_cast<uint2 *>(sm + OP_KB + pkb * 16384 + sr) = ob;
+            *reinterpret_cast<uint2 *>(sm + lo_ak + sr) = lq;
+            *reinterpret_cast<uint2 *>(sm + lo_ak + sr64) = la;
+            *reinterpret_cast<uint2 *>(sm + LO_KB + pkb * 8192 + sr) = lb;
         }
         tc::fence_async_smem();
         __syncthreads();   // operands and eM visible
-        KDA_MARK(ci, 2);
         // ---- D1. round 1a: A = [Qh; Ka] Kb^T (independent of the state), issued
         // before Sm^T is written so that the L extraction can start earlier
         if (tid == 0) {
             tc::fence_after_sync();
             constexpr uint32_t id_a = tc::idesc_bf16(128, 64, false, false);
+            // hi hi' + lo hi' + hi lo': A to fp32 accuracy (the lo lo' term is below it)
+            const uint64_t dAKlo = tc::desc_k(sbase + LO_AK0, 0), dKBlo = tc::desc_k(sbase + LO_KB, 0);
 #pragma unroll
             for (int k = 0; k < 8; ++k)
                 tc::mma_bf16(tbase + COL_A, dAK + (k >> 2) * 1024 + (k & 3) * 2, dKB + (k >> 2) * 1024 + (k & 3) * 2,
                              id_a, k > 0);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                tc::mma_bf16(tbase + COL_A, dAKlo + (k >> 2) * 1024 + (k & 3) * 2,
+                             dKB + (k >> 2) * 1024 + (k & 3) * 2, id_a, 1);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                tc::mma_bf16(tbase + COL_A, dAK + (k >> 2) * 1024 + (k & 3) * 2,
+                             dKBlo + (k >> 2) * 512 + (k & 3) * 2, id_a, 1);
             tc::mma_commit(bar_a);
         }
         // ---- Sm^T = (Diag(e^m) S_0)^T (bf16, K-major B operand of round 1b) ----
@@ -299,7 +322,6 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
         }
         tc::fence_async_smem();
         __syncthreads();
-        KDA_MARK(ci, 3);
         // ---- D2. round 1b: [R'; O] = [Qh; Ka] Sm; then the next chunk's loads ----
         if (tid == 0) {
             tc::fence_after_sync();
@@ -318,7 +340,6 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
         // wait is acted on at the block-wide vote after phase E
         ok = tc::bar_wait(warp < 4 ? bar_a : bar_b, (uint32_t)(ci & 1));
         tc::fence_after_sync();
-        KDA_MARK(ci, 4);
         // ---- E. warps 0,1: A_qk (masked bf16 operand). Warps 2,3: L = Diag(beta)
         // A_kk (fp32), then the inverses X of its four 16x16 diagonal blocks by
         // forward substitution (each warp owns two blocks: no block-wide sync).
@@ -414,7 +435,6 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
         tc::fence_async_smem();
         tc::fence_before_sync();
         if (!__syncthreads_and(ok)) { ok = false; break; }
-        KDA_MARK(ci, 5);
         // ---- F. W = (I + L)^{-1} Diag(beta) R by block forward substitution on bf16
         // mma.sync (fp32 accumulate): W_R = X_RR (beta R_R - sum_{J<R} L_RJ W_J).
         // Warp w owns the eight d_v columns 8w..8w+7, so the four block rows need
@@ -423,7 +443,6 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
         {
             const int g = lane >> 2, t = lane & 3, c0 = 8 * warp;
             __nv_bfloat16 *ws = Wsc + warp * 8 * 72;                // [8 cols][72]
-            KDA_MARK(ci, 14);
 #pragma unroll
             for (int R = 0; R < 4; ++R) {
                 const int r0 = 16 * R + g, r1 = r0 + 8;
@@ -478,13 +497,11 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
                 *reinterpret_cast<uint32_t *>(sm + OP_W + tc::sw128(r0, warp) + 4 * t) = pack_bf16(w[0], w[1]);
                 *reinterpret_cast<uint32_t *>(sm + OP_W + tc::sw128(r1, warp) + 4 * t) = pack_bf16(w[2], w[3]);
                 __syncwarp();
-                KDA_MARK(ci, 10 + R);
             }
         }
         tc::fence_async_smem();
         tc::fence_before_sync();
         __syncthreads();
-        KDA_MARK(ci, 7);
         // ---- H. round 3: O += A_qk W ; D = Kb^T W ---------------------------------------
         if (tid == 0) {
             tc::fence_after_sync();
@@ -503,7 +520,6 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
         mma_phase ^= 1;
         if (!__syncthreads_and(ok)) { ok = false; break; }
         tc::fence_after_sync();
-        KDA_MARK(ci, 8);
         // ---- I. outputs, state update, snapshot -------------------------------------------
         {
             float a[32];
@@ -533,7 +549,6 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
         }
         tc::fence_before_sync();
         __syncthreads();
-        KDA_MARK(ci, 9);
     }
 
     if (ok && p.state_out) {
@@ -590,16 +605,15 @@ inline kda_status launch_prefill_tc(PrefillParams &p, const kda_dims &d, int64_t
         !encode_map(&P.tm_k, p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, T, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_map(&P.tm_v, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, T, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_map(&P.tm_g, p.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, T, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return KDA_ERR_CUDA;
+        return fail_text("cuTensorMapEncodeTiled failed for q, k, v or g");
     P.p = p;
     P.p.n_items = p.n_seq * H * 2;
     static std::atomic<unsigned long long> attr_done{0};
-    if (!set_smem_limit_once((const void *)prefill_tc_kernel, (int)tcp::SMEM_BYTES, attr_done))
-        return KDA_ERR_CUDA;
+    const kda_status r = set_smem_limit_once((const void *)prefill_tc_kernel, (int)tcp::SMEM_BYTES, attr_done);
+    if (r != KDA_OK) return r;
     if (!gate()) return KDA_ERR_CUDA;
     prefill_tc_kernel<<<P.p.n_items, tcp::NT, tcp::SMEM_BYTES, st>>>(P);
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    return launch_result();
 }
 
 }  // namespace kda

@@ -47,6 +47,8 @@ _SIGNATURES = {
     "kda_prefill_noalloc_capacity": (ctypes.c_size_t, []),
     "kda_decode": (_I32, [_P, _I32, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P]),
     "kda_verify": (_I32, [_P, _I32, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P]),
+    "kda_verify_commit": (_I32, [_P, _I32, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _I64, _P, _P,
+                                 _P, _P, _P, _P, _P, _I32, _P, _P, _P]),
     "kda_snapshot": (_I32, [_I32, _P, _P, _P, _I64, _P, _I64, _I32, _I32, _I32, _P]),
     "kda_status_string": (ctypes.c_char_p, [_I32]),
     "kda_check_device_status": (_I32, [_P]),
@@ -212,6 +214,29 @@ def kda_verify(q, k, v, g, beta, cu_draft, slots, state_pool, token_states, o, s
                             _dptr(v), _dptr(g), _dptr(beta), _dptr(slots), state_pool.shape[0],
                             _dptr(state_pool), _dptr(token_states), _dptr(o), _stream(stream)),
            "kda_verify")
+
+
+def kda_verify_commit(prev, n_accept, cu_prev, q, k, v, g, beta, cu_draft, slots, state_pool, o,
+                      pos=None, snap_interval=0, snap_row=None, snapshots=None, scale=0.0,
+                      stream=None):
+    """Speculative step with the previous step's commit fused in (see include/kda.h).
+
+    ``prev``: dict of the previous batch's device tensors k, v, g, beta (packed by
+    ``cu_prev``), or None when it is empty; ``n_accept``: device int32 [n_seq].
+    """
+    cp = _host_array(cu_prev, np.int32)
+    cd = _host_array(cu_draft, np.int32)
+    if len(cp) != len(cd):
+        raise KDAError(1, "cu_prev and cu_draft must describe the same sequences")
+    dims = _dims(q, v, 0, scale)
+    pv = prev or {}
+    n_rows = 0 if snapshots is None else snapshots.shape[0]
+    _check(lib().kda_verify_commit(
+        ctypes.byref(dims), len(cd) - 1, _hptr(cp), _dptr(pv.get("k")), _dptr(pv.get("v")),
+        _dptr(pv.get("g")), _dptr(pv.get("beta")), _dptr(n_accept), _dptr(pos), int(snap_interval),
+        _dptr(snap_row), _dptr(snapshots), n_rows, _hptr(cd), _dptr(q), _dptr(k), _dptr(v),
+        _dptr(g), _dptr(beta), _dptr(slots), state_pool.shape[0], _dptr(state_pool), _dptr(o),
+        _stream(stream)), "kda_verify_commit")
 
 
 def kda_snapshot(src_idx, dst_idx, src, dst, stream=None):

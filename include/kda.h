@@ -24,7 +24,10 @@
  *  - Pointers suffixed _h are host memory read during the call only. All other
  *    pointers are device memory owned by the caller; the library allocates no
  *    memory and keeps no state between calls except a device status word.
- *    Scratch memory, where a call can use it, is a caller-provided workspace.
+ *    Scratch memory, where a call can use it, is a caller-provided workspace,
+ *    with one exception: kda_prefill_noalloc uses a fixed device array of
+ *    kda_prefill_noalloc_capacity() bytes that the library's module holds on
+ *    every device it is loaded on, from module load until process exit.
  *  - Every device pointer must be 16-byte aligned (KDA_ERR_ALIGN otherwise).
  *  - Calls are asynchronous on `stream`: argument errors return synchronously
  *    before anything is launched; device-side range errors and bounded-wait
@@ -132,8 +135,11 @@ kda_status kda_prefill_workspace_size(const kda_dims *dims, int32_t n_seq,
  * Errors (before launch): KDA_ERR_INVALID, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGN,
  * KDA_ERR_WORKSPACE (non-null workspace below kda_prefill_workspace_size).
  * Device status KDA_ERR_RANGE: a chunk whose per-channel decay exceeds the
- * tensor-core path's range (sum of g over one chunk below -170 in some channel;
- * the outputs of that chunk are then not reliable).
+ * tensor-core path's range: with b_r = g_0 + ... + g_r summed over the chunk's
+ * tokens r = 0..63, some channel has -b_31 > 80 or b_31 - b_last > 80 (80 nats of
+ * decay from the chunk's middle in either direction; any chunk whose total decay
+ * sum(g) stays above -80 in every channel is within range). The outputs of that
+ * chunk are then not reliable.
  */
 kda_status kda_prefill(const kda_dims *dims, int32_t n_seq, const int32_t *cu_seqlens_h,
                        const int64_t *start_pos_h, const void *q, const void *k,
@@ -148,9 +154,15 @@ kda_status kda_prefill(const kda_dims *dims, int32_t n_seq, const int32_t *cu_se
  * kda_prefill_noalloc_capacity() bytes (a module-level array, resident from the
  * library's first use on a device) whenever kda_prefill_workspace_size fits in
  * it, and the single-launch path otherwise. Arguments, layouts and errors as
- * kda_prefill. The scratch is shared by all calls on a device: calls that may
- * run concurrently (different streams, threads or processes sharing a context)
- * must be ordered by the caller, e.g. issued on one stream.
+ * kda_prefill. For callers that cannot allocate device memory at the point of
+ * the call (code running inside a captured or replayed stream region, or a host
+ * that forbids allocation after start-up) and cannot set a workspace aside.
+ * The scratch is shared by all calls on a device of this process and keeps the
+ * last call's contents (every call writes what it reads): calls that could
+ * overlap on the GPU (issued on different streams, or from different host
+ * threads) race, so the caller must order them, e.g. issue them on one stream.
+ * The scratch's device address is looked up once per device, on the first call
+ * that uses it; make that first call before any stream capture.
  */
 kda_status kda_prefill_noalloc(const kda_dims *dims, int32_t n_seq, const int32_t *cu_seqlens_h,
                                const int64_t *start_pos_h, const void *q, const void *k,
@@ -162,9 +174,13 @@ kda_status kda_prefill_noalloc(const kda_dims *dims, int32_t n_seq, const int32_
 size_t kda_prefill_noalloc_capacity(void);
 
 /*
- * kda_decode — one token per sequence against a pool of live states (the
- * recurrence above for a single t), updating each state in place with one
- * read and one write of it.
+ * kda_decode — one token per sequence against a pool of live states, updating
+ * each state in place with one read and one write of it. This is one step t of
+ * the recurrence at the top of this header (Kimi K3 technical FAQ, "What is KDA,
+ * and why does a serving engineer care?": the fixed d_k x d_v state per head is
+ * all a decode step reads and rewrites, instead of a growing KV cache; runtimewire,
+ * "The architecture is built around inference cost": KDA layers carry a
+ * fixed-size recurrent state).
  *   q, k, g [n_seq, H, dk]; v, o [n_seq, H, dv]; beta [n_seq, H].
  *   slots [n_seq] (device int32): row of state_pool used by each sequence;
  *               slots must be distinct (a repeated slot is a data race).
@@ -177,11 +193,15 @@ kda_status kda_decode(const kda_dims *dims, int32_t n_seq, const void *q, const 
                       int32_t n_slots, float *state_pool, void *o, kda_stream_t stream);
 
 /*
- * kda_verify — speculative verify: sequence s runs its draft tokens
- * [cu_draft_h[s], cu_draft_h[s+1]) (packed like prefill) from the state
- * state_pool[slots[s]], which is only read, and writes the output and the
- * state after every token, so that the caller can commit the state of the
- * last accepted token with kda_snapshot (rollback of rejected drafts).
+ * kda_verify — speculative verify (runtimewire, "A third party tripled
+ * single-user decoding speed": a draft model proposes several tokens and the
+ * target accepts a prefix of them per step, 2.61 to 4.73 on average; Kimi K3
+ * technical FAQ, "What is the speculative-decoding story?"). Sequence s runs its
+ * draft tokens [cu_draft_h[s], cu_draft_h[s+1]) (packed like prefill) through the
+ * recurrence at the top of this header from the state state_pool[slots[s]],
+ * which is only read, and writes the output and the state after every token, so
+ * that the caller can commit the state of the last accepted token with
+ * kda_snapshot (rollback of rejected drafts).
  *   token_states [cu_draft_h[n_seq], H, dk, dv]: state after each token.
  * Errors as kda_decode.
  */
@@ -190,6 +210,46 @@ kda_status kda_verify(const kda_dims *dims, int32_t n_seq, const int32_t *cu_dra
                       const float *beta, const int32_t *slots, int32_t n_slots,
                       const float *state_pool, float *token_states, void *o,
                       kda_stream_t stream);
+
+/*
+ * kda_verify_commit — one speculative step with the previous step's commit fused
+ * in, so that no per-token state is ever written (vLLM day-0 blog, "Kimi Delta
+ * Attention": the recurrent state lives in state blocks and is snapshotted at
+ * block boundaries; runtimewire, "A third party tripled single-user decoding
+ * speed": each step accepts a prefix of its draft tokens). Acceptance of a step
+ * is known only after every layer has verified it, so the commit of step n-1
+ * runs inside the verify of step n. For sequence s, with S = state_pool[slots[s]]
+ * holding the state before the previous step's tokens:
+ *   1. commit: the first n_accept[s] tokens of the previous step's batch
+ *      [cu_prev_h[s], cu_prev_h[s+1]) (k_prev, v_prev, g_prev, beta_prev, packed
+ *      like kda_verify's input; their q is not needed) run through the
+ *      recurrence at the top of this header and S is written back in place (not
+ *      written when n_accept[s] == 0). With snap_interval > 0 and snap_row[s] >= 0,
+ *      the state after the committed token at absolute position p = pos[s] + j + 1
+ *      with p % snap_interval == 0, if one of the committed tokens is there, is
+ *      also written to snapshots[snap_row[s]] (at most one such p when
+ *      snap_interval >= the batch length).
+ *   2. verify: this step's tokens [cu_draft_h[s], cu_draft_h[s+1]) (q, k, v, g,
+ *      beta) run from the committed state; their outputs go to o [cu_draft_h[n_seq],
+ *      H, dv]; the state is not written.
+ * The state after step 1 is bit-identical to kda_verify's state after token
+ * n_accept[s] - 1 of the previous batch, and the outputs of step 2 to kda_verify's
+ * from that state. A pipeline drains with a call whose draft batch is empty.
+ *   n_accept [n_seq] (device int32), 0 <= n_accept[s] <= cu_prev_h[s+1] - cu_prev_h[s].
+ *   pos [n_seq] (device int64, required with snapshots): tokens absorbed by S.
+ *   snap_row [n_seq] (device int64, nullable), snapshots [n_snap_rows, H, dk, dv].
+ * Device status KDA_ERR_RANGE (that sequence is skipped: neither S nor its outputs
+ * are written) for a slot outside [0, n_slots), n_accept outside its range, or a
+ * snap_row >= n_snap_rows. Other errors as kda_verify.
+ */
+kda_status kda_verify_commit(const kda_dims *dims, int32_t n_seq, const int32_t *cu_prev_h,
+                             const void *k_prev, const void *v_prev, const float *g_prev,
+                             const float *beta_prev, const int32_t *n_accept, const int64_t *pos,
+                             int32_t snap_interval, const int64_t *snap_row, float *snapshots,
+                             int64_t n_snap_rows, const int32_t *cu_draft_h, const void *q,
+                             const void *k, const void *v, const float *g, const float *beta,
+                             const int32_t *slots, int32_t n_slots, float *state_pool, void *o,
+                             kda_stream_t stream);
 
 /*
  * kda_snapshot — bit-exact copies of whole states between pools: for i < n,
@@ -216,8 +276,9 @@ const char *kda_status_string(kda_status s);
  */
 kda_status kda_check_device_status(kda_stream_t stream);
 
-/* Text of the CUDA error behind the most recent KDA_ERR_CUDA (static storage;
- * "no error" if there was none). */
+/* Text behind the most recent KDA_ERR_CUDA (static storage): the CUDA error, a
+ * failed tensor-map encoding, or an injected launch failure; "no error" if there
+ * was none. */
 const char *kda_last_cuda_error(void);
 
 /* Number of kernel launches the library has issued in this process (for

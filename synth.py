@@ -185,9 +185,10 @@ def states(seed: int, n: int, H: int, dk: int, dv: int, std: float = 0.1, tag: s
     return torch.from_numpy(x.reshape(n, H, dk, dv))
 
 
-def draft_lengths(seed: int, n: int, lo: int = 1, hi: int = 8) -> list[int]:
-    """n integers uniform in {lo..hi} (speculative draft lengths)."""
-    u = uniform(seed, "draft", n)
+def draft_lengths(seed: int, n: int, lo: int = 1, hi: int = 8, start: int = 0) -> list[int]:
+    """n integers uniform in {lo..hi} (speculative draft lengths), elements start..
+    start+n-1 of the stream."""
+    u = uniform(seed, "draft", n, start=start)
     return [lo + int(x * (hi - lo + 1)) for x in u]
 
 
@@ -207,6 +208,82 @@ def randint(seed: int, tag: str, n: int, lo: int, hi: int) -> list[int]:
     """n integers uniform in {lo..hi}."""
     u = uniform(seed, tag, n)
     return [lo + int(x * (hi - lo + 1)) for x in u]
+
+
+# ---------------------------------------------------------------------------
+# The same streams drawn on a CUDA device (torch, int64 with wrapping arithmetic
+# standing in for uint64), for benchmark inputs of tens of GB that the host would
+# take minutes to draw. The bits of every stream are identical to the host's; the
+# fp64 log/cos/sqrt/exp of the device library can differ from the host's in the
+# last bit, so an element can differ by one rounding step after the cast to the I/O
+# type. Parity tests use the host generator above.
+# ---------------------------------------------------------------------------
+def _s64(x: int) -> int:
+    return x - (1 << 64) if x >= (1 << 63) else x
+
+
+_GAMMA_S, _M1_S, _M2_S = _s64(int(GAMMA)), _s64(int(_M1)), _s64(int(_M2))
+
+
+def _srl(z: torch.Tensor, s: int) -> torch.Tensor:
+    return (z >> s) & ((1 << (64 - s)) - 1)
+
+
+def _mix_dev(z: torch.Tensor) -> torch.Tensor:
+    z = (z ^ _srl(z, 30)) * _M1_S
+    z = (z ^ _srl(z, 27)) * _M2_S
+    return z ^ _srl(z, 31)
+
+
+def _normal_dev(key: np.uint64, start: int, n: int, device) -> torch.Tensor:
+    """float64 normals of elements start .. start+n-1 of a stream, on `device`."""
+    k = _s64(int(key))
+    idx = torch.arange(2 * start + 1, 2 * start + 2 * n + 1, dtype=torch.int64, device=device)
+    b = _mix_dev(k + idx * _GAMMA_S)
+    u = (_srl(b, 11).to(torch.float64) + 0.5) * (1.0 / 9007199254740992.0)
+    u1, u2 = u[0::2], u[1::2]
+    return torch.sqrt(-2.0 * torch.log(u1)) * torch.cos(2.0 * math.pi * u2)
+
+
+def _rows_dev(seed, tag, t0, T, H, d, io, device, normalise):
+    out = torch.empty((T, H, d), dtype=torch.bfloat16 if io == "bf16" else torch.float32,
+                      device=device)
+    key = stream_key(seed, TAG[tag])
+    rows = max(1, (1 << 24) // (H * d))
+    for r0 in range(0, T, rows):
+        r1 = min(T, r0 + rows)
+        x = _normal_dev(key, (t0 + r0) * H * d, (r1 - r0) * H * d, device).view(r1 - r0, H, d)
+        if normalise:
+            x = x / torch.sqrt((x * x).sum(dim=-1, keepdim=True))
+        out[r0:r1] = x.float().to(out.dtype)
+    return out
+
+
+def _flat_dev(seed, tag, start, n, device, transform):
+    out = torch.empty(n, dtype=torch.float32, device=device)
+    key = stream_key(seed, TAG[tag])
+    blk = 1 << 24
+    for o in range(0, n, blk):
+        m = min(blk, n - o)
+        out[o:o + m] = transform(_normal_dev(key, start + o, m, device)).float()
+    return out
+
+
+def token_inputs_device(seed: int, T: int, H: int, dk: int, dv: int, io: str = "bf16",
+                        t0: int = 0, device="cuda") -> dict:
+    """token_inputs drawn on a CUDA device (see the note above)."""
+    gate = lambda x: -(torch.clamp(x, min=0.0) + torch.log1p(torch.exp(-x.abs()))) * 0.1  # noqa: E731
+    return {"q": _rows_dev(seed, "q", t0, T, H, dk, io, device, True),
+            "k": _rows_dev(seed, "k", t0, T, H, dk, io, device, True),
+            "v": _rows_dev(seed, "v", t0, T, H, dv, io, device, False),
+            "g": _flat_dev(seed, "g", t0 * H * dk, T * H * dk, device, gate).view(T, H, dk),
+            "beta": _flat_dev(seed, "beta", t0 * H, T * H, device, torch.sigmoid).view(T, H)}
+
+
+def states_device(seed: int, n: int, H: int, dk: int, dv: int, std: float = 0.1,
+                  tag: str = "state", device="cuda") -> torch.Tensor:
+    """states drawn on a CUDA device (see the note above)."""
+    return _flat_dev(seed, tag, 0, n * H * dk * dv, device, lambda z: z * std).view(n, H, dk, dv)
 
 
 # ---------------------------------------------------------------------------

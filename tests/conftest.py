@@ -27,3 +27,10 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.fail("GPU test collected without a CUDA device")
     return torch.device("cuda", 0)
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """Write the parity measures of this session to $KDA_PARITY_REPORT (when set)."""
+    mod = sys.modules.get("kda_cases")
+    if mod is not None:
+        mod.write_report()

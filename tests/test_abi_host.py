@@ -177,6 +177,29 @@ def test_decode_verify_snapshot_validation():
     assert L.kda_snapshot(0, None, None, None, 0, None, 0, 4, 128, 128, None) == 0
 
 
+def test_verify_commit_validation():
+    L = K.lib()
+    d = _dims()
+    cu2 = np.array([0, 3, 5], dtype=np.int32)
+    bad = np.array([0, 3, 2], dtype=np.int32)
+    P = lambda a: a.ctypes.data_as(ctypes.c_void_p)  # noqa: E731
+
+    def call(dims=d, n=2, cp=cu2, cd=cu2, kp=A, na=A, pos=None, snap=0, srow=None, sn=None,
+             q=A, slots=A, pool=A, o=A):
+        return L.kda_verify_commit(ctypes.byref(dims), n, P(cp), kp, A, A, A, na, pos, snap, srow,
+                                   sn, 0, P(cd), q, A, A, A, A, slots, 8, pool, o, None)
+    assert call(dims=_dims(d=48)) == 2                   # unsupported head dim
+    assert call(n=-1) == 1
+    assert call(cp=bad) == 1 and call(cd=bad) == 1       # decreasing offsets
+    assert call(kp=None) == 1                            # previous batch without its tensors
+    assert call(na=None) == 1                            # acceptance counts are required
+    assert call(q=None) == 1
+    assert call(snap=256, srow=A) == 1                   # snapshot rows without positions
+    assert call(o=MIS) == 3
+    assert call(na=MIS) == 3
+    assert call(n=0) == 0
+
+
 def test_no_launch_issued_by_host_tests():
     # the validation failures above must not have launched anything
     assert K.kda_launch_count() == 0

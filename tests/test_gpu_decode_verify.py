@@ -11,7 +11,7 @@ import torch
 
 import synth
 from hybrid_linear_attention_04_b200 import kda as K
-from kda_cases import TOL_BF16, TOL_FP32, blockwise_err, to_np
+from kda_cases import TOL_BF16, TOL_FP32, blockwise_err, check_outputs, check_states, to_np
 from oracle import native
 
 pytestmark = pytest.mark.gpu
@@ -49,9 +49,9 @@ def test_decode_matches_oracle(cuda_device, d, io, H, n_seq):
     assert K.kda_check_device_status() == 0
     o_ref, S_ref = _oracle_decode(x, pool, slots)
     tol = TOL_BF16 if io == "bf16" else TOL_FP32
-    assert blockwise_err(to_np(o), o_ref, (2,)) <= tol
+    check_outputs("o", to_np(o), o_ref, tol, np.arange(n_seq + 1))
     got = to_np(pool_d)
-    assert blockwise_err(got[slots.numpy()], S_ref, (2, 3)) <= tol
+    check_states("state", got[slots.numpy()], S_ref, tol, (2, 3))
     # rows that no sequence uses are untouched, bit for bit
     unused = sorted(set(range(pool.shape[0])) - set(slots.tolist()))
     assert torch.equal(pool_d[unused].cpu(), pool[unused])
@@ -93,12 +93,16 @@ def test_verify_matches_oracle_and_rollback(cuda_device, d, io, H, n_seq):
     assert torch.equal(pool_d.cpu(), pool)           # the source pool is only read
     tol = TOL_BF16 if io == "bf16" else TOL_FP32
     o_got, ts_got = to_np(o), ts.cpu().numpy()
+    o_all, ts_all = np.zeros_like(o_got), np.zeros(ts_got.shape)
     for s in range(n_seq):
         a, b = int(cu[s]), int(cu[s + 1])
         oo, _, sn = native.oracle_sequence(x["q"][a:b], x["k"][a:b], x["v"][a:b], x["g"][a:b],
                                            x["beta"][a:b], pool[int(slots[s])], None, 0, 1)
         assert blockwise_err(o_got[a:b], oo, (2,)) <= tol, s
         assert blockwise_err(ts_got[a:b], sn, (2, 3)) <= tol, s
+        o_all[a:b], ts_all[a:b] = oo, sn
+    check_outputs("o", o_got, o_all, tol, cu)
+    check_states("token states", ts_got, ts_all, tol, (2, 3))
     # rollback: commit the state of a seeded accepted prefix into the live slot
     acc = synth.randint(200 + d, "misc", n_seq, 0, 8)
     src = [int(cu[s]) + min(acc[s], int(cu[s + 1] - cu[s])) - 1 for s in range(n_seq)]

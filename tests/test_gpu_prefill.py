@@ -12,7 +12,8 @@ import torch
 
 import synth
 from hybrid_linear_attention_04_b200 import kda as K
-from kda_cases import blockwise_err, oracle_prefill, packed_inputs, to_np, tol_for
+from kda_cases import (blockwise_err, check_outputs, check_states, oracle_prefill, packed_inputs,
+                       to_np, tol_for)
 
 pytestmark = pytest.mark.gpu
 
@@ -49,18 +50,18 @@ def run_prefill(dev, cu, H, d, chunk, io, start=None, s0=None, snap=0, device=No
     return o, sout, snaps, offs
 
 
-def check(o, sout, snaps, offs, ref, io):
+def check(o, sout, snaps, offs, ref, io, cu=None):
     tol = tol_for(io)
     o_ref, s_ref, sn_ref = ref
-    assert blockwise_err(to_np(o), o_ref, (2,)) <= tol
-    assert blockwise_err(to_np(sout), s_ref, (2, 3)) <= tol
+    check_outputs("o", to_np(o), o_ref, tol, cu)
+    check_states("state", to_np(sout), s_ref, tol, (2, 3))
     n_snap = int(offs[-1])
     got = snaps.cpu().numpy()
     assert sn_ref.shape[0] == n_snap
     assert torch.isnan(snaps[n_snap]).all()                      # spare row untouched
     if n_snap:
         assert not np.isnan(got[:n_snap]).any()
-        assert blockwise_err(got[:n_snap], sn_ref, (2, 3)) <= tol
+        check_states("snapshots", got[:n_snap], sn_ref, tol, (2, 3))
 
 
 def test_tiny_fp32_workload(cuda_device, path):
@@ -81,7 +82,7 @@ def test_ragged_with_state_and_snapshots(cuda_device, path, d, chunk, io):
     snap = 2 * chunk
     o, sout, snaps, offs = run_prefill(dev, cu, H, d, chunk, io, start, s0.to(cuda_device), snap,
                                        cuda_device)
-    check(o, sout, snaps, offs, oracle_prefill(x, cu, start, s0, snap), io)
+    check(o, sout, snaps, offs, oracle_prefill(x, cu, start, s0, snap), io, cu)
 
 
 def test_snapshot_after_every_chunk(cuda_device, path):
@@ -96,7 +97,7 @@ def test_snapshot_after_every_chunk(cuda_device, path):
     o, sout, snaps, offs = run_prefill(dev, cu, H, d, C, "bf16", start, s0.to(cuda_device), C,
                                        cuda_device)
     assert int(offs[-1]) == 3 + 1 + 2 + 0
-    check(o, sout, snaps, offs, oracle_prefill(x, cu, start, s0, C), "bf16")
+    check(o, sout, snaps, offs, oracle_prefill(x, cu, start, s0, C), "bf16", cu)
 
 
 def test_zero_length_sequence_passes_state_through(cuda_device, path):
@@ -167,7 +168,7 @@ def test_more_sequences_than_one_launch(cuda_device, path):
     s0 = synth.states(31, n_seq, H, d, d, std=0.1)
     o, sout, snaps, offs = run_prefill(dev, cu, H, d, 64, "bf16", start, s0.to(cuda_device), 128,
                                        cuda_device)
-    check(o, sout, snaps, offs, oracle_prefill(x, cu, start, s0, 128), "bf16")
+    check(o, sout, snaps, offs, oracle_prefill(x, cu, start, s0, 128), "bf16", cu)
 
 
 @pytest.mark.parametrize("ws", ["auto", None])

@@ -15,7 +15,8 @@ import torch
 import synth
 from hybrid_linear_attention_04_b200 import build as kbuild
 from hybrid_linear_attention_04_b200 import kda as K
-from kda_cases import blockwise_err, oracle_prefill, packed_inputs, to_np, tol_for
+from kda_cases import (blockwise_err, check_outputs, check_states, oracle_prefill, packed_inputs,
+                       to_np, tol_for)
 
 PACKET = 75776      # workspace bytes per (64-token chunk row, head)
 
@@ -70,9 +71,9 @@ def test_fits_in_scratch_two_launches_and_matches(cuda_device):
     assert K.kda_launch_count() - n0 == 2
     ref = oracle_prefill(x, cu, start, s0, 128)
     tol = tol_for("bf16")
-    assert blockwise_err(to_np(got[0]), ref[0], (2,)) <= tol
-    assert blockwise_err(to_np(got[1]), ref[1], (2, 3)) <= tol
-    assert blockwise_err(got[2].cpu().numpy(), ref[2], (2, 3)) <= tol
+    check_outputs("o", to_np(got[0]), ref[0], tol, cu)
+    check_states("state", to_np(got[1]), ref[1], tol, (2, 3))
+    check_states("snapshots", got[2].cpu().numpy(), ref[2], tol, (2, 3))
     ws = torch.empty(K.kda_prefill_workspace_size(dev["q"], dev["v"], cu), dtype=torch.uint8,
                      device=cuda_device)
     again = _run(K.kda_prefill, x, dev, cu, H, d, start, s0, 128, workspace=ws)
@@ -92,12 +93,12 @@ def test_larger_than_scratch_runs_single_launch(cuda_device):
     assert K.kda_launch_count() - n0 == 1
     ref = oracle_prefill(x, cu, None, None, 256)
     tol = tol_for("bf16")
-    # outputs normwise per head over all tokens (as for the 8192-token workload): from a
-    # zero state the first tokens' output rows are tiny, and a per-row ratio would measure
-    # bf16 rounding against a near-zero norm
-    assert blockwise_err(to_np(got[0]), ref[0], (0, 2)) <= tol
-    assert blockwise_err(to_np(got[1]), ref[1], (2, 3)) <= tol
-    assert blockwise_err(got[2].cpu().numpy(), ref[2], (2, 3)) <= tol
+    # outputs per (token, head) row as well as per head: from a zero state the first
+    # tokens' rows scale with q.k, and only an fp32-accurate decayed QK^T keeps them
+    # within the tolerance where that product nearly cancels
+    check_outputs("o", to_np(got[0]), ref[0], tol, cu)
+    check_states("state", to_np(got[1]), ref[1], tol, (2, 3))
+    check_states("snapshots", got[2].cpu().numpy(), ref[2], tol, (2, 3))
     again = _run(K.kda_prefill, x, dev, cu, H, d, None, None, 256, workspace=None)
     for a, b in zip(got, again):
         assert torch.equal(a, b)
