@@ -45,7 +45,83 @@ struct DecodeParams {
     float scale;
     int32_t tok0[kMaxSeqsPerLaunch + 1];  // verify: packed token offsets (relative)
     int64_t tok_base;                     // verify: absolute offset of tok0[0]
+    // q/k front-end (taps == 0: q and k are used as given)
+    int32_t taps;
+    const float *wq, *wk;    // [H, D, taps] conv weights
+    float *conv;             // conv states [n_slots, 2, H, D, taps-1]: decode and verify+commit
+                             // update them in place, verify only reads them
+    float *conv_tok;         // verify: conv state after each token [T, 2, H, D, taps-1] (nullable)
 };
+
+// ---- q/k front-end (Kimi K3 technical FAQ, "What is KDA": queries and keys pass
+// through a short convolution, Swish and L2 normalisation). Per head and key channel,
+// a causal depthwise convolution y_t = sum_j w[j] x_{t-(taps-1)+j} (tap taps-1 on the
+// current token, no bias) over the raw inputs, z = y sigmoid(y), then z / max(|z|, 1e-6)
+// over the d_k channels of the token. The conv state of a sequence is its last taps-1
+// raw inputs, oldest first. Thread c < D owns channel c: its weights and window are
+// registers, and tokens pass through it in order.
+constexpr int kMaxTaps = 4;
+constexpr float kNormEps = 1e-6f;
+
+struct ConvWin {
+    float wq[kMaxTaps], wk[kMaxTaps];
+    float hq[kMaxTaps - 1], hk[kMaxTaps - 1];
+};
+
+__device__ __forceinline__ int64_t conv_index(int64_t row2, int H, int h, int D, int c, int taps) {
+    // row2 = 2 * (slot or token) + (0 for q, 1 for k)
+    return ((row2 * H + h) * D + c) * (int64_t)(taps - 1);
+}
+
+// weights and window of channel c from conv state row `row` (slot or token) of `src`
+__device__ __forceinline__ void conv_begin(ConvWin &w, const DecodeParams &p, const float *src, int64_t row,
+                                           int h, int D, int c) {
+    const int K = p.taps;
+#pragma unroll
+    for (int j = 0; j < kMaxTaps; ++j) {
+        w.wq[j] = j < K ? p.wq[((int64_t)h * D + c) * K + j] : 0.f;
+        w.wk[j] = j < K ? p.wk[((int64_t)h * D + c) * K + j] : 0.f;
+    }
+    const float *sq = src + conv_index(2 * row, p.H, h, D, c, K);
+    const float *sk = src + conv_index(2 * row + 1, p.H, h, D, c, K);
+#pragma unroll
+    for (int j = 0; j < kMaxTaps - 1; ++j) {
+        w.hq[j] = j < K - 1 ? sq[j] : 0.f;
+        w.hk[j] = j < K - 1 ? sk[j] : 0.f;
+    }
+}
+
+__device__ __forceinline__ void conv_store(const ConvWin &w, const DecodeParams &p, float *dst, int64_t row,
+                                           int h, int D, int c) {
+    const int K = p.taps;
+    float *dq = dst + conv_index(2 * row, p.H, h, D, c, K);
+    float *dk = dst + conv_index(2 * row + 1, p.H, h, D, c, K);
+#pragma unroll
+    for (int j = 0; j < kMaxTaps - 1; ++j)
+        if (j < K - 1) { dq[j] = w.hq[j]; dk[j] = w.hk[j]; }
+}
+
+// one causal conv step of raw input x through weights wt and window hs (shifted in place)
+// (every index is a compile-time constant after unrolling, so window and weights stay
+// in registers)
+__device__ __forceinline__ float conv_step(const float (&wt)[kMaxTaps], float (&hs)[kMaxTaps - 1], int K, float x) {
+    float wl = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxTaps; ++j)
+        if (j == K - 1) wl = wt[j];
+    float y = wl * x;
+#pragma unroll
+    for (int j = 0; j < kMaxTaps - 1; ++j)
+        if (j < K - 1) y = fmaf(wt[j], hs[j], y);
+#pragma unroll
+    for (int j = 0; j < kMaxTaps - 1; ++j) {
+        if (j < K - 2) hs[j] = hs[j + 1];
+        else if (j == K - 2) hs[j] = x;
+    }
+    return y;
+}
+
+__device__ __forceinline__ float swish(float y) { return y / (1.f + expf(-y)); }
 
 // Per-token vectors staged in shared memory. 16-byte aligned (and padded to a
 // multiple of 16 bytes) because the step reads v with float4 loads.
@@ -78,16 +154,67 @@ __device__ __forceinline__ void load_token(TokVec<D> &tv, const DecodeParams &p,
     load_vectors<D, TIO>(tv, p.q, p.k, p.v, p.g, p.beta, row);
 }
 
+// Stage a token whose raw q, k pass through the front-end: the conv and Swish here
+// (thread c < D, channel c, window w), the L2 normalisation in token_finish. With
+// q_ == nullptr only the q window advances (a token whose output is not needed still
+// moves the conv state).
+template <int D, typename TIO>
+__device__ __forceinline__ void load_vectors_conv(TokVec<D> &tv, ConvWin &w, int K, const void *q_, const void *k_,
+                                                  const void *v_, const float *g_, const float *beta,
+                                                  int64_t row, bool want_q) {
+    const int c = threadIdx.x;
+    if (c < D) {
+        const float xq = IO<TIO>::ld(static_cast<const TIO *>(q_) + row * D + c);
+        const float xk = IO<TIO>::ld(static_cast<const TIO *>(k_) + row * D + c);
+        const float yq = conv_step(w.wq, w.hq, K, xq);
+        const float yk = conv_step(w.wk, w.hk, K, xk);
+        tv.q[c] = want_q ? swish(yq) : 0.f;
+        tv.k[c] = swish(yk);
+        tv.v[c] = IO<TIO>::ld(static_cast<const TIO *>(v_) + row * D + c);
+        tv.a[c] = expf(g_[row * D + c]);
+    }
+    if (threadIdx.x == 0) tv.beta = beta[row];
+}
+
+// One warp finishes a staged token: L2-normalises k and q when the front-end is on,
+// then k . q (fixed reduction order) when q is used.
+template <int D>
+__device__ __forceinline__ void token_finish(TokVec<D> &tv, bool normalise, bool with_q) {
+    const int lane = threadIdx.x & 31;
+    if (normalise) {
+        float sk = 0.f, sq = 0.f;
+#pragma unroll
+        for (int i = lane; i < D; i += 32) {
+            sk = fmaf(tv.k[i], tv.k[i], sk);
+            sq = fmaf(tv.q[i], tv.q[i], sq);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            sk += __shfl_xor_sync(0xffffffffu, sk, off);
+            sq += __shfl_xor_sync(0xffffffffu, sq, off);
+        }
+        const float rk = 1.f / fmaxf(sqrtf(sk), kNormEps), rq = 1.f / fmaxf(sqrtf(sq), kNormEps);
+#pragma unroll
+        for (int i = lane; i < D; i += 32) {
+            tv.k[i] *= rk;
+            tv.q[i] *= rq;
+        }
+        __syncwarp();
+    }
+    if (with_q) {
+        float s = 0.f;
+#pragma unroll
+        for (int i = lane; i < D; i += 32) s = fmaf(tv.k[i], tv.q[i], s);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (lane == 0) tv.kq = s;
+    }
+}
+
 // k . q for a staged token, by one warp, fixed reduction order.
 template <int D>
 __device__ __forceinline__ void token_kq(TokVec<D> &tv) {
-    int lane = threadIdx.x & 31;
-    float s = 0.f;
-#pragma unroll
-    for (int i = lane; i < D; i += 32) s = fmaf(tv.k[i], tv.q[i], s);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    if (lane == 0) tv.kq = s;
+    token_finish<D>(tv, false, true);
 }
 
 // One recurrence step on the register-resident state. red: [NW][2][D] scratch
@@ -187,9 +314,16 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
                      : "l"(src));
     }
     const int64_t row = (int64_t)s * p.H + h;
-    load_token<D, TIO>(tv, p, row);
+    if (p.taps) {
+        ConvWin w;
+        if (t < D) conv_begin(w, p, p.conv, slot, h, D, t);
+        load_vectors_conv<D, TIO>(tv, w, p.taps, p.q, p.k, p.v, p.g, p.beta, row, true);
+        if (t < D) conv_store(w, p, p.conv, slot, h, D, t);
+    } else {
+        load_token<D, TIO>(tv, p, row);
+    }
     __syncthreads();
-    if (t < 32) token_kq<D>(tv);
+    if (t < 32) token_finish<D>(tv, p.taps > 0, true);
     __syncthreads();
     const float4 o = kda_step<D>(st, tv, red, p.scale);
 #pragma unroll
@@ -221,16 +355,25 @@ verify_kernel(const __grid_constant__ DecodeParams p) {
     float4 st[Sh::R];
 #pragma unroll
     for (int m = 0; m < Sh::R; ++m) st[m] = ld_stream(S + (int64_t)(rs + Sh::RS * m) * D + cg * 4);
+    ConvWin w;
+    if (p.taps && t < D) conv_begin(w, p, p.conv, slot, h, D, t);
     int parity = 0;
     for (int j0 = 0; j0 < n_tok; j0 += kTokBatch) {
         const int nb = min(kTokBatch, n_tok - j0);
         __syncthreads();  // previous batch's vectors are no longer read
-        for (int j = 0; j < nb; ++j)
-            load_token<D, TIO>(tv[j], p, (tok_first + j0 + j) * p.H + h);
+        for (int j = 0; j < nb; ++j) {
+            const int64_t tok = tok_first + j0 + j;
+            if (p.taps) {
+                load_vectors_conv<D, TIO>(tv[j], w, p.taps, p.q, p.k, p.v, p.g, p.beta, tok * p.H + h, true);
+                if (p.conv_tok && t < D) conv_store(w, p, p.conv_tok, tok, h, D, t);
+            } else {
+                load_token<D, TIO>(tv[j], p, tok * p.H + h);
+            }
+        }
         __syncthreads();
-        if (warp < nb) token_kq<D>(tv[warp]);
+        if (warp < nb) token_finish<D>(tv[warp], p.taps > 0, true);
         for (int j = Sh::NW; j < nb; ++j)
-            if (warp == 0) token_kq<D>(tv[j]);
+            if (warp == 0) token_finish<D>(tv[j], p.taps > 0, true);
         __syncthreads();
         for (int j = 0; j < nb; ++j) {
             const float4 o = kda_step<D>(st, tv[j], red[parity], p.scale);
@@ -255,6 +398,8 @@ namespace kda {
 // only), it is written back once, and this step's draft tokens run from it with
 // outputs only. No per-token state is written.
 struct CommitParams {
+    const void *q;              // the previous step's raw q (front-end on: advances the q window)
+    float *conv_snapshots;      // front-end on: conv state at the boundary [rows, 2, H, D, taps-1]
     const void *k, *v;          // the previous step's tokens (packed like verify's)
     const float *g, *beta;
     const int32_t *n_accept;    // [n_seq] leading tokens of the previous batch to commit
@@ -305,14 +450,29 @@ verify_commit_kernel(const __grid_constant__ VerifyCommitParams P) {
                      : "l"(src));
     }
     int parity = 0;
+    ConvWin w;
+    if (p.taps && t < D) conv_begin(w, p, p.conv, slot, h, D, t);
     // 1. commit: replay the accepted prefix of the previous batch (state only)
     const int64_t prev_first = c.tok_base + c.tok0[s];
     for (int j0 = 0; j0 < na; j0 += kTokBatch) {
         const int nb = min(kTokBatch, na - j0);
         __syncthreads();
-        for (int j = 0; j < nb; ++j)
-            load_vectors<D, TIO>(tv[j], nullptr, c.k, c.v, c.g, c.beta, (prev_first + j0 + j) * p.H + h);
+        for (int j = 0; j < nb; ++j) {
+            const int64_t row = (prev_first + j0 + j) * p.H + h;
+            if (p.taps) {
+                load_vectors_conv<D, TIO>(tv[j], w, p.taps, c.q, c.k, c.v, c.g, c.beta, row, false);
+                if (j0 + j == jsnap && t < D) conv_store(w, p, c.conv_snapshots, srow, h, D, t);
+            } else {
+                load_vectors<D, TIO>(tv[j], nullptr, c.k, c.v, c.g, c.beta, row);
+            }
+        }
         __syncthreads();
+        if (p.taps) {
+            if (warp < nb) token_finish<D>(tv[warp], true, false);
+            for (int j = Sh::NW; j < nb; ++j)
+                if (warp == 0) token_finish<D>(tv[j], true, false);
+            __syncthreads();
+        }
         for (int j = 0; j < nb; ++j) {
             kda_step<D, false>(st, tv[j], red[parity], 0.f);
             parity ^= 1;
@@ -326,6 +486,7 @@ verify_commit_kernel(const __grid_constant__ VerifyCommitParams P) {
     if (na > 0) {
 #pragma unroll
         for (int m = 0; m < Sh::R; ++m) st_stream(S + (int64_t)(rs + Sh::RS * m) * D + cg * 4, st[m]);
+        if (p.taps && t < D) conv_store(w, p, p.conv, slot, h, D, t);
     }
     // 2. verify this step's tokens from the committed state: outputs only
     const int n_tok = p.tok0[s + 1] - p.tok0[s];
@@ -333,12 +494,17 @@ verify_commit_kernel(const __grid_constant__ VerifyCommitParams P) {
     for (int j0 = 0; j0 < n_tok; j0 += kTokBatch) {
         const int nb = min(kTokBatch, n_tok - j0);
         __syncthreads();
-        for (int j = 0; j < nb; ++j)
-            load_token<D, TIO>(tv[j], p, (tok_first + j0 + j) * p.H + h);
+        for (int j = 0; j < nb; ++j) {
+            const int64_t row = (tok_first + j0 + j) * p.H + h;
+            if (p.taps)
+                load_vectors_conv<D, TIO>(tv[j], w, p.taps, p.q, p.k, p.v, p.g, p.beta, row, true);
+            else
+                load_token<D, TIO>(tv[j], p, row);
+        }
         __syncthreads();
-        if (warp < nb) token_kq<D>(tv[warp]);
+        if (warp < nb) token_finish<D>(tv[warp], p.taps > 0, true);
         for (int j = Sh::NW; j < nb; ++j)
-            if (warp == 0) token_kq<D>(tv[j]);
+            if (warp == 0) token_finish<D>(tv[j], p.taps > 0, true);
         __syncthreads();
         for (int j = 0; j < nb; ++j) {
             const float4 o = kda_step<D>(st, tv[j], red[parity], p.scale);

@@ -13,10 +13,12 @@
 
 #include "common.cuh"
 #include "decode.cuh"
+#include "frontend.cuh"
 #include "prefill_simt.cuh"
 #include "prefill_tc.cuh"
 #include "prefill_split.cuh"
 #include "snapshot.cuh"
+#include "statemap.cuh"
 
 namespace kda {
 
@@ -113,6 +115,17 @@ static kda_status dispatch_simt(int D, int C, const PrefillParams &p, cudaStream
     KDA_CASE(128, 16) KDA_CASE(128, 32) KDA_CASE(128, 64)
 #undef KDA_CASE
     return KDA_ERR_UNSUPPORTED;
+}
+
+template <int D, typename TIO>
+static kda_status launch_frontend(const FrontendParams &P, int64_t n_blocks, cudaStream_t st) {
+    static std::atomic<unsigned long long> attr_done{0};
+    const kda_status r = set_smem_limit_once((const void *)qk_frontend_kernel<D, TIO>,
+                                             (int)FrontendShape<D>::smem_bytes, attr_done);
+    if (r != KDA_OK) return r;
+    if (!launch_gate()) return KDA_ERR_CUDA;
+    qk_frontend_kernel<D, TIO><<<(unsigned)n_blocks, D, FrontendShape<D>::smem_bytes, st>>>(P);
+    return last_launch_status();
 }
 
 // Forced path selection for tests: 0 = automatic, 1 = CUDA-core path only.
@@ -300,34 +313,72 @@ kda_status kda_prefill_noalloc(const kda_dims *dims, int32_t n_seq, const int32_
 
 size_t kda_prefill_noalloc_capacity(void) { return kNoallocScratchBytes; }
 
-kda_status kda_decode(const kda_dims *dims, int32_t n_seq, const void *q, const void *k,
-                      const void *v, const float *g, const float *beta, const int32_t *slots,
-                      int32_t n_slots, float *pool, void *o, kda_stream_t stream) {
+static kda_status check_conv(const kda_conv *conv) {
+    if (!conv) return KDA_OK;
+    if (conv->taps < 2 || conv->taps > kMaxTaps || !conv->w_q || !conv->w_k) return KDA_ERR_INVALID;
+    if (!aligned16(conv->w_q) || !aligned16(conv->w_k)) return KDA_ERR_ALIGN;
+    return KDA_OK;
+}
+
+static void set_conv(DecodeParams &p, const kda_conv *conv, float *pool, float *tok) {
+    p.taps = conv ? conv->taps : 0;
+    p.wq = conv ? conv->w_q : nullptr;
+    p.wk = conv ? conv->w_k : nullptr;
+    p.conv = conv ? pool : nullptr;
+    p.conv_tok = conv ? tok : nullptr;
+}
+
+static kda_status decode_impl(const kda_dims *dims, const kda_conv *conv, int32_t n_seq,
+                              const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, const int32_t *slots, int32_t n_slots, float *pool,
+                              float *conv_pool, void *o, kda_stream_t stream) {
     kda_status st = check_dims(dims, false);
     if (st != KDA_OK) return st;
+    if ((st = check_conv(conv)) != KDA_OK) return st;
     if (n_seq < 0 || n_slots < 0) return KDA_ERR_INVALID;
     if (n_seq == 0) return KDA_OK;
     if (!q || !k || !v || !g || !beta || !slots || !pool || !o) return KDA_ERR_INVALID;
-    const void *ptrs[] = {q, k, v, g, beta, slots, pool, o};
+    if (conv && !conv_pool) return KDA_ERR_INVALID;
+    const void *ptrs[] = {q, k, v, g, beta, slots, pool, o, conv_pool};
     for (const void *ptr : ptrs)
-        if (!aligned16(ptr)) return KDA_ERR_ALIGN;
+        if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
     if ((int64_t)n_seq * dims->H > 0x7fffffffLL) return KDA_ERR_INVALID;
     static thread_local DecodeParams p;
     std::memset(&p, 0, sizeof(p));
     p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.slots = slots; p.pool = pool; p.o = o;
     p.n_seq = n_seq; p.H = dims->H; p.n_slots = n_slots; p.scale = eff_scale(dims);
+    set_conv(p, conv, conv_pool, nullptr);
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     return dims->io == KDA_IO_BF16
                ? dispatch_decode<__nv_bfloat16>(dims->dk, p, n_seq * dims->H, cs, false)
                : dispatch_decode<float>(dims->dk, p, n_seq * dims->H, cs, false);
 }
 
-kda_status kda_verify(const kda_dims *dims, int32_t n_seq, const int32_t *cu_draft,
-                      const void *q, const void *k, const void *v, const float *g,
-                      const float *beta, const int32_t *slots, int32_t n_slots,
-                      const float *pool, float *token_states, void *o, kda_stream_t stream) {
+kda_status kda_decode(const kda_dims *dims, int32_t n_seq, const void *q, const void *k,
+                      const void *v, const float *g, const float *beta, const int32_t *slots,
+                      int32_t n_slots, float *pool, void *o, kda_stream_t stream) {
+    return decode_impl(dims, nullptr, n_seq, q, k, v, g, beta, slots, n_slots, pool, nullptr, o,
+                       stream);
+}
+
+kda_status kda_decode_conv(const kda_dims *dims, const kda_conv *conv, int32_t n_seq,
+                           const void *q, const void *k, const void *v, const float *g,
+                           const float *beta, const int32_t *slots, int32_t n_slots,
+                           float *pool, float *conv_pool, void *o, kda_stream_t stream) {
+    if (!conv) return KDA_ERR_INVALID;
+    return decode_impl(dims, conv, n_seq, q, k, v, g, beta, slots, n_slots, pool, conv_pool, o,
+                       stream);
+}
+
+static kda_status verify_impl(const kda_dims *dims, const kda_conv *conv, int32_t n_seq,
+                              const int32_t *cu_draft, const void *q, const void *k, const void *v,
+                              const float *g, const float *beta, const int32_t *slots,
+                              int32_t n_slots, const float *pool, const float *conv_pool,
+                              float *token_states, float *conv_tok, void *o, kda_stream_t stream) {
     kda_status st = check_dims(dims, false);
     if (st != KDA_OK) return st;
+    if ((st = check_conv(conv)) != KDA_OK) return st;
+    if (conv && !conv_pool) return KDA_ERR_INVALID;
     if (n_seq < 0 || n_slots < 0) return KDA_ERR_INVALID;
     if (n_seq == 0) return KDA_OK;
     if (!cu_draft || cu_draft[0] != 0) return KDA_ERR_INVALID;
@@ -336,7 +387,7 @@ kda_status kda_verify(const kda_dims *dims, int32_t n_seq, const int32_t *cu_dra
     const int64_t T = cu_draft[n_seq];
     if (!slots || !pool) return KDA_ERR_INVALID;
     if (T > 0 && (!q || !k || !v || !g || !beta || !token_states || !o)) return KDA_ERR_INVALID;
-    const void *ptrs[] = {q, k, v, g, beta, slots, pool, token_states, o};
+    const void *ptrs[] = {q, k, v, g, beta, slots, pool, token_states, o, conv_pool, conv_tok};
     for (const void *ptr : ptrs)
         if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
@@ -348,6 +399,7 @@ kda_status kda_verify(const kda_dims *dims, int32_t n_seq, const int32_t *cu_dra
         p.pool = const_cast<float *>(pool); p.token_states = token_states; p.o = o;
         p.n_seq = ng; p.H = dims->H; p.n_slots = n_slots; p.scale = eff_scale(dims);
         p.tok_base = cu_draft[g0];
+        set_conv(p, conv, const_cast<float *>(conv_pool), conv_tok);
         for (int i = 0; i <= ng; ++i) p.tok0[i] = cu_draft[g0 + i] - cu_draft[g0];
         st = dims->io == KDA_IO_BF16
                  ? dispatch_decode<__nv_bfloat16>(dims->dk, p, ng * dims->H, cs, true)
@@ -357,16 +409,37 @@ kda_status kda_verify(const kda_dims *dims, int32_t n_seq, const int32_t *cu_dra
     return KDA_OK;
 }
 
-kda_status kda_verify_commit(const kda_dims *dims, int32_t n_seq, const int32_t *cu_prev,
-                             const void *k_prev, const void *v_prev, const float *g_prev,
-                             const float *beta_prev, const int32_t *n_accept, const int64_t *pos,
-                             int32_t snap_interval, const int64_t *snap_row, float *snapshots,
-                             int64_t n_snap_rows, const int32_t *cu_draft, const void *q,
-                             const void *k, const void *v, const float *g, const float *beta,
-                             const int32_t *slots, int32_t n_slots, float *pool, void *o,
-                             kda_stream_t stream) {
+kda_status kda_verify(const kda_dims *dims, int32_t n_seq, const int32_t *cu_draft,
+                      const void *q, const void *k, const void *v, const float *g,
+                      const float *beta, const int32_t *slots, int32_t n_slots,
+                      const float *pool, float *token_states, void *o, kda_stream_t stream) {
+    return verify_impl(dims, nullptr, n_seq, cu_draft, q, k, v, g, beta, slots, n_slots, pool,
+                       nullptr, token_states, nullptr, o, stream);
+}
+
+kda_status kda_verify_conv(const kda_dims *dims, const kda_conv *conv, int32_t n_seq,
+                           const int32_t *cu_draft, const void *q, const void *k, const void *v,
+                           const float *g, const float *beta, const int32_t *slots,
+                           int32_t n_slots, const float *pool, const float *conv_pool,
+                           float *token_states, float *conv_token_states, void *o,
+                           kda_stream_t stream) {
+    if (!conv) return KDA_ERR_INVALID;
+    return verify_impl(dims, conv, n_seq, cu_draft, q, k, v, g, beta, slots, n_slots, pool,
+                       conv_pool, token_states, conv_token_states, o, stream);
+}
+
+static kda_status verify_commit_impl(
+    const kda_dims *dims, const kda_conv *conv, int32_t n_seq, const int32_t *cu_prev,
+    const void *q_prev, const void *k_prev, const void *v_prev, const float *g_prev,
+    const float *beta_prev, const int32_t *n_accept, const int64_t *pos, int32_t snap_interval,
+    const int64_t *snap_row, float *snapshots, float *conv_snapshots, int64_t n_snap_rows,
+    const int32_t *cu_draft, const void *q, const void *k, const void *v, const float *g,
+    const float *beta, const int32_t *slots, int32_t n_slots, float *pool, float *conv_pool,
+    void *o, kda_stream_t stream) {
     kda_status st = check_dims(dims, false);
     if (st != KDA_OK) return st;
+    if ((st = check_conv(conv)) != KDA_OK) return st;
+    if (conv && !conv_pool) return KDA_ERR_INVALID;
     if (n_seq < 0 || n_slots < 0 || snap_interval < 0 || n_snap_rows < 0) return KDA_ERR_INVALID;
     if (n_seq == 0) return KDA_OK;
     if (!cu_prev || !cu_draft || cu_prev[0] != 0 || cu_draft[0] != 0) return KDA_ERR_INVALID;
@@ -374,11 +447,13 @@ kda_status kda_verify_commit(const kda_dims *dims, int32_t n_seq, const int32_t 
         if (cu_prev[s + 1] < cu_prev[s] || cu_draft[s + 1] < cu_draft[s]) return KDA_ERR_INVALID;
     const int64_t Tp = cu_prev[n_seq], T = cu_draft[n_seq];
     if (!slots || !pool || !n_accept) return KDA_ERR_INVALID;
-    if (Tp > 0 && (!k_prev || !v_prev || !g_prev || !beta_prev)) return KDA_ERR_INVALID;
+    if (Tp > 0 && (!k_prev || !v_prev || !g_prev || !beta_prev || (conv && !q_prev)))
+        return KDA_ERR_INVALID;
     if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID;
-    if (snap_interval > 0 && snap_row && (!pos || !snapshots)) return KDA_ERR_INVALID;
-    const void *ptrs[] = {k_prev, v_prev, g_prev, beta_prev, n_accept, pos, snap_row, snapshots,
-                          q, k, v, g, beta, slots, pool, o};
+    if (snap_interval > 0 && snap_row && (!pos || !snapshots || (conv && !conv_snapshots)))
+        return KDA_ERR_INVALID;
+    const void *ptrs[] = {q_prev, k_prev, v_prev, g_prev, beta_prev, n_accept, pos, snap_row,
+                          snapshots, conv_snapshots, q, k, v, g, beta, slots, pool, conv_pool, o};
     for (const void *ptr : ptrs)
         if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
@@ -392,7 +467,10 @@ kda_status kda_verify_commit(const kda_dims *dims, int32_t n_seq, const int32_t 
         p.n_seq = ng; p.H = dims->H; p.n_slots = n_slots; p.scale = eff_scale(dims);
         p.tok_base = cu_draft[g0];
         for (int i = 0; i <= ng; ++i) p.tok0[i] = cu_draft[g0 + i] - cu_draft[g0];
+        set_conv(p, conv, conv_pool, nullptr);
         CommitParams &c = P.c;
+        c.q = conv ? q_prev : nullptr;
+        c.conv_snapshots = conv ? conv_snapshots : nullptr;
         c.k = k_prev; c.v = v_prev; c.g = g_prev; c.beta = beta_prev;
         c.n_accept = n_accept + g0;
         c.pos = pos ? pos + g0 : nullptr;
@@ -402,6 +480,95 @@ kda_status kda_verify_commit(const kda_dims *dims, int32_t n_seq, const int32_t 
         for (int i = 0; i <= ng; ++i) c.tok0[i] = cu_prev[g0 + i] - cu_prev[g0];
         st = dims->io == KDA_IO_BF16 ? dispatch_verify_commit<__nv_bfloat16>(dims->dk, P, ng * dims->H, cs)
                                      : dispatch_verify_commit<float>(dims->dk, P, ng * dims->H, cs);
+        if (st != KDA_OK) return st;
+    }
+    return KDA_OK;
+}
+
+kda_status kda_verify_commit(const kda_dims *dims, int32_t n_seq, const int32_t *cu_prev,
+                             const void *k_prev, const void *v_prev, const float *g_prev,
+                             const float *beta_prev, const int32_t *n_accept, const int64_t *pos,
+                             int32_t snap_interval, const int64_t *snap_row, float *snapshots,
+                             int64_t n_snap_rows, const int32_t *cu_draft, const void *q,
+                             const void *k, const void *v, const float *g, const float *beta,
+                             const int32_t *slots, int32_t n_slots, float *pool, void *o,
+                             kda_stream_t stream) {
+    return verify_commit_impl(dims, nullptr, n_seq, cu_prev, nullptr, k_prev, v_prev, g_prev,
+                              beta_prev, n_accept, pos, snap_interval, snap_row, snapshots, nullptr,
+                              n_snap_rows, cu_draft, q, k, v, g, beta, slots, n_slots, pool,
+                              nullptr, o, stream);
+}
+
+kda_status kda_verify_commit_conv(const kda_dims *dims, const kda_conv *conv, int32_t n_seq,
+                                  const int32_t *cu_prev, const void *q_prev, const void *k_prev,
+                                  const void *v_prev, const float *g_prev, const float *beta_prev,
+                                  const int32_t *n_accept, const int64_t *pos,
+                                  int32_t snap_interval, const int64_t *snap_row,
+                                  float *snapshots, float *conv_snapshots, int64_t n_snap_rows,
+                                  const int32_t *cu_draft, const void *q, const void *k,
+                                  const void *v, const float *g, const float *beta,
+                                  const int32_t *slots, int32_t n_slots, float *pool,
+                                  float *conv_pool, void *o, kda_stream_t stream) {
+    if (!conv) return KDA_ERR_INVALID;
+    return verify_commit_impl(dims, conv, n_seq, cu_prev, q_prev, k_prev, v_prev, g_prev,
+                              beta_prev, n_accept, pos, snap_interval, snap_row, snapshots,
+                              conv_snapshots, n_snap_rows, cu_draft, q, k, v, g, beta, slots,
+                              n_slots, pool, conv_pool, o, stream);
+}
+
+kda_status kda_qk_frontend(const kda_dims *dims, const kda_conv *conv, int32_t n_seq,
+                           const int32_t *cu, const int64_t *start_pos, const void *q,
+                           const void *k, const float *conv_in, float *conv_out, void *q_out,
+                           void *k_out, int32_t snap_interval, float *conv_snapshots,
+                           kda_stream_t stream) {
+    kda_status st = check_dims(dims, true);
+    if (st != KDA_OK) return st;
+    if (!conv) return KDA_ERR_INVALID;
+    if ((st = check_conv(conv)) != KDA_OK) return st;
+    if (n_seq < 0 || snap_interval < 0) return KDA_ERR_INVALID;
+    if (n_seq == 0) return KDA_OK;
+    if (!cu) return KDA_ERR_INVALID;
+    const int C = dims->chunk, D = dims->dk, H = dims->H;
+    std::vector<int64_t> offs(n_seq + 1);
+    st = kda_snapshot_plan(n_seq, cu, start_pos, snap_interval, offs.data(), nullptr);
+    if (st != KDA_OK) return st;
+    if (snap_interval > 0) {
+        if (snap_interval % C != 0) return KDA_ERR_INVALID;
+        for (int s = 0; s < n_seq && start_pos; ++s)
+            if (start_pos[s] % C != 0) return KDA_ERR_INVALID;
+    }
+    const int64_t T = cu[n_seq];
+    if (T > 0 && (!q || !k || !q_out || !k_out)) return KDA_ERR_INVALID;
+    if (offs[n_seq] > 0 && !conv_snapshots) return KDA_ERR_INVALID;
+    const void *ptrs[] = {q, k, conv_in, conv_out, q_out, k_out, conv_snapshots};
+    for (const void *ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    static thread_local FrontendParams P;
+    const int64_t cstate = (int64_t)2 * H * D * (conv->taps - 1);
+    for (int g0 = 0; g0 < n_seq; g0 += kPrefillSeqs) {
+        const int ng = std::min(kPrefillSeqs, n_seq - g0);
+        std::memset(&P, 0, sizeof(P));
+        P.q = q; P.k = k; P.q_out = q_out; P.k_out = k_out; P.wq = conv->w_q; P.wk = conv->w_k;
+        P.conv_in = conv_in ? conv_in + g0 * cstate : nullptr;
+        P.conv_out = conv_out ? conv_out + g0 * cstate : nullptr;
+        P.conv_snap = conv_snapshots;
+        P.H = H; P.taps = conv->taps; P.n_seq = ng; P.C = C; P.tok_first = cu[g0];
+        P.snap_interval = snap_interval;
+        for (int i = 0; i < ng; ++i) {
+            P.tok0[i] = cu[g0 + i];
+            P.len[i] = cu[g0 + i + 1] - cu[g0 + i];
+            P.start_pos[i] = start_pos ? start_pos[g0 + i] : 0;
+            P.snap_off[i] = offs[g0 + i];
+        }
+        const int64_t rows = ((int64_t)cu[g0 + ng] - cu[g0]) / C + ng;
+        if (rows * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+        const bool bf = dims->io == KDA_IO_BF16;
+        switch (D) {
+        case 32: st = bf ? launch_frontend<32, __nv_bfloat16>(P, rows * H, cs) : launch_frontend<32, float>(P, rows * H, cs); break;
+        case 64: st = bf ? launch_frontend<64, __nv_bfloat16>(P, rows * H, cs) : launch_frontend<64, float>(P, rows * H, cs); break;
+        default: st = bf ? launch_frontend<128, __nv_bfloat16>(P, rows * H, cs) : launch_frontend<128, float>(P, rows * H, cs); break;
+        }
         if (st != KDA_OK) return st;
     }
     return KDA_OK;
@@ -432,6 +599,23 @@ kda_status kda_snapshot(int32_t n, const int64_t *src_idx, const int64_t *dst_id
         if (st != KDA_OK) return st;
     }
     return KDA_OK;
+}
+
+kda_status kda_state_map_apply(int64_t n, int32_t dk, int32_t dv, const float *M, const float *X,
+                               const float *N, float *out, kda_stream_t stream) {
+    if (n < 0 || dk < 1 || dv < 1) return KDA_ERR_INVALID;
+    if (n == 0) return KDA_OK;
+    if (!M || !X || !out) return KDA_ERR_INVALID;
+    if (out == X || out == M) return KDA_ERR_INVALID;      // out may alias N only
+    const void *ptrs[] = {M, X, N, out};
+    for (const void *ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
+    const int64_t tiles = (int64_t)((dk + 63) / 64) * ((dv + 63) / 64);
+    if (n * tiles > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    StateMapParams p{M, X, N, out, n, dk, dv};
+    if (!launch_gate()) return KDA_ERR_CUDA;
+    state_map_kernel<<<(unsigned)(n * tiles), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+    return last_launch_status();
 }
 
 kda_status kda_check_device_status(kda_stream_t stream) {

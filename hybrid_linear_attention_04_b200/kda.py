@@ -35,6 +35,10 @@ class kda_dims(ctypes.Structure):
                 ("chunk", ctypes.c_int32), ("io", ctypes.c_int32), ("scale", ctypes.c_float)]
 
 
+class kda_conv(ctypes.Structure):
+    _fields_ = [("taps", ctypes.c_int32), ("w_q", ctypes.c_void_p), ("w_k", ctypes.c_void_p)]
+
+
 _P = ctypes.c_void_p
 _I32, _I64 = ctypes.c_int32, ctypes.c_int64
 
@@ -50,6 +54,13 @@ _SIGNATURES = {
     "kda_verify_commit": (_I32, [_P, _I32, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _I64, _P, _P,
                                  _P, _P, _P, _P, _P, _I32, _P, _P, _P]),
     "kda_snapshot": (_I32, [_I32, _P, _P, _P, _I64, _P, _I64, _I32, _I32, _I32, _P]),
+    "kda_state_map_apply": (_I32, [_I64, _I32, _I32, _P, _P, _P, _P, _P]),
+    "kda_qk_frontend": (_I32, [_P, _P, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P]),
+    "kda_decode_conv": (_I32, [_P, _P, _I32, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P]),
+    "kda_verify_conv": (_I32, [_P, _P, _I32, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P, _P,
+                               _P]),
+    "kda_verify_commit_conv": (_I32, [_P, _P, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P,
+                                      _P, _I64, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P]),
     "kda_status_string": (ctypes.c_char_p, [_I32]),
     "kda_check_device_status": (_I32, [_P]),
     "kda_launch_count": (_I64, []),
@@ -237,6 +248,86 @@ def kda_verify_commit(prev, n_accept, cu_prev, q, k, v, g, beta, cu_draft, slots
         _dptr(snap_row), _dptr(snapshots), n_rows, _hptr(cd), _dptr(q), _dptr(k), _dptr(v),
         _dptr(g), _dptr(beta), _dptr(slots), state_pool.shape[0], _dptr(state_pool), _dptr(o),
         _stream(stream)), "kda_verify_commit")
+
+
+def _conv(w_q, w_k):
+    """kda_conv for weight tensors [H, dk, taps] (fp32, device)."""
+    if w_q.shape != w_k.shape or w_q.dtype != torch.float32:
+        raise KDAError(1, "conv weights must be fp32 [H, dk, taps], the same for q and k")
+    _dptr(w_q), _dptr(w_k)
+    return kda_conv(int(w_q.shape[-1]), w_q.data_ptr(), w_k.data_ptr())
+
+
+def kda_qk_frontend(q_raw, k_raw, w_q, w_k, cu_seqlens, q_out, k_out, conv_in=None,
+                    conv_out=None, start_pos=None, snap_interval=0, conv_snapshots=None,
+                    chunk=64, stream=None):
+    """Short conv + Swish + L2 front-end of a packed prefill batch (see include/kda.h)."""
+    cu = _host_array(cu_seqlens, np.int32)
+    sp = _host_array(start_pos, np.int64)
+    dims = _dims(q_raw, q_raw, chunk)
+    conv = _conv(w_q, w_k)
+    _check(lib().kda_qk_frontend(ctypes.byref(dims), ctypes.byref(conv), len(cu) - 1, _hptr(cu),
+                                 _hptr(sp), _dptr(q_raw), _dptr(k_raw), _dptr(conv_in),
+                                 _dptr(conv_out), _dptr(q_out), _dptr(k_out), int(snap_interval),
+                                 _dptr(conv_snapshots), _stream(stream)), "kda_qk_frontend")
+
+
+def kda_decode_conv(q, k, v, g, beta, slots, state_pool, conv_pool, o, w_q, w_k, scale=0.0,
+                    stream=None):
+    """kda_decode with the q/k front-end fused in (raw q, k; see include/kda.h)."""
+    dims = _dims(q, v, 0, scale)
+    conv = _conv(w_q, w_k)
+    _check(lib().kda_decode_conv(ctypes.byref(dims), ctypes.byref(conv), q.shape[0], _dptr(q),
+                                 _dptr(k), _dptr(v), _dptr(g), _dptr(beta), _dptr(slots),
+                                 state_pool.shape[0], _dptr(state_pool), _dptr(conv_pool),
+                                 _dptr(o), _stream(stream)), "kda_decode_conv")
+
+
+def kda_verify_conv(q, k, v, g, beta, cu_draft, slots, state_pool, conv_pool, token_states, o,
+                    w_q, w_k, conv_token_states=None, scale=0.0, stream=None):
+    """kda_verify with the q/k front-end fused in (see include/kda.h)."""
+    cu = _host_array(cu_draft, np.int32)
+    dims = _dims(q, v, 0, scale)
+    conv = _conv(w_q, w_k)
+    _check(lib().kda_verify_conv(ctypes.byref(dims), ctypes.byref(conv), len(cu) - 1, _hptr(cu),
+                                 _dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(beta),
+                                 _dptr(slots), state_pool.shape[0], _dptr(state_pool),
+                                 _dptr(conv_pool), _dptr(token_states),
+                                 _dptr(conv_token_states), _dptr(o), _stream(stream)),
+           "kda_verify_conv")
+
+
+def kda_verify_commit_conv(prev, n_accept, cu_prev, q, k, v, g, beta, cu_draft, slots,
+                           state_pool, conv_pool, o, w_q, w_k, pos=None, snap_interval=0,
+                           snap_row=None, snapshots=None, conv_snapshots=None, scale=0.0,
+                           stream=None):
+    """kda_verify_commit with the q/k front-end fused in; ``prev`` holds raw q too."""
+    cp = _host_array(cu_prev, np.int32)
+    cd = _host_array(cu_draft, np.int32)
+    if len(cp) != len(cd):
+        raise KDAError(1, "cu_prev and cu_draft must describe the same sequences")
+    dims = _dims(q, v, 0, scale)
+    conv = _conv(w_q, w_k)
+    pv = prev or {}
+    n_rows = 0 if snapshots is None else snapshots.shape[0]
+    _check(lib().kda_verify_commit_conv(
+        ctypes.byref(dims), ctypes.byref(conv), len(cd) - 1, _hptr(cp), _dptr(pv.get("q")),
+        _dptr(pv.get("k")), _dptr(pv.get("v")), _dptr(pv.get("g")), _dptr(pv.get("beta")),
+        _dptr(n_accept), _dptr(pos), int(snap_interval), _dptr(snap_row), _dptr(snapshots),
+        _dptr(conv_snapshots), n_rows, _hptr(cd), _dptr(q), _dptr(k), _dptr(v), _dptr(g),
+        _dptr(beta), _dptr(slots), state_pool.shape[0], _dptr(state_pool), _dptr(conv_pool),
+        _dptr(o), _stream(stream)), "kda_verify_commit_conv")
+
+
+def kda_state_map_apply(M, X, out, N=None, stream=None):
+    """out = M X + N per leading index (see include/kda.h): M [..., dk, dk], X, N, out
+    [..., dk, dv] fp32 device tensors; the leading dimensions are flattened."""
+    dk, dv = X.shape[-2], X.shape[-1]
+    n = X.numel() // (dk * dv)
+    if M.shape[-2:] != (dk, dk) or M.numel() // (dk * dk) != n or out.shape != X.shape:
+        raise KDAError(1, "kda_state_map_apply: shapes do not match")
+    _check(lib().kda_state_map_apply(n, dk, dv, _dptr(M), _dptr(X), _dptr(N), _dptr(out),
+                                     _stream(stream)), "kda_state_map_apply")
 
 
 def kda_snapshot(src_idx, dst_idx, src, dst, stream=None):

@@ -76,6 +76,28 @@ typedef struct {
 #define KDA_SEQS_PER_LAUNCH 1024
 
 /*
+ * The q/k front-end (Kimi K3 technical FAQ, "What is KDA, and why does a serving
+ * engineer care?": queries and keys go through a short convolution, Swish and L2
+ * normalization before the recurrence). Per head h and key channel c, over the raw
+ * inputs x of one sequence (q and k each with their own weights):
+ *     y_t = sum_{j=0}^{taps-1} w[h][c][j] * x_{t-(taps-1)+j}   (causal, depthwise,
+ *                                                              no bias; tap taps-1
+ *                                                              on the current token)
+ *     z_t = y_t * sigmoid(y_t)                                 (Swish)
+ *     out_t = z_t / max(||z_t||_2, 1e-6)                        (over the dk channels)
+ * A sequence's conv state is its last taps-1 raw inputs (zeros for a fresh
+ * sequence), fp32, laid out [2 (q then k), H, dk, taps-1], oldest input first; pools
+ * of conv states are [n, 2, H, dk, taps-1]. Conv states travel with the recurrent
+ * states: the calls below carry them across calls and snapshot them at the same
+ * block boundaries.
+ */
+typedef struct {
+    int32_t taps;          /* 2, 3 or 4 */
+    const float *w_q;      /* [H, dk, taps] fp32, device */
+    const float *w_k;      /* [H, dk, taps] fp32, device */
+} kda_conv;
+
+/*
  * kda_snapshot_plan — where each sequence's snapshots go (host only, no GPU).
  * Snapshot rule of the vLLM day-0 blog, "Kimi Delta Attention" (snapshots at
  * block boundaries): sequence s (tokens cu_seqlens_h[s] .. cu_seqlens_h[s+1]-1,
@@ -264,6 +286,79 @@ kda_status kda_verify_commit(const kda_dims *dims, int32_t n_seq, const int32_t 
 kda_status kda_snapshot(int32_t n, const int64_t *src_idx, const int64_t *dst_idx,
                         const float *src, int64_t n_src, float *dst, int64_t n_dst,
                         int32_t H, int32_t dk, int32_t dv, kda_stream_t stream);
+
+/*
+ * kda_qk_frontend — the front-end above over a packed prefill batch, producing the
+ * normalised q and k that kda_prefill takes. Sequences, start_pos_h, snap_interval
+ * and the snapshot rule are as in kda_prefill (the same kda_snapshot_plan rows).
+ *   q_raw, k_raw [T_total, H, dk] (bf16 or fp32 as dims->io): raw inputs.
+ *   conv_in  [n_seq, 2, H, dk, taps-1] (nullable = zeros), conv_out (nullable): the
+ *            conv state before and after each sequence.
+ *   q_out, k_out [T_total, H, dk]: normalised outputs (may not alias the inputs).
+ *   conv_snapshots [kda_snapshot_plan total, 2, H, dk, taps-1] (required when a
+ *            snapshot is due): the conv state after each snapshot position.
+ * Errors: as kda_prefill, and KDA_ERR_INVALID for a null conv, taps outside 2..4
+ * or null weights.
+ */
+kda_status kda_qk_frontend(const kda_dims *dims, const kda_conv *conv, int32_t n_seq,
+                           const int32_t *cu_seqlens_h, const int64_t *start_pos_h,
+                           const void *q_raw, const void *k_raw, const float *conv_in,
+                           float *conv_out, void *q_out, void *k_out, int32_t snap_interval,
+                           float *conv_snapshots, kda_stream_t stream);
+
+/*
+ * kda_decode_conv, kda_verify_conv, kda_verify_commit_conv — kda_decode, kda_verify
+ * and kda_verify_commit with the front-end fused into their token loads: q and k
+ * (and q_prev, k_prev) are raw inputs, and each sequence's conv state is carried
+ * next to its recurrent state in conv_pool [n_slots, 2, H, dk, taps-1]:
+ *   decode:        conv_pool[slots[s]] is updated in place with the state slot.
+ *   verify:        conv_pool is only read; conv_token_states [T, 2, H, dk, taps-1]
+ *                  (nullable) receives the conv state after every draft token, the
+ *                  companion of token_states for rollback.
+ *   verify_commit: the replay of the accepted prefix advances conv_pool[slots[s]]
+ *                  (written with the state); q_prev is required (it moves the q
+ *                  conv state); a block-boundary snapshot also writes the conv state
+ *                  to conv_snapshots[snap_row[s]] ([n_snap_rows, 2, H, dk, taps-1]).
+ * Other arguments, layouts and errors as the calls without the front-end.
+ */
+kda_status kda_decode_conv(const kda_dims *dims, const kda_conv *conv, int32_t n_seq,
+                           const void *q, const void *k, const void *v, const float *g,
+                           const float *beta, const int32_t *slots, int32_t n_slots,
+                           float *state_pool, float *conv_pool, void *o, kda_stream_t stream);
+kda_status kda_verify_conv(const kda_dims *dims, const kda_conv *conv, int32_t n_seq,
+                           const int32_t *cu_draft_h, const void *q, const void *k,
+                           const void *v, const float *g, const float *beta,
+                           const int32_t *slots, int32_t n_slots, const float *state_pool,
+                           const float *conv_pool, float *token_states,
+                           float *conv_token_states, void *o, kda_stream_t stream);
+kda_status kda_verify_commit_conv(const kda_dims *dims, const kda_conv *conv, int32_t n_seq,
+                                  const int32_t *cu_prev_h, const void *q_prev,
+                                  const void *k_prev, const void *v_prev, const float *g_prev,
+                                  const float *beta_prev, const int32_t *n_accept,
+                                  const int64_t *pos, int32_t snap_interval,
+                                  const int64_t *snap_row, float *snapshots,
+                                  float *conv_snapshots, int64_t n_snap_rows,
+                                  const int32_t *cu_draft_h, const void *q, const void *k,
+                                  const void *v, const float *g, const float *beta,
+                                  const int32_t *slots, int32_t n_slots, float *state_pool,
+                                  float *conv_pool, void *o, kda_stream_t stream);
+
+/*
+ * kda_state_map_apply — out[i] = M[i] X[i] + N[i] for i < n, fp32 (N nullable = 0).
+ * Splitting one long sequence across workers (runtimewire, "The architecture is
+ * built around inference cost": KDA carries a fixed-size recurrent state over a
+ * 1M-token context): each step S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1}
+ * + beta_t k_t v_t^T is affine in the state, so a token segment maps its entering
+ * state S to M S + N, where M (dk x dk) is kda_prefill's final state for the segment
+ * with v = 0 from the identity state (dv = dk), and N its final state from zero.
+ * Maps compose as (M2, N2) o (M1, N1) = (M2 M1, M2 N1 + N2): two calls of this
+ * function. A worker holding segment r applies the maps of segments 0..r-1 to the
+ * sequence's initial state, then runs kda_prefill of its segment from the result.
+ *   M [n, dk, dk]; X, N, out [n, dk, dv] (per head: n = segments x H), device fp32.
+ *   out may alias N; it must not overlap M or X (KDA_ERR_INVALID when equal).
+ */
+kda_status kda_state_map_apply(int64_t n, int32_t dk, int32_t dv, const float *M, const float *X,
+                               const float *N, float *out, kda_stream_t stream);
 
 /* Human-readable name of a status code (static storage). */
 const char *kda_status_string(kda_status s);

@@ -38,7 +38,8 @@ _M2 = np.uint64(0x94D049BB133111EB)
 
 # stream tags, one per drawn quantity
 TAG = {"q": 1, "k": 2, "v": 3, "g": 4, "beta": 5, "state": 6, "lens": 7,
-       "draft": 8, "resume": 9, "perm": 10, "slots": 11, "misc": 12}
+       "draft": 8, "resume": 9, "perm": 10, "slots": 11, "misc": 12, "conv": 13,
+       "convstate": 14}
 
 _BLOCK = 1 << 22
 
@@ -175,6 +176,27 @@ def token_inputs(seed: int, T: int, H: int, dk: int, dv: int, io: str = "bf16",
     beta = torch.from_numpy(normal(seed, "beta", T * H, start=t0 * H, out_dtype=np.float32,
                                    transform=_sigmoid).reshape(T, H))
     return {"q": q, "k": k, "v": v, "g": g, "beta": beta}
+
+
+def raw_qk(seed: int, T: int, H: int, dk: int, io: str = "bf16", t0: int = 0) -> dict:
+    """Raw (pre-front-end) q and k of tokens [t0, t0+T): N(0, 1) per element, rounded
+    to the I/O type (tags q and k of the same streams as token_inputs, unnormalised)."""
+    return {"q": _plain_rows(seed, "q", t0, T, H, dk, io),
+            "k": _plain_rows(seed, "k", t0, T, H, dk, io)}
+
+
+def conv_weights(seed: int, H: int, dk: int, taps: int) -> tuple:
+    """Short-conv weights for q and k, [H, dk, taps] fp32 each: N(0, 1) / sqrt(taps)."""
+    x = normal(seed, "conv", 2 * H * dk * taps, out_dtype=np.float32,
+               transform=lambda z: z / math.sqrt(taps)).reshape(2, H, dk, taps)
+    return torch.from_numpy(x[0].copy()), torch.from_numpy(x[1].copy())
+
+
+def conv_states(seed: int, n: int, H: int, dk: int, taps: int, io: str = "bf16") -> torch.Tensor:
+    """n conv states [n, 2, H, dk, taps-1] fp32 holding earlier raw inputs: N(0, 1)
+    values rounded to the I/O type (what a carried conv state contains)."""
+    x = normal(seed, "convstate", n * 2 * H * dk * (taps - 1)).reshape(n, 2, H, dk, taps - 1)
+    return _to_io(x, io).float()
 
 
 def states(seed: int, n: int, H: int, dk: int, dv: int, std: float = 0.1, tag: str = "state",

@@ -200,6 +200,45 @@ def test_verify_commit_validation():
     assert call(n=0) == 0
 
 
+def test_frontend_validation():
+    L = K.lib()
+    d = _dims()
+    cu = np.array([0, 64, 100], dtype=np.int32)
+    P = lambda a: a.ctypes.data_as(ctypes.c_void_p)  # noqa: E731
+    conv = K.kda_conv(4, 0x10000, 0x10000)
+    bad_taps = K.kda_conv(5, 0x10000, 0x10000)
+    no_w = K.kda_conv(4, None, 0x10000)
+    mis_w = K.kda_conv(4, 0x10008, 0x10000)
+
+    def fe(cv=conv, n=2, c=cu, snap=0, sn=None, qo=A, start=None):
+        return L.kda_qk_frontend(ctypes.byref(d), None if cv is None else ctypes.byref(cv), n, P(c),
+                                 start, A, A, None, None, qo, A, snap, sn, None)
+    assert fe(cv=None) == 1 and fe(cv=bad_taps) == 1 and fe(cv=no_w) == 1
+    assert fe(cv=mis_w) == 3
+    assert fe(c=np.array([0, 64, 10], np.int32)) == 1
+    assert fe(snap=96) == 1                        # not a multiple of the chunk
+    assert fe(snap=64) == 1                        # snapshots due, no conv snapshot pool
+    assert fe(qo=None) == 1 and fe(qo=MIS) == 3
+    assert fe(n=0) == 0
+    st = np.array([32, 0], dtype=np.int64)
+    assert fe(snap=64, sn=A, start=P(st)) == 1     # start position off the chunk grid
+    # decode / verify / verify+commit with the front-end
+    assert L.kda_decode_conv(ctypes.byref(d), None, 4, A, A, A, A, A, A, 8, A, A, A, None) == 1
+    assert L.kda_decode_conv(ctypes.byref(d), ctypes.byref(conv), 4, A, A, A, A, A, A, 8, A, None,
+                             A, None) == 1         # no conv pool
+    assert L.kda_decode_conv(ctypes.byref(d), ctypes.byref(bad_taps), 4, A, A, A, A, A, A, 8, A, A,
+                             A, None) == 1
+    c2 = np.array([0, 3, 5], dtype=np.int32)
+    assert L.kda_verify_conv(ctypes.byref(d), ctypes.byref(conv), 2, P(c2), A, A, A, A, A, A, 8, A,
+                             None, A, None, A, None) == 1
+    assert L.kda_verify_conv(ctypes.byref(d), ctypes.byref(conv), 2, P(c2), A, A, A, A, A, A, 8, A,
+                             A, A, MIS, A, None) == 3
+    # verify+commit with the front-end needs the previous batch's raw q
+    assert L.kda_verify_commit_conv(ctypes.byref(d), ctypes.byref(conv), 2, P(c2), None, A, A, A, A,
+                                    A, None, 0, None, None, None, 0, P(c2), A, A, A, A, A, A, 8, A,
+                                    A, A, None) == 1
+
+
 def test_no_launch_issued_by_host_tests():
     # the validation failures above must not have launched anything
     assert K.kda_launch_count() == 0
