@@ -383,6 +383,7 @@ def run_ours(args):
         del wl.p_ws, wl.ts
         torch.cuda.empty_cache()
         extra["tiny"] = bench_tiny(K, dev, args.steps, args.warmup)
+        extra.update(bench_frontend(K, dev, args.steps, args.warmup, peaks))
         extra["ragged"] = bench_ragged(K, dev, args.steps, args.warmup, peaks)
         torch.cuda.empty_cache()
         extra["long"] = bench_long(K, dev, max(3, args.steps // 4), args.warmup, peaks)
@@ -593,6 +594,60 @@ def bench_long(K, dev, steps, warmup, peaks):
             "launches_per_pass": launches, "path": "split",
             "workload": "1,048,576 tokens x 64 heads as 16 calls of 65,536 (state handed "
                         "across calls), snapshots /4096; one pass = 16 calls"}
+
+
+def bench_frontend(K, dev, steps, warmup, peaks):
+    """The q/k front-end (short conv, Swish, L2): kda_qk_frontend over the 8192-token
+    prefill workload (raw q, k; conv states carried and snapshotted every 256 tokens),
+    and kda_decode_conv, the decode step with the front-end fused in, on 512 x 64 states."""
+    taps = 4
+    T, n_seq = PREFILL_T, N_SEQ
+    raw = synth.raw_qk(1001, T, H, D, io="bf16")
+    rd = {k: v.to(dev) for k, v in raw.items()}
+    wq, wk = (w.to(dev) for w in synth.conv_weights(1001, H, D, taps))
+    qo, ko = torch.empty_like(rd["q"]), torch.empty_like(rd["k"])
+    cu = np.array([0, T], dtype=np.int32)
+    cin = synth.conv_states(1001, 1, H, D, taps).to(dev)
+    cout = torch.empty_like(cin)
+    csn = torch.empty((T // SNAP, 2, H, D, taps - 1), device=dev)
+
+    def fe():
+        K.kda_qk_frontend(rd["q"], rd["k"], wq, wk, cu, qo, ko, conv_in=cin, conv_out=cout,
+                          snap_interval=SNAP, conv_snapshots=csn, chunk=C)
+    ms_fe = time_calls(fe, steps, warmup, dev)
+    cstate = 2 * H * D * (taps - 1) * 4
+    b_fe = T * H * D * 2 * 4 + (2 + T // SNAP) * cstate
+    x = synth.token_inputs(1002, n_seq, H, D, D, io="bf16")
+    xd = {k: v.to(dev) for k, v in x.items()}
+    rq = {k: v.to(dev) for k, v in synth.raw_qk(1002, n_seq, H, D, io="bf16").items()}
+    pool = synth.states(1002, n_seq, H, D, D, std=0.1).to(dev)
+    cpool = synth.conv_states(1002, n_seq, H, D, taps).to(dev)
+    slots = torch.arange(n_seq, dtype=torch.int32, device=dev)
+    o = torch.empty((n_seq, H, D), dtype=torch.bfloat16, device=dev)
+
+    def dc():
+        K.kda_decode_conv(rq["q"], rq["k"], xd["v"], xd["g"], xd["beta"], slots, pool, cpool, o,
+                          wq, wk)
+    ms_dc = time_calls(dc, steps, warmup, dev)
+    b_dc = decode_bytes(n_seq) + n_seq * 2 * cstate
+    st = K.kda_check_device_status()
+    if st != 0:
+        raise RuntimeError(f"front-end workloads: device status {K.kda_status_string(st)}")
+    hbm = peaks["hbm_gbs"]
+    return {
+        "frontend_prefill": {"ms": round(ms_fe, 4), "value": T / (ms_fe * 1e-3), "unit": "tok/s",
+                             "tokens": T, "algorithmic_bytes": b_fe,
+                             "achieved_gbs": round(b_fe / (ms_fe * 1e-3) / 1e9, 1),
+                             "hbm_frac": round(b_fe / (ms_fe * 1e-3) / 1e9 / hbm, 4),
+                             "workload": "kda_qk_frontend, 8192 tokens x 64 heads, 4 taps, raw bf16 "
+                                         "q/k in, normalised bf16 q/k out, conv snapshots /256"},
+        "decode_conv": {"ms": round(ms_dc, 4), "value": n_seq * H / (ms_dc * 1e-3),
+                        "unit": "state-steps/s", "algorithmic_bytes": b_dc,
+                        "achieved_gbs": round(b_dc / (ms_dc * 1e-3) / 1e9, 1),
+                        "hbm_frac": round(b_dc / (ms_dc * 1e-3) / 1e9 / hbm, 4),
+                        "workload": "kda_decode_conv, 512 sequences x 64 heads, 4 taps, conv "
+                                    "states updated in place with the fp32 states"},
+    }
 
 
 def time_calls(fn, steps, warmup, dev):

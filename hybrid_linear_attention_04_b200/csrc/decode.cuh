@@ -12,12 +12,19 @@
 //     S  = S' + k w^T
 //     o  = scale (y + (k . q) w)            (= scale * S^T q, read after update)
 //
-// Thread map: thread t owns column group cg = t % (D/4) (four adjacent d_v
-// columns, one float4) and rows rs, rs + RS, ... with rs = t / (D/4). Column
-// sums over d_k reduce first across lanes of a warp that share cg (shuffles),
-// then across warps through shared memory in a fixed order (deterministic).
-// Decode and verify run the same step function, so verify's state after its
-// j-th token is bit-identical to j decode calls.
+// The d_v columns of S evolve independently (w, the update and o are per column),
+// so warp w owns the 16 columns 16w .. 16w+15 over all d_k rows: lane l holds the
+// float4 of columns 16w + 4 (l % 4) .. +3 in rows l / 4 + 8 m, m < D / 8. The column
+// sums over d_k reduce inside the lane, then across the 8 lanes that share the
+// column group (three butterfly shuffles, so every lane holds the same sum); a
+// token step has no barrier and no shared-memory reduction. Decode, verify and the
+// commit replay run the same step function, so verify's state after its j-th token
+// is bit-identical to j decode calls.
+//
+// Token vectors are staged in shared memory a batch at a time: threads t < D own
+// channel t of q and k (and run the q/k front-end's conv window in token order),
+// threads t >= D channel t - D of v and g; each thread issues all its loads for the
+// batch before it uses any.
 #pragma once
 #include "common.cuh"
 
@@ -26,12 +33,10 @@ namespace kda {
 constexpr int kMaxSeqsPerLaunch = KDA_SEQS_PER_LAUNCH;
 
 template <int D> struct DecodeShape {
-    static constexpr int NT = D == 128 ? 256 : (D == 64 ? 128 : 64);  // threads per CTA
-    static constexpr int CG = D / 4;                                    // column groups
-    static constexpr int RS = NT / CG;                                  // row slots
-    static constexpr int R = D / RS;                                    // rows per thread
-    static constexpr int NW = NT / 32;                                  // warps
-    static_assert(CG <= 32 && 32 % CG == 0, "column groups must tile a warp");
+    static constexpr int NT = 2 * D;     // threads per CTA: 256, 128, 64
+    static constexpr int NW = NT / 32;   // warps, 16 d_v columns each
+    static constexpr int R = D / 8;      // rows per lane
+    static_assert(NW * 16 == D, "warps must tile the columns");
 };
 
 struct DecodeParams {
@@ -131,49 +136,86 @@ template <int D> struct __align__(16) TokVec {
 };
 static_assert(sizeof(TokVec<128>) % 16 == 0 && sizeof(TokVec<32>) % 16 == 0, "TokVec padding");
 
-// Stage the vectors of token row `row` (= token * H + head); q may be null (a token
-// whose output is not needed). D threads (or fewer, looping) fill the vectors.
-template <int D, typename TIO>
-__device__ __forceinline__ void load_vectors(TokVec<D> &tv, const void *q_, const void *k_, const void *v_,
-                                             const float *g_, const float *beta, int64_t row) {
-    const TIO *q = q_ ? static_cast<const TIO *>(q_) + row * D : nullptr;
-    const TIO *k = static_cast<const TIO *>(k_) + row * D;
-    const TIO *v = static_cast<const TIO *>(v_) + row * D;
-    const float *g = g_ + row * D;
-    for (int i = threadIdx.x; i < D; i += blockDim.x) {
-        tv.k[i] = IO<TIO>::ld(k + i);
-        tv.q[i] = q ? IO<TIO>::ld(q + i) : 0.f;
-        tv.v[i] = IO<TIO>::ld(v + i);
-        tv.a[i] = expf(g[i]);
-    }
-    if (threadIdx.x == 0) tv.beta = beta[row];
-}
+// Verify: tokens are processed in batches of kTokBatch staged in shared memory.
+constexpr int kTokBatch = 8;
 
-template <int D, typename TIO>
-__device__ __forceinline__ void load_token(TokVec<D> &tv, const DecodeParams &p, int64_t row) {
-    load_vectors<D, TIO>(tv, p.q, p.k, p.v, p.g, p.beta, row);
-}
+// Where the front-end's conv state goes while a batch is staged (front-end on only):
+// after every token into rows tok0 + j of `tok` (nullable), and after token snap_j
+// (batch-relative; -1 = none) into row snap_row of `snap`.
+struct ConvOut {
+    float *tok;
+    int64_t tok0;
+    float *snap;
+    int64_t snap_row;
+    int snap_j;
+};
 
-// Stage a token whose raw q, k pass through the front-end: the conv and Swish here
-// (thread c < D, channel c, window w), the L2 normalisation in token_finish. With
-// q_ == nullptr only the q window advances (a token whose output is not needed still
-// moves the conv state).
-template <int D, typename TIO>
-__device__ __forceinline__ void load_vectors_conv(TokVec<D> &tv, ConvWin &w, int K, const void *q_, const void *k_,
-                                                  const void *v_, const float *g_, const float *beta,
-                                                  int64_t row, bool want_q) {
-    const int c = threadIdx.x;
-    if (c < D) {
-        const float xq = IO<TIO>::ld(static_cast<const TIO *>(q_) + row * D + c);
-        const float xk = IO<TIO>::ld(static_cast<const TIO *>(k_) + row * D + c);
-        const float yq = conv_step(w.wq, w.hq, K, xq);
-        const float yk = conv_step(w.wk, w.hk, K, xk);
-        tv.q[c] = want_q ? swish(yq) : 0.f;
-        tv.k[c] = swish(yk);
-        tv.v[c] = IO<TIO>::ld(static_cast<const TIO *>(v_) + row * D + c);
-        tv.a[c] = expf(g_[row * D + c]);
+// Stage nb <= kTokBatch tokens, rows row0 + j * rstride (= token * H + head) of the
+// packed arrays, into tv[0..nb). q_ may be null (a replayed token whose output is not
+// needed: with the front-end its q still moves the conv window). With CONV, q and k
+// are raw and pass through the conv and Swish here (window w of the thread's
+// channel); token_finish normalises them.
+template <int D, typename TIO, bool CONV>
+__device__ __forceinline__ void stage_batch(TokVec<D> *tv, int nb, int64_t row0, int64_t rstride,
+                                            const void *q_, const void *k_, const void *v_,
+                                            const float *g_, const float *beta, ConvWin &w,
+                                            const DecodeParams &p, int h, const ConvOut &co) {
+    constexpr int L = kTokBatch / 2;      // loads in flight per array (register budget)
+    const int t = threadIdx.x;
+    if (t < D) {
+        const TIO *q = static_cast<const TIO *>(q_), *k = static_cast<const TIO *>(k_);
+        for (int j0 = 0; j0 < nb; j0 += L) {
+            float xq[L], xk[L];
+#pragma unroll
+            for (int j = 0; j < L; ++j) {
+                if (j0 + j < nb) {
+                    const int64_t off = (row0 + (j0 + j) * rstride) * D + t;
+                    xq[j] = (q_ != nullptr) ? IO<TIO>::ld(q + off) : 0.f;
+                    xk[j] = IO<TIO>::ld(k + off);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < L; ++j) {
+                const int jj = j0 + j;
+                if (jj < nb) {
+                    if (CONV) {
+                        const float yq = conv_step(w.wq, w.hq, p.taps, xq[j]);
+                        const float yk = conv_step(w.wk, w.hk, p.taps, xk[j]);
+                        tv[jj].q[t] = q_ != nullptr ? swish(yq) : 0.f;
+                        tv[jj].k[t] = swish(yk);
+                        if (co.tok) conv_store(w, p, co.tok, co.tok0 + jj, h, D, t);
+                        if (jj == co.snap_j) conv_store(w, p, co.snap, co.snap_row, h, D, t);
+                    } else {
+                        tv[jj].q[t] = xq[j];
+                        tv[jj].k[t] = xk[j];
+                    }
+                }
+            }
+        }
+    } else {
+        const int c = t - D;
+        const TIO *v = static_cast<const TIO *>(v_);
+        const float b = c < nb ? beta[row0 + c * rstride] : 0.f;
+        for (int j0 = 0; j0 < nb; j0 += L) {
+            float xv[L], xg[L];
+#pragma unroll
+            for (int j = 0; j < L; ++j) {
+                if (j0 + j < nb) {
+                    const int64_t off = (row0 + (j0 + j) * rstride) * D + c;
+                    xv[j] = IO<TIO>::ld(v + off);
+                    xg[j] = g_[off];
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < L; ++j) {
+                if (j0 + j < nb) {
+                    tv[j0 + j].v[c] = xv[j];
+                    tv[j0 + j].a[c] = expf(xg[j]);
+                }
+            }
+        }
+        if (c < nb) tv[c].beta = b;
     }
-    if (threadIdx.x == 0) tv.beta = beta[row];
 }
 
 // One warp finishes a staged token: L2-normalises k and q when the front-end is on,
@@ -211,26 +253,30 @@ __device__ __forceinline__ void token_finish(TokVec<D> &tv, bool normalise, bool
     }
 }
 
-// k . q for a staged token, by one warp, fixed reduction order.
+// Finish nb staged tokens (warp j takes token j, warp 0 the rest) between barriers.
 template <int D>
-__device__ __forceinline__ void token_kq(TokVec<D> &tv) {
-    token_finish<D>(tv, false, true);
+__device__ __forceinline__ void finish_batch(TokVec<D> *tv, int nb, bool normalise, bool with_q) {
+    const int warp = threadIdx.x >> 5;
+    __syncthreads();
+    if (warp < nb) token_finish<D>(tv[warp], normalise, with_q);
+    for (int j = DecodeShape<D>::NW; j < nb; ++j)
+        if (warp == 0) token_finish<D>(tv[j], normalise, with_q);
+    __syncthreads();
 }
 
-// One recurrence step on the register-resident state. red: [NW][2][D] scratch
-// in shared memory; the caller separates reuses of `red` by a barrier. With
-// OUT = false the output read (y and o) is skipped; the state arithmetic is the
-// same instruction for instruction, so both forms give bit-identical states.
+// One recurrence step on the register-resident columns of this warp. With OUT =
+// false the output read (y and o) is skipped; the state arithmetic is the same
+// instruction for instruction, so both forms give bit-identical states. The
+// returned o (OUT) holds the lane's four columns; every lane of a column group has it.
 template <int D, bool OUT = true>
-__device__ __forceinline__ float4 kda_step(float4 (&st)[DecodeShape<D>::R], const TokVec<D> &tv,
-                                           float *red, float scale) {
+__device__ __forceinline__ float4 kda_step(float4 (&st)[DecodeShape<D>::R], const TokVec<D> &tv, float scale) {
     using Sh = DecodeShape<D>;
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const int cg = t % Sh::CG, rs = t / Sh::CG;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int cg = lane & 3, rg = lane >> 2;
     float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
 #pragma unroll
     for (int m = 0; m < Sh::R; ++m) {
-        const int r = rs + Sh::RS * m;
+        const int r = rg + 8 * m;
         const float a = tv.a[r], kr = tv.k[r];
         float4 s = st[m];
         s.x *= a; s.y *= a; s.z *= a; s.w *= a;
@@ -244,7 +290,7 @@ __device__ __forceinline__ float4 kda_step(float4 (&st)[DecodeShape<D>::R], cons
         }
     }
 #pragma unroll
-    for (int off = Sh::CG; off < 32; off <<= 1) {
+    for (int off = 4; off < 32; off <<= 1) {
         x.x += __shfl_xor_sync(0xffffffffu, x.x, off);
         x.y += __shfl_xor_sync(0xffffffffu, x.y, off);
         x.z += __shfl_xor_sync(0xffffffffu, x.z, off);
@@ -256,28 +302,13 @@ __device__ __forceinline__ float4 kda_step(float4 (&st)[DecodeShape<D>::R], cons
             y.w += __shfl_xor_sync(0xffffffffu, y.w, off);
         }
     }
-    if (lane < Sh::CG) {
-        *reinterpret_cast<float4 *>(red + (warp * 2 + 0) * D + cg * 4) = x;
-        if (OUT) *reinterpret_cast<float4 *>(red + (warp * 2 + 1) * D + cg * 4) = y;
-    }
-    __syncthreads();
-    float4 X = make_float4(0.f, 0.f, 0.f, 0.f), Y = X;
-#pragma unroll
-    for (int w = 0; w < Sh::NW; ++w) {
-        float4 a = *reinterpret_cast<const float4 *>(red + (w * 2 + 0) * D + cg * 4);
-        X.x += a.x; X.y += a.y; X.z += a.z; X.w += a.w;
-        if (OUT) {
-            float4 b = *reinterpret_cast<const float4 *>(red + (w * 2 + 1) * D + cg * 4);
-            Y.x += b.x; Y.y += b.y; Y.z += b.z; Y.w += b.w;
-        }
-    }
-    const float4 vv = *reinterpret_cast<const float4 *>(tv.v + cg * 4);
+    const float4 vv = *reinterpret_cast<const float4 *>(tv.v + 16 * warp + 4 * cg);
     float4 wv;
-    wv.x = tv.beta * (vv.x - X.x); wv.y = tv.beta * (vv.y - X.y);
-    wv.z = tv.beta * (vv.z - X.z); wv.w = tv.beta * (vv.w - X.w);
+    wv.x = tv.beta * (vv.x - x.x); wv.y = tv.beta * (vv.y - x.y);
+    wv.z = tv.beta * (vv.z - x.z); wv.w = tv.beta * (vv.w - x.w);
 #pragma unroll
     for (int m = 0; m < Sh::R; ++m) {
-        const float kr = tv.k[rs + Sh::RS * m];
+        const float kr = tv.k[rg + 8 * m];
         float4 s = st[m];
         s.x = fmaf(kr, wv.x, s.x); s.y = fmaf(kr, wv.y, s.y);
         s.z = fmaf(kr, wv.z, s.z); s.w = fmaf(kr, wv.w, s.w);
@@ -285,63 +316,70 @@ __device__ __forceinline__ float4 kda_step(float4 (&st)[DecodeShape<D>::R], cons
     }
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
     if (OUT) {
-        o.x = scale * fmaf(tv.kq, wv.x, Y.x); o.y = scale * fmaf(tv.kq, wv.y, Y.y);
-        o.z = scale * fmaf(tv.kq, wv.z, Y.z); o.w = scale * fmaf(tv.kq, wv.w, Y.w);
+        o.x = scale * fmaf(tv.kq, wv.x, y.x); o.y = scale * fmaf(tv.kq, wv.y, y.y);
+        o.z = scale * fmaf(tv.kq, wv.z, y.z); o.w = scale * fmaf(tv.kq, wv.w, y.w);
     }
     return o;
 }
 
-template <int D, typename TIO>
-__global__ void __launch_bounds__(DecodeShape<D>::NT)
+// offset of the lane's float4 in row m of a state
+template <int D>
+__device__ __forceinline__ int64_t lane_off(int m) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    return (int64_t)((lane >> 2) + 8 * m) * D + 16 * warp + 4 * (lane & 3);
+}
+template <int D>
+__device__ __forceinline__ int lane_col() {
+    return 16 * (threadIdx.x >> 5) + 4 * (threadIdx.x & 3);
+}
+
+template <int D>
+__device__ __forceinline__ void load_state(float4 (&st)[DecodeShape<D>::R], const float *S) {
+#pragma unroll
+    for (int m = 0; m < DecodeShape<D>::R; ++m) {
+        const float *src = S + lane_off<D>(m);
+        asm volatile("ld.global.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
+                     : "=f"(st[m].x), "=f"(st[m].y), "=f"(st[m].z), "=f"(st[m].w)
+                     : "l"(src));
+    }
+}
+template <int D>
+__device__ __forceinline__ void store_state(const float4 (&st)[DecodeShape<D>::R], float *S) {
+#pragma unroll
+    for (int m = 0; m < DecodeShape<D>::R; ++m) st_stream(S + lane_off<D>(m), st[m]);
+}
+
+template <int D, typename TIO, bool CONV>
+__global__ void __launch_bounds__(DecodeShape<D>::NT, 2)
 decode_kernel(const __grid_constant__ DecodeParams p) {
-    using Sh = DecodeShape<D>;
     __shared__ TokVec<D> tv;
-    __shared__ __align__(16) float red[Sh::NW * 2 * D];
     const int s = blockIdx.x / p.H, h = blockIdx.x % p.H;
     const int32_t slot = p.slots[s];
     if (slot < 0 || slot >= p.n_slots) {
         if (threadIdx.x == 0) record_status(KDA_ERR_RANGE);
         return;
     }
-    const int t = threadIdx.x, cg = t % Sh::CG, rs = t / Sh::CG;
+    const int t = threadIdx.x;
     float *S = p.pool + ((int64_t)slot * p.H + h) * (int64_t)D * D;
-    float4 st[Sh::R];
-#pragma unroll
-    for (int m = 0; m < Sh::R; ++m) {
-        const float *src = S + (int64_t)(rs + Sh::RS * m) * D + cg * 4;
-        asm volatile("ld.global.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
-                     : "=f"(st[m].x), "=f"(st[m].y), "=f"(st[m].z), "=f"(st[m].w)
-                     : "l"(src));
-    }
+    float4 st[DecodeShape<D>::R];
+    load_state<D>(st, S);
     const int64_t row = (int64_t)s * p.H + h;
-    if (p.taps) {
-        ConvWin w;
-        if (t < D) conv_begin(w, p, p.conv, slot, h, D, t);
-        load_vectors_conv<D, TIO>(tv, w, p.taps, p.q, p.k, p.v, p.g, p.beta, row, true);
-        if (t < D) conv_store(w, p, p.conv, slot, h, D, t);
-    } else {
-        load_token<D, TIO>(tv, p, row);
-    }
-    __syncthreads();
-    if (t < 32) token_finish<D>(tv, p.taps > 0, true);
-    __syncthreads();
-    const float4 o = kda_step<D>(st, tv, red, p.scale);
-#pragma unroll
-    for (int m = 0; m < Sh::R; ++m)
-        st_stream(S + (int64_t)(rs + Sh::RS * m) * D + cg * 4, st[m]);
-    if (rs == 0) IO<TIO>::st4(static_cast<TIO *>(p.o) + row * D + cg * 4, o);
+    ConvWin w;
+    if (CONV && t < D) conv_begin(w, p, p.conv, slot, h, D, t);
+    const ConvOut none{nullptr, 0, nullptr, 0, -1};
+    stage_batch<D, TIO, CONV>(&tv, 1, row, 0, p.q, p.k, p.v, p.g, p.beta, w, p, h, none);
+    if (CONV && t < D) conv_store(w, p, p.conv, slot, h, D, t);
+    finish_batch<D>(&tv, 1, CONV, true);
+    const float4 o = kda_step<D>(st, tv, p.scale);
+    store_state<D>(st, S);
+    if ((t & 31) < 4) IO<TIO>::st4(static_cast<TIO *>(p.o) + row * D + lane_col<D>(), o);
 }
 
-// Verify: tokens are processed in batches of kTokBatch staged in shared memory.
-constexpr int kTokBatch = 8;
-
 // two CTAs per SM (register cap) keep enough state loads and stores in flight
-template <int D, typename TIO>
+template <int D, typename TIO, bool CONV>
 __global__ void __launch_bounds__(DecodeShape<D>::NT, 2)
 verify_kernel(const __grid_constant__ DecodeParams p) {
-    using Sh = DecodeShape<D>;
     __shared__ TokVec<D> tv[kTokBatch];
-    __shared__ __align__(16) float red[2][Sh::NW * 2 * D];
     const int s = blockIdx.x / p.H, h = blockIdx.x % p.H;
     const int32_t slot = p.slots[s];
     if (slot < 0 || slot >= p.n_slots) {
@@ -350,47 +388,28 @@ verify_kernel(const __grid_constant__ DecodeParams p) {
     }
     const int n_tok = p.tok0[s + 1] - p.tok0[s];
     const int64_t tok_first = p.tok_base + p.tok0[s];
-    const int t = threadIdx.x, cg = t % Sh::CG, rs = t / Sh::CG, warp = t >> 5;
+    const int t = threadIdx.x;
     const float *S = p.pool + ((int64_t)slot * p.H + h) * (int64_t)D * D;
-    float4 st[Sh::R];
+    float4 st[DecodeShape<D>::R];
 #pragma unroll
-    for (int m = 0; m < Sh::R; ++m) st[m] = ld_stream(S + (int64_t)(rs + Sh::RS * m) * D + cg * 4);
+    for (int m = 0; m < DecodeShape<D>::R; ++m) st[m] = ld_stream(S + lane_off<D>(m));
     ConvWin w;
-    if (p.taps && t < D) conv_begin(w, p, p.conv, slot, h, D, t);
-    int parity = 0;
+    if (CONV && t < D) conv_begin(w, p, p.conv, slot, h, D, t);
     for (int j0 = 0; j0 < n_tok; j0 += kTokBatch) {
         const int nb = min(kTokBatch, n_tok - j0);
         __syncthreads();  // previous batch's vectors are no longer read
+        const ConvOut co{p.conv_tok, tok_first + j0, nullptr, 0, -1};
+        stage_batch<D, TIO, CONV>(tv, nb, (tok_first + j0) * p.H + h, p.H, p.q, p.k, p.v, p.g, p.beta,
+                                  w, p, h, co);
+        finish_batch<D>(tv, nb, CONV, true);
         for (int j = 0; j < nb; ++j) {
-            const int64_t tok = tok_first + j0 + j;
-            if (p.taps) {
-                load_vectors_conv<D, TIO>(tv[j], w, p.taps, p.q, p.k, p.v, p.g, p.beta, tok * p.H + h, true);
-                if (p.conv_tok && t < D) conv_store(w, p, p.conv_tok, tok, h, D, t);
-            } else {
-                load_token<D, TIO>(tv[j], p, tok * p.H + h);
-            }
-        }
-        __syncthreads();
-        if (warp < nb) token_finish<D>(tv[warp], p.taps > 0, true);
-        for (int j = Sh::NW; j < nb; ++j)
-            if (warp == 0) token_finish<D>(tv[j], p.taps > 0, true);
-        __syncthreads();
-        for (int j = 0; j < nb; ++j) {
-            const float4 o = kda_step<D>(st, tv[j], red[parity], p.scale);
-            parity ^= 1;
+            const float4 o = kda_step<D>(st, tv[j], p.scale);
             const int64_t row = (tok_first + j0 + j) * p.H + h;
-            float *dst = p.token_states + row * (int64_t)D * D;
-#pragma unroll
-            for (int m = 0; m < Sh::R; ++m)
-                st_stream(dst + (int64_t)(rs + Sh::RS * m) * D + cg * 4, st[m]);
-            if (rs == 0) IO<TIO>::st4(static_cast<TIO *>(p.o) + row * D + cg * 4, o);
+            store_state<D>(st, p.token_states + row * (int64_t)D * D);
+            if ((t & 31) < 4) IO<TIO>::st4(static_cast<TIO *>(p.o) + row * D + lane_col<D>(), o);
         }
     }
 }
-
-}  // namespace kda
-
-namespace kda {
 
 // ---------------------------------------------------------------- verify + commit
 // One speculative step with the previous step's commit fused in: the live state is
@@ -405,6 +424,7 @@ struct CommitParams {
     const int32_t *n_accept;    // [n_seq] leading tokens of the previous batch to commit
     const int64_t *pos;         // [n_seq] tokens absorbed by the live state (snapshots only)
     const int64_t *snap_row;    // [n_seq] snapshot row for a boundary crossed, or < 0
+    const uint8_t *commit_new;  // [n_seq] nonzero: this step's tokens are committed too (nullable)
     float *snapshots;
     int64_t n_snap_rows;
     int32_t snap_interval;
@@ -417,14 +437,12 @@ struct VerifyCommitParams {
     CommitParams c;
 };
 
-template <int D, typename TIO>
+template <int D, typename TIO, bool CONV>
 __global__ void __launch_bounds__(DecodeShape<D>::NT, 2)
 verify_commit_kernel(const __grid_constant__ VerifyCommitParams P) {
-    using Sh = DecodeShape<D>;
     const DecodeParams &p = P.p;
     const CommitParams &c = P.c;
     __shared__ TokVec<D> tv[kTokBatch];
-    __shared__ __align__(16) float red[2][Sh::NW * 2 * D];
     const int s = blockIdx.x / p.H, h = blockIdx.x % p.H;
     const int32_t slot = p.slots[s];
     const int m_prev = c.tok0[s + 1] - c.tok0[s];
@@ -439,79 +457,56 @@ verify_commit_kernel(const __grid_constant__ VerifyCommitParams P) {
         if (threadIdx.x == 0) record_status(KDA_ERR_RANGE);
         return;
     }
-    const int t = threadIdx.x, cg = t % Sh::CG, rs = t / Sh::CG, warp = t >> 5;
+    const int n_tok = p.tok0[s + 1] - p.tok0[s];
+    // committed tokens: the replayed prefix, then (mixed step) this step's tokens;
+    // jsnap indexes that sequence
+    const bool cnew = c.commit_new != nullptr && c.commit_new[s] != 0 && n_tok > 0;
+    const int t = threadIdx.x;
     float *S = p.pool + ((int64_t)slot * p.H + h) * (int64_t)D * D;
-    float4 st[Sh::R];
-#pragma unroll
-    for (int m = 0; m < Sh::R; ++m) {
-        const float *src = S + (int64_t)(rs + Sh::RS * m) * D + cg * 4;
-        asm volatile("ld.global.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
-                     : "=f"(st[m].x), "=f"(st[m].y), "=f"(st[m].z), "=f"(st[m].w)
-                     : "l"(src));
-    }
-    int parity = 0;
+    float4 st[DecodeShape<D>::R];
+    load_state<D>(st, S);
     ConvWin w;
-    if (p.taps && t < D) conv_begin(w, p, p.conv, slot, h, D, t);
+    if (CONV && t < D) conv_begin(w, p, p.conv, slot, h, D, t);
     // 1. commit: replay the accepted prefix of the previous batch (state only)
     const int64_t prev_first = c.tok_base + c.tok0[s];
     for (int j0 = 0; j0 < na; j0 += kTokBatch) {
         const int nb = min(kTokBatch, na - j0);
         __syncthreads();
+        const int sj = (jsnap >= j0 && jsnap < j0 + nb) ? (int)(jsnap - j0) : -1;
+        const ConvOut co{nullptr, 0, c.conv_snapshots, srow, sj};
+        stage_batch<D, TIO, CONV>(tv, nb, prev_first * p.H + h + (int64_t)j0 * p.H, p.H,
+                                  CONV ? c.q : nullptr, c.k, c.v, c.g, c.beta, w, p, h, co);
+        finish_batch<D>(tv, nb, CONV, false);
         for (int j = 0; j < nb; ++j) {
-            const int64_t row = (prev_first + j0 + j) * p.H + h;
-            if (p.taps) {
-                load_vectors_conv<D, TIO>(tv[j], w, p.taps, c.q, c.k, c.v, c.g, c.beta, row, false);
-                if (j0 + j == jsnap && t < D) conv_store(w, p, c.conv_snapshots, srow, h, D, t);
-            } else {
-                load_vectors<D, TIO>(tv[j], nullptr, c.k, c.v, c.g, c.beta, row);
-            }
-        }
-        __syncthreads();
-        if (p.taps) {
-            if (warp < nb) token_finish<D>(tv[warp], true, false);
-            for (int j = Sh::NW; j < nb; ++j)
-                if (warp == 0) token_finish<D>(tv[j], true, false);
-            __syncthreads();
-        }
-        for (int j = 0; j < nb; ++j) {
-            kda_step<D, false>(st, tv[j], red[parity], 0.f);
-            parity ^= 1;
-            if (j0 + j == jsnap) {
-                float *dst = c.snapshots + (srow * p.H + h) * (int64_t)D * D;
-#pragma unroll
-                for (int m = 0; m < Sh::R; ++m) st_stream(dst + (int64_t)(rs + Sh::RS * m) * D + cg * 4, st[m]);
-            }
+            kda_step<D, false>(st, tv[j], 0.f);
+            if (j0 + j == jsnap) store_state<D>(st, c.snapshots + (srow * p.H + h) * (int64_t)D * D);
         }
     }
-    if (na > 0) {
-#pragma unroll
-        for (int m = 0; m < Sh::R; ++m) st_stream(S + (int64_t)(rs + Sh::RS * m) * D + cg * 4, st[m]);
-        if (p.taps && t < D) conv_store(w, p, p.conv, slot, h, D, t);
+    if (na > 0 && !cnew) {
+        store_state<D>(st, S);
+        if (CONV && t < D) conv_store(w, p, p.conv, slot, h, D, t);
     }
-    // 2. verify this step's tokens from the committed state: outputs only
-    const int n_tok = p.tok0[s + 1] - p.tok0[s];
+    // 2. this step's tokens from the committed state: outputs; with commit_new the
+    // state after them is written too (decode, or a short prefill appended in the step)
     const int64_t tok_first = p.tok_base + p.tok0[s];
     for (int j0 = 0; j0 < n_tok; j0 += kTokBatch) {
         const int nb = min(kTokBatch, n_tok - j0);
         __syncthreads();
+        const int64_t js = cnew ? jsnap - na - j0 : -1;      // snapshot inside this batch?
+        const ConvOut co{nullptr, 0, c.conv_snapshots, srow, (js >= 0 && js < nb) ? (int)js : -1};
+        stage_batch<D, TIO, CONV>(tv, nb, (tok_first + j0) * p.H + h, p.H, p.q, p.k, p.v, p.g, p.beta,
+                                  w, p, h, co);
+        finish_batch<D>(tv, nb, CONV, true);
         for (int j = 0; j < nb; ++j) {
+            const float4 o = kda_step<D>(st, tv[j], p.scale);
             const int64_t row = (tok_first + j0 + j) * p.H + h;
-            if (p.taps)
-                load_vectors_conv<D, TIO>(tv[j], w, p.taps, p.q, p.k, p.v, p.g, p.beta, row, true);
-            else
-                load_token<D, TIO>(tv[j], p, row);
+            if ((t & 31) < 4) IO<TIO>::st4(static_cast<TIO *>(p.o) + row * D + lane_col<D>(), o);
+            if (j == js) store_state<D>(st, c.snapshots + (srow * p.H + h) * (int64_t)D * D);
         }
-        __syncthreads();
-        if (warp < nb) token_finish<D>(tv[warp], p.taps > 0, true);
-        for (int j = Sh::NW; j < nb; ++j)
-            if (warp == 0) token_finish<D>(tv[j], p.taps > 0, true);
-        __syncthreads();
-        for (int j = 0; j < nb; ++j) {
-            const float4 o = kda_step<D>(st, tv[j], red[parity], p.scale);
-            parity ^= 1;
-            const int64_t row = (tok_first + j0 + j) * p.H + h;
-            if (rs == 0) IO<TIO>::st4(static_cast<TIO *>(p.o) + row * D + cg * 4, o);
-        }
+    }
+    if (cnew) {
+        store_state<D>(st, S);
+        if (CONV && t < D) conv_store(w, p, p.conv, slot, h, D, t);
     }
 }
 

@@ -64,10 +64,14 @@ static float eff_scale(const kda_dims *d) {
 template <int D, typename TIO>
 static kda_status launch_decode(DecodeParams &p, int n_blocks, cudaStream_t st, bool verify) {
     if (!launch_gate()) return KDA_ERR_CUDA;
-    if (verify)
-        verify_kernel<D, TIO><<<n_blocks, DecodeShape<D>::NT, 0, st>>>(p);
-    else
-        decode_kernel<D, TIO><<<n_blocks, DecodeShape<D>::NT, 0, st>>>(p);
+    const bool conv = p.taps > 0;
+    if (verify) {
+        if (conv) verify_kernel<D, TIO, true><<<n_blocks, DecodeShape<D>::NT, 0, st>>>(p);
+        else verify_kernel<D, TIO, false><<<n_blocks, DecodeShape<D>::NT, 0, st>>>(p);
+    } else {
+        if (conv) decode_kernel<D, TIO, true><<<n_blocks, DecodeShape<D>::NT, 0, st>>>(p);
+        else decode_kernel<D, TIO, false><<<n_blocks, DecodeShape<D>::NT, 0, st>>>(p);
+    }
     return last_launch_status();
 }
 
@@ -85,11 +89,16 @@ template <typename TIO>
 static kda_status dispatch_verify_commit(int D, VerifyCommitParams &P, int n_blocks, cudaStream_t st) {
     if (D != 32 && D != 64 && D != 128) return KDA_ERR_UNSUPPORTED;
     if (!launch_gate()) return KDA_ERR_CUDA;
+    const bool conv = P.p.taps > 0;
+#define KDA_VC(d)                                                                                    \
+    if (conv) verify_commit_kernel<d, TIO, true><<<n_blocks, DecodeShape<d>::NT, 0, st>>>(P);        \
+    else verify_commit_kernel<d, TIO, false><<<n_blocks, DecodeShape<d>::NT, 0, st>>>(P);
     switch (D) {
-    case 32: verify_commit_kernel<32, TIO><<<n_blocks, DecodeShape<32>::NT, 0, st>>>(P); break;
-    case 64: verify_commit_kernel<64, TIO><<<n_blocks, DecodeShape<64>::NT, 0, st>>>(P); break;
-    default: verify_commit_kernel<128, TIO><<<n_blocks, DecodeShape<128>::NT, 0, st>>>(P); break;
+    case 32: KDA_VC(32) break;
+    case 64: KDA_VC(64) break;
+    default: KDA_VC(128) break;
     }
+#undef KDA_VC
     return last_launch_status();
 }
 
@@ -434,8 +443,8 @@ static kda_status verify_commit_impl(
     const float *beta_prev, const int32_t *n_accept, const int64_t *pos, int32_t snap_interval,
     const int64_t *snap_row, float *snapshots, float *conv_snapshots, int64_t n_snap_rows,
     const int32_t *cu_draft, const void *q, const void *k, const void *v, const float *g,
-    const float *beta, const int32_t *slots, int32_t n_slots, float *pool, float *conv_pool,
-    void *o, kda_stream_t stream) {
+    const float *beta, const uint8_t *commit_new, const int32_t *slots, int32_t n_slots,
+    float *pool, float *conv_pool, void *o, kda_stream_t stream) {
     kda_status st = check_dims(dims, false);
     if (st != KDA_OK) return st;
     if ((st = check_conv(conv)) != KDA_OK) return st;
@@ -453,7 +462,8 @@ static kda_status verify_commit_impl(
     if (snap_interval > 0 && snap_row && (!pos || !snapshots || (conv && !conv_snapshots)))
         return KDA_ERR_INVALID;
     const void *ptrs[] = {q_prev, k_prev, v_prev, g_prev, beta_prev, n_accept, pos, snap_row,
-                          snapshots, conv_snapshots, q, k, v, g, beta, slots, pool, conv_pool, o};
+                          snapshots, conv_snapshots, q, k, v, g, beta, slots, pool, conv_pool, o,
+                          commit_new};
     for (const void *ptr : ptrs)
         if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
@@ -475,6 +485,7 @@ static kda_status verify_commit_impl(
         c.n_accept = n_accept + g0;
         c.pos = pos ? pos + g0 : nullptr;
         c.snap_row = (snap_interval > 0 && snap_row) ? snap_row + g0 : nullptr;
+        c.commit_new = commit_new ? commit_new + g0 : nullptr;
         c.snapshots = snapshots; c.n_snap_rows = n_snap_rows; c.snap_interval = snap_interval;
         c.tok_base = cu_prev[g0];
         for (int i = 0; i <= ng; ++i) c.tok0[i] = cu_prev[g0 + i] - cu_prev[g0];
@@ -491,12 +502,12 @@ kda_status kda_verify_commit(const kda_dims *dims, int32_t n_seq, const int32_t 
                              int32_t snap_interval, const int64_t *snap_row, float *snapshots,
                              int64_t n_snap_rows, const int32_t *cu_draft, const void *q,
                              const void *k, const void *v, const float *g, const float *beta,
-                             const int32_t *slots, int32_t n_slots, float *pool, void *o,
-                             kda_stream_t stream) {
+                             const uint8_t *commit_new, const int32_t *slots, int32_t n_slots,
+                             float *pool, void *o, kda_stream_t stream) {
     return verify_commit_impl(dims, nullptr, n_seq, cu_prev, nullptr, k_prev, v_prev, g_prev,
                               beta_prev, n_accept, pos, snap_interval, snap_row, snapshots, nullptr,
-                              n_snap_rows, cu_draft, q, k, v, g, beta, slots, n_slots, pool,
-                              nullptr, o, stream);
+                              n_snap_rows, cu_draft, q, k, v, g, beta, commit_new, slots, n_slots,
+                              pool, nullptr, o, stream);
 }
 
 kda_status kda_verify_commit_conv(const kda_dims *dims, const kda_conv *conv, int32_t n_seq,
@@ -507,13 +518,14 @@ kda_status kda_verify_commit_conv(const kda_dims *dims, const kda_conv *conv, in
                                   float *snapshots, float *conv_snapshots, int64_t n_snap_rows,
                                   const int32_t *cu_draft, const void *q, const void *k,
                                   const void *v, const float *g, const float *beta,
-                                  const int32_t *slots, int32_t n_slots, float *pool,
-                                  float *conv_pool, void *o, kda_stream_t stream) {
+                                  const uint8_t *commit_new, const int32_t *slots,
+                                  int32_t n_slots, float *pool, float *conv_pool, void *o,
+                                  kda_stream_t stream) {
     if (!conv) return KDA_ERR_INVALID;
     return verify_commit_impl(dims, conv, n_seq, cu_prev, q_prev, k_prev, v_prev, g_prev,
                               beta_prev, n_accept, pos, snap_interval, snap_row, snapshots,
-                              conv_snapshots, n_snap_rows, cu_draft, q, k, v, g, beta, slots,
-                              n_slots, pool, conv_pool, o, stream);
+                              conv_snapshots, n_snap_rows, cu_draft, q, k, v, g, beta, commit_new,
+                              slots, n_slots, pool, conv_pool, o, stream);
 }
 
 kda_status kda_qk_frontend(const kda_dims *dims, const kda_conv *conv, int32_t n_seq,

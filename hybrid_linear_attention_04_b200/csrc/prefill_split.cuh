@@ -87,10 +87,15 @@ __host__ __device__ constexpr uint32_t u_piece(int hf, int wg, int q4, int r) {
 }
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RANGE_LIMIT2 = 80.f * LOG2E;      // 80 nats, in log2 units
+// raw q, k and b of the channels beyond that range ([kMaxFast][64] fp32 each), in the tail
+// of g's buffer (free once the cumsum has read g, until A_qk is staged after the correction)
+constexpr int kMaxFast = 8;
+constexpr uint32_t P_FQ = P_G + 24576, P_FK = P_FQ + kMaxFast * 256, P_FB = P_FK + kMaxFast * 256;
 static_assert(P_WSC + 8 * 8 * 72 * 2 <= P_AQK && P_AQK + 8192 <= P_TOT && P_AQK % 1024 == 0,
               "solve scratch overlaps");
 static_assert(P_KBLO + 16384 <= P_TOT && P_LO1 % 1024 == 0 && P_KBLO % 1024 == 0,
               "low parts overlap live data");
+static_assert(P_FQ >= P_KBLO + 16384 && P_FB + kMaxFast * 256 <= P_TOT, "fast-channel staging");
 static_assert(2 * (P_SMEM + 1024) <= 233472, "two prep CTAs per SM");
 static_assert(STAGE % 1024 == 0 && PACKET % 16 == 0 && C_O % 1024 == 0 && C_SN % 1024 == 0, "alignment");
 static_assert(C_SMEM <= 232448, "chain shared memory");
@@ -130,9 +135,21 @@ __device__ __forceinline__ float2 bf16x2_unpack(uint32_t u) {
 // a, b -> (bf16 pair hi, bf16 pair lo) with hi + lo = (a, b) to about 2^-17 relative:
 // the operands of a three-term bf16 product hi*hi' + lo*hi' + hi*lo' that is accurate to
 // fp32 level although the tensor cores take bf16
+// The same pair by integer round-to-nearest-even on the ALU (finite inputs; bit-identical
+// to the conversion instruction): the prep kernel's conversion/MUFU pipe is its busiest
+// unit, held by the exponentials, while its integer pipe has room.
+__device__ __forceinline__ uint32_t bf16x2_alu(float a, float b) {
+    uint32_t ua = __float_as_uint(a), ub = __float_as_uint(b);
+    ua += 0x7fffu + ((ua >> 16) & 1u);
+    ub += 0x7fffu + ((ub >> 16) & 1u);
+    return __byte_perm(ua, ub, 0x7632);
+}
+__device__ __forceinline__ uint4 bf16x8_alu(const float *a, float s) {
+    return make_uint4(bf16x2_alu(s * a[0], s * a[1]), bf16x2_alu(s * a[2], s * a[3]),
+                      bf16x2_alu(s * a[4], s * a[5]), bf16x2_alu(s * a[6], s * a[7]));
+}
 __device__ __forceinline__ void bf16x2_split(float a, float b, uint32_t &hi, uint32_t &lo) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-    hi = *reinterpret_cast<const uint32_t *>(&h);
+    hi = bf16x2_alu(a, b);
     // the residuals are exact in fp32; they are truncated to bf16 (their upper halves,
     // one byte permute instead of a second conversion): error below 2^-17 of a, b
     const float ra = a - __uint_as_float(hi << 16), rb = b - __uint_as_float(hi & 0xffff0000u);
@@ -225,7 +242,8 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
             for (int e = 0; e < 4; ++e) b[i][e] += b[i - 1][e];
         *reinterpret_cast<float4 *>(Tot + warp * 128 + 4 * lane) = make_float4(b[7][0], b[7][1], b[7][2], b[7][3]);
         __syncthreads();
-        float m2[4] = {0.f, 0.f, 0.f, 0.f};
+        float m2[4] = {0.f, 0.f, 0.f, 0.f}, r1[4], r2[4];
+        int n_fast;                       // channels on the second reference (block-uniform)
         {
             float off[4] = {0.f, 0.f, 0.f, 0.f}, bc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -243,18 +261,57 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
             for (int i = 0; i < 8; ++i)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) b[i][e] += off[e];
+            // references per channel: the chunk middle, or (beyond the range) 0 and b_C
+            bool fast[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                fast[e] = -m2[e] > RANGE_LIMIT2 || m2[e] - bc[e] > RANGE_LIMIT2;
+                r1[e] = fast[e] ? 0.f : m2[e];
+                r2[e] = fast[e] ? bc[e] : m2[e];
+            }
+            n_fast = fast_channels(fast).n;
             if (warp == 0) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int ch = 4 * lane + e;
-                    eM[ch] = tc::ex2(m2[e]);
-                    eC[ch] = tc::ex2(bc[e] - m2[e]);
+                    eM[ch] = tc::ex2(r1[e]);
+                    eC[ch] = tc::ex2(bc[e] - r2[e]);
                     gC[ch] = tc::ex2(bc[e]);
-                    if (-m2[e] > RANGE_LIMIT2 || m2[e] - bc[e] > RANGE_LIMIT2) record_status(KDA_ERR_RANGE);
                 }
+                if (lane == 0 && n_fast > kMaxFast) record_status(KDA_ERR_RANGE);
             }
         }
-        // ---- Qh = q 2^(b-m), Ka = k 2^(b-m) in place; Kb = k 2^(m-b)
+        if (n_fast > 0) {
+            // raw q, k and b of the channels on the second reference (r1 != r2), for
+            // fast_correct, read before the pass below scales q and k in place
+            const int pkb = lane >> 4, pchk = (lane & 15) >> 1, phf = (lane & 1) * 8;
+            bool fast[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) fast[e] = r1[e] != r2[e];
+            const FastChannels fch = fast_channels(fast);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int r = 8 * warp + i;
+                const uint32_t so = tc::sw128(r, pchk) + phf;
+                const uint2 qv = *reinterpret_cast<const uint2 *>(sm + P_QK + pkb * 16384 + so);
+                const uint2 kv = *reinterpret_cast<const uint2 *>(sm + P_QK + pkb * 16384 + 8192 + so);
+                const float2 q01 = bf16x2_unpack(qv.x), q23 = bf16x2_unpack(qv.y);
+                const float2 k01 = bf16x2_unpack(kv.x), k23 = bf16x2_unpack(kv.y);
+                const float qr[4] = {q01.x, q01.y, q23.x, q23.y}, kr[4] = {k01.x, k01.y, k23.x, k23.y};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int f = fast[e] ? fast_index(fch, lane, e) : kMaxFast;
+                    if (f < kMaxFast) {
+                        const bool live = r < n;
+                        reinterpret_cast<float *>(sm + P_FQ)[f * 64 + r] = live ? qr[e] : 0.f;
+                        reinterpret_cast<float *>(sm + P_FK)[f * 64 + r] = live ? kr[e] : 0.f;
+                        reinterpret_cast<float *>(sm + P_FB)[f * 64 + r] = live ? b[i][e] : 0.f;
+                    }
+                }
+            }
+            __syncwarp();
+        }
+        // ---- Qh = q 2^(b-r1), Ka = k 2^(b-r1) in place; Kb = k 2^(r2-b)
         {
             const int pkb = lane >> 4, pchk = (lane & 15) >> 1, phf = (lane & 1) * 8;
 #pragma unroll
@@ -270,9 +327,8 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
                 float e1[4], e2[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float d = b[i][e] - m2[e];
-                    e1[e] = tc::ex2(d);
-                    e2[e] = tc::ex2(-d);
+                    e1[e] = tc::ex2(b[i][e] - r1[e]);
+                    e2[e] = tc::ex2(r2[e] - b[i][e]);
                 }
                 // high parts in place of q and k (and Kb), low parts in the P_LO* slabs
                 uint2 qh = make_uint2(0u, 0u), ql = qh, ah = qh, al = qh, bh = qh, bl = qh;
@@ -335,6 +391,17 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
             tc::tma_load3(sm + P_V + 8192, &P.tm_v, 64, h, z, bar_v);
             v_issued = true;
         }
+        if (n_fast > 0) {
+            // the pairwise part of the channels beyond the range, into A (TMEM)
+            if (warp < 4)
+                fast_correct<kMaxFast>(tbase + tlane + P_COL_A, 32 * warp + lane, n_fast,
+                                       reinterpret_cast<const float *>(sm + P_FQ),
+                                       reinterpret_cast<const float *>(sm + P_FK),
+                                       reinterpret_cast<const float *>(sm + P_FB));
+            tc::fence_before_sync();
+            __syncthreads();
+            tc::fence_after_sync();
+        }
         if (warp < 2) {
             // A_qk, masked to i <= r, into its staging image (bulk-stored after this phase)
             const int r = 32 * warp + lane;
@@ -349,7 +416,7 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int jj = 32 * half + 8 * q4 + 2 * e;
-                        w[e] = bf16x2(jj <= r ? a[8 * q4 + 2 * e] : 0.f, jj + 1 <= r ? a[8 * q4 + 2 * e + 1] : 0.f);
+                        w[e] = bf16x2_alu(jj <= r ? a[8 * q4 + 2 * e] : 0.f, jj + 1 <= r ? a[8 * q4 + 2 * e + 1] : 0.f);
                     }
                     *reinterpret_cast<uint4 *>(sm + P_AQK + tc::sw128(r, 4 * half + q4)) =
                         make_uint4(w[0], w[1], w[2], w[3]);
@@ -375,7 +442,7 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
                         l[e] = jj < r ? br * a[8 * q4 + e] : 0.f;
                         if (jj >= dblk && jj < dblk + 16) Ls[r * 17 + (jj - dblk)] = l[e];
                     }
-                    *reinterpret_cast<uint4 *>(Lb + r * 72 + 32 * half + 8 * q4) = bf16x8(l, 1.f);
+                    *reinterpret_cast<uint4 *>(Lb + r * 72 + 32 * half + 8 * q4) = bf16x8_alu(l, 1.f);
                 }
             }
             __syncwarp();
@@ -460,8 +527,8 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
                 // T Diag(beta) (bf16, K-major A operand of the next MMAs: W' = T Diag(beta) Ka,
                 // U = T Diag(beta) V); columns c0 + 2t, c0 + 2t + 1 are in 16-byte chunk `warp`
                 const float b0 = bet[c0 + 2 * t], b1 = bet[c0 + 2 * t + 1];
-                *reinterpret_cast<uint32_t *>(sm + P_TI + tc::sw128(r0, warp) + 4 * t) = bf16x2(w[0] * b0, w[1] * b1);
-                *reinterpret_cast<uint32_t *>(sm + P_TI + tc::sw128(r1, warp) + 4 * t) = bf16x2(w[2] * b0, w[3] * b1);
+                *reinterpret_cast<uint32_t *>(sm + P_TI + tc::sw128(r0, warp) + 4 * t) = bf16x2_alu(w[0] * b0, w[1] * b1);
+                *reinterpret_cast<uint32_t *>(sm + P_TI + tc::sw128(r1, warp) + 4 * t) = bf16x2_alu(w[2] * b0, w[3] * b1);
                 __syncwarp();
             }
         }
@@ -505,7 +572,7 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
                         for (int q4 = 0; q4 < 4; ++q4) {
                             const uint32_t off = mat ? P_G + u_piece(wh, hh, q4, r) - PK_U + 16384
                                                      : P_G + wh * 8192 + tc::sw128(r, 4 * hh + q4);
-                            *reinterpret_cast<uint4 *>(sm + off) = bf16x8(a + 8 * q4, 1.f);
+                            *reinterpret_cast<uint4 *>(sm + off) = bf16x8_alu(a + 8 * q4, 1.f);
                         }
                     }
                 }

@@ -72,6 +72,11 @@ constexpr uint32_t COL_A = 0, COL_O = 64, COL_S = 128, TMEM_COLS = 256;
 constexpr uint32_t CHUNK_TX = 16384 + 16384 + 32768 + 8192;   // bytes per chunk of loads
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RANGE_LIMIT2 = 80.f * LOG2E;    // 80 nats, in log2 units
+// raw q, k and b of the channels beyond that range ([kMaxFast][64] fp32 each) in TOT (read
+// only by the cumsum before them; a barrier separates the two when the staging is used)
+constexpr int kMaxFast = 4;
+constexpr uint32_t FQ = TOT, FK = TOT + kMaxFast * 256, FB = TOT + 2 * kMaxFast * 256;
+static_assert(3 * kMaxFast * 256 <= 8 * 128 * 4, "fast-channel staging");
 }  // namespace tcp
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -221,7 +226,8 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
             bnext = (ci + 1 < n_chunks && tid < nn) ? p.beta[(int64_t)(sq.tok0 + (ci + 1) * C + tid) * H + h] : 0.f;
         }
         __syncthreads();
-        float m2[4] = {0.f, 0.f, 0.f, 0.f};
+        float m2[4] = {0.f, 0.f, 0.f, 0.f}, r1[4], r2[4];
+        int n_fast;                       // channels on the second reference (block-uniform)
         {
             float off[4] = {0.f, 0.f, 0.f, 0.f}, bc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -239,18 +245,28 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
             for (int i = 0; i < 8; ++i)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) b[i][e] += off[e];
+            // references per channel: the chunk middle, or (beyond the range) 0 and b_C
+            // (b <= 0, so row 0 is at most -m above the middle)
+            bool fast[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                fast[e] = -m2[e] > RANGE_LIMIT2 || m2[e] - bc[e] > RANGE_LIMIT2;
+                r1[e] = fast[e] ? 0.f : m2[e];
+                r2[e] = fast[e] ? bc[e] : m2[e];
+            }
+            n_fast = fast_channels(fast).n;
             if (warp == 0) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int c = 4 * lane + e;
-                    eM[c] = tc::ex2(m2[e]);
-                    eC[c] = tc::ex2(bc[e] - m2[e]);
+                    eM[c] = tc::ex2(r1[e]);
+                    eC[c] = tc::ex2(bc[e] - r2[e]);
                     gC[c] = tc::ex2(bc[e]);
-                    // b <= 0, so row 0 is at most -m above the reference
-                    if (-m2[e] > RANGE_LIMIT2 || m2[e] - bc[e] > RANGE_LIMIT2) record_status(KDA_ERR_RANGE);
                 }
+                if (lane == 0 && n_fast > kMaxFast) record_status(KDA_ERR_RANGE);
             }
         }
+        if (n_fast > 0) __syncthreads();   // TOT (the cumsum totals) becomes the staging below
         // ---- C. scaled bf16 operands Qh = q 2^(b-m), Ka = k 2^(b-m), Kb = k 2^(m-b)
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -263,9 +279,26 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
             float e1[4], e2[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float d = b[i][e] - m2[e];
-                e1[e] = tc::ex2(d);
-                e2[e] = tc::ex2(-d);
+                e1[e] = tc::ex2(b[i][e] - r1[e]);
+                e2[e] = tc::ex2(r2[e] - b[i][e]);
+            }
+            if (n_fast > 0) {
+                // raw values of the channels on the second reference (r1 != r2), for fast_correct
+                const float qr[4] = {q01.x, q01.y, q23.x, q23.y}, kr[4] = {k01.x, k01.y, k23.x, k23.y};
+                bool fast[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) fast[e] = r1[e] != r2[e];
+                const FastChannels fch = fast_channels(fast);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int f = fast[e] ? fast_index(fch, lane, e) : kMaxFast;
+                    if (f < kMaxFast) {
+                        const bool live = r < n;
+                        reinterpret_cast<float *>(sm + FQ)[f * 64 + r] = live ? qr[e] : 0.f;
+                        reinterpret_cast<float *>(sm + FK)[f * 64 + r] = live ? kr[e] : 0.f;
+                        reinterpret_cast<float *>(sm + FB)[f * 64 + r] = live ? b[i][e] : 0.f;
+                    }
+                }
             }
             // high parts (the MMA operands) and low parts (for the fp32-accurate A)
             uint2 oq = make_uint2(0u, 0u), lq = oq, oa = oq, la = oq, ob = oq, lb = oq;
@@ -340,6 +373,12 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
         // wait is acted on at the block-wide vote after phase E
         ok = tc::bar_wait(warp < 4 ? bar_a : bar_b, (uint32_t)(ci & 1));
         tc::fence_after_sync();
+        // the pairwise part of the channels beyond the range, into A (each warp its own rows)
+        if (n_fast > 0 && warp < 4)
+            fast_correct<kMaxFast>(tbase + tlane + COL_A, 32 * warp + lane, n_fast,
+                                   reinterpret_cast<const float *>(sm + FQ),
+                                   reinterpret_cast<const float *>(sm + FK),
+                                   reinterpret_cast<const float *>(sm + FB));
         // ---- E. warps 0,1: A_qk (masked bf16 operand). Warps 2,3: L = Diag(beta)
         // A_kk (fp32), then the inverses X of its four 16x16 diagonal blocks by
         // forward substitution (each warp owns two blocks: no block-wide sync).

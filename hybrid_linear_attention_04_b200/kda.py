@@ -52,7 +52,7 @@ _SIGNATURES = {
     "kda_decode": (_I32, [_P, _I32, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P]),
     "kda_verify": (_I32, [_P, _I32, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P]),
     "kda_verify_commit": (_I32, [_P, _I32, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _I64, _P, _P,
-                                 _P, _P, _P, _P, _P, _I32, _P, _P, _P]),
+                                 _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P]),
     "kda_snapshot": (_I32, [_I32, _P, _P, _P, _I64, _P, _I64, _I32, _I32, _I32, _P]),
     "kda_state_map_apply": (_I32, [_I64, _I32, _I32, _P, _P, _P, _P, _P]),
     "kda_qk_frontend": (_I32, [_P, _P, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P]),
@@ -60,7 +60,8 @@ _SIGNATURES = {
     "kda_verify_conv": (_I32, [_P, _P, _I32, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P, _P,
                                _P]),
     "kda_verify_commit_conv": (_I32, [_P, _P, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P,
-                                      _P, _I64, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P]),
+                                      _P, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P,
+                                      _P]),
     "kda_status_string": (ctypes.c_char_p, [_I32]),
     "kda_check_device_status": (_I32, [_P]),
     "kda_launch_count": (_I64, []),
@@ -228,12 +229,13 @@ def kda_verify(q, k, v, g, beta, cu_draft, slots, state_pool, token_states, o, s
 
 
 def kda_verify_commit(prev, n_accept, cu_prev, q, k, v, g, beta, cu_draft, slots, state_pool, o,
-                      pos=None, snap_interval=0, snap_row=None, snapshots=None, scale=0.0,
-                      stream=None):
+                      pos=None, snap_interval=0, snap_row=None, snapshots=None, commit_new=None,
+                      scale=0.0, stream=None):
     """Speculative step with the previous step's commit fused in (see include/kda.h).
 
     ``prev``: dict of the previous batch's device tensors k, v, g, beta (packed by
-    ``cu_prev``), or None when it is empty; ``n_accept``: device int32 [n_seq].
+    ``cu_prev``), or None when it is empty; ``n_accept``: device int32 [n_seq];
+    ``commit_new``: device uint8 [n_seq] (mixed step: commit this step's tokens too).
     """
     cp = _host_array(cu_prev, np.int32)
     cd = _host_array(cu_draft, np.int32)
@@ -246,8 +248,8 @@ def kda_verify_commit(prev, n_accept, cu_prev, q, k, v, g, beta, cu_draft, slots
         ctypes.byref(dims), len(cd) - 1, _hptr(cp), _dptr(pv.get("k")), _dptr(pv.get("v")),
         _dptr(pv.get("g")), _dptr(pv.get("beta")), _dptr(n_accept), _dptr(pos), int(snap_interval),
         _dptr(snap_row), _dptr(snapshots), n_rows, _hptr(cd), _dptr(q), _dptr(k), _dptr(v),
-        _dptr(g), _dptr(beta), _dptr(slots), state_pool.shape[0], _dptr(state_pool), _dptr(o),
-        _stream(stream)), "kda_verify_commit")
+        _dptr(g), _dptr(beta), _dptr(commit_new), _dptr(slots), state_pool.shape[0],
+        _dptr(state_pool), _dptr(o), _stream(stream)), "kda_verify_commit")
 
 
 def _conv(w_q, w_k):
@@ -299,8 +301,8 @@ def kda_verify_conv(q, k, v, g, beta, cu_draft, slots, state_pool, conv_pool, to
 
 def kda_verify_commit_conv(prev, n_accept, cu_prev, q, k, v, g, beta, cu_draft, slots,
                            state_pool, conv_pool, o, w_q, w_k, pos=None, snap_interval=0,
-                           snap_row=None, snapshots=None, conv_snapshots=None, scale=0.0,
-                           stream=None):
+                           snap_row=None, snapshots=None, conv_snapshots=None, commit_new=None,
+                           scale=0.0, stream=None):
     """kda_verify_commit with the q/k front-end fused in; ``prev`` holds raw q too."""
     cp = _host_array(cu_prev, np.int32)
     cd = _host_array(cu_draft, np.int32)
@@ -315,8 +317,8 @@ def kda_verify_commit_conv(prev, n_accept, cu_prev, q, k, v, g, beta, cu_draft, 
         _dptr(pv.get("k")), _dptr(pv.get("v")), _dptr(pv.get("g")), _dptr(pv.get("beta")),
         _dptr(n_accept), _dptr(pos), int(snap_interval), _dptr(snap_row), _dptr(snapshots),
         _dptr(conv_snapshots), n_rows, _hptr(cd), _dptr(q), _dptr(k), _dptr(v), _dptr(g),
-        _dptr(beta), _dptr(slots), state_pool.shape[0], _dptr(state_pool), _dptr(conv_pool),
-        _dptr(o), _stream(stream)), "kda_verify_commit_conv")
+        _dptr(beta), _dptr(commit_new), _dptr(slots), state_pool.shape[0], _dptr(state_pool),
+        _dptr(conv_pool), _dptr(o), _stream(stream)), "kda_verify_commit_conv")
 
 
 def kda_state_map_apply(M, X, out, N=None, stream=None):

@@ -156,12 +156,14 @@ kda_status kda_prefill_workspace_size(const kda_dims *dims, int32_t n_seq,
  * A zero-length sequence writes state_out = state_in and no snapshots.
  * Errors (before launch): KDA_ERR_INVALID, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGN,
  * KDA_ERR_WORKSPACE (non-null workspace below kda_prefill_workspace_size).
- * Device status KDA_ERR_RANGE: a chunk whose per-channel decay exceeds the
- * tensor-core path's range: with b_r = g_0 + ... + g_r summed over the chunk's
- * tokens r = 0..63, some channel has -b_31 > 80 or b_31 - b_last > 80 (80 nats of
- * decay from the chunk's middle in either direction; any chunk whose total decay
- * sum(g) stays above -80 in every channel is within range). The outputs of that
- * chunk are then not reliable.
+ * Gate range on the tensor-core path: with b_r = g_0 + ... + g_r summed over a
+ * chunk's tokens r = 0..63, a key channel with -b_31 > 80 or b_31 - b_last > 80
+ * (more than 80 nats of decay from the chunk's middle in either direction) is
+ * computed on a second, bounded reference with its part of the intra-chunk
+ * products from pairwise exponentials; results are as for any other chunk. Up to 8
+ * such channels per chunk and head (two-launch path) or 4 (single launch) are
+ * handled; a chunk with more records device status KDA_ERR_RANGE and its outputs
+ * are then not reliable. The CUDA-core path has no such limit.
  */
 kda_status kda_prefill(const kda_dims *dims, int32_t n_seq, const int32_t *cu_seqlens_h,
                        const int64_t *start_pos_h, const void *q, const void *k,
@@ -254,9 +256,17 @@ kda_status kda_verify(const kda_dims *dims, int32_t n_seq, const int32_t *cu_dra
  *   2. verify: this step's tokens [cu_draft_h[s], cu_draft_h[s+1]) (q, k, v, g,
  *      beta) run from the committed state; their outputs go to o [cu_draft_h[n_seq],
  *      H, dv]; the state is not written.
+ * Mixed step (a serving step of continuous batching in one launch): with
+ * commit_new[s] != 0 (device uint8 [n_seq], nullable = all zero) the tokens of step 2
+ * are committed too, i.e. S is written after them (after step 1's tokens otherwise):
+ * a decode token (n_accept[s] = 0, one token), or a short prefill appended to a live
+ * sequence, runs in the same launch as the speculative sequences. A block-boundary
+ * snapshot then counts the committed tokens of both steps, in order.
  * The state after step 1 is bit-identical to kda_verify's state after token
  * n_accept[s] - 1 of the previous batch, and the outputs of step 2 to kda_verify's
- * from that state. A pipeline drains with a call whose draft batch is empty.
+ * from that state (with commit_new, the state written to kda_verify's state after the
+ * last token, and for one token to kda_decode's). A pipeline drains with a call
+ * whose draft batch is empty.
  *   n_accept [n_seq] (device int32), 0 <= n_accept[s] <= cu_prev_h[s+1] - cu_prev_h[s].
  *   pos [n_seq] (device int64, required with snapshots): tokens absorbed by S.
  *   snap_row [n_seq] (device int64, nullable), snapshots [n_snap_rows, H, dk, dv].
@@ -270,8 +280,8 @@ kda_status kda_verify_commit(const kda_dims *dims, int32_t n_seq, const int32_t 
                              int32_t snap_interval, const int64_t *snap_row, float *snapshots,
                              int64_t n_snap_rows, const int32_t *cu_draft_h, const void *q,
                              const void *k, const void *v, const float *g, const float *beta,
-                             const int32_t *slots, int32_t n_slots, float *state_pool, void *o,
-                             kda_stream_t stream);
+                             const uint8_t *commit_new, const int32_t *slots, int32_t n_slots,
+                             float *state_pool, void *o, kda_stream_t stream);
 
 /*
  * kda_snapshot — bit-exact copies of whole states between pools: for i < n,
@@ -340,8 +350,9 @@ kda_status kda_verify_commit_conv(const kda_dims *dims, const kda_conv *conv, in
                                   float *conv_snapshots, int64_t n_snap_rows,
                                   const int32_t *cu_draft_h, const void *q, const void *k,
                                   const void *v, const float *g, const float *beta,
-                                  const int32_t *slots, int32_t n_slots, float *state_pool,
-                                  float *conv_pool, void *o, kda_stream_t stream);
+                                  const uint8_t *commit_new, const int32_t *slots,
+                                  int32_t n_slots, float *state_pool, float *conv_pool, void *o,
+                                  kda_stream_t stream);
 
 /*
  * kda_state_map_apply — out[i] = M[i] X[i] + N[i] for i < n, fp32 (N nullable = 0).

@@ -187,7 +187,7 @@ def test_verify_commit_validation():
     def call(dims=d, n=2, cp=cu2, cd=cu2, kp=A, na=A, pos=None, snap=0, srow=None, sn=None,
              q=A, slots=A, pool=A, o=A):
         return L.kda_verify_commit(ctypes.byref(dims), n, P(cp), kp, A, A, A, na, pos, snap, srow,
-                                   sn, 0, P(cd), q, A, A, A, A, slots, 8, pool, o, None)
+                                   sn, 0, P(cd), q, A, A, A, A, None, slots, 8, pool, o, None)
     assert call(dims=_dims(d=48)) == 2                   # unsupported head dim
     assert call(n=-1) == 1
     assert call(cp=bad) == 1 and call(cd=bad) == 1       # decreasing offsets
@@ -235,8 +235,8 @@ def test_frontend_validation():
                              A, A, MIS, A, None) == 3
     # verify+commit with the front-end needs the previous batch's raw q
     assert L.kda_verify_commit_conv(ctypes.byref(d), ctypes.byref(conv), 2, P(c2), None, A, A, A, A,
-                                    A, None, 0, None, None, None, 0, P(c2), A, A, A, A, A, A, 8, A,
-                                    A, A, None) == 1
+                                    A, None, 0, None, None, None, 0, P(c2), A, A, A, A, A, None, A,
+                                    8, A, A, A, None) == 1
 
 
 def test_no_launch_issued_by_host_tests():

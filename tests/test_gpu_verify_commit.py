@@ -168,3 +168,74 @@ def test_verify_commit_drain_and_range(cuda_device):
         _, st, _ = native.oracle_sequence(xp["q"][a:a + na], xp["k"][a:a + na], xp["v"][a:a + na],
                                           xp["g"][a:a + na], xp["beta"][a:a + na], c["pool"][slot])
         check_states("drained state", got[slot].double().numpy()[None], st[None], TOL_BF16, (2, 3))
+
+
+def test_mixed_step_decode_append_and_verify_in_one_launch(cuda_device):
+    """One launch serving three kinds of sequences (continuous batching): plain decode
+    (one token, committed), a short prefill appended to a live sequence (several tokens,
+    committed) and speculative sequences (the previous step's accepted prefix committed,
+    this step's drafts only verified). Committed states equal kda_decode / kda_verify's
+    per-token states bit for bit, outputs equal kda_verify's, and a block-boundary
+    snapshot falling among appended tokens is written."""
+    H, d, n_seq, snap = 8, 128, 12, 64
+    c = _case(1201, n_seq, H, d, "bf16", cuda_device)
+    cp, cd = c["cp"], c["cd"]
+    kind = ["decode", "append", "verify"] * 4
+    # decode and append sequences commit nothing of the previous batch
+    acc = [a if kind[s] == "verify" else 0 for s, a in enumerate(c["acc"])]
+    lens = np.diff(cd).tolist()
+    for s in range(n_seq):
+        if kind[s] == "decode":
+            lens[s] = 1
+    cd = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    xc = synth.token_inputs(1202, int(cd[-1]), H, d, d, io="bf16")
+    dc = {k: v.to(cuda_device) for k, v in xc.items()}
+    pos = [snap * (s + 1) - 2 for s in range(n_seq)]          # boundaries 2 tokens ahead
+    sn = torch.full((n_seq, H, d, d), float("nan"), device=cuda_device)
+    pool_b = c["pool"].to(cuda_device)
+    o = torch.empty((int(cd[-1]), H, d), dtype=torch.bfloat16, device=cuda_device)
+    cnew = torch.tensor([k != "verify" for k in kind], dtype=torch.uint8, device=cuda_device)
+    K.kda_verify_commit(c["dp"], torch.tensor(acc, dtype=torch.int32, device=cuda_device), cp,
+                        dc["q"], dc["k"], dc["v"], dc["g"], dc["beta"], cd, c["slots_d"], pool_b, o,
+                        pos=torch.tensor(pos, dtype=torch.int64, device=cuda_device),
+                        snap_interval=snap,
+                        snap_row=torch.arange(n_seq, dtype=torch.int64, device=cuda_device),
+                        snapshots=sn, commit_new=cnew)
+    assert K.kda_check_device_status() == 0
+    # reference: commit the verify sequences' accepted prefix, then kda_verify of this batch
+    pool_a = c["pool"].to(cuda_device)
+    dp = c["dp"]
+    ts = torch.empty((int(cp[-1]), H, d, d), device=cuda_device)
+    K.kda_verify(dp["q"], dp["k"], dp["v"], dp["g"], dp["beta"], cp, c["slots_d"], pool_a, ts,
+                 torch.empty_like(dp["v"]))
+    keep = [s for s in range(n_seq) if acc[s] > 0]
+    K.kda_snapshot(torch.tensor([int(cp[s]) + acc[s] - 1 for s in keep], dtype=torch.int64,
+                                device=cuda_device),
+                   torch.tensor([c["slots"][s] for s in keep], dtype=torch.int64, device=cuda_device),
+                   ts, pool_a)
+    ts2 = torch.empty((int(cd[-1]), H, d, d), device=cuda_device)
+    o_ref = torch.empty_like(o)
+    K.kda_verify(dc["q"], dc["k"], dc["v"], dc["g"], dc["beta"], cd, c["slots_d"], pool_a, ts2, o_ref)
+    assert torch.equal(o, o_ref)
+    for s in range(n_seq):
+        slot = c["slots"][s]
+        if kind[s] == "verify":
+            assert torch.equal(pool_b[slot], pool_a[slot]), s
+            assert torch.isnan(sn[s]).all() or acc[s] >= 2
+        else:
+            assert torch.equal(pool_b[slot], ts2[int(cd[s + 1]) - 1]), s   # after the last token
+            if lens[s] >= 2:                                              # boundary at token 1
+                assert torch.equal(sn[s], ts2[int(cd[s]) + 1]), s
+            else:
+                assert torch.isnan(sn[s]).all(), s
+    # the decode sequences equal kda_decode itself
+    dec = [s for s in range(n_seq) if kind[s] == "decode"]
+    rows = torch.tensor([int(cd[s]) for s in dec], device=cuda_device)
+    pool_d = c["pool"].to(cuda_device)
+    od = torch.empty((len(dec), H, d), dtype=torch.bfloat16, device=cuda_device)
+    K.kda_decode(dc["q"][rows].contiguous(), dc["k"][rows].contiguous(), dc["v"][rows].contiguous(),
+                 dc["g"][rows].contiguous(), dc["beta"][rows].contiguous(),
+                 c["slots_d"][dec].contiguous(), pool_d, od)
+    for i, s in enumerate(dec):
+        assert torch.equal(pool_d[c["slots"][s]], pool_b[c["slots"][s]])
+        assert torch.equal(od[i], o[int(cd[s])])
