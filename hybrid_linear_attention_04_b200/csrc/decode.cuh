@@ -27,6 +27,7 @@
 // batch before it uses any.
 #pragma once
 #include "common.cuh"
+#include "tc_util.cuh"
 
 namespace kda {
 
@@ -349,6 +350,112 @@ __device__ __forceinline__ void store_state(const float4 (&st)[DecodeShape<D>::R
     for (int m = 0; m < DecodeShape<D>::R; ++m) st_stream(S + lane_off<D>(m), st[m]);
 }
 
+// ---- token rows staged by bulk copies (verify, verify + commit) ----------------
+// A CTA's tokens form one stream of batches of up to kTokBatch tokens (verify+commit:
+// the replayed prefix, then this step's tokens). Thread 0 copies a batch's raw q, k, v
+// and g rows into one of two shared-memory buffers with bulk asynchronous copies that
+// complete on that buffer's mbarrier, two batches ahead of their use, so the rows of
+// every batch arrive while the state is loaded and the previous batch is stepped.
+template <int D, typename TIO> struct RawTok {
+    static constexpr uint32_t QB = D * sizeof(TIO);     // one q, k or v row
+    static constexpr uint32_t BYTES = 3 * QB + D * 4;   // + one g row (fp32)
+    static constexpr uint32_t SMEM = 2 * kTokBatch * BYTES;   // dynamic shared memory
+};
+
+struct TokSrc {                 // tokens row0, row0 + H, ... of packed arrays
+    const void *q, *k, *v;      // q null: not staged (a replayed token without front-end)
+    const float *g, *beta;
+    int64_t row0;
+    int n;
+};
+
+template <int D, typename TIO>
+__device__ __forceinline__ void issue_rows(uint8_t *raw, const TokSrc &src, int j0, int nb, int H,
+                                           uint64_t *bar) {
+    using RT = RawTok<D, TIO>;
+    const uint32_t per = src.q ? RT::BYTES : RT::BYTES - RT::QB;   // every row keeps its slot
+    tc::bar_expect_tx(bar, per * (uint32_t)nb);
+    for (int j = 0; j < nb; ++j) {
+        const int64_t row = src.row0 + (int64_t)(j0 + j) * H;
+        uint8_t *dst = raw + j * RT::BYTES;
+        if (src.q) tc::bulk_load(dst, static_cast<const TIO *>(src.q) + row * D, RT::QB, bar);
+        tc::bulk_load(dst + RT::QB, static_cast<const TIO *>(src.k) + row * D, RT::QB, bar);
+        tc::bulk_load(dst + 2 * RT::QB, static_cast<const TIO *>(src.v) + row * D, RT::QB, bar);
+        tc::bulk_load(dst + 3 * RT::QB, src.g + row * D, D * 4, bar);
+    }
+}
+
+// Staged raw rows -> token vectors (the front-end's conv and Swish with CONV): threads
+// t < D channel t of q and k, in token order; threads t >= D channel t - D of v and g.
+// b: this thread's beta (threads D .. D + nb - 1), loaded ahead.
+template <int D, typename TIO, bool CONV>
+__device__ __forceinline__ void convert_batch(TokVec<D> *tv, const uint8_t *raw, int nb, bool read_q,
+                                              bool with_q, float b, ConvWin &w, const DecodeParams &p, int h,
+                                              const ConvOut &co) {
+    using RT = RawTok<D, TIO>;
+    const int t = threadIdx.x;
+    if (t < D) {
+        for (int j = 0; j < nb; ++j) {
+            const uint8_t *rj = raw + j * RT::BYTES;
+            const float xq = read_q ? IO<TIO>::ld(reinterpret_cast<const TIO *>(rj) + t) : 0.f;
+            const float xk = IO<TIO>::ld(reinterpret_cast<const TIO *>(rj + RT::QB) + t);
+            if (CONV) {
+                const float yq = conv_step(w.wq, w.hq, p.taps, xq);
+                const float yk = conv_step(w.wk, w.hk, p.taps, xk);
+                tv[j].q[t] = with_q ? swish(yq) : 0.f;
+                tv[j].k[t] = swish(yk);
+                if (co.tok) conv_store(w, p, co.tok, co.tok0 + j, h, D, t);
+                if (j == co.snap_j) conv_store(w, p, co.snap, co.snap_row, h, D, t);
+            } else {
+                tv[j].q[t] = with_q ? xq : 0.f;
+                tv[j].k[t] = xk;
+            }
+        }
+    } else {
+        const int c = t - D;
+        for (int j = 0; j < nb; ++j) {
+            const uint8_t *rj = raw + j * RT::BYTES;
+            tv[j].v[c] = IO<TIO>::ld(reinterpret_cast<const TIO *>(rj + 2 * RT::QB) + c);
+            tv[j].a[c] = expf(reinterpret_cast<const float *>(rj + 3 * RT::QB)[c]);
+        }
+        if (c < nb) tv[c].beta = b;
+    }
+}
+
+// The batch stream of one CTA: batches of src[0] (n0 tokens), then of src[1].
+struct TokStream {
+    TokSrc src[2];
+    int nb0, nbat;              // batches of src[0]; all batches
+    __device__ __forceinline__ void locate(int bi, int &which, int &j0, int &nb) const {
+        which = bi < nb0 ? 0 : 1;
+        j0 = (which ? bi - nb0 : bi) * kTokBatch;
+        nb = min(kTokBatch, src[which].n - j0);
+    }
+};
+
+__device__ __forceinline__ TokStream make_stream(const TokSrc &a, const TokSrc &b) {
+    TokStream s;
+    s.src[0] = a;
+    s.src[1] = b;
+    s.nb0 = (a.n + kTokBatch - 1) / kTokBatch;
+    s.nbat = s.nb0 + (b.n + kTokBatch - 1) / kTokBatch;
+    return s;
+}
+
+template <int D, typename TIO>
+__device__ __forceinline__ void issue_batch(const TokStream &ts, int bi, uint8_t *raw, uint64_t *bar, int H) {
+    int which, j0, nb;
+    ts.locate(bi, which, j0, nb);
+    issue_rows<D, TIO>(raw, ts.src[which], j0, nb, H, bar);
+}
+
+// beta of token c of batch bi (threads D + c), issued early as a plain load
+__device__ __forceinline__ float batch_beta(const TokStream &ts, int bi, int c, int H) {
+    int which, j0, nb;
+    ts.locate(bi, which, j0, nb);
+    return c < nb ? ts.src[which].beta[ts.src[which].row0 + (int64_t)(j0 + c) * H] : 0.f;
+}
+
 template <int D, typename TIO, bool CONV>
 __global__ void __launch_bounds__(DecodeShape<D>::NT, 2)
 decode_kernel(const __grid_constant__ DecodeParams p) {
@@ -379,7 +486,11 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
 template <int D, typename TIO, bool CONV>
 __global__ void __launch_bounds__(DecodeShape<D>::NT, 2)
 verify_kernel(const __grid_constant__ DecodeParams p) {
+    using RT = RawTok<D, TIO>;
     __shared__ TokVec<D> tv[kTokBatch];
+    extern __shared__ __align__(128) uint8_t dyn_smem[];   // two raw row buffers
+    uint8_t *raw[2] = {dyn_smem, dyn_smem + kTokBatch * RT::BYTES};
+    __shared__ uint64_t bars[2];
     const int s = blockIdx.x / p.H, h = blockIdx.x % p.H;
     const int32_t slot = p.slots[s];
     if (slot < 0 || slot >= p.n_slots) {
@@ -388,27 +499,49 @@ verify_kernel(const __grid_constant__ DecodeParams p) {
     }
     const int n_tok = p.tok0[s + 1] - p.tok0[s];
     const int64_t tok_first = p.tok_base + p.tok0[s];
-    const int t = threadIdx.x;
+    const int t = threadIdx.x, warp = t >> 5;
+    const TokSrc none{nullptr, nullptr, nullptr, nullptr, nullptr, 0, 0};
+    const TokStream ts = make_stream(TokSrc{p.q, p.k, p.v, p.g, p.beta, tok_first * p.H + h, n_tok}, none);
+    if (t == 0) {
+        tc::bar_init(&bars[0], 1);
+        tc::bar_init(&bars[1], 1);
+        tc::bar_init_fence();
+        for (int bi = 0; bi < 2 && bi < ts.nbat; ++bi) issue_batch<D, TIO>(ts, bi, raw[bi], &bars[bi], p.H);
+    }
+    float bnext = (t >= D && ts.nbat > 0) ? batch_beta(ts, 0, t - D, p.H) : 0.f;
     const float *S = p.pool + ((int64_t)slot * p.H + h) * (int64_t)D * D;
     float4 st[DecodeShape<D>::R];
 #pragma unroll
     for (int m = 0; m < DecodeShape<D>::R; ++m) st[m] = ld_stream(S + lane_off<D>(m));
     ConvWin w;
     if (CONV && t < D) conv_begin(w, p, p.conv, slot, h, D, t);
-    for (int j0 = 0; j0 < n_tok; j0 += kTokBatch) {
-        const int nb = min(kTokBatch, n_tok - j0);
-        __syncthreads();  // previous batch's vectors are no longer read
+    __syncthreads();  // barrier initialisation visible
+    bool ok = true;
+    for (int bi = 0; bi < ts.nbat; ++bi) {
+        int which, j0, nb;
+        ts.locate(bi, which, j0, nb);
+        const float b = bnext;
+        if (t >= D && bi + 1 < ts.nbat) bnext = batch_beta(ts, bi + 1, t - D, p.H);
+        ok = tc::bar_wait(&bars[bi & 1], (uint32_t)((bi >> 1) & 1)) && ok;
         const ConvOut co{p.conv_tok, tok_first + j0, nullptr, 0, -1};
-        stage_batch<D, TIO, CONV>(tv, nb, (tok_first + j0) * p.H + h, p.H, p.q, p.k, p.v, p.g, p.beta,
-                                  w, p, h, co);
-        finish_batch<D>(tv, nb, CONV, true);
+        convert_batch<D, TIO, CONV>(tv, raw[bi & 1], nb, true, true, b, w, p, h, co);
+        __syncthreads();  // vectors staged, raw buffer read
+        if (t == 0 && bi + 2 < ts.nbat) issue_batch<D, TIO>(ts, bi + 2, raw[bi & 1], &bars[bi & 1], p.H);
+        if (warp < nb) token_finish<D>(tv[warp], CONV, true);
+        for (int j = DecodeShape<D>::NW; j < nb; ++j)
+            if (warp == 0) token_finish<D>(tv[j], CONV, true);
+        __syncthreads();
         for (int j = 0; j < nb; ++j) {
             const float4 o = kda_step<D>(st, tv[j], p.scale);
             const int64_t row = (tok_first + j0 + j) * p.H + h;
             store_state<D>(st, p.token_states + row * (int64_t)D * D);
             if ((t & 31) < 4) IO<TIO>::st4(static_cast<TIO *>(p.o) + row * D + lane_col<D>(), o);
         }
+        __syncthreads();  // the vectors are free for the next batch
     }
+    if (!ok && t == 0)  // copies still in flight land before the shared memory is released
+        for (int bi = ts.nbat - 2 < 0 ? 0 : ts.nbat - 2; bi < ts.nbat; ++bi)
+            tc::bar_wait(&bars[bi & 1], (uint32_t)((bi >> 1) & 1), 1u << 16);
 }
 
 // ---------------------------------------------------------------- verify + commit
@@ -440,9 +573,13 @@ struct VerifyCommitParams {
 template <int D, typename TIO, bool CONV>
 __global__ void __launch_bounds__(DecodeShape<D>::NT, 2)
 verify_commit_kernel(const __grid_constant__ VerifyCommitParams P) {
+    using RT = RawTok<D, TIO>;
     const DecodeParams &p = P.p;
     const CommitParams &c = P.c;
     __shared__ TokVec<D> tv[kTokBatch];
+    extern __shared__ __align__(128) uint8_t dyn_smem[];   // two raw row buffers
+    uint8_t *raw[2] = {dyn_smem, dyn_smem + kTokBatch * RT::BYTES};
+    __shared__ uint64_t bars[2];
     const int s = blockIdx.x / p.H, h = blockIdx.x % p.H;
     const int32_t slot = p.slots[s];
     const int m_prev = c.tok0[s + 1] - c.tok0[s];
@@ -461,53 +598,74 @@ verify_commit_kernel(const __grid_constant__ VerifyCommitParams P) {
     // committed tokens: the replayed prefix, then (mixed step) this step's tokens;
     // jsnap indexes that sequence
     const bool cnew = c.commit_new != nullptr && c.commit_new[s] != 0 && n_tok > 0;
-    const int t = threadIdx.x;
+    const int t = threadIdx.x, warp = t >> 5;
+    // the stream: the replayed prefix of the previous batch (its q only for the front-end's
+    // window), then this step's tokens
+    const int64_t prev_first = c.tok_base + c.tok0[s];
+    const int64_t tok_first = p.tok_base + p.tok0[s];
+    const TokStream ts = make_stream(TokSrc{CONV ? c.q : nullptr, c.k, c.v, c.g, c.beta, prev_first * p.H + h, na},
+                                     TokSrc{p.q, p.k, p.v, p.g, p.beta, tok_first * p.H + h, n_tok});
+    if (t == 0) {
+        tc::bar_init(&bars[0], 1);
+        tc::bar_init(&bars[1], 1);
+        tc::bar_init_fence();
+        for (int bi = 0; bi < 2 && bi < ts.nbat; ++bi) issue_batch<D, TIO>(ts, bi, raw[bi], &bars[bi], p.H);
+    }
+    float bnext = (t >= D && ts.nbat > 0) ? batch_beta(ts, 0, t - D, p.H) : 0.f;
     float *S = p.pool + ((int64_t)slot * p.H + h) * (int64_t)D * D;
     float4 st[DecodeShape<D>::R];
     load_state<D>(st, S);
     ConvWin w;
     if (CONV && t < D) conv_begin(w, p, p.conv, slot, h, D, t);
-    // 1. commit: replay the accepted prefix of the previous batch (state only)
-    const int64_t prev_first = c.tok_base + c.tok0[s];
-    for (int j0 = 0; j0 < na; j0 += kTokBatch) {
-        const int nb = min(kTokBatch, na - j0);
+    __syncthreads();  // barrier initialisation visible
+    bool ok = true;
+    for (int bi = 0; bi < ts.nbat; ++bi) {
+        int which, j0, nb;
+        ts.locate(bi, which, j0, nb);
+        const bool replay = which == 0;
+        const float b = bnext;
+        if (t >= D && bi + 1 < ts.nbat) bnext = batch_beta(ts, bi + 1, t - D, p.H);
+        ok = tc::bar_wait(&bars[bi & 1], (uint32_t)((bi >> 1) & 1)) && ok;
+        // the committed-token index of this batch's first token, and a snapshot inside it
+        const int64_t c0 = replay ? j0 : (cnew ? na + j0 : -1);
+        const int64_t js = (c0 >= 0 && jsnap >= c0 && jsnap < c0 + nb) ? jsnap - c0 : -1;
+        const ConvOut co{nullptr, 0, c.conv_snapshots, srow, (int)js};
+        convert_batch<D, TIO, CONV>(tv, raw[bi & 1], nb, CONV || !replay, !replay, b, w, p, h, co);
+        __syncthreads();  // vectors staged, raw buffer read
+        if (t == 0 && bi + 2 < ts.nbat) issue_batch<D, TIO>(ts, bi + 2, raw[bi & 1], &bars[bi & 1], p.H);
+        if (warp < nb) token_finish<D>(tv[warp], CONV, !replay);
+        for (int j = DecodeShape<D>::NW; j < nb; ++j)
+            if (warp == 0) token_finish<D>(tv[j], CONV, !replay);
         __syncthreads();
-        const int sj = (jsnap >= j0 && jsnap < j0 + nb) ? (int)(jsnap - j0) : -1;
-        const ConvOut co{nullptr, 0, c.conv_snapshots, srow, sj};
-        stage_batch<D, TIO, CONV>(tv, nb, prev_first * p.H + h + (int64_t)j0 * p.H, p.H,
-                                  CONV ? c.q : nullptr, c.k, c.v, c.g, c.beta, w, p, h, co);
-        finish_batch<D>(tv, nb, CONV, false);
-        for (int j = 0; j < nb; ++j) {
-            kda_step<D, false>(st, tv[j], 0.f);
-            if (j0 + j == jsnap) store_state<D>(st, c.snapshots + (srow * p.H + h) * (int64_t)D * D);
+        if (replay) {
+            // 1. commit: the accepted prefix, state only
+            for (int j = 0; j < nb; ++j) {
+                kda_step<D, false>(st, tv[j], 0.f);
+                if (j == js) store_state<D>(st, c.snapshots + (srow * p.H + h) * (int64_t)D * D);
+            }
+            if (bi == ts.nb0 - 1 && !cnew) {
+                store_state<D>(st, S);
+                if (CONV && t < D) conv_store(w, p, p.conv, slot, h, D, t);
+            }
+        } else {
+            // 2. this step's tokens from the committed state: outputs (and with commit_new
+            // their state is committed too)
+            for (int j = 0; j < nb; ++j) {
+                const float4 o = kda_step<D>(st, tv[j], p.scale);
+                const int64_t row = (tok_first + j0 + j) * p.H + h;
+                if ((t & 31) < 4) IO<TIO>::st4(static_cast<TIO *>(p.o) + row * D + lane_col<D>(), o);
+                if (j == js) store_state<D>(st, c.snapshots + (srow * p.H + h) * (int64_t)D * D);
+            }
         }
-    }
-    if (na > 0 && !cnew) {
-        store_state<D>(st, S);
-        if (CONV && t < D) conv_store(w, p, p.conv, slot, h, D, t);
-    }
-    // 2. this step's tokens from the committed state: outputs; with commit_new the
-    // state after them is written too (decode, or a short prefill appended in the step)
-    const int64_t tok_first = p.tok_base + p.tok0[s];
-    for (int j0 = 0; j0 < n_tok; j0 += kTokBatch) {
-        const int nb = min(kTokBatch, n_tok - j0);
-        __syncthreads();
-        const int64_t js = cnew ? jsnap - na - j0 : -1;      // snapshot inside this batch?
-        const ConvOut co{nullptr, 0, c.conv_snapshots, srow, (js >= 0 && js < nb) ? (int)js : -1};
-        stage_batch<D, TIO, CONV>(tv, nb, (tok_first + j0) * p.H + h, p.H, p.q, p.k, p.v, p.g, p.beta,
-                                  w, p, h, co);
-        finish_batch<D>(tv, nb, CONV, true);
-        for (int j = 0; j < nb; ++j) {
-            const float4 o = kda_step<D>(st, tv[j], p.scale);
-            const int64_t row = (tok_first + j0 + j) * p.H + h;
-            if ((t & 31) < 4) IO<TIO>::st4(static_cast<TIO *>(p.o) + row * D + lane_col<D>(), o);
-            if (j == js) store_state<D>(st, c.snapshots + (srow * p.H + h) * (int64_t)D * D);
-        }
+        __syncthreads();  // the vectors are free for the next batch
     }
     if (cnew) {
         store_state<D>(st, S);
         if (CONV && t < D) conv_store(w, p, p.conv, slot, h, D, t);
     }
+    if (!ok && t == 0)  // copies still in flight land before the shared memory is released
+        for (int bi = ts.nbat - 2 < 0 ? 0 : ts.nbat - 2; bi < ts.nbat; ++bi)
+            tc::bar_wait(&bars[bi & 1], (uint32_t)((bi >> 1) & 1), 1u << 16);
 }
 
 }  // namespace kda

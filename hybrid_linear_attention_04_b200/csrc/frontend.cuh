@@ -7,12 +7,12 @@
 // sequence's conv state is its last taps-1 raw inputs, oldest first, laid out
 // [2 (q, k), H, D, taps-1] per sequence.
 //
-// One CTA (D threads; thread c owns channel c for q and k) per (sequence, C-token
-// tile, head): the tile's raw rows are read once, coalesced, with the window of the
-// previous taps-1 inputs in registers (from the sequence's conv state for its first
-// tile, from the rows before it otherwise); Swish outputs are staged in shared memory;
-// each warp then normalises whole rows and writes them out. The tile that ends on a
-// snapshot boundary writes the conv state there, the last tile the final conv state.
+// One warp per (sequence, C-token tile, head), four per CTA; lane l owns the D/32
+// consecutive channels from D/32 l for q and k, with their weights and conv windows in
+// registers (the window from the sequence's conv state for its first tile, from the
+// rows before it otherwise). Rows go in groups of four with all their loads issued
+// first; each row's L2 norm is a warp reduction. The tile that ends on a snapshot
+// boundary writes the conv state there, the last tile the final conv state.
 #pragma once
 #include "decode.cuh"
 #include "prefill_common.cuh"
@@ -35,104 +35,142 @@ struct FrontendParams {
 
 template <int D>
 struct FrontendShape {
-    static constexpr int NT = D, NW = D / 32, ROWS = 64;
-    static constexpr uint32_t smem_bytes = 2u * ROWS * D * 4u;   // Swish outputs of q and k
+    static constexpr int WARPS = 4;          // independent (tile, head) items per CTA
+    static constexpr int NT = 32 * WARPS;
+    static constexpr int CPL = D / 32;       // channels per lane: 4 lane .. (CPL lane + CPL - 1)
+    static constexpr int G = 4;              // rows whose loads are issued together
 };
 
+// CPL consecutive elements of a row (one vector access)
+template <typename TIO, int CPL>
+__device__ __forceinline__ void ld_vec(const TIO *p, float (&x)[CPL]) {
+    if (CPL == 4) {
+        const float4 v = IO<TIO>::ld4(p);
+        x[0] = v.x; x[1] = v.y; x[2 % CPL] = v.z; x[3 % CPL] = v.w;
+    } else {
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) x[e] = IO<TIO>::ld(p + e);
+    }
+}
+template <typename TIO, int CPL>
+__device__ __forceinline__ void st_vec(TIO *p, const float (&x)[CPL], float s) {
+    if (CPL == 4) {
+        IO<TIO>::st4(p, make_float4(x[0] * s, x[1 % CPL] * s, x[2 % CPL] * s, x[3 % CPL] * s));
+    } else {
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) IO<TIO>::st(p + e, x[e] * s);
+    }
+}
+
 template <int D, typename TIO>
-__global__ void __launch_bounds__(D) qk_frontend_kernel(const __grid_constant__ FrontendParams P) {
+__global__ void __launch_bounds__(FrontendShape<D>::NT) qk_frontend_kernel(const __grid_constant__ FrontendParams P) {
     using Sh = FrontendShape<D>;
-    extern __shared__ float fsm[];
-    float *zq = fsm, *zk = fsm + Sh::ROWS * D;
+    constexpr int CPL = Sh::CPL, G = Sh::G;
     const int H = P.H, K = P.taps, C = P.C;
-    const int h = blockIdx.x % H, row = blockIdx.x / H;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t item = (int64_t)blockIdx.x * Sh::WARPS + warp;
+    const int h = (int)(item % H);
+    const int64_t row = item / H;
     // owner sequence: the last one whose first tile row is <= row (rows of different
     // sequences never collide; see prefill_split.cuh for the same indexing)
-    auto first_row = [&](int i) { return (P.tok0[i] - P.tok_first) / C + i; };
+    auto first_row = [&](int i) { return (int64_t)(P.tok0[i] - P.tok_first) / C + i; };
     int lo = 0, hi = P.n_seq - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (first_row(mid) <= row) lo = mid; else hi = mid - 1;
     }
-    const int i = lo, b = row - first_row(i), len = P.len[i];
-    if (b < 0 || (b > 0 && b * C >= len)) return;          // an unused row (block-uniform)
-    const int c = threadIdx.x, warp = c >> 5, lane = c & 31;
+    const int i = lo, len = P.len[i];
+    const int64_t bt = row - first_row(i);
+    if (bt < 0 || (bt > 0 && bt * C >= len)) return;        // an unused row (warp-uniform)
+    const int b = (int)bt;
     const int n = max(0, min(C, len - b * C));
     const int64_t t0 = (int64_t)P.tok0[i] + (int64_t)b * C;
+    const int c0 = CPL * lane;
     const TIO *q = static_cast<const TIO *>(P.q), *k = static_cast<const TIO *>(P.k);
-    ConvWin w;
+    // weights and windows of the lane's channels
+    float wq[CPL][kMaxTaps], wk[CPL][kMaxTaps], hq[CPL][kMaxTaps - 1], hk[CPL][kMaxTaps - 1];
 #pragma unroll
-    for (int j = 0; j < kMaxTaps; ++j) {
-        w.wq[j] = j < K ? P.wq[((int64_t)h * D + c) * K + j] : 0.f;
-        w.wk[j] = j < K ? P.wk[((int64_t)h * D + c) * K + j] : 0.f;
+    for (int e = 0; e < CPL; ++e) {
+#pragma unroll
+        for (int j = 0; j < kMaxTaps; ++j) {
+            wq[e][j] = j < K ? P.wq[((int64_t)h * D + c0 + e) * K + j] : 0.f;
+            wk[e][j] = j < K ? P.wk[((int64_t)h * D + c0 + e) * K + j] : 0.f;
+        }
     }
-    // the window before the tile: conv state (first tile) or the raw rows before it
 #pragma unroll
     for (int j = 0; j < kMaxTaps - 1; ++j) {
-        float a = 0.f, bb = 0.f;
+        float xa[CPL], xb[CPL];
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) xa[e] = xb[e] = 0.f;
         if (j < K - 1) {
             if (b == 0) {
                 if (P.conv_in) {
-                    a = P.conv_in[conv_index(2 * i, H, h, D, c, K) + j];
-                    bb = P.conv_in[conv_index(2 * i + 1, H, h, D, c, K) + j];
+#pragma unroll
+                    for (int e = 0; e < CPL; ++e) {
+                        xa[e] = P.conv_in[conv_index(2 * i, H, h, D, c0 + e, K) + j];
+                        xb[e] = P.conv_in[conv_index(2 * i + 1, H, h, D, c0 + e, K) + j];
+                    }
                 }
             } else {
-                const int64_t r = t0 - (K - 1) + j;         // inside this sequence (b * C >= K - 1)
-                a = IO<TIO>::ld(q + (r * H + h) * D + c);
-                bb = IO<TIO>::ld(k + (r * H + h) * D + c);
+                const int64_t r = t0 - (K - 1) + j;             // inside this sequence (b * C >= K - 1)
+                ld_vec<TIO, CPL>(q + (r * H + h) * D + c0, xa);
+                ld_vec<TIO, CPL>(k + (r * H + h) * D + c0, xb);
             }
         }
-        w.hq[j] = a;
-        w.hk[j] = bb;
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) {
+            hq[e][j] = xa[e];
+            hk[e][j] = xb[e];
+        }
     }
-    for (int r = 0; r < n; ++r) {
-        const int64_t off = ((t0 + r) * H + h) * D + c;
-        zq[r * D + c] = swish(conv_step(w.wq, w.hq, K, IO<TIO>::ld(q + off)));
-        zk[r * D + c] = swish(conv_step(w.wk, w.hk, K, IO<TIO>::ld(k + off)));
+    TIO *qo = static_cast<TIO *>(P.q_out), *ko = static_cast<TIO *>(P.k_out);
+    for (int r0 = 0; r0 < n; r0 += G) {
+        float xq[G][CPL], xk[G][CPL];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            if (r0 + g < n) {
+                const int64_t off = ((t0 + r0 + g) * H + h) * D + c0;
+                ld_vec<TIO, CPL>(q + off, xq[g]);
+                ld_vec<TIO, CPL>(k + off, xk[g]);
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            if (r0 + g < n) {
+                float zq[CPL], zk[CPL], sq = 0.f, sk = 0.f;
+#pragma unroll
+                for (int e = 0; e < CPL; ++e) {
+                    zq[e] = swish(conv_step(wq[e], hq[e], K, xq[g][e]));
+                    zk[e] = swish(conv_step(wk[e], hk[e], K, xk[g][e]));
+                    sq = fmaf(zq[e], zq[e], sq);
+                    sk = fmaf(zk[e], zk[e], sk);
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                    sk += __shfl_xor_sync(0xffffffffu, sk, o);
+                }
+                const int64_t off = ((t0 + r0 + g) * H + h) * D + c0;
+                st_vec<TIO, CPL>(qo + off, zq, 1.f / fmaxf(sqrtf(sq), kNormEps));
+                st_vec<TIO, CPL>(ko + off, zk, 1.f / fmaxf(sqrtf(sk), kNormEps));
+            }
+        }
     }
     // conv states: at a snapshot boundary that ends this tile, and after the last token
+    auto put = [&](float *dst, int64_t srow) {
+#pragma unroll
+        for (int e = 0; e < CPL; ++e)
+#pragma unroll
+            for (int jj = 0; jj < kMaxTaps - 1; ++jj)
+                if (jj < K - 1) {
+                    dst[conv_index(2 * srow, H, h, D, c0 + e, K) + jj] = hq[e][jj];
+                    dst[conv_index(2 * srow + 1, H, h, D, c0 + e, K) + jj] = hk[e][jj];
+                }
+    };
     const int64_t p_end = P.start_pos[i] + (int64_t)b * C + n;
-    if (P.conv_snap && P.snap_interval > 0 && n == C && p_end % P.snap_interval == 0) {
-        const int64_t j = p_end / P.snap_interval - P.start_pos[i] / P.snap_interval - 1;
-        const int64_t srow = P.snap_off[i] + j;
-#pragma unroll
-        for (int jj = 0; jj < kMaxTaps - 1; ++jj)
-            if (jj < K - 1) {
-                P.conv_snap[conv_index(2 * srow, H, h, D, c, K) + jj] = w.hq[jj];
-                P.conv_snap[conv_index(2 * srow + 1, H, h, D, c, K) + jj] = w.hk[jj];
-            }
-    }
-    if (P.conv_out && (b + 1) * C >= len) {
-#pragma unroll
-        for (int jj = 0; jj < kMaxTaps - 1; ++jj)
-            if (jj < K - 1) {
-                P.conv_out[conv_index(2 * i, H, h, D, c, K) + jj] = w.hq[jj];
-                P.conv_out[conv_index(2 * i + 1, H, h, D, c, K) + jj] = w.hk[jj];
-            }
-    }
-    __syncthreads();
-    // L2 normalisation of whole rows, one warp per row
-    TIO *qo = static_cast<TIO *>(P.q_out), *ko = static_cast<TIO *>(P.k_out);
-    for (int r = warp; r < n; r += Sh::NW) {
-        float sq = 0.f, sk = 0.f;
-#pragma unroll
-        for (int e = lane; e < D; e += 32) {
-            sq = fmaf(zq[r * D + e], zq[r * D + e], sq);
-            sk = fmaf(zk[r * D + e], zk[r * D + e], sk);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            sq += __shfl_xor_sync(0xffffffffu, sq, o);
-            sk += __shfl_xor_sync(0xffffffffu, sk, o);
-        }
-        const float rq = 1.f / fmaxf(sqrtf(sq), kNormEps), rk = 1.f / fmaxf(sqrtf(sk), kNormEps);
-        const int64_t base = ((t0 + r) * H + h) * D;
-#pragma unroll
-        for (int e = lane; e < D; e += 32) {
-            IO<TIO>::st(qo + base + e, zq[r * D + e] * rq);
-            IO<TIO>::st(ko + base + e, zk[r * D + e] * rk);
-        }
-    }
+    if (P.conv_snap && P.snap_interval > 0 && n == C && p_end % P.snap_interval == 0)
+        put(P.conv_snap, P.snap_off[i] + p_end / P.snap_interval - P.start_pos[i] / P.snap_interval - 1);
+    if (P.conv_out && (b + 1) * C >= len) put(P.conv_out, i);
 }
 
 }  // namespace kda

@@ -63,11 +63,18 @@ static float eff_scale(const kda_dims *d) {
 // ---------------------------------------------------------------- decode ----
 template <int D, typename TIO>
 static kda_status launch_decode(DecodeParams &p, int n_blocks, cudaStream_t st, bool verify) {
-    if (!launch_gate()) return KDA_ERR_CUDA;
     const bool conv = p.taps > 0;
+    constexpr uint32_t dyn = RawTok<D, TIO>::SMEM;
     if (verify) {
-        if (conv) verify_kernel<D, TIO, true><<<n_blocks, DecodeShape<D>::NT, 0, st>>>(p);
-        else verify_kernel<D, TIO, false><<<n_blocks, DecodeShape<D>::NT, 0, st>>>(p);
+        static std::atomic<unsigned long long> attr[2]{{0}, {0}};
+        const kda_status r = conv ? set_smem_limit_once((const void *)verify_kernel<D, TIO, true>, dyn, attr[1])
+                                  : set_smem_limit_once((const void *)verify_kernel<D, TIO, false>, dyn, attr[0]);
+        if (r != KDA_OK) return r;
+    }
+    if (!launch_gate()) return KDA_ERR_CUDA;
+    if (verify) {
+        if (conv) verify_kernel<D, TIO, true><<<n_blocks, DecodeShape<D>::NT, dyn, st>>>(p);
+        else verify_kernel<D, TIO, false><<<n_blocks, DecodeShape<D>::NT, dyn, st>>>(p);
     } else {
         if (conv) decode_kernel<D, TIO, true><<<n_blocks, DecodeShape<D>::NT, 0, st>>>(p);
         else decode_kernel<D, TIO, false><<<n_blocks, DecodeShape<D>::NT, 0, st>>>(p);
@@ -88,11 +95,26 @@ static kda_status dispatch_decode(int D, DecodeParams &p, int n_blocks, cudaStre
 template <typename TIO>
 static kda_status dispatch_verify_commit(int D, VerifyCommitParams &P, int n_blocks, cudaStream_t st) {
     if (D != 32 && D != 64 && D != 128) return KDA_ERR_UNSUPPORTED;
-    if (!launch_gate()) return KDA_ERR_CUDA;
     const bool conv = P.p.taps > 0;
+    static std::atomic<unsigned long long> attr[3][2]{};
+    const int di = D == 32 ? 0 : D == 64 ? 1 : 2;
+    kda_status r = KDA_OK;
+#define KDA_VC_ATTR(d)                                                                                 \
+    r = conv ? set_smem_limit_once((const void *)verify_commit_kernel<d, TIO, true>,                    \
+                                   RawTok<d, TIO>::SMEM, attr[di][1])                                   \
+             : set_smem_limit_once((const void *)verify_commit_kernel<d, TIO, false>,                   \
+                                   RawTok<d, TIO>::SMEM, attr[di][0]);
+    switch (D) {
+    case 32: KDA_VC_ATTR(32) break;
+    case 64: KDA_VC_ATTR(64) break;
+    default: KDA_VC_ATTR(128) break;
+    }
+#undef KDA_VC_ATTR
+    if (r != KDA_OK) return r;
+    if (!launch_gate()) return KDA_ERR_CUDA;
 #define KDA_VC(d)                                                                                    \
-    if (conv) verify_commit_kernel<d, TIO, true><<<n_blocks, DecodeShape<d>::NT, 0, st>>>(P);        \
-    else verify_commit_kernel<d, TIO, false><<<n_blocks, DecodeShape<d>::NT, 0, st>>>(P);
+    if (conv) verify_commit_kernel<d, TIO, true><<<n_blocks, DecodeShape<d>::NT, RawTok<d, TIO>::SMEM, st>>>(P); \
+    else verify_commit_kernel<d, TIO, false><<<n_blocks, DecodeShape<d>::NT, RawTok<d, TIO>::SMEM, st>>>(P);
     switch (D) {
     case 32: KDA_VC(32) break;
     case 64: KDA_VC(64) break;
@@ -127,13 +149,10 @@ static kda_status dispatch_simt(int D, int C, const PrefillParams &p, cudaStream
 }
 
 template <int D, typename TIO>
-static kda_status launch_frontend(const FrontendParams &P, int64_t n_blocks, cudaStream_t st) {
-    static std::atomic<unsigned long long> attr_done{0};
-    const kda_status r = set_smem_limit_once((const void *)qk_frontend_kernel<D, TIO>,
-                                             (int)FrontendShape<D>::smem_bytes, attr_done);
-    if (r != KDA_OK) return r;
+static kda_status launch_frontend(const FrontendParams &P, int64_t n_items, cudaStream_t st) {
+    using Sh = FrontendShape<D>;
     if (!launch_gate()) return KDA_ERR_CUDA;
-    qk_frontend_kernel<D, TIO><<<(unsigned)n_blocks, D, FrontendShape<D>::smem_bytes, st>>>(P);
+    qk_frontend_kernel<D, TIO><<<(unsigned)((n_items + Sh::WARPS - 1) / Sh::WARPS), Sh::NT, 0, st>>>(P);
     return last_launch_status();
 }
 

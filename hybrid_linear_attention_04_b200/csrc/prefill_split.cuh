@@ -135,21 +135,8 @@ __device__ __forceinline__ float2 bf16x2_unpack(uint32_t u) {
 // a, b -> (bf16 pair hi, bf16 pair lo) with hi + lo = (a, b) to about 2^-17 relative:
 // the operands of a three-term bf16 product hi*hi' + lo*hi' + hi*lo' that is accurate to
 // fp32 level although the tensor cores take bf16
-// The same pair by integer round-to-nearest-even on the ALU (finite inputs; bit-identical
-// to the conversion instruction): the prep kernel's conversion/MUFU pipe is its busiest
-// unit, held by the exponentials, while its integer pipe has room.
-__device__ __forceinline__ uint32_t bf16x2_alu(float a, float b) {
-    uint32_t ua = __float_as_uint(a), ub = __float_as_uint(b);
-    ua += 0x7fffu + ((ua >> 16) & 1u);
-    ub += 0x7fffu + ((ub >> 16) & 1u);
-    return __byte_perm(ua, ub, 0x7632);
-}
-__device__ __forceinline__ uint4 bf16x8_alu(const float *a, float s) {
-    return make_uint4(bf16x2_alu(s * a[0], s * a[1]), bf16x2_alu(s * a[2], s * a[3]),
-                      bf16x2_alu(s * a[4], s * a[5]), bf16x2_alu(s * a[6], s * a[7]));
-}
 __device__ __forceinline__ void bf16x2_split(float a, float b, uint32_t &hi, uint32_t &lo) {
-    hi = bf16x2_alu(a, b);
+    hi = bf16x2(a, b);
     // the residuals are exact in fp32; they are truncated to bf16 (their upper halves,
     // one byte permute instead of a second conversion): error below 2^-17 of a, b
     const float ra = a - __uint_as_float(hi << 16), rb = b - __uint_as_float(hi & 0xffff0000u);
@@ -416,7 +403,7 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int jj = 32 * half + 8 * q4 + 2 * e;
-                        w[e] = bf16x2_alu(jj <= r ? a[8 * q4 + 2 * e] : 0.f, jj + 1 <= r ? a[8 * q4 + 2 * e + 1] : 0.f);
+                        w[e] = bf16x2(jj <= r ? a[8 * q4 + 2 * e] : 0.f, jj + 1 <= r ? a[8 * q4 + 2 * e + 1] : 0.f);
                     }
                     *reinterpret_cast<uint4 *>(sm + P_AQK + tc::sw128(r, 4 * half + q4)) =
                         make_uint4(w[0], w[1], w[2], w[3]);
@@ -442,7 +429,7 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
                         l[e] = jj < r ? br * a[8 * q4 + e] : 0.f;
                         if (jj >= dblk && jj < dblk + 16) Ls[r * 17 + (jj - dblk)] = l[e];
                     }
-                    *reinterpret_cast<uint4 *>(Lb + r * 72 + 32 * half + 8 * q4) = bf16x8_alu(l, 1.f);
+                    *reinterpret_cast<uint4 *>(Lb + r * 72 + 32 * half + 8 * q4) = bf16x8(l, 1.f);
                 }
             }
             __syncwarp();
@@ -527,8 +514,8 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
                 // T Diag(beta) (bf16, K-major A operand of the next MMAs: W' = T Diag(beta) Ka,
                 // U = T Diag(beta) V); columns c0 + 2t, c0 + 2t + 1 are in 16-byte chunk `warp`
                 const float b0 = bet[c0 + 2 * t], b1 = bet[c0 + 2 * t + 1];
-                *reinterpret_cast<uint32_t *>(sm + P_TI + tc::sw128(r0, warp) + 4 * t) = bf16x2_alu(w[0] * b0, w[1] * b1);
-                *reinterpret_cast<uint32_t *>(sm + P_TI + tc::sw128(r1, warp) + 4 * t) = bf16x2_alu(w[2] * b0, w[3] * b1);
+                *reinterpret_cast<uint32_t *>(sm + P_TI + tc::sw128(r0, warp) + 4 * t) = bf16x2(w[0] * b0, w[1] * b1);
+                *reinterpret_cast<uint32_t *>(sm + P_TI + tc::sw128(r1, warp) + 4 * t) = bf16x2(w[2] * b0, w[3] * b1);
                 __syncwarp();
             }
         }
@@ -572,7 +559,7 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
                         for (int q4 = 0; q4 < 4; ++q4) {
                             const uint32_t off = mat ? P_G + u_piece(wh, hh, q4, r) - PK_U + 16384
                                                      : P_G + wh * 8192 + tc::sw128(r, 4 * hh + q4);
-                            *reinterpret_cast<uint4 *>(sm + off) = bf16x8_alu(a + 8 * q4, 1.f);
+                            *reinterpret_cast<uint4 *>(sm + off) = bf16x8(a + 8 * q4, 1.f);
                         }
                     }
                 }
