@@ -69,9 +69,14 @@ struct DecodeParams {
 constexpr int kMaxTaps = 4;
 constexpr float kNormEps = 1e-6f;
 
+// One channel's conv weights (tap 0 .. taps-1) and window (its last taps-1 raw inputs,
+// oldest first), as scalars with the tap count branched on explicitly: an array form
+// indexed through the runtime tap count lands in local memory.
+struct Win {
+    float w0, w1, w2, w3, h0, h1, h2;
+};
 struct ConvWin {
-    float wq[kMaxTaps], wk[kMaxTaps];
-    float hq[kMaxTaps - 1], hk[kMaxTaps - 1];
+    Win q, k;
 };
 
 __device__ __forceinline__ int64_t conv_index(int64_t row2, int H, int h, int D, int c, int taps) {
@@ -79,52 +84,54 @@ __device__ __forceinline__ int64_t conv_index(int64_t row2, int H, int h, int D,
     return ((row2 * H + h) * D + c) * (int64_t)(taps - 1);
 }
 
-// weights and window of channel c from conv state row `row` (slot or token) of `src`
+// weights w[0..K-1] and the window state[0..K-2] (null: zeros)
+__device__ __forceinline__ void win_load(Win &c, const float *w, const float *state, int K) {
+    c.w0 = w[0];
+    c.w1 = w[1];
+    c.w2 = K > 2 ? w[2] : 0.f;
+    c.w3 = K > 3 ? w[3] : 0.f;
+    c.h0 = state ? state[0] : 0.f;
+    c.h1 = (state && K > 2) ? state[1] : 0.f;
+    c.h2 = (state && K > 3) ? state[2] : 0.f;
+}
+__device__ __forceinline__ void win_store(const Win &c, float *dst, int K) {
+    dst[0] = c.h0;
+    if (K > 2) dst[1] = c.h1;
+    if (K > 3) dst[2] = c.h2;
+}
+
+// one causal conv step: y = sum_j w_j x_{t-(K-1)+j} over the window and x, then shift x in
+__device__ __forceinline__ float conv_step(Win &c, int K, float x) {
+    float y;
+    if (K == 4) {
+        y = c.w3 * x;
+        y = fmaf(c.w0, c.h0, y); y = fmaf(c.w1, c.h1, y); y = fmaf(c.w2, c.h2, y);
+        c.h0 = c.h1; c.h1 = c.h2; c.h2 = x;
+    } else if (K == 3) {
+        y = c.w2 * x;
+        y = fmaf(c.w0, c.h0, y); y = fmaf(c.w1, c.h1, y);
+        c.h0 = c.h1; c.h1 = x;
+    } else {
+        y = c.w1 * x;
+        y = fmaf(c.w0, c.h0, y);
+        c.h0 = x;
+    }
+    return y;
+}
+
+// weights and windows of channel c from conv state row `row` (slot or token) of `src`
 __device__ __forceinline__ void conv_begin(ConvWin &w, const DecodeParams &p, const float *src, int64_t row,
                                            int h, int D, int c) {
     const int K = p.taps;
-#pragma unroll
-    for (int j = 0; j < kMaxTaps; ++j) {
-        w.wq[j] = j < K ? p.wq[((int64_t)h * D + c) * K + j] : 0.f;
-        w.wk[j] = j < K ? p.wk[((int64_t)h * D + c) * K + j] : 0.f;
-    }
-    const float *sq = src + conv_index(2 * row, p.H, h, D, c, K);
-    const float *sk = src + conv_index(2 * row + 1, p.H, h, D, c, K);
-#pragma unroll
-    for (int j = 0; j < kMaxTaps - 1; ++j) {
-        w.hq[j] = j < K - 1 ? sq[j] : 0.f;
-        w.hk[j] = j < K - 1 ? sk[j] : 0.f;
-    }
+    win_load(w.q, p.wq + ((int64_t)h * D + c) * K, src + conv_index(2 * row, p.H, h, D, c, K), K);
+    win_load(w.k, p.wk + ((int64_t)h * D + c) * K, src + conv_index(2 * row + 1, p.H, h, D, c, K), K);
 }
 
 __device__ __forceinline__ void conv_store(const ConvWin &w, const DecodeParams &p, float *dst, int64_t row,
                                            int h, int D, int c) {
     const int K = p.taps;
-    float *dq = dst + conv_index(2 * row, p.H, h, D, c, K);
-    float *dk = dst + conv_index(2 * row + 1, p.H, h, D, c, K);
-#pragma unroll
-    for (int j = 0; j < kMaxTaps - 1; ++j)
-        if (j < K - 1) { dq[j] = w.hq[j]; dk[j] = w.hk[j]; }
-}
-
-// one causal conv step of raw input x through weights wt and window hs (shifted in place)
-// (every index is a compile-time constant after unrolling, so window and weights stay
-// in registers)
-__device__ __forceinline__ float conv_step(const float (&wt)[kMaxTaps], float (&hs)[kMaxTaps - 1], int K, float x) {
-    float wl = 0.f;
-#pragma unroll
-    for (int j = 0; j < kMaxTaps; ++j)
-        if (j == K - 1) wl = wt[j];
-    float y = wl * x;
-#pragma unroll
-    for (int j = 0; j < kMaxTaps - 1; ++j)
-        if (j < K - 1) y = fmaf(wt[j], hs[j], y);
-#pragma unroll
-    for (int j = 0; j < kMaxTaps - 1; ++j) {
-        if (j < K - 2) hs[j] = hs[j + 1];
-        else if (j == K - 2) hs[j] = x;
-    }
-    return y;
+    win_store(w.q, dst + conv_index(2 * row, p.H, h, D, c, K), K);
+    win_store(w.k, dst + conv_index(2 * row + 1, p.H, h, D, c, K), K);
 }
 
 __device__ __forceinline__ float swish(float y) { return y / (1.f + expf(-y)); }
@@ -180,8 +187,8 @@ __device__ __forceinline__ void stage_batch(TokVec<D> *tv, int nb, int64_t row0,
                 const int jj = j0 + j;
                 if (jj < nb) {
                     if (CONV) {
-                        const float yq = conv_step(w.wq, w.hq, p.taps, xq[j]);
-                        const float yk = conv_step(w.wk, w.hk, p.taps, xk[j]);
+                        const float yq = conv_step(w.q, p.taps, xq[j]);
+                        const float yk = conv_step(w.k, p.taps, xk[j]);
                         tv[jj].q[t] = q_ != nullptr ? swish(yq) : 0.f;
                         tv[jj].k[t] = swish(yk);
                         if (co.tok) conv_store(w, p, co.tok, co.tok0 + jj, h, D, t);
@@ -400,8 +407,8 @@ __device__ __forceinline__ void convert_batch(TokVec<D> *tv, const uint8_t *raw,
             const float xq = read_q ? IO<TIO>::ld(reinterpret_cast<const TIO *>(rj) + t) : 0.f;
             const float xk = IO<TIO>::ld(reinterpret_cast<const TIO *>(rj + RT::QB) + t);
             if (CONV) {
-                const float yq = conv_step(w.wq, w.hq, p.taps, xq);
-                const float yk = conv_step(w.wk, w.hk, p.taps, xk);
+                const float yq = conv_step(w.q, p.taps, xq);
+                const float yk = conv_step(w.k, p.taps, xk);
                 tv[j].q[t] = with_q ? swish(yq) : 0.f;
                 tv[j].k[t] = swish(yk);
                 if (co.tok) conv_store(w, p, co.tok, co.tok0 + j, h, D, t);
@@ -422,21 +429,33 @@ __device__ __forceinline__ void convert_batch(TokVec<D> *tv, const uint8_t *raw,
     }
 }
 
-// The batch stream of one CTA: batches of src[0] (n0 tokens), then of src[1].
+// The batch stream of one CTA: batches of a, then of b. (Two members and selects, not
+// an array indexed at run time, so that the stream stays in registers.)
 struct TokStream {
-    TokSrc src[2];
-    int nb0, nbat;              // batches of src[0]; all batches
+    TokSrc a, b;
+    int nb0, nbat;              // batches of a; all batches
     __device__ __forceinline__ void locate(int bi, int &which, int &j0, int &nb) const {
         which = bi < nb0 ? 0 : 1;
         j0 = (which ? bi - nb0 : bi) * kTokBatch;
-        nb = min(kTokBatch, src[which].n - j0);
+        nb = min(kTokBatch, (which ? b.n : a.n) - j0);
+    }
+    __device__ __forceinline__ TokSrc pick(int which) const {
+        TokSrc r;
+        r.q = which ? b.q : a.q;
+        r.k = which ? b.k : a.k;
+        r.v = which ? b.v : a.v;
+        r.g = which ? b.g : a.g;
+        r.beta = which ? b.beta : a.beta;
+        r.row0 = which ? b.row0 : a.row0;
+        r.n = which ? b.n : a.n;
+        return r;
     }
 };
 
 __device__ __forceinline__ TokStream make_stream(const TokSrc &a, const TokSrc &b) {
     TokStream s;
-    s.src[0] = a;
-    s.src[1] = b;
+    s.a = a;
+    s.b = b;
     s.nb0 = (a.n + kTokBatch - 1) / kTokBatch;
     s.nbat = s.nb0 + (b.n + kTokBatch - 1) / kTokBatch;
     return s;
@@ -446,14 +465,15 @@ template <int D, typename TIO>
 __device__ __forceinline__ void issue_batch(const TokStream &ts, int bi, uint8_t *raw, uint64_t *bar, int H) {
     int which, j0, nb;
     ts.locate(bi, which, j0, nb);
-    issue_rows<D, TIO>(raw, ts.src[which], j0, nb, H, bar);
+    issue_rows<D, TIO>(raw, ts.pick(which), j0, nb, H, bar);
 }
 
 // beta of token c of batch bi (threads D + c), issued early as a plain load
 __device__ __forceinline__ float batch_beta(const TokStream &ts, int bi, int c, int H) {
     int which, j0, nb;
     ts.locate(bi, which, j0, nb);
-    return c < nb ? ts.src[which].beta[ts.src[which].row0 + (int64_t)(j0 + c) * H] : 0.f;
+    const TokSrc src = ts.pick(which);
+    return c < nb ? src.beta[src.row0 + (int64_t)(j0 + c) * H] : 0.f;
 }
 
 template <int D, typename TIO, bool CONV>
@@ -489,7 +509,7 @@ verify_kernel(const __grid_constant__ DecodeParams p) {
     using RT = RawTok<D, TIO>;
     __shared__ TokVec<D> tv[kTokBatch];
     extern __shared__ __align__(128) uint8_t dyn_smem[];   // two raw row buffers
-    uint8_t *raw[2] = {dyn_smem, dyn_smem + kTokBatch * RT::BYTES};
+    auto raw = [&](int i) { return dyn_smem + i * (kTokBatch * RT::BYTES); };
     __shared__ uint64_t bars[2];
     const int s = blockIdx.x / p.H, h = blockIdx.x % p.H;
     const int32_t slot = p.slots[s];
@@ -506,7 +526,7 @@ verify_kernel(const __grid_constant__ DecodeParams p) {
         tc::bar_init(&bars[0], 1);
         tc::bar_init(&bars[1], 1);
         tc::bar_init_fence();
-        for (int bi = 0; bi < 2 && bi < ts.nbat; ++bi) issue_batch<D, TIO>(ts, bi, raw[bi], &bars[bi], p.H);
+        for (int bi = 0; bi < 2 && bi < ts.nbat; ++bi) issue_batch<D, TIO>(ts, bi, raw(bi), &bars[bi], p.H);
     }
     float bnext = (t >= D && ts.nbat > 0) ? batch_beta(ts, 0, t - D, p.H) : 0.f;
     const float *S = p.pool + ((int64_t)slot * p.H + h) * (int64_t)D * D;
@@ -524,9 +544,9 @@ verify_kernel(const __grid_constant__ DecodeParams p) {
         if (t >= D && bi + 1 < ts.nbat) bnext = batch_beta(ts, bi + 1, t - D, p.H);
         ok = tc::bar_wait(&bars[bi & 1], (uint32_t)((bi >> 1) & 1)) && ok;
         const ConvOut co{p.conv_tok, tok_first + j0, nullptr, 0, -1};
-        convert_batch<D, TIO, CONV>(tv, raw[bi & 1], nb, true, true, b, w, p, h, co);
+        convert_batch<D, TIO, CONV>(tv, raw(bi & 1), nb, true, true, b, w, p, h, co);
         __syncthreads();  // vectors staged, raw buffer read
-        if (t == 0 && bi + 2 < ts.nbat) issue_batch<D, TIO>(ts, bi + 2, raw[bi & 1], &bars[bi & 1], p.H);
+        if (t == 0 && bi + 2 < ts.nbat) issue_batch<D, TIO>(ts, bi + 2, raw(bi & 1), &bars[bi & 1], p.H);
         if (warp < nb) token_finish<D>(tv[warp], CONV, true);
         for (int j = DecodeShape<D>::NW; j < nb; ++j)
             if (warp == 0) token_finish<D>(tv[j], CONV, true);
@@ -578,7 +598,7 @@ verify_commit_kernel(const __grid_constant__ VerifyCommitParams P) {
     const CommitParams &c = P.c;
     __shared__ TokVec<D> tv[kTokBatch];
     extern __shared__ __align__(128) uint8_t dyn_smem[];   // two raw row buffers
-    uint8_t *raw[2] = {dyn_smem, dyn_smem + kTokBatch * RT::BYTES};
+    auto raw = [&](int i) { return dyn_smem + i * (kTokBatch * RT::BYTES); };
     __shared__ uint64_t bars[2];
     const int s = blockIdx.x / p.H, h = blockIdx.x % p.H;
     const int32_t slot = p.slots[s];
@@ -609,7 +629,7 @@ verify_commit_kernel(const __grid_constant__ VerifyCommitParams P) {
         tc::bar_init(&bars[0], 1);
         tc::bar_init(&bars[1], 1);
         tc::bar_init_fence();
-        for (int bi = 0; bi < 2 && bi < ts.nbat; ++bi) issue_batch<D, TIO>(ts, bi, raw[bi], &bars[bi], p.H);
+        for (int bi = 0; bi < 2 && bi < ts.nbat; ++bi) issue_batch<D, TIO>(ts, bi, raw(bi), &bars[bi], p.H);
     }
     float bnext = (t >= D && ts.nbat > 0) ? batch_beta(ts, 0, t - D, p.H) : 0.f;
     float *S = p.pool + ((int64_t)slot * p.H + h) * (int64_t)D * D;
@@ -630,9 +650,9 @@ verify_commit_kernel(const __grid_constant__ VerifyCommitParams P) {
         const int64_t c0 = replay ? j0 : (cnew ? na + j0 : -1);
         const int64_t js = (c0 >= 0 && jsnap >= c0 && jsnap < c0 + nb) ? jsnap - c0 : -1;
         const ConvOut co{nullptr, 0, c.conv_snapshots, srow, (int)js};
-        convert_batch<D, TIO, CONV>(tv, raw[bi & 1], nb, CONV || !replay, !replay, b, w, p, h, co);
+        convert_batch<D, TIO, CONV>(tv, raw(bi & 1), nb, CONV || !replay, !replay, b, w, p, h, co);
         __syncthreads();  // vectors staged, raw buffer read
-        if (t == 0 && bi + 2 < ts.nbat) issue_batch<D, TIO>(ts, bi + 2, raw[bi & 1], &bars[bi & 1], p.H);
+        if (t == 0 && bi + 2 < ts.nbat) issue_batch<D, TIO>(ts, bi + 2, raw(bi & 1), &bars[bi & 1], p.H);
         if (warp < nb) token_finish<D>(tv[warp], CONV, !replay);
         for (int j = DecodeShape<D>::NW; j < nb; ++j)
             if (warp == 0) token_finish<D>(tv[j], CONV, !replay);

@@ -88,40 +88,34 @@ __global__ void __launch_bounds__(FrontendShape<D>::NT) qk_frontend_kernel(const
     const int c0 = CPL * lane;
     const TIO *q = static_cast<const TIO *>(P.q), *k = static_cast<const TIO *>(P.k);
     // weights and windows of the lane's channels
-    float wq[CPL][kMaxTaps], wk[CPL][kMaxTaps], hq[CPL][kMaxTaps - 1], hk[CPL][kMaxTaps - 1];
-#pragma unroll
-    for (int e = 0; e < CPL; ++e) {
-#pragma unroll
-        for (int j = 0; j < kMaxTaps; ++j) {
-            wq[e][j] = j < K ? P.wq[((int64_t)h * D + c0 + e) * K + j] : 0.f;
-            wk[e][j] = j < K ? P.wk[((int64_t)h * D + c0 + e) * K + j] : 0.f;
-        }
-    }
+    Win cq[CPL], ck[CPL];
+    float hist[kMaxTaps - 1][2][CPL];      // the window before the tile, oldest first
 #pragma unroll
     for (int j = 0; j < kMaxTaps - 1; ++j) {
-        float xa[CPL], xb[CPL];
 #pragma unroll
-        for (int e = 0; e < CPL; ++e) xa[e] = xb[e] = 0.f;
+        for (int e = 0; e < CPL; ++e) hist[j][0][e] = hist[j][1][e] = 0.f;
         if (j < K - 1) {
             if (b == 0) {
                 if (P.conv_in) {
 #pragma unroll
                     for (int e = 0; e < CPL; ++e) {
-                        xa[e] = P.conv_in[conv_index(2 * i, H, h, D, c0 + e, K) + j];
-                        xb[e] = P.conv_in[conv_index(2 * i + 1, H, h, D, c0 + e, K) + j];
+                        hist[j][0][e] = P.conv_in[conv_index(2 * i, H, h, D, c0 + e, K) + j];
+                        hist[j][1][e] = P.conv_in[conv_index(2 * i + 1, H, h, D, c0 + e, K) + j];
                     }
                 }
             } else {
                 const int64_t r = t0 - (K - 1) + j;             // inside this sequence (b * C >= K - 1)
-                ld_vec<TIO, CPL>(q + (r * H + h) * D + c0, xa);
-                ld_vec<TIO, CPL>(k + (r * H + h) * D + c0, xb);
+                ld_vec<TIO, CPL>(q + (r * H + h) * D + c0, hist[j][0]);
+                ld_vec<TIO, CPL>(k + (r * H + h) * D + c0, hist[j][1]);
             }
         }
+    }
 #pragma unroll
-        for (int e = 0; e < CPL; ++e) {
-            hq[e][j] = xa[e];
-            hk[e][j] = xb[e];
-        }
+    for (int e = 0; e < CPL; ++e) {
+        const float sq[3] = {hist[0][0][e], hist[1][0][e], hist[2][0][e]};
+        const float sk[3] = {hist[0][1][e], hist[1][1][e], hist[2][1][e]};
+        win_load(cq[e], P.wq + ((int64_t)h * D + c0 + e) * K, sq, K);
+        win_load(ck[e], P.wk + ((int64_t)h * D + c0 + e) * K, sk, K);
     }
     TIO *qo = static_cast<TIO *>(P.q_out), *ko = static_cast<TIO *>(P.k_out);
     for (int r0 = 0; r0 < n; r0 += G) {
@@ -140,8 +134,8 @@ __global__ void __launch_bounds__(FrontendShape<D>::NT) qk_frontend_kernel(const
                 float zq[CPL], zk[CPL], sq = 0.f, sk = 0.f;
 #pragma unroll
                 for (int e = 0; e < CPL; ++e) {
-                    zq[e] = swish(conv_step(wq[e], hq[e], K, xq[g][e]));
-                    zk[e] = swish(conv_step(wk[e], hk[e], K, xk[g][e]));
+                    zq[e] = swish(conv_step(cq[e], K, xq[g][e]));
+                    zk[e] = swish(conv_step(ck[e], K, xk[g][e]));
                     sq = fmaf(zq[e], zq[e], sq);
                     sk = fmaf(zk[e], zk[e], sk);
                 }
@@ -159,13 +153,10 @@ __global__ void __launch_bounds__(FrontendShape<D>::NT) qk_frontend_kernel(const
     // conv states: at a snapshot boundary that ends this tile, and after the last token
     auto put = [&](float *dst, int64_t srow) {
 #pragma unroll
-        for (int e = 0; e < CPL; ++e)
-#pragma unroll
-            for (int jj = 0; jj < kMaxTaps - 1; ++jj)
-                if (jj < K - 1) {
-                    dst[conv_index(2 * srow, H, h, D, c0 + e, K) + jj] = hq[e][jj];
-                    dst[conv_index(2 * srow + 1, H, h, D, c0 + e, K) + jj] = hk[e][jj];
-                }
+        for (int e = 0; e < CPL; ++e) {
+            win_store(cq[e], dst + conv_index(2 * srow, H, h, D, c0 + e, K), K);
+            win_store(ck[e], dst + conv_index(2 * srow + 1, H, h, D, c0 + e, K), K);
+        }
     };
     const int64_t p_end = P.start_pos[i] + (int64_t)b * C + n;
     if (P.conv_snap && P.snap_interval > 0 && n == C && p_end % P.snap_interval == 0)
