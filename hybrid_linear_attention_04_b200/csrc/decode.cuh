@@ -136,17 +136,6 @@ __device__ __forceinline__ void conv_store(const ConvWin &w, const DecodeParams 
 
 __device__ __forceinline__ float swish(float y) { return y / (1.f + expf(-y)); }
 
-// Per-token vectors staged in shared memory. 16-byte aligned (and padded to a
-// multiple of 16 bytes) because the step reads v with float4 loads.
-template <int D> struct __align__(16) TokVec {
-    float k[D], q[D], a[D], v[D];
-    float beta, kq;
-};
-static_assert(sizeof(TokVec<128>) % 16 == 0 && sizeof(TokVec<32>) % 16 == 0, "TokVec padding");
-
-// Verify: tokens are processed in batches of kTokBatch staged in shared memory.
-constexpr int kTokBatch = 8;
-
 // Where the front-end's conv state goes while a batch is staged (front-end on only):
 // after every token into rows tok0 + j of `tok` (nullable), and after token snap_j
 // (batch-relative; -1 = none) into row snap_row of `snap`.
@@ -158,72 +147,70 @@ struct ConvOut {
     int snap_j;
 };
 
-// Stage nb <= kTokBatch tokens, rows row0 + j * rstride (= token * H + head) of the
-// packed arrays, into tv[0..nb). q_ may be null (a replayed token whose output is not
-// needed: with the front-end its q still moves the conv window). With CONV, q and k
-// are raw and pass through the conv and Swish here (window w of the thread's
-// channel); token_finish normalises them.
-template <int D, typename TIO, bool CONV>
-__device__ __forceinline__ void stage_batch(TokVec<D> *tv, int nb, int64_t row0, int64_t rstride,
-                                            const void *q_, const void *k_, const void *v_,
-                                            const float *g_, const float *beta, ConvWin &w,
-                                            const DecodeParams &p, int h, const ConvOut &co) {
-    constexpr int L = kTokBatch / 2;      // loads in flight per array (register budget)
-    const int t = threadIdx.x;
-    if (t < D) {
-        const TIO *q = static_cast<const TIO *>(q_), *k = static_cast<const TIO *>(k_);
-        for (int j0 = 0; j0 < nb; j0 += L) {
-            float xq[L], xk[L];
-#pragma unroll
-            for (int j = 0; j < L; ++j) {
-                if (j0 + j < nb) {
-                    const int64_t off = (row0 + (j0 + j) * rstride) * D + t;
-                    xq[j] = (q_ != nullptr) ? IO<TIO>::ld(q + off) : 0.f;
-                    xk[j] = IO<TIO>::ld(k + off);
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < L; ++j) {
-                const int jj = j0 + j;
-                if (jj < nb) {
-                    if (CONV) {
-                        const float yq = conv_step(w.q, p.taps, xq[j]);
-                        const float yk = conv_step(w.k, p.taps, xk[j]);
-                        tv[jj].q[t] = q_ != nullptr ? swish(yq) : 0.f;
-                        tv[jj].k[t] = swish(yk);
-                        if (co.tok) conv_store(w, p, co.tok, co.tok0 + jj, h, D, t);
-                        if (jj == co.snap_j) conv_store(w, p, co.snap, co.snap_row, h, D, t);
-                    } else {
-                        tv[jj].q[t] = xq[j];
-                        tv[jj].k[t] = xk[j];
-                    }
-                }
-            }
-        }
-    } else {
-        const int c = t - D;
-        const TIO *v = static_cast<const TIO *>(v_);
-        const float b = c < nb ? beta[row0 + c * rstride] : 0.f;
-        for (int j0 = 0; j0 < nb; j0 += L) {
-            float xv[L], xg[L];
-#pragma unroll
-            for (int j = 0; j < L; ++j) {
-                if (j0 + j < nb) {
-                    const int64_t off = (row0 + (j0 + j) * rstride) * D + c;
-                    xv[j] = IO<TIO>::ld(v + off);
-                    xg[j] = g_[off];
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < L; ++j) {
-                if (j0 + j < nb) {
-                    tv[j0 + j].v[c] = xv[j];
-                    tv[j0 + j].a[c] = expf(xg[j]);
-                }
-            }
-        }
-        if (c < nb) tv[c].beta = b;
+// ---- packed fp32 pairs (sm_100 f32x2 arithmetic) --------------------------------
+// One instruction does the work of two fp32 lanes; each element is rounded exactly as
+// the scalar fmul / fmaf would round it, so the pairing changes no result bit.
+using f2 = unsigned long long;
+__device__ __forceinline__ f2 pk2(float lo, float hi) {
+    f2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 up2(f2 x) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(x));
+    return r;
+}
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+    f2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+    f2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// ---- per-token vectors in shared memory ----------------------------------------
+// A lane reads the gate a = exp(g), k and q at its rows rg + 8 m (rg = lane / 4,
+// m < D / 8). They are stored permuted, channel c at (c % 8) * STR + c / 8, so that one
+// 128-bit load gives a lane rows m .. m + 3; STR pads each row group so that the 8
+// distinct addresses of a warp's load, and a warp's 32 scalar stores, hit distinct banks.
+template <int D> struct TokLayout {
+    static constexpr int R = D / 8;                                  // rows per lane
+    static constexpr int STR = ((R + 4) / 4) % 2 ? R + 4 : R + 8;   // floats per row group
+    static constexpr int SZ = 8 * STR;
+    static_assert(R % 4 == 0 && (STR * 4) % 16 == 0, "128-bit rows");
+};
+template <int D> __device__ __forceinline__ int perm(int c) { return (c & 7) * TokLayout<D>::STR + (c >> 3); }
+
+template <int D> struct __align__(16) TokVec {
+    float a[TokLayout<D>::SZ], k[TokLayout<D>::SZ], q[TokLayout<D>::SZ];   // permuted
+    float v[D];                                                          // natural order
+    float beta, kq, pad0, pad1;
+};
+
+// Channel c of q and k into a token vector: with CONV through the front-end's conv window
+// and Swish (token_finish normalises), else as given. with_q false: q is zero (a replayed
+// token whose output is not needed; its raw q still moves the conv window).
+template <int D, bool CONV>
+__device__ __forceinline__ void put_qk(TokVec<D> &tv, int c, float xq, float xk, bool with_q, ConvWin &w,
+                                       int taps) {
+    float q = xq, k = xk;
+    if (CONV) {
+        const float yq = conv_step(w.q, taps, xq);
+        const float yk = conv_step(w.k, taps, xk);
+        q = swish(yq);
+        k = swish(yk);
     }
+    tv.q[perm<D>(c)] = with_q ? q : 0.f;
+    tv.k[perm<D>(c)] = k;
+}
+template <int D>
+__device__ __forceinline__ void put_vg(TokVec<D> &tv, int c, float xv, float xg) {
+    tv.v[c] = xv;
+    tv.a[perm<D>(c)] = expf(xg);
 }
 
 // One warp finishes a staged token: L2-normalises k and q when the front-end is on,
@@ -234,9 +221,10 @@ __device__ __forceinline__ void token_finish(TokVec<D> &tv, bool normalise, bool
     if (normalise) {
         float sk = 0.f, sq = 0.f;
 #pragma unroll
-        for (int i = lane; i < D; i += 32) {
-            sk = fmaf(tv.k[i], tv.k[i], sk);
-            sq = fmaf(tv.q[i], tv.q[i], sq);
+        for (int c = lane; c < D; c += 32) {
+            const float k = tv.k[perm<D>(c)], q = tv.q[perm<D>(c)];
+            sk = fmaf(k, k, sk);
+            sq = fmaf(q, q, sq);
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
@@ -245,31 +233,74 @@ __device__ __forceinline__ void token_finish(TokVec<D> &tv, bool normalise, bool
         }
         const float rk = 1.f / fmaxf(sqrtf(sk), kNormEps), rq = 1.f / fmaxf(sqrtf(sq), kNormEps);
 #pragma unroll
-        for (int i = lane; i < D; i += 32) {
-            tv.k[i] *= rk;
-            tv.q[i] *= rq;
+        for (int c = lane; c < D; c += 32) {
+            tv.k[perm<D>(c)] *= rk;
+            tv.q[perm<D>(c)] *= rq;
         }
         __syncwarp();
     }
     if (with_q) {
         float s = 0.f;
 #pragma unroll
-        for (int i = lane; i < D; i += 32) s = fmaf(tv.k[i], tv.q[i], s);
+        for (int c = lane; c < D; c += 32) s = fmaf(tv.k[perm<D>(c)], tv.q[perm<D>(c)], s);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
         if (lane == 0) tv.kq = s;
     }
 }
 
-// Finish nb staged tokens (warp j takes token j, warp 0 the rest) between barriers.
+// ---- the state in registers ------------------------------------------------------
+// Lane (warp w, rg = lane / 4, cg = lane % 4) holds columns 16 w + 4 cg + e (e < 4) of
+// rows rg + 8 m (m < R): P[i][e] pairs rows m = 2 i (low half) and 2 i + 1 (high half)
+// of column e, so the gate, both column sums and the rank-1 update run as f32x2 pairs.
+template <int D> using StatePairs = f2[TokLayout<D>::R / 2][4];
+
 template <int D>
-__device__ __forceinline__ void finish_batch(TokVec<D> *tv, int nb, bool normalise, bool with_q) {
-    const int warp = threadIdx.x >> 5;
-    __syncthreads();
-    if (warp < nb) token_finish<D>(tv[warp], normalise, with_q);
-    for (int j = DecodeShape<D>::NW; j < nb; ++j)
-        if (warp == 0) token_finish<D>(tv[j], normalise, with_q);
-    __syncthreads();
+__device__ __forceinline__ int64_t lane_off(int m) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    return (int64_t)((lane >> 2) + 8 * m) * D + 16 * warp + 4 * (lane & 3);
+}
+__device__ __forceinline__ int lane_col() { return 16 * (threadIdx.x >> 5) + 4 * (threadIdx.x & 3); }
+
+__device__ __forceinline__ void set_rows(f2 (&p)[4], const float4 &e, const float4 &o) {
+    p[0] = pk2(e.x, o.x); p[1] = pk2(e.y, o.y); p[2] = pk2(e.z, o.z); p[3] = pk2(e.w, o.w);
+}
+__device__ __forceinline__ void get_rows(const f2 (&p)[4], float4 &e, float4 &o) {
+    const float2 a = up2(p[0]), b = up2(p[1]), c = up2(p[2]), d = up2(p[3]);
+    e = make_float4(a.x, b.x, c.x, d.x);
+    o = make_float4(a.y, b.y, c.y, d.y);
+}
+// from global memory (read once: no L1 allocation)
+template <int D>
+__device__ __forceinline__ void load_state(StatePairs<D> &P, const float *S) {
+#pragma unroll
+    for (int i = 0; i < TokLayout<D>::R / 2; ++i) {
+        float4 e, o;
+        const float *se = S + lane_off<D>(2 * i), *so = S + lane_off<D>(2 * i + 1);
+        asm volatile("ld.global.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
+                     : "=f"(e.x), "=f"(e.y), "=f"(e.z), "=f"(e.w) : "l"(se));
+        asm volatile("ld.global.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
+                     : "=f"(o.x), "=f"(o.y), "=f"(o.z), "=f"(o.w) : "l"(so));
+        set_rows(P[i], e, o);
+    }
+}
+// from a row-major copy in shared memory
+template <int D>
+__device__ __forceinline__ void load_state_smem(StatePairs<D> &P, const float *S) {
+#pragma unroll
+    for (int i = 0; i < TokLayout<D>::R / 2; ++i)
+        set_rows(P[i], *reinterpret_cast<const float4 *>(S + lane_off<D>(2 * i)),
+                 *reinterpret_cast<const float4 *>(S + lane_off<D>(2 * i + 1)));
+}
+template <int D>
+__device__ __forceinline__ void store_state(const StatePairs<D> &P, float *S) {
+#pragma unroll
+    for (int i = 0; i < TokLayout<D>::R / 2; ++i) {
+        float4 e, o;
+        get_rows(P[i], e, o);
+        st_stream(S + lane_off<D>(2 * i), e);
+        st_stream(S + lane_off<D>(2 * i + 1), o);
+    }
 }
 
 // One recurrence step on the register-resident columns of this warp. With OUT =
@@ -277,205 +308,74 @@ __device__ __forceinline__ void finish_batch(TokVec<D> *tv, int nb, bool normali
 // instruction for instruction, so both forms give bit-identical states. The
 // returned o (OUT) holds the lane's four columns; every lane of a column group has it.
 template <int D, bool OUT = true>
-__device__ __forceinline__ float4 kda_step(float4 (&st)[DecodeShape<D>::R], const TokVec<D> &tv, float scale) {
-    using Sh = DecodeShape<D>;
+__device__ __forceinline__ float4 kda_step(StatePairs<D> &P, const TokVec<D> &tv, float scale) {
+    using L = TokLayout<D>;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int cg = lane & 3, rg = lane >> 2;
-    float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
+    const int rg = lane >> 2, cg = lane & 3;
+    const float *ap = tv.a + rg * L::STR, *kp = tv.k + rg * L::STR, *qp = tv.q + rg * L::STR;
+    f2 xa[4] = {0ull, 0ull, 0ull, 0ull}, ya[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-    for (int m = 0; m < Sh::R; ++m) {
-        const int r = rg + 8 * m;
-        const float a = tv.a[r], kr = tv.k[r];
-        float4 s = st[m];
-        s.x *= a; s.y *= a; s.z *= a; s.w *= a;
-        st[m] = s;
-        x.x = fmaf(kr, s.x, x.x); x.y = fmaf(kr, s.y, x.y);
-        x.z = fmaf(kr, s.z, x.z); x.w = fmaf(kr, s.w, x.w);
+    for (int i = 0; i < L::R / 4; ++i) {
+        const float4 a4 = *reinterpret_cast<const float4 *>(ap + 4 * i);
+        const float4 k4 = *reinterpret_cast<const float4 *>(kp + 4 * i);
+        const f2 a01 = pk2(a4.x, a4.y), a23 = pk2(a4.z, a4.w);
+        const f2 k01 = pk2(k4.x, k4.y), k23 = pk2(k4.z, k4.w);
+        f2 q01 = 0ull, q23 = 0ull;
         if (OUT) {
-            const float qr = tv.q[r];
-            y.x = fmaf(qr, s.x, y.x); y.y = fmaf(qr, s.y, y.y);
-            y.z = fmaf(qr, s.z, y.z); y.w = fmaf(qr, s.w, y.w);
+            const float4 q4 = *reinterpret_cast<const float4 *>(qp + 4 * i);
+            q01 = pk2(q4.x, q4.y);
+            q23 = pk2(q4.z, q4.w);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const f2 s0 = mul2(P[2 * i][e], a01), s1 = mul2(P[2 * i + 1][e], a23);
+            P[2 * i][e] = s0;
+            P[2 * i + 1][e] = s1;
+            xa[e] = fma2(k23, s1, fma2(k01, s0, xa[e]));
+            if (OUT) ya[e] = fma2(q23, s1, fma2(q01, s0, ya[e]));
+        }
+    }
+    float x[4], y[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 xs = up2(xa[e]);
+        x[e] = xs.x + xs.y;
+        if (OUT) {
+            const float2 ys = up2(ya[e]);
+            y[e] = ys.x + ys.y;
         }
     }
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-        x.x += __shfl_xor_sync(0xffffffffu, x.x, off);
-        x.y += __shfl_xor_sync(0xffffffffu, x.y, off);
-        x.z += __shfl_xor_sync(0xffffffffu, x.z, off);
-        x.w += __shfl_xor_sync(0xffffffffu, x.w, off);
-        if (OUT) {
-            y.x += __shfl_xor_sync(0xffffffffu, y.x, off);
-            y.y += __shfl_xor_sync(0xffffffffu, y.y, off);
-            y.z += __shfl_xor_sync(0xffffffffu, y.z, off);
-            y.w += __shfl_xor_sync(0xffffffffu, y.w, off);
+    for (int off = 4; off < 32; off <<= 1)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            x[e] += __shfl_xor_sync(0xffffffffu, x[e], off);
+            if (OUT) y[e] += __shfl_xor_sync(0xffffffffu, y[e], off);
         }
-    }
     const float4 vv = *reinterpret_cast<const float4 *>(tv.v + 16 * warp + 4 * cg);
-    float4 wv;
-    wv.x = tv.beta * (vv.x - x.x); wv.y = tv.beta * (vv.y - x.y);
-    wv.z = tv.beta * (vv.z - x.z); wv.w = tv.beta * (vv.w - x.w);
+    const float w0 = tv.beta * (vv.x - x[0]), w1 = tv.beta * (vv.y - x[1]);
+    const float w2 = tv.beta * (vv.z - x[2]), w3 = tv.beta * (vv.w - x[3]);
+    const f2 ww[4] = {pk2(w0, w0), pk2(w1, w1), pk2(w2, w2), pk2(w3, w3)};
 #pragma unroll
-    for (int m = 0; m < Sh::R; ++m) {
-        const float kr = tv.k[rg + 8 * m];
-        float4 s = st[m];
-        s.x = fmaf(kr, wv.x, s.x); s.y = fmaf(kr, wv.y, s.y);
-        s.z = fmaf(kr, wv.z, s.z); s.w = fmaf(kr, wv.w, s.w);
-        st[m] = s;
+    for (int i = 0; i < L::R / 4; ++i) {
+        const float4 k4 = *reinterpret_cast<const float4 *>(kp + 4 * i);
+        const f2 k01 = pk2(k4.x, k4.y), k23 = pk2(k4.z, k4.w);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            P[2 * i][e] = fma2(k01, ww[e], P[2 * i][e]);
+            P[2 * i + 1][e] = fma2(k23, ww[e], P[2 * i + 1][e]);
+        }
     }
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
     if (OUT) {
-        o.x = scale * fmaf(tv.kq, wv.x, y.x); o.y = scale * fmaf(tv.kq, wv.y, y.y);
-        o.z = scale * fmaf(tv.kq, wv.z, y.z); o.w = scale * fmaf(tv.kq, wv.w, y.w);
+        o.x = scale * fmaf(tv.kq, w0, y[0]); o.y = scale * fmaf(tv.kq, w1, y[1]);
+        o.z = scale * fmaf(tv.kq, w2, y[2]); o.w = scale * fmaf(tv.kq, w3, y[3]);
     }
     return o;
 }
 
-// offset of the lane's float4 in row m of a state
-template <int D>
-__device__ __forceinline__ int64_t lane_off(int m) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    return (int64_t)((lane >> 2) + 8 * m) * D + 16 * warp + 4 * (lane & 3);
-}
-template <int D>
-__device__ __forceinline__ int lane_col() {
-    return 16 * (threadIdx.x >> 5) + 4 * (threadIdx.x & 3);
-}
-
-template <int D>
-__device__ __forceinline__ void load_state(float4 (&st)[DecodeShape<D>::R], const float *S) {
-#pragma unroll
-    for (int m = 0; m < DecodeShape<D>::R; ++m) {
-        const float *src = S + lane_off<D>(m);
-        asm volatile("ld.global.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
-                     : "=f"(st[m].x), "=f"(st[m].y), "=f"(st[m].z), "=f"(st[m].w)
-                     : "l"(src));
-    }
-}
-template <int D>
-__device__ __forceinline__ void store_state(const float4 (&st)[DecodeShape<D>::R], float *S) {
-#pragma unroll
-    for (int m = 0; m < DecodeShape<D>::R; ++m) st_stream(S + lane_off<D>(m), st[m]);
-}
-
-// ---- token rows staged by bulk copies (verify, verify + commit) ----------------
-// A CTA's tokens form one stream of batches of up to kTokBatch tokens (verify+commit:
-// the replayed prefix, then this step's tokens). Thread 0 copies a batch's raw q, k, v
-// and g rows into one of two shared-memory buffers with bulk asynchronous copies that
-// complete on that buffer's mbarrier, two batches ahead of their use, so the rows of
-// every batch arrive while the state is loaded and the previous batch is stepped.
-template <int D, typename TIO> struct RawTok {
-    static constexpr uint32_t QB = D * sizeof(TIO);     // one q, k or v row
-    static constexpr uint32_t BYTES = 3 * QB + D * 4;   // + one g row (fp32)
-    static constexpr uint32_t SMEM = 2 * kTokBatch * BYTES;   // dynamic shared memory
-};
-
-struct TokSrc {                 // tokens row0, row0 + H, ... of packed arrays
-    const void *q, *k, *v;      // q null: not staged (a replayed token without front-end)
-    const float *g, *beta;
-    int64_t row0;
-    int n;
-};
-
-template <int D, typename TIO>
-__device__ __forceinline__ void issue_rows(uint8_t *raw, const TokSrc &src, int j0, int nb, int H,
-                                           uint64_t *bar) {
-    using RT = RawTok<D, TIO>;
-    const uint32_t per = src.q ? RT::BYTES : RT::BYTES - RT::QB;   // every row keeps its slot
-    tc::bar_expect_tx(bar, per * (uint32_t)nb);
-    for (int j = 0; j < nb; ++j) {
-        const int64_t row = src.row0 + (int64_t)(j0 + j) * H;
-        uint8_t *dst = raw + j * RT::BYTES;
-        if (src.q) tc::bulk_load(dst, static_cast<const TIO *>(src.q) + row * D, RT::QB, bar);
-        tc::bulk_load(dst + RT::QB, static_cast<const TIO *>(src.k) + row * D, RT::QB, bar);
-        tc::bulk_load(dst + 2 * RT::QB, static_cast<const TIO *>(src.v) + row * D, RT::QB, bar);
-        tc::bulk_load(dst + 3 * RT::QB, src.g + row * D, D * 4, bar);
-    }
-}
-
-// Staged raw rows -> token vectors (the front-end's conv and Swish with CONV): threads
-// t < D channel t of q and k, in token order; threads t >= D channel t - D of v and g.
-// b: this thread's beta (threads D .. D + nb - 1), loaded ahead.
-template <int D, typename TIO, bool CONV>
-__device__ __forceinline__ void convert_batch(TokVec<D> *tv, const uint8_t *raw, int nb, bool read_q,
-                                              bool with_q, float b, ConvWin &w, const DecodeParams &p, int h,
-                                              const ConvOut &co) {
-    using RT = RawTok<D, TIO>;
-    const int t = threadIdx.x;
-    if (t < D) {
-        for (int j = 0; j < nb; ++j) {
-            const uint8_t *rj = raw + j * RT::BYTES;
-            const float xq = read_q ? IO<TIO>::ld(reinterpret_cast<const TIO *>(rj) + t) : 0.f;
-            const float xk = IO<TIO>::ld(reinterpret_cast<const TIO *>(rj + RT::QB) + t);
-            if (CONV) {
-                const float yq = conv_step(w.q, p.taps, xq);
-                const float yk = conv_step(w.k, p.taps, xk);
-                tv[j].q[t] = with_q ? swish(yq) : 0.f;
-                tv[j].k[t] = swish(yk);
-                if (co.tok) conv_store(w, p, co.tok, co.tok0 + j, h, D, t);
-                if (j == co.snap_j) conv_store(w, p, co.snap, co.snap_row, h, D, t);
-            } else {
-                tv[j].q[t] = with_q ? xq : 0.f;
-                tv[j].k[t] = xk;
-            }
-        }
-    } else {
-        const int c = t - D;
-        for (int j = 0; j < nb; ++j) {
-            const uint8_t *rj = raw + j * RT::BYTES;
-            tv[j].v[c] = IO<TIO>::ld(reinterpret_cast<const TIO *>(rj + 2 * RT::QB) + c);
-            tv[j].a[c] = expf(reinterpret_cast<const float *>(rj + 3 * RT::QB)[c]);
-        }
-        if (c < nb) tv[c].beta = b;
-    }
-}
-
-// The batch stream of one CTA: batches of a, then of b. (Two members and selects, not
-// an array indexed at run time, so that the stream stays in registers.)
-struct TokStream {
-    TokSrc a, b;
-    int nb0, nbat;              // batches of a; all batches
-    __device__ __forceinline__ void locate(int bi, int &which, int &j0, int &nb) const {
-        which = bi < nb0 ? 0 : 1;
-        j0 = (which ? bi - nb0 : bi) * kTokBatch;
-        nb = min(kTokBatch, (which ? b.n : a.n) - j0);
-    }
-    __device__ __forceinline__ TokSrc pick(int which) const {
-        TokSrc r;
-        r.q = which ? b.q : a.q;
-        r.k = which ? b.k : a.k;
-        r.v = which ? b.v : a.v;
-        r.g = which ? b.g : a.g;
-        r.beta = which ? b.beta : a.beta;
-        r.row0 = which ? b.row0 : a.row0;
-        r.n = which ? b.n : a.n;
-        return r;
-    }
-};
-
-__device__ __forceinline__ TokStream make_stream(const TokSrc &a, const TokSrc &b) {
-    TokStream s;
-    s.a = a;
-    s.b = b;
-    s.nb0 = (a.n + kTokBatch - 1) / kTokBatch;
-    s.nbat = s.nb0 + (b.n + kTokBatch - 1) / kTokBatch;
-    return s;
-}
-
-template <int D, typename TIO>
-__device__ __forceinline__ void issue_batch(const TokStream &ts, int bi, uint8_t *raw, uint64_t *bar, int H) {
-    int which, j0, nb;
-    ts.locate(bi, which, j0, nb);
-    issue_rows<D, TIO>(raw, ts.pick(which), j0, nb, H, bar);
-}
-
-// beta of token c of batch bi (threads D + c), issued early as a plain load
-__device__ __forceinline__ float batch_beta(const TokStream &ts, int bi, int c, int H) {
-    int which, j0, nb;
-    ts.locate(bi, which, j0, nb);
-    const TokSrc src = ts.pick(which);
-    return c < nb ? src.beta[src.row0 + (int64_t)(j0 + c) * H] : 0.f;
-}
-
+// ---------------------------------------------------------------- decode
+// One token per (sequence, head): one CTA each, the state read and written once.
 template <int D, typename TIO, bool CONV>
 __global__ void __launch_bounds__(DecodeShape<D>::NT, 2)
 decode_kernel(const __grid_constant__ DecodeParams p) {
@@ -488,87 +388,33 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
     }
     const int t = threadIdx.x;
     float *S = p.pool + ((int64_t)slot * p.H + h) * (int64_t)D * D;
-    float4 st[DecodeShape<D>::R];
-    load_state<D>(st, S);
+    StatePairs<D> P;
+    load_state<D>(P, S);
     const int64_t row = (int64_t)s * p.H + h;
-    ConvWin w;
-    if (CONV && t < D) conv_begin(w, p, p.conv, slot, h, D, t);
-    const ConvOut none{nullptr, 0, nullptr, 0, -1};
-    stage_batch<D, TIO, CONV>(&tv, 1, row, 0, p.q, p.k, p.v, p.g, p.beta, w, p, h, none);
-    if (CONV && t < D) conv_store(w, p, p.conv, slot, h, D, t);
-    finish_batch<D>(&tv, 1, CONV, true);
-    const float4 o = kda_step<D>(st, tv, p.scale);
-    store_state<D>(st, S);
-    if ((t & 31) < 4) IO<TIO>::st4(static_cast<TIO *>(p.o) + row * D + lane_col<D>(), o);
+    if (t < D) {
+        ConvWin w;
+        if (CONV) conv_begin(w, p, p.conv, slot, h, D, t);
+        const float xq = IO<TIO>::ld(static_cast<const TIO *>(p.q) + row * D + t);
+        const float xk = IO<TIO>::ld(static_cast<const TIO *>(p.k) + row * D + t);
+        put_qk<D, CONV>(tv, t, xq, xk, true, w, p.taps);
+        if (CONV) conv_store(w, p, p.conv, slot, h, D, t);
+    } else {
+        const int c = t - D;
+        put_vg<D>(tv, c, IO<TIO>::ld(static_cast<const TIO *>(p.v) + row * D + c), p.g[row * D + c]);
+        if (c == 0) tv.beta = p.beta[row];
+    }
+    __syncthreads();
+    if (t < 32) token_finish<D>(tv, CONV, true);
+    __syncthreads();
+    const float4 o = kda_step<D>(P, tv, p.scale);
+    store_state<D>(P, S);
+    if ((t & 31) < 4) IO<TIO>::st4(static_cast<TIO *>(p.o) + row * D + lane_col(), o);
 }
 
-// two CTAs per SM (register cap) keep enough state loads and stores in flight
-template <int D, typename TIO, bool CONV>
-__global__ void __launch_bounds__(DecodeShape<D>::NT, 2)
-verify_kernel(const __grid_constant__ DecodeParams p) {
-    using RT = RawTok<D, TIO>;
-    __shared__ TokVec<D> tv[kTokBatch];
-    extern __shared__ __align__(128) uint8_t dyn_smem[];   // two raw row buffers
-    auto raw = [&](int i) { return dyn_smem + i * (kTokBatch * RT::BYTES); };
-    __shared__ uint64_t bars[2];
-    const int s = blockIdx.x / p.H, h = blockIdx.x % p.H;
-    const int32_t slot = p.slots[s];
-    if (slot < 0 || slot >= p.n_slots) {
-        if (threadIdx.x == 0) record_status(KDA_ERR_RANGE);
-        return;
-    }
-    const int n_tok = p.tok0[s + 1] - p.tok0[s];
-    const int64_t tok_first = p.tok_base + p.tok0[s];
-    const int t = threadIdx.x, warp = t >> 5;
-    const TokSrc none{nullptr, nullptr, nullptr, nullptr, nullptr, 0, 0};
-    const TokStream ts = make_stream(TokSrc{p.q, p.k, p.v, p.g, p.beta, tok_first * p.H + h, n_tok}, none);
-    if (t == 0) {
-        tc::bar_init(&bars[0], 1);
-        tc::bar_init(&bars[1], 1);
-        tc::bar_init_fence();
-        for (int bi = 0; bi < 2 && bi < ts.nbat; ++bi) issue_batch<D, TIO>(ts, bi, raw(bi), &bars[bi], p.H);
-    }
-    float bnext = (t >= D && ts.nbat > 0) ? batch_beta(ts, 0, t - D, p.H) : 0.f;
-    const float *S = p.pool + ((int64_t)slot * p.H + h) * (int64_t)D * D;
-    float4 st[DecodeShape<D>::R];
-#pragma unroll
-    for (int m = 0; m < DecodeShape<D>::R; ++m) st[m] = ld_stream(S + lane_off<D>(m));
-    ConvWin w;
-    if (CONV && t < D) conv_begin(w, p, p.conv, slot, h, D, t);
-    __syncthreads();  // barrier initialisation visible
-    bool ok = true;
-    for (int bi = 0; bi < ts.nbat; ++bi) {
-        int which, j0, nb;
-        ts.locate(bi, which, j0, nb);
-        const float b = bnext;
-        if (t >= D && bi + 1 < ts.nbat) bnext = batch_beta(ts, bi + 1, t - D, p.H);
-        ok = tc::bar_wait(&bars[bi & 1], (uint32_t)((bi >> 1) & 1)) && ok;
-        const ConvOut co{p.conv_tok, tok_first + j0, nullptr, 0, -1};
-        convert_batch<D, TIO, CONV>(tv, raw(bi & 1), nb, true, true, b, w, p, h, co);
-        __syncthreads();  // vectors staged, raw buffer read
-        if (t == 0 && bi + 2 < ts.nbat) issue_batch<D, TIO>(ts, bi + 2, raw(bi & 1), &bars[bi & 1], p.H);
-        if (warp < nb) token_finish<D>(tv[warp], CONV, true);
-        for (int j = DecodeShape<D>::NW; j < nb; ++j)
-            if (warp == 0) token_finish<D>(tv[j], CONV, true);
-        __syncthreads();
-        for (int j = 0; j < nb; ++j) {
-            const float4 o = kda_step<D>(st, tv[j], p.scale);
-            const int64_t row = (tok_first + j0 + j) * p.H + h;
-            store_state<D>(st, p.token_states + row * (int64_t)D * D);
-            if ((t & 31) < 4) IO<TIO>::st4(static_cast<TIO *>(p.o) + row * D + lane_col<D>(), o);
-        }
-        __syncthreads();  // the vectors are free for the next batch
-    }
-    if (!ok && t == 0)  // copies still in flight land before the shared memory is released
-        for (int bi = ts.nbat - 2 < 0 ? 0 : ts.nbat - 2; bi < ts.nbat; ++bi)
-            tc::bar_wait(&bars[bi & 1], (uint32_t)((bi >> 1) & 1), 1u << 16);
-}
-
-// ---------------------------------------------------------------- verify + commit
-// One speculative step with the previous step's commit fused in: the live state is
-// read once, the previous step's first n_accept tokens are replayed into it (state
-// only), it is written back once, and this step's draft tokens run from it with
-// outputs only. No per-token state is written.
+// ---------------------------------------------------------------- verify, verify + commit
+// The previous step's commit, for verify + commit: the live state is read once, the
+// previous step's first n_accept tokens are replayed into it (state only), it is written
+// back once, and this step's draft tokens run from it with outputs only.
 struct CommitParams {
     const void *q;              // the previous step's raw q (front-end on: advances the q window)
     float *conv_snapshots;      // front-end on: conv state at the boundary [rows, 2, H, D, taps-1]
@@ -585,107 +431,333 @@ struct CommitParams {
     int32_t tok0[kMaxSeqsPerLaunch + 1];  // previous batch offsets (relative)
 };
 
-struct VerifyCommitParams {
-    DecodeParams p;   // this step: q, k, v, g, beta, o, tok0/tok_base, slots, pool (in/out)
-    CommitParams c;
+// A persistent grid: CTA b owns the contiguous items [b per_cta, (b + 1) per_cta) of the
+// (sequence, head) list, so that its items share few sequences. Warp 0 is the producer:
+// one bulk copy brings the next item's state (and conv window and weights) into shared
+// memory while the current item runs from registers, and the item's token rows come in
+// batches of TB by 3-D TMA tiles (channels x 1 head x TB rows) into two buffers, two
+// batches ahead across item boundaries.
+struct SpecParams {
+    CUtensorMap mq, mk, mv, mg;       // this step's q, k, v, g rows: (D, H, rows), box (D, 1, TB)
+    CUtensorMap pq, pk, pv, pg;       // the previous step's (replay; pq with the front-end only)
+    DecodeParams p;                   // verify: token_states, conv_tok; pool read-only
+    CommitParams c;                   // verify + commit only
+    int32_t n_items, per_cta;
 };
 
-template <int D, typename TIO, bool CONV>
-__global__ void __launch_bounds__(DecodeShape<D>::NT, 2)
-verify_commit_kernel(const __grid_constant__ VerifyCommitParams P) {
-    using RT = RawTok<D, TIO>;
-    const DecodeParams &p = P.p;
-    const CommitParams &c = P.c;
-    __shared__ TokVec<D> tv[kTokBatch];
-    extern __shared__ __align__(128) uint8_t dyn_smem[];   // two raw row buffers
-    auto raw = [&](int i) { return dyn_smem + i * (kTokBatch * RT::BYTES); };
-    __shared__ uint64_t bars[2];
-    const int s = blockIdx.x / p.H, h = blockIdx.x % p.H;
-    const int32_t slot = p.slots[s];
-    const int m_prev = c.tok0[s + 1] - c.tok0[s];
-    const int32_t na = c.n_accept[s];
-    int64_t srow = -1, jsnap = -1;          // snapshot row, and the replayed token after which it falls
-    if (c.snap_interval > 0 && c.snap_row != nullptr && c.snap_row[s] >= 0) {
-        srow = c.snap_row[s];
-        const int64_t p0 = c.pos[s];
-        jsnap = (p0 / c.snap_interval + 1) * c.snap_interval - p0 - 1;
+template <typename TIO> struct SpecShape {
+    static constexpr int TB = sizeof(TIO) == 2 ? 8 : 4;   // tokens per batch
+};
+constexpr int kSpecSeqs = 16;         // sequence records per CTA (the host keeps ranges within it)
+
+struct SeqMeta {
+    int32_t slot, na, n_prev, n_tok, cnew, ok;
+    int64_t srow, jsnap;  // snapshot row, and the committed-token index after which it falls
+};
+
+template <int D, typename TIO> struct SpecSmem {
+    static constexpr int TB = SpecShape<TIO>::TB;
+    static constexpr uint32_t ROW = D * sizeof(TIO);
+    static constexpr uint32_t ST = 0;                                  // state [D][D] fp32
+    static constexpr uint32_t CW = ST + D * D * 4;                     // conv: q, k windows, q, k weights
+    static constexpr uint32_t CW_K = D * (kMaxTaps - 1) * 4, CW_WQ = 2 * CW_K, CW_WK = CW_WQ + D * kMaxTaps * 4;
+    static constexpr uint32_t RAW0 = CW + CW_WK + D * kMaxTaps * 4;    // raw batches: q, k, v, g rows
+    static constexpr uint32_t RAW = TB * (3 * ROW + D * 4);
+    static constexpr uint32_t TV = RAW0 + 2 * RAW;                     // token vectors [TB]
+    static constexpr uint32_t META = TV + TB * sizeof(TokVec<D>);      // SeqMeta [kSpecSeqs]
+    static constexpr uint32_t BARS = META + kSpecSeqs * sizeof(SeqMeta);   // state, raw 0, raw 1
+    static constexpr uint32_t PROD = BARS + 32;                        // producer cursors
+    static constexpr uint32_t BYTES = PROD + 32 + 128;                 // + alignment slack
+    static_assert(RAW0 % 128 == 0 && RAW % 128 == 0 && (TB * ROW) % 128 == 0 && TV % 16 == 0, "alignment");
+};
+
+struct ItemInfo {
+    int s, h, na, n_tok, nb0, nbat;
+    bool valid, cnew;
+    int32_t slot;
+    int64_t srow, jsnap, prev_first, tok_first;
+};
+
+template <int D, typename TIO, bool COMMIT>
+__device__ __forceinline__ ItemInfo item_info(const SpecParams &P, const SeqMeta *meta, int s0, int it) {
+    constexpr int TB = SpecShape<TIO>::TB;
+    ItemInfo I;
+    I.s = it / P.p.H;
+    I.h = it - I.s * P.p.H;
+    const SeqMeta &m = meta[I.s - s0];
+    I.slot = m.slot;
+    I.valid = m.ok != 0;
+    I.n_tok = m.n_tok;
+    I.na = COMMIT ? m.na : 0;
+    I.cnew = COMMIT && m.cnew != 0;
+    I.srow = m.srow;
+    I.jsnap = m.jsnap;
+    I.nb0 = (I.na + TB - 1) / TB;
+    I.nbat = I.nb0 + (I.n_tok + TB - 1) / TB;
+    I.prev_first = COMMIT ? P.c.tok_base + P.c.tok0[I.s] : 0;
+    I.tok_first = P.p.tok_base + P.p.tok0[I.s];
+    return I;
+}
+
+struct ProdCursor {
+    int kb, bb, nb_issued;     // batch cursor: local item, batch within it; batches issued
+    int ks, ns_issued;         // state cursor: next local item to consider; states issued
+};
+
+// warp 0: issue the next batch of token rows (lane 0 the copies, lanes c < nb the
+// loads of their beta, kept in breg until the batch is converted)
+template <int D, typename TIO, bool CONV, bool COMMIT>
+__device__ __forceinline__ void produce_batch(const SpecParams &P, uint8_t *sm, const SeqMeta *meta, int s0,
+                                              int i0, int n_local, float &b0, float &b1) {
+    using SM = SpecSmem<D, TIO>;
+    constexpr int TB = SM::TB;
+    ProdCursor *cur = reinterpret_cast<ProdCursor *>(sm + SM::PROD);
+    const int lane = threadIdx.x & 31;
+    int kb = cur->kb, bb = cur->bb;
+    ItemInfo I;
+    for (;; ++kb, bb = 0) {
+        if (kb >= n_local) return;
+        I = item_info<D, TIO, COMMIT>(P, meta, s0, i0 + kb);
+        if (I.valid && bb < I.nbat) break;
     }
-    if (slot < 0 || slot >= p.n_slots || na < 0 || na > m_prev || srow >= c.n_snap_rows) {
-        if (threadIdx.x == 0) record_status(KDA_ERR_RANGE);
+    const bool replay = bb < I.nb0;
+    const int j0 = (replay ? bb : bb - I.nb0) * TB;
+    const int nb = min(TB, (replay ? I.na : I.n_tok) - j0);
+    const int64_t row0 = (replay ? I.prev_first : I.tok_first) + j0;
+    const int slot = cur->nb_issued & 1;
+    __syncwarp();
+    if (lane == 0) {
+        uint64_t *bar = reinterpret_cast<uint64_t *>(sm + SM::BARS) + 1 + slot;
+        uint8_t *raw = sm + SM::RAW0 + slot * SM::RAW;
+        const bool with_q = !replay || CONV;
+        tc::bar_expect_tx(bar, (uint32_t)TB * ((with_q ? 3u : 2u) * SM::ROW + D * 4u));
+        const int z = (int)row0;
+        if (with_q) tc::tma_load3(raw, replay ? &P.pq : &P.mq, 0, I.h, z, bar);
+        tc::tma_load3(raw + TB * SM::ROW, replay ? &P.pk : &P.mk, 0, I.h, z, bar);
+        tc::tma_load3(raw + 2 * TB * SM::ROW, replay ? &P.pv : &P.mv, 0, I.h, z, bar);
+        tc::tma_load3(raw + 3 * TB * SM::ROW, replay ? &P.pg : &P.mg, 0, I.h, z, bar);
+        cur->kb = kb;
+        cur->bb = bb + 1;
+        cur->nb_issued += 1;
+    }
+    if (lane < nb) {
+        const float *beta = replay ? P.c.beta : P.p.beta;
+        const float b = beta[(row0 + lane) * P.p.H + I.h];
+        if (slot) b1 = b;
+        else b0 = b;
+    }
+    __syncwarp();
+}
+
+// thread 0: issue the state (and conv window and weights) of the next item that needs it
+template <int D, typename TIO, bool CONV, bool COMMIT>
+__device__ __forceinline__ void produce_state(const SpecParams &P, uint8_t *sm, const SeqMeta *meta, int s0,
+                                              int i0, int n_local) {
+    using SM = SpecSmem<D, TIO>;
+    ProdCursor *cur = reinterpret_cast<ProdCursor *>(sm + SM::PROD);
+    for (int ks = cur->ks; ks < n_local; ++ks) {
+        const ItemInfo I = item_info<D, TIO, COMMIT>(P, meta, s0, i0 + ks);
+        if (!I.valid || I.nbat == 0) continue;
+        const DecodeParams &p = P.p;
+        uint64_t *bar = reinterpret_cast<uint64_t *>(sm + SM::BARS);
+        const int K = p.taps;
+        const uint32_t wb = CONV ? (uint32_t)(D * (K - 1) * 4) : 0u, cb = CONV ? (uint32_t)(D * K * 4) : 0u;
+        tc::bar_expect_tx(bar, (uint32_t)(D * D * 4) + 2 * wb + 2 * cb);
+        tc::bulk_load(sm + SM::ST, p.pool + ((int64_t)I.slot * p.H + I.h) * (int64_t)D * D, D * D * 4, bar);
+        if (CONV) {
+            tc::bulk_load(sm + SM::CW, p.conv + conv_index(2 * (int64_t)I.slot, p.H, I.h, D, 0, K), wb, bar);
+            tc::bulk_load(sm + SM::CW + SM::CW_K, p.conv + conv_index(2 * (int64_t)I.slot + 1, p.H, I.h, D, 0, K),
+                          wb, bar);
+            tc::bulk_load(sm + SM::CW + SM::CW_WQ, p.wq + (int64_t)I.h * D * K, cb, bar);
+            tc::bulk_load(sm + SM::CW + SM::CW_WK, p.wk + (int64_t)I.h * D * K, cb, bar);
+        }
+        cur->ks = ks + 1;
+        cur->ns_issued += 1;
         return;
     }
-    const int n_tok = p.tok0[s + 1] - p.tok0[s];
-    // committed tokens: the replayed prefix, then (mixed step) this step's tokens;
-    // jsnap indexes that sequence
-    const bool cnew = c.commit_new != nullptr && c.commit_new[s] != 0 && n_tok > 0;
-    const int t = threadIdx.x, warp = t >> 5;
-    // the stream: the replayed prefix of the previous batch (its q only for the front-end's
-    // window), then this step's tokens
-    const int64_t prev_first = c.tok_base + c.tok0[s];
-    const int64_t tok_first = p.tok_base + p.tok0[s];
-    const TokStream ts = make_stream(TokSrc{CONV ? c.q : nullptr, c.k, c.v, c.g, c.beta, prev_first * p.H + h, na},
-                                     TokSrc{p.q, p.k, p.v, p.g, p.beta, tok_first * p.H + h, n_tok});
-    if (t == 0) {
-        tc::bar_init(&bars[0], 1);
-        tc::bar_init(&bars[1], 1);
-        tc::bar_init_fence();
-        for (int bi = 0; bi < 2 && bi < ts.nbat; ++bi) issue_batch<D, TIO>(ts, bi, raw(bi), &bars[bi], p.H);
-    }
-    float bnext = (t >= D && ts.nbat > 0) ? batch_beta(ts, 0, t - D, p.H) : 0.f;
-    float *S = p.pool + ((int64_t)slot * p.H + h) * (int64_t)D * D;
-    float4 st[DecodeShape<D>::R];
-    load_state<D>(st, S);
-    ConvWin w;
-    if (CONV && t < D) conv_begin(w, p, p.conv, slot, h, D, t);
-    __syncthreads();  // barrier initialisation visible
-    bool ok = true;
-    for (int bi = 0; bi < ts.nbat; ++bi) {
-        int which, j0, nb;
-        ts.locate(bi, which, j0, nb);
-        const bool replay = which == 0;
-        const float b = bnext;
-        if (t >= D && bi + 1 < ts.nbat) bnext = batch_beta(ts, bi + 1, t - D, p.H);
-        ok = tc::bar_wait(&bars[bi & 1], (uint32_t)((bi >> 1) & 1)) && ok;
-        // the committed-token index of this batch's first token, and a snapshot inside it
-        const int64_t c0 = replay ? j0 : (cnew ? na + j0 : -1);
-        const int64_t js = (c0 >= 0 && jsnap >= c0 && jsnap < c0 + nb) ? jsnap - c0 : -1;
-        const ConvOut co{nullptr, 0, c.conv_snapshots, srow, (int)js};
-        convert_batch<D, TIO, CONV>(tv, raw(bi & 1), nb, CONV || !replay, !replay, b, w, p, h, co);
-        __syncthreads();  // vectors staged, raw buffer read
-        if (t == 0 && bi + 2 < ts.nbat) issue_batch<D, TIO>(ts, bi + 2, raw(bi & 1), &bars[bi & 1], p.H);
-        if (warp < nb) token_finish<D>(tv[warp], CONV, !replay);
-        for (int j = DecodeShape<D>::NW; j < nb; ++j)
-            if (warp == 0) token_finish<D>(tv[j], CONV, !replay);
-        __syncthreads();
-        if (replay) {
-            // 1. commit: the accepted prefix, state only
-            for (int j = 0; j < nb; ++j) {
-                kda_step<D, false>(st, tv[j], 0.f);
-                if (j == js) store_state<D>(st, c.snapshots + (srow * p.H + h) * (int64_t)D * D);
-            }
-            if (bi == ts.nb0 - 1 && !cnew) {
-                store_state<D>(st, S);
-                if (CONV && t < D) conv_store(w, p, p.conv, slot, h, D, t);
-            }
-        } else {
-            // 2. this step's tokens from the committed state: outputs (and with commit_new
-            // their state is committed too)
-            for (int j = 0; j < nb; ++j) {
-                const float4 o = kda_step<D>(st, tv[j], p.scale);
-                const int64_t row = (tok_first + j0 + j) * p.H + h;
-                if ((t & 31) < 4) IO<TIO>::st4(static_cast<TIO *>(p.o) + row * D + lane_col<D>(), o);
-                if (j == js) store_state<D>(st, c.snapshots + (srow * p.H + h) * (int64_t)D * D);
+    cur->ks = n_local;
+}
+
+// Raw rows of a batch -> token vectors: threads t < D channel t of q and k (the
+// front-end's conv window in token order with CONV), threads t >= D channel t - D of v
+// and g, warp-0 lanes j < nb the beta they loaded.
+template <int D, typename TIO, bool CONV>
+__device__ __forceinline__ void convert_batch(TokVec<D> *tv, const uint8_t *raw, int nb, bool read_q, bool with_q,
+                                              float b, ConvWin &w, const DecodeParams &p, int h, const ConvOut &co) {
+    constexpr int TB = SpecShape<TIO>::TB;
+    constexpr uint32_t ROW = D * sizeof(TIO);
+    const int t = threadIdx.x;
+    if (t < D) {
+        const TIO *rq = reinterpret_cast<const TIO *>(raw), *rk = reinterpret_cast<const TIO *>(raw + TB * ROW);
+        for (int j = 0; j < nb; ++j) {
+            const float xq = read_q ? IO<TIO>::ld(rq + j * D + t) : 0.f;
+            const float xk = IO<TIO>::ld(rk + j * D + t);
+            put_qk<D, CONV>(tv[j], t, xq, xk, with_q, w, p.taps);
+            if (CONV) {
+                if (co.tok) conv_store(w, p, co.tok, co.tok0 + j, h, D, t);
+                if (j == co.snap_j) conv_store(w, p, co.snap, co.snap_row, h, D, t);
             }
         }
-        __syncthreads();  // the vectors are free for the next batch
+        if (t < nb) tv[t].beta = b;
+    } else {
+        const int c = t - D;
+        const TIO *rv = reinterpret_cast<const TIO *>(raw + 2 * TB * ROW);
+        const float *rgt = reinterpret_cast<const float *>(raw + 3 * TB * ROW);
+        for (int j = 0; j < nb; ++j) put_vg<D>(tv[j], c, IO<TIO>::ld(rv + j * D + c), rgt[j * D + c]);
     }
-    if (cnew) {
-        store_state<D>(st, S);
-        if (CONV && t < D) conv_store(w, p, p.conv, slot, h, D, t);
+}
+
+// COMMIT = false: verify. Every token gives its output and its state (token_states row),
+// and with the front-end its conv state (conv_tok row); the pool is only read.
+// COMMIT = true: verify + commit. The stream of an item is the replayed prefix (state
+// only; the state is written back to the pool after it, or after this step's tokens with
+// commit_new), then this step's tokens (outputs); a snapshot at a crossed boundary.
+template <int D, typename TIO, bool CONV, bool COMMIT>
+__global__ void __launch_bounds__(DecodeShape<D>::NT, 2)
+spec_kernel(const __grid_constant__ SpecParams P) {
+    using SM = SpecSmem<D, TIO>;
+    using Sh = DecodeShape<D>;
+    constexpr int TB = SM::TB;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    const DecodeParams &p = P.p;
+    const CommitParams &c = P.c;
+    TokVec<D> *tv = reinterpret_cast<TokVec<D> *>(sm + SM::TV);
+    SeqMeta *meta = reinterpret_cast<SeqMeta *>(sm + SM::META);
+    uint64_t *bar_s = reinterpret_cast<uint64_t *>(sm + SM::BARS), *bar_t = bar_s + 1;
+    ProdCursor *cur = reinterpret_cast<ProdCursor *>(sm + SM::PROD);
+    const int t = threadIdx.x, warp = t >> 5;
+
+    const int i0 = blockIdx.x * P.per_cta;
+    const int n_local = max(0, min(P.n_items, i0 + P.per_cta) - i0);
+    if (n_local == 0) return;
+    const int s0 = i0 / p.H, n_meta = (i0 + n_local - 1) / p.H - s0 + 1;
+    if (n_meta > kSpecSeqs) {                   // the host never launches this
+        if (t == 0) record_status(KDA_ERR_INVALID);
+        return;
     }
-    if (!ok && t == 0)  // copies still in flight land before the shared memory is released
-        for (int bi = ts.nbat - 2 < 0 ? 0 : ts.nbat - 2; bi < ts.nbat; ++bi)
-            tc::bar_wait(&bars[bi & 1], (uint32_t)((bi >> 1) & 1), 1u << 16);
+    // per-sequence records of this CTA's range
+    if (t < n_meta) {
+        const int s = s0 + t;
+        SeqMeta m;
+        m.slot = p.slots[s];
+        m.n_tok = p.tok0[s + 1] - p.tok0[s];
+        m.ok = m.slot >= 0 && m.slot < p.n_slots;
+        m.na = 0; m.n_prev = 0; m.cnew = 0; m.srow = -1; m.jsnap = -1;
+        if (COMMIT) {
+            m.na = c.n_accept[s];
+            m.n_prev = c.tok0[s + 1] - c.tok0[s];
+            m.cnew = c.commit_new != nullptr && c.commit_new[s] != 0 && m.n_tok > 0;
+            if (c.snap_interval > 0 && c.snap_row != nullptr && c.snap_row[s] >= 0) {
+                m.srow = c.snap_row[s];
+                const int64_t p0 = c.pos[s];
+                m.jsnap = (p0 / c.snap_interval + 1) * c.snap_interval - p0 - 1;
+            }
+            m.ok = m.ok && m.na >= 0 && m.na <= m.n_prev && m.srow < c.n_snap_rows;
+        }
+        meta[t] = m;
+    }
+    if (t == 0) {
+        tc::bar_init(bar_s, 1);
+        tc::bar_init(&bar_t[0], 1);
+        tc::bar_init(&bar_t[1], 1);
+        tc::bar_init_fence();
+        cur->kb = 0; cur->bb = 0; cur->nb_issued = 0; cur->ks = 0; cur->ns_issued = 0;
+    }
+    __syncthreads();
+    float b0 = 0.f, b1 = 0.f;   // warp 0: beta of the batches in the two raw buffers
+    if (t == 0) produce_state<D, TIO, CONV, COMMIT>(P, sm, meta, s0, i0, n_local);
+    if (warp == 0) {
+        produce_batch<D, TIO, CONV, COMMIT>(P, sm, meta, s0, i0, n_local, b0, b1);
+        produce_batch<D, TIO, CONV, COMMIT>(P, sm, meta, s0, i0, n_local, b0, b1);
+    }
+
+    bool ok = true;
+    int g = 0, vs = 0;          // batches and states consumed
+    for (int kl = 0; kl < n_local && ok; ++kl) {
+        int nbat;
+        {
+            const ItemInfo I = item_info<D, TIO, COMMIT>(P, meta, s0, i0 + kl);
+            if (!I.valid) {
+                if (t == 0) record_status(KDA_ERR_RANGE);
+                continue;
+            }
+            nbat = I.nbat;
+        }
+        if (nbat == 0) continue;
+        const bool sok = tc::bar_wait(bar_s, (uint32_t)(vs & 1));
+        vs += sok;
+        ok = ok && sok;
+        StatePairs<D> Pr;
+        load_state_smem<D>(Pr, reinterpret_cast<const float *>(sm + SM::ST));
+        ConvWin w;
+        if (CONV && t < D) {
+            const float *cw = reinterpret_cast<const float *>(sm + SM::CW);
+            const int K = p.taps;
+            win_load(w.q, cw + SM::CW_WQ / 4 + t * K, cw + t * (K - 1), K);
+            win_load(w.k, cw + SM::CW_WK / 4 + t * K, cw + SM::CW_K / 4 + t * (K - 1), K);
+        }
+        __syncthreads();        // the state buffer is free
+        if (t == 0 && ok) produce_state<D, TIO, CONV, COMMIT>(P, sm, meta, s0, i0, n_local);
+        for (int bi = 0; bi < nbat; ++bi) {
+            // the item's fields are re-read from shared memory after every barrier rather
+            // than held in registers through the steps
+            const ItemInfo I = item_info<D, TIO, COMMIT>(P, meta, s0, i0 + kl);
+            const bool replay = bi < I.nb0;
+            const int j0 = (replay ? bi : bi - I.nb0) * TB;
+            const int nb = min(TB, (replay ? I.na : I.n_tok) - j0);
+            // the committed-token index of this batch's first token, and a snapshot in it
+            const int64_t c0 = !COMMIT ? -1 : replay ? j0 : (I.cnew ? I.na + j0 : -1);
+            const int js = (c0 >= 0 && I.jsnap >= c0 && I.jsnap < c0 + nb) ? (int)(I.jsnap - c0) : -1;
+            const ConvOut co = COMMIT ? ConvOut{nullptr, 0, c.conv_snapshots, I.srow, js}
+                                      : ConvOut{p.conv_tok, I.tok_first + j0, nullptr, 0, -1};
+            const bool bok = tc::bar_wait(&bar_t[g & 1], (uint32_t)((g >> 1) & 1));
+            convert_batch<D, TIO, CONV>(tv, sm + SM::RAW0 + (g & 1) * SM::RAW, nb, CONV || !replay, !replay,
+                                        (g & 1) ? b1 : b0, w, p, I.h, co);
+            ok = __syncthreads_and(ok && bok);   // vectors staged, raw buffer read
+            if (!ok) break;
+            ++g;
+            if (warp == 0) produce_batch<D, TIO, CONV, COMMIT>(P, sm, meta, s0, i0, n_local, b0, b1);
+            for (int j = warp; j < nb; j += Sh::NW) token_finish<D>(tv[j], CONV, !replay);
+            __syncthreads();
+            const int64_t hh = I.h;
+            if (replay) {
+                const bool store_after = bi == I.nb0 - 1 && !I.cnew;
+                float *snap = js >= 0 ? c.snapshots + (I.srow * p.H + hh) * (int64_t)D * D : nullptr;
+                for (int j = 0; j < nb; ++j) {
+                    kda_step<D, false>(Pr, tv[j], 0.f);
+                    if (j == js) store_state<D>(Pr, snap);
+                }
+                if (store_after) {
+                    store_state<D>(Pr, p.pool + ((int64_t)I.slot * p.H + hh) * (int64_t)D * D);
+                    if (CONV && t < D) conv_store(w, p, p.conv, I.slot, I.h, D, t);
+                }
+            } else {
+                float *snap = js >= 0 ? c.snapshots + (I.srow * p.H + hh) * (int64_t)D * D : nullptr;
+                const int64_t row0 = (I.tok_first + j0) * p.H + hh;
+                for (int j = 0; j < nb; ++j) {
+                    const float4 o = kda_step<D>(Pr, tv[j], p.scale);
+                    const int64_t row = row0 + (int64_t)j * p.H;
+                    if ((t & 31) < 4) IO<TIO>::st4(static_cast<TIO *>(p.o) + row * D + lane_col(), o);
+                    if (!COMMIT) store_state<D>(Pr, p.token_states + row * (int64_t)D * D);
+                    if (COMMIT && j == js) store_state<D>(Pr, snap);
+                }
+            }
+            __syncthreads();                  // the vectors are free for the next batch
+        }
+        if (ok) {
+            const ItemInfo I = item_info<D, TIO, COMMIT>(P, meta, s0, i0 + kl);
+            if (I.cnew) {
+                store_state<D>(Pr, p.pool + ((int64_t)I.slot * p.H + I.h) * (int64_t)D * D);
+                if (CONV && t < D) conv_store(w, p, p.conv, I.slot, I.h, D, t);
+            }
+        }
+    }
+    if (t == 0) {
+        // copies still in flight land before the shared memory is released
+        for (; vs < cur->ns_issued; ++vs) tc::bar_wait(bar_s, (uint32_t)(vs & 1), 1u << 16);
+        for (; g < cur->nb_issued; ++g) tc::bar_wait(&bar_t[g & 1], (uint32_t)((g >> 1) & 1), 1u << 16);
+    }
 }
 
 }  // namespace kda

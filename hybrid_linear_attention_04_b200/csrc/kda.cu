@@ -62,66 +62,115 @@ static float eff_scale(const kda_dims *d) {
 
 // ---------------------------------------------------------------- decode ----
 template <int D, typename TIO>
-static kda_status launch_decode(DecodeParams &p, int n_blocks, cudaStream_t st, bool verify) {
-    const bool conv = p.taps > 0;
-    constexpr uint32_t dyn = RawTok<D, TIO>::SMEM;
-    if (verify) {
-        static std::atomic<unsigned long long> attr[2]{{0}, {0}};
-        const kda_status r = conv ? set_smem_limit_once((const void *)verify_kernel<D, TIO, true>, dyn, attr[1])
-                                  : set_smem_limit_once((const void *)verify_kernel<D, TIO, false>, dyn, attr[0]);
-        if (r != KDA_OK) return r;
-    }
+static kda_status launch_decode(DecodeParams &p, int n_blocks, cudaStream_t st) {
     if (!launch_gate()) return KDA_ERR_CUDA;
-    if (verify) {
-        if (conv) verify_kernel<D, TIO, true><<<n_blocks, DecodeShape<D>::NT, dyn, st>>>(p);
-        else verify_kernel<D, TIO, false><<<n_blocks, DecodeShape<D>::NT, dyn, st>>>(p);
-    } else {
-        if (conv) decode_kernel<D, TIO, true><<<n_blocks, DecodeShape<D>::NT, 0, st>>>(p);
-        else decode_kernel<D, TIO, false><<<n_blocks, DecodeShape<D>::NT, 0, st>>>(p);
-    }
+    if (p.taps > 0) decode_kernel<D, TIO, true><<<n_blocks, DecodeShape<D>::NT, 0, st>>>(p);
+    else decode_kernel<D, TIO, false><<<n_blocks, DecodeShape<D>::NT, 0, st>>>(p);
     return last_launch_status();
 }
 
 template <typename TIO>
-static kda_status dispatch_decode(int D, DecodeParams &p, int n_blocks, cudaStream_t st, bool verify) {
+static kda_status dispatch_decode(int D, DecodeParams &p, int n_blocks, cudaStream_t st) {
     switch (D) {
-    case 32: return launch_decode<32, TIO>(p, n_blocks, st, verify);
-    case 64: return launch_decode<64, TIO>(p, n_blocks, st, verify);
-    case 128: return launch_decode<128, TIO>(p, n_blocks, st, verify);
+    case 32: return launch_decode<32, TIO>(p, n_blocks, st);
+    case 64: return launch_decode<64, TIO>(p, n_blocks, st);
+    case 128: return launch_decode<128, TIO>(p, n_blocks, st);
     }
     return KDA_ERR_UNSUPPORTED;
 }
 
-template <typename TIO>
-static kda_status dispatch_verify_commit(int D, VerifyCommitParams &P, int n_blocks, cudaStream_t st) {
-    if (D != 32 && D != 64 && D != 128) return KDA_ERR_UNSUPPORTED;
-    const bool conv = P.p.taps > 0;
-    static std::atomic<unsigned long long> attr[3][2]{};
-    const int di = D == 32 ? 0 : D == 64 ? 1 : 2;
-    kda_status r = KDA_OK;
-#define KDA_VC_ATTR(d)                                                                                 \
-    r = conv ? set_smem_limit_once((const void *)verify_commit_kernel<d, TIO, true>,                    \
-                                   RawTok<d, TIO>::SMEM, attr[di][1])                                   \
-             : set_smem_limit_once((const void *)verify_commit_kernel<d, TIO, false>,                   \
-                                   RawTok<d, TIO>::SMEM, attr[di][0]);
-    switch (D) {
-    case 32: KDA_VC_ATTR(32) break;
-    case 64: KDA_VC_ATTR(64) break;
-    default: KDA_VC_ATTR(128) break;
+// ---------------------------------------------------- verify, verify + commit ----
+constexpr int kMaxDevices = 64;     // devices whose scratch address is cached
+
+static int sm_count() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    static std::atomic<int> cache[kMaxDevices];
+    int n = dev < kMaxDevices ? cache[dev].load(std::memory_order_relaxed) : 0;
+    if (n == 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        if (dev < kMaxDevices) cache[dev].store(n, std::memory_order_relaxed);
     }
-#undef KDA_VC_ATTR
+    return n;
+}
+
+// Token rows of one packed [rows, H, D] array as a 3-D tensor (channel, head, row) read
+// in boxes of D channels x 1 head x `box_rows` rows. An empty or absent array gets a
+// zeroed map, which no launch then reads.
+static bool encode_rows(CUtensorMap *m, const void *base, bool bf16, int D, int H, int64_t rows, int box_rows) {
+    std::memset(m, 0, sizeof(*m));
+    if (!base || rows <= 0) return true;
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t es = bf16 ? 2 : 4;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
+    cuuint64_t strides[2] = {(cuuint64_t)D * es, (cuuint64_t)H * D * es};
+    cuuint32_t box[3] = {(cuuint32_t)D, 1, (cuuint32_t)box_rows};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+               const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, typename TIO, bool CONV, bool COMMIT>
+static kda_status launch_spec_t(SpecParams &P, cudaStream_t st) {
+    using SM = SpecSmem<D, TIO>;
+    const void *fn = (const void *)spec_kernel<D, TIO, CONV, COMMIT>;
+    static std::atomic<unsigned long long> attr{0};
+    static std::atomic<int> occ_cache{0};
+    kda_status r = set_smem_limit_once(fn, (int)SM::BYTES, attr);
     if (r != KDA_OK) return r;
-    if (!launch_gate()) return KDA_ERR_CUDA;
-#define KDA_VC(d)                                                                                    \
-    if (conv) verify_commit_kernel<d, TIO, true><<<n_blocks, DecodeShape<d>::NT, RawTok<d, TIO>::SMEM, st>>>(P); \
-    else verify_commit_kernel<d, TIO, false><<<n_blocks, DecodeShape<d>::NT, RawTok<d, TIO>::SMEM, st>>>(P);
-    switch (D) {
-    case 32: KDA_VC(32) break;
-    case 64: KDA_VC(64) break;
-    default: KDA_VC(128) break;
+    int occ = occ_cache.load(std::memory_order_relaxed);
+    if (occ == 0) {
+        const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, DecodeShape<D>::NT, SM::BYTES);
+        if (e != cudaSuccess) return fail_cuda(e);
+        if (occ < 1) return fail_text("the verify kernel does not fit on an SM");
+        occ_cache.store(occ, std::memory_order_relaxed);
     }
-#undef KDA_VC
+    const int sms = sm_count();
+    if (sms < 1) return fail_text("no multiprocessor count");
+    // resident CTAs on every SM, each a contiguous range of (sequence, head) items that
+    // spans at most kSpecSeqs sequences
+    const int64_t n_items = P.n_items, H = P.p.H;
+    const int64_t grid0 = std::max<int64_t>(1, std::min<int64_t>(n_items, (int64_t)occ * sms));
+    int64_t per = (n_items + grid0 - 1) / grid0;
+    per = std::max<int64_t>(1, std::min<int64_t>(per, (kSpecSeqs - 2) * H + 2));
+    const int64_t grid = (n_items + per - 1) / per;
+    if (grid > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    P.per_cta = (int32_t)per;
+    if (!launch_gate()) return KDA_ERR_CUDA;
+    spec_kernel<D, TIO, CONV, COMMIT><<<(unsigned)grid, DecodeShape<D>::NT, SM::BYTES, st>>>(P);
     return last_launch_status();
+}
+
+// verify (commit false) or verify + commit over one group of sequences; T and Tp: rows of
+// this step's and the previous step's packed token arrays
+template <typename TIO>
+static kda_status launch_spec(int D, SpecParams &P, bool commit, int64_t T, int64_t Tp, cudaStream_t st) {
+    if (D != 32 && D != 64 && D != 128) return KDA_ERR_UNSUPPORTED;
+    constexpr bool bf = sizeof(TIO) == 2;
+    constexpr int TB = SpecShape<TIO>::TB;
+    const DecodeParams &p = P.p;
+    const CommitParams &c = P.c;
+    const int H = p.H;
+    if (!encode_rows(&P.mq, p.q, bf, D, H, T, TB) || !encode_rows(&P.mk, p.k, bf, D, H, T, TB) ||
+        !encode_rows(&P.mv, p.v, bf, D, H, T, TB) || !encode_rows(&P.mg, p.g, false, D, H, T, TB) ||
+        !encode_rows(&P.pq, commit ? c.q : nullptr, bf, D, H, Tp, TB) ||
+        !encode_rows(&P.pk, commit ? c.k : nullptr, bf, D, H, Tp, TB) ||
+        !encode_rows(&P.pv, commit ? c.v : nullptr, bf, D, H, Tp, TB) ||
+        !encode_rows(&P.pg, commit ? c.g : nullptr, false, D, H, Tp, TB))
+        return fail_text("cuTensorMapEncodeTiled failed for the token rows");
+    const bool conv = p.taps > 0;
+#define KDA_SPEC(d)                                                                                  \
+    if (commit) return conv ? launch_spec_t<d, TIO, true, true>(P, st) : launch_spec_t<d, TIO, false, true>(P, st); \
+    return conv ? launch_spec_t<d, TIO, true, false>(P, st) : launch_spec_t<d, TIO, false, false>(P, st);
+    switch (D) {
+    case 32: KDA_SPEC(32)
+    case 64: KDA_SPEC(64)
+    default: KDA_SPEC(128)
+    }
+#undef KDA_SPEC
 }
 
 // --------------------------------------------------------------- prefill ----
@@ -162,7 +211,6 @@ static std::atomic<int> g_prefill_path{0};
 // Scratch of kda_prefill_noalloc: a fixed module-level device array, so that call needs
 // neither an allocation nor a caller buffer. Its size bounds the workspaces it can serve.
 constexpr size_t kNoallocScratchBytes = size_t(64) << 20;
-constexpr int kMaxDevices = 64;     // devices whose scratch address is cached
 __device__ __align__(1024) uint8_t g_noalloc_scratch[kNoallocScratchBytes];
 
 }  // namespace kda
@@ -378,8 +426,8 @@ static kda_status decode_impl(const kda_dims *dims, const kda_conv *conv, int32_
     set_conv(p, conv, conv_pool, nullptr);
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     return dims->io == KDA_IO_BF16
-               ? dispatch_decode<__nv_bfloat16>(dims->dk, p, n_seq * dims->H, cs, false)
-               : dispatch_decode<float>(dims->dk, p, n_seq * dims->H, cs, false);
+               ? dispatch_decode<__nv_bfloat16>(dims->dk, p, n_seq * dims->H, cs)
+               : dispatch_decode<float>(dims->dk, p, n_seq * dims->H, cs);
 }
 
 kda_status kda_decode(const kda_dims *dims, int32_t n_seq, const void *q, const void *k,
@@ -419,19 +467,21 @@ static kda_status verify_impl(const kda_dims *dims, const kda_conv *conv, int32_
     for (const void *ptr : ptrs)
         if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-    static thread_local DecodeParams p;
+    static thread_local SpecParams P;
     for (int g0 = 0; g0 < n_seq; g0 += kMaxSeqsPerLaunch) {
         const int ng = std::min(kMaxSeqsPerLaunch, n_seq - g0);
-        std::memset(&p, 0, sizeof(p));
+        std::memset(&P, 0, sizeof(P));
+        DecodeParams &p = P.p;
         p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.slots = slots + g0;
         p.pool = const_cast<float *>(pool); p.token_states = token_states; p.o = o;
         p.n_seq = ng; p.H = dims->H; p.n_slots = n_slots; p.scale = eff_scale(dims);
         p.tok_base = cu_draft[g0];
         set_conv(p, conv, const_cast<float *>(conv_pool), conv_tok);
         for (int i = 0; i <= ng; ++i) p.tok0[i] = cu_draft[g0 + i] - cu_draft[g0];
-        st = dims->io == KDA_IO_BF16
-                 ? dispatch_decode<__nv_bfloat16>(dims->dk, p, ng * dims->H, cs, true)
-                 : dispatch_decode<float>(dims->dk, p, ng * dims->H, cs, true);
+        if ((int64_t)ng * dims->H > 0x7fffffffLL) return KDA_ERR_INVALID;
+        P.n_items = ng * dims->H;
+        st = dims->io == KDA_IO_BF16 ? launch_spec<__nv_bfloat16>(dims->dk, P, false, T, 0, cs)
+                                     : launch_spec<float>(dims->dk, P, false, T, 0, cs);
         if (st != KDA_OK) return st;
     }
     return KDA_OK;
@@ -486,7 +536,7 @@ static kda_status verify_commit_impl(
     for (const void *ptr : ptrs)
         if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-    static thread_local VerifyCommitParams P;
+    static thread_local SpecParams P;
     for (int g0 = 0; g0 < n_seq; g0 += kMaxSeqsPerLaunch) {
         const int ng = std::min(kMaxSeqsPerLaunch, n_seq - g0);
         std::memset(&P, 0, sizeof(P));
@@ -508,8 +558,10 @@ static kda_status verify_commit_impl(
         c.snapshots = snapshots; c.n_snap_rows = n_snap_rows; c.snap_interval = snap_interval;
         c.tok_base = cu_prev[g0];
         for (int i = 0; i <= ng; ++i) c.tok0[i] = cu_prev[g0 + i] - cu_prev[g0];
-        st = dims->io == KDA_IO_BF16 ? dispatch_verify_commit<__nv_bfloat16>(dims->dk, P, ng * dims->H, cs)
-                                     : dispatch_verify_commit<float>(dims->dk, P, ng * dims->H, cs);
+        if ((int64_t)ng * dims->H > 0x7fffffffLL) return KDA_ERR_INVALID;
+        P.n_items = ng * dims->H;
+        st = dims->io == KDA_IO_BF16 ? launch_spec<__nv_bfloat16>(dims->dk, P, true, T, Tp, cs)
+                                     : launch_spec<float>(dims->dk, P, true, T, Tp, cs);
         if (st != KDA_OK) return st;
     }
     return KDA_OK;

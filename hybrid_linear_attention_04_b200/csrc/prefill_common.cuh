@@ -80,7 +80,9 @@ __device__ __forceinline__ int fast_index(const FastChannels &f, int lane, int e
 // Add the pairwise part of the channels on the second reference to the A tile in TMEM
 // (rows 0-63 A_qk with q, rows 64-127 A_kk with k; columns i <= r, resp. i < r, of 64):
 // the calling warp's 32 lanes = rows 32 (warp % 4) + lane. fq, fk, fb: [kMaxFast][64] raw
-// q, raw k and b (log2 units) of those channels, zero on rows past the chunk's length.
+// q, raw k and b (log2 units) of those channels; past the chunk's length q and k are zero
+// and b stays at its last live value, so that every exponent taken here is <= 0 (a zero b
+// there would overflow 2^(b_r - b_i) and put 0 * inf into the rows past the length).
 template <int kMaxFast>
 __device__ __forceinline__ void fast_correct(uint32_t taddr_row, int r, int nf, const float *fq,
                                              const float *fk, const float *fb) {

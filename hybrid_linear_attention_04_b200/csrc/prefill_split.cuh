@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(256, 2) prefill_prep_kernel(const __grid_const
                         const bool live = r < n;
                         reinterpret_cast<float *>(sm + P_FQ)[f * 64 + r] = live ? qr[e] : 0.f;
                         reinterpret_cast<float *>(sm + P_FK)[f * 64 + r] = live ? kr[e] : 0.f;
-                        reinterpret_cast<float *>(sm + P_FB)[f * 64 + r] = live ? b[i][e] : 0.f;
+                        reinterpret_cast<float *>(sm + P_FB)[f * 64 + r] = b[i][e];   // b_(n-1) past n
                     }
                 }
             }
@@ -752,17 +752,50 @@ __global__ void __launch_bounds__(256, 1) prefill_chain_kernel(const __grid_cons
                 *reinterpret_cast<uint4 *>(sm + C_W + tc::sw128(r_w, 4 * wh + q4)) = bf16x8(w, 1.f);
             }
             tc::fence_async_smem();
-        } else if (ci > 0) {
-            // O of chunk ci - 1: its MMAs were committed before this chunk's barrier below, so
-            // the phase awaited is bar_o's latest
-            ok = tc::bar_wait(bar_o, (uint32_t)((ci - 1) & 1));
-            tc::fence_after_sync();
-            tc::tmem_ld32(tbase + tlane + C_COL_R1 + 64 * ((ci - 1) & 1) + 32 * wh, ov);
-            tc::tmem_ld_wait();
-        }
-        if (stores_pending) {                 // staging tiles may be written after the barrier
-            tc::bulk_wait_read_all();
-            stores_pending = false;
+        } else {
+            // O warps, while round 1 runs: the outputs of chunk ci - 1 (its MMAs were committed
+            // before the previous chunk's end barrier, so the phase awaited is bar_o's latest)
+            // and half 0 of a pending snapshot leave through the staging tiles now, off the
+            // recurrence's critical path
+            const int pn = min(C, sq.len - (ci - 1) * C);
+            const int r = 32 * wq + lane;
+            const bool tiled = ci > 0 && pn == C;
+            const bool snap = snap_pend >= 0 && snap_half == 0;
+            if (ci > 0) {
+                ok = tc::bar_wait(bar_o, (uint32_t)((ci - 1) & 1));
+                tc::fence_after_sync();
+                tc::tmem_ld32(tbase + tlane + C_COL_R1 + 64 * ((ci - 1) & 1) + 32 * wh, ov);
+                tc::tmem_ld_wait();
+            }
+            if (ci > 0 && !tiled && r < pn) {
+                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) +
+                                                       ((int64_t)(sq.tok0 + (ci - 1) * C + r) * H + h) * D + j0 + 32 * wh);
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) dst[q4] = bf16x8(ov + 8 * q4, p.scale);
+            }
+            // thread 32's stores of the previous chunk have read the tiles (issued a chunk ago:
+            // no wait in practice), before anyone writes them again
+            if (stores_pending) {
+                tc::bulk_wait_read_all();
+                stores_pending = false;
+            }
+            if (tiled || snap) {
+                tc::named_sync(1, 128);
+                if (tiled) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        *reinterpret_cast<uint4 *>(sm + C_O + tc::sw128(r, 4 * wh + q4)) = bf16x8(ov + 8 * q4, p.scale);
+                }
+                if (snap) stage_snapshot(S);
+                tc::fence_async_smem();
+                tc::named_sync(1, 128);
+                if (tid == 32) {
+                    if (tiled) tc::tma_store3(&CP.tm_o, sm + C_O, j0, h, sq.tok0 + (ci - 1) * C);
+                    if (snap) store_snapshot_half(snap_pend, 0);
+                    tc::bulk_commit();
+                    stores_pending = true;
+                }
+            }
         }
         tc::fence_before_sync();
         __syncthreads();
@@ -781,36 +814,8 @@ __global__ void __launch_bounds__(256, 1) prefill_chain_kernel(const __grid_cons
             for (int k = 0; k < 4; ++k) tc::mma_bf16(tbase + col_r1, dAQK + 2 * k, dW + 128 * k, id_o, 1);
             tc::mma_commit(bar_o);
         }
-        // ---- while this chunk's MMAs run: outputs of chunk ci - 1 and half of a pending
-        // snapshot go through the staging tiles
-        if (!wwarp) {
-            const int pn = min(C, sq.len - (ci - 1) * C);
-            const int r = 32 * wq + lane;
-            const bool tiled = ci > 0 && pn == C;
-            if (ci > 0 && !tiled && r < pn) {
-                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) +
-                                                       ((int64_t)(sq.tok0 + (ci - 1) * C + r) * H + h) * D + j0 + 32 * wh);
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) dst[q4] = bf16x8(ov + 8 * q4, p.scale);
-            }
-            if (tiled) {
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    *reinterpret_cast<uint4 *>(sm + C_O + tc::sw128(r, 4 * wh + q4)) = bf16x8(ov + 8 * q4, p.scale);
-            }
-            const bool snap = snap_pend >= 0 && snap_half == 0;
-            if (snap) stage_snapshot(S);
-            if (tiled || snap) {
-                tc::fence_async_smem();
-                tc::named_sync(1, 128);
-                if (tid == 32) {
-                    if (tiled) tc::tma_store3(&CP.tm_o, sm + C_O, j0, h, sq.tok0 + (ci - 1) * C);
-                    if (snap) store_snapshot_half(snap_pend, 0);
-                    tc::bulk_commit();
-                    stores_pending = true;
-                }
-            }
-        } else if (snap_pend >= 0 && snap_half == 1) {
+        // ---- while this chunk's MMAs run: the W warps send half 1 of a pending snapshot
+        if (wwarp && snap_pend >= 0 && snap_half == 1) {
             stage_snapshot(Ss);
             tc::fence_async_smem();
             tc::named_sync(2, 128);
@@ -855,6 +860,12 @@ __global__ void __launch_bounds__(256, 1) prefill_chain_kernel(const __grid_cons
                 ++snap_row;
             }
             ok = ok && okd;
+        }
+        // thread 64's half-1 snapshot stores have read the tile before the end barrier: the O
+        // warps may stage the next snapshot's half 0 into it early in the next chunk
+        if (wwarp && stores_pending) {
+            tc::bulk_wait_read_all();
+            stores_pending = false;
         }
         tc::fence_before_sync();
         ok = __syncthreads_and(ok);

@@ -296,7 +296,7 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
                         const bool live = r < n;
                         reinterpret_cast<float *>(sm + FQ)[f * 64 + r] = live ? qr[e] : 0.f;
                         reinterpret_cast<float *>(sm + FK)[f * 64 + r] = live ? kr[e] : 0.f;
-                        reinterpret_cast<float *>(sm + FB)[f * 64 + r] = live ? b[i][e] : 0.f;
+                        reinterpret_cast<float *>(sm + FB)[f * 64 + r] = b[i][e];   // b_(n-1) past n
                     }
                 }
             }
