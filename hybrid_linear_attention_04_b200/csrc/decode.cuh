@@ -463,7 +463,8 @@ template <int D, typename TIO> struct SpecSmem {
     static constexpr uint32_t CW_K = D * (kMaxTaps - 1) * 4, CW_WQ = 2 * CW_K, CW_WK = CW_WQ + D * kMaxTaps * 4;
     static constexpr uint32_t RAW0 = CW + CW_WK + D * kMaxTaps * 4;    // raw batches: q, k, v, g rows
     static constexpr uint32_t RAW = TB * (3 * ROW + D * 4);
-    static constexpr uint32_t TV = RAW0 + 2 * RAW;                     // token vectors [TB]
+    static constexpr uint32_t BETA = RAW0 + 2 * RAW;                   // beta of the raw batches [2][TB]
+    static constexpr uint32_t TV = BETA + 128;                         // token vectors [TB]
     static constexpr uint32_t META = TV + TB * sizeof(TokVec<D>);      // SeqMeta [kSpecSeqs]
     static constexpr uint32_t BARS = META + kSpecSeqs * sizeof(SeqMeta);   // state, raw 0, raw 1
     static constexpr uint32_t PROD = BARS + 32;                        // producer cursors
@@ -504,11 +505,11 @@ struct ProdCursor {
     int ks, ns_issued;         // state cursor: next local item to consider; states issued
 };
 
-// warp 0: issue the next batch of token rows (lane 0 the copies, lanes c < nb the
-// loads of their beta, kept in breg until the batch is converted)
+// warp 0: issue the next batch of token rows (lane 0 the tiles, lanes c < nb a copy of
+// their token's beta; all complete on the buffer's mbarrier)
 template <int D, typename TIO, bool CONV, bool COMMIT>
 __device__ __forceinline__ void produce_batch(const SpecParams &P, uint8_t *sm, const SeqMeta *meta, int s0,
-                                              int i0, int n_local, float &b0, float &b1) {
+                                              int i0, int n_local) {
     using SM = SpecSmem<D, TIO>;
     constexpr int TB = SM::TB;
     ProdCursor *cur = reinterpret_cast<ProdCursor *>(sm + SM::PROD);
@@ -525,9 +526,15 @@ __device__ __forceinline__ void produce_batch(const SpecParams &P, uint8_t *sm, 
     const int nb = min(TB, (replay ? I.na : I.n_tok) - j0);
     const int64_t row0 = (replay ? I.prev_first : I.tok_first) + j0;
     const int slot = cur->nb_issued & 1;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + SM::BARS) + 1 + slot;
+    if (lane < nb) {
+        // before the tiles' arrival below, so that the phase cannot complete without them
+        const float *beta = replay ? P.c.beta : P.p.beta;
+        tc::cp_async4(reinterpret_cast<float *>(sm + SM::BETA) + slot * TB + lane, beta + (row0 + lane) * P.p.H + I.h);
+        tc::cp_async_arrive(bar);
+    }
     __syncwarp();
     if (lane == 0) {
-        uint64_t *bar = reinterpret_cast<uint64_t *>(sm + SM::BARS) + 1 + slot;
         uint8_t *raw = sm + SM::RAW0 + slot * SM::RAW;
         const bool with_q = !replay || CONV;
         tc::bar_expect_tx(bar, (uint32_t)TB * ((with_q ? 3u : 2u) * SM::ROW + D * 4u));
@@ -539,12 +546,6 @@ __device__ __forceinline__ void produce_batch(const SpecParams &P, uint8_t *sm, 
         cur->kb = kb;
         cur->bb = bb + 1;
         cur->nb_issued += 1;
-    }
-    if (lane < nb) {
-        const float *beta = replay ? P.c.beta : P.p.beta;
-        const float b = beta[(row0 + lane) * P.p.H + I.h];
-        if (slot) b1 = b;
-        else b0 = b;
     }
     __syncwarp();
 }
@@ -580,10 +581,11 @@ __device__ __forceinline__ void produce_state(const SpecParams &P, uint8_t *sm, 
 
 // Raw rows of a batch -> token vectors: threads t < D channel t of q and k (the
 // front-end's conv window in token order with CONV), threads t >= D channel t - D of v
-// and g, warp-0 lanes j < nb the beta they loaded.
+// and g, threads t < nb token t's beta.
 template <int D, typename TIO, bool CONV>
-__device__ __forceinline__ void convert_batch(TokVec<D> *tv, const uint8_t *raw, int nb, bool read_q, bool with_q,
-                                              float b, ConvWin &w, const DecodeParams &p, int h, const ConvOut &co) {
+__device__ __forceinline__ void convert_batch(TokVec<D> *tv, const uint8_t *raw, const float *beta, int nb,
+                                              bool read_q, bool with_q, ConvWin &w, const DecodeParams &p, int h,
+                                              const ConvOut &co) {
     constexpr int TB = SpecShape<TIO>::TB;
     constexpr uint32_t ROW = D * sizeof(TIO);
     const int t = threadIdx.x;
@@ -598,7 +600,7 @@ __device__ __forceinline__ void convert_batch(TokVec<D> *tv, const uint8_t *raw,
                 if (j == co.snap_j) conv_store(w, p, co.snap, co.snap_row, h, D, t);
             }
         }
-        if (t < nb) tv[t].beta = b;
+        if (t < nb) tv[t].beta = beta[t];
     } else {
         const int c = t - D;
         const TIO *rv = reinterpret_cast<const TIO *>(raw + 2 * TB * ROW);
@@ -665,11 +667,10 @@ spec_kernel(const __grid_constant__ SpecParams P) {
         cur->kb = 0; cur->bb = 0; cur->nb_issued = 0; cur->ks = 0; cur->ns_issued = 0;
     }
     __syncthreads();
-    float b0 = 0.f, b1 = 0.f;   // warp 0: beta of the batches in the two raw buffers
     if (t == 0) produce_state<D, TIO, CONV, COMMIT>(P, sm, meta, s0, i0, n_local);
     if (warp == 0) {
-        produce_batch<D, TIO, CONV, COMMIT>(P, sm, meta, s0, i0, n_local, b0, b1);
-        produce_batch<D, TIO, CONV, COMMIT>(P, sm, meta, s0, i0, n_local, b0, b1);
+        produce_batch<D, TIO, CONV, COMMIT>(P, sm, meta, s0, i0, n_local);
+        produce_batch<D, TIO, CONV, COMMIT>(P, sm, meta, s0, i0, n_local);
     }
 
     bool ok = true;
@@ -712,12 +713,13 @@ spec_kernel(const __grid_constant__ SpecParams P) {
             const ConvOut co = COMMIT ? ConvOut{nullptr, 0, c.conv_snapshots, I.srow, js}
                                       : ConvOut{p.conv_tok, I.tok_first + j0, nullptr, 0, -1};
             const bool bok = tc::bar_wait(&bar_t[g & 1], (uint32_t)((g >> 1) & 1));
-            convert_batch<D, TIO, CONV>(tv, sm + SM::RAW0 + (g & 1) * SM::RAW, nb, CONV || !replay, !replay,
-                                        (g & 1) ? b1 : b0, w, p, I.h, co);
+            convert_batch<D, TIO, CONV>(tv, sm + SM::RAW0 + (g & 1) * SM::RAW,
+                                        reinterpret_cast<const float *>(sm + SM::BETA) + (g & 1) * TB, nb,
+                                        CONV || !replay, !replay, w, p, I.h, co);
             ok = __syncthreads_and(ok && bok);   // vectors staged, raw buffer read
             if (!ok) break;
             ++g;
-            if (warp == 0) produce_batch<D, TIO, CONV, COMMIT>(P, sm, meta, s0, i0, n_local, b0, b1);
+            if (warp == 0) produce_batch<D, TIO, CONV, COMMIT>(P, sm, meta, s0, i0, n_local);
             for (int j = warp; j < nb; j += Sh::NW) token_finish<D>(tv[j], CONV, !replay);
             __syncthreads();
             const int64_t hh = I.h;

@@ -225,6 +225,16 @@ __device__ __forceinline__ void bulk_wait_read_all() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
+// ---- element copies global -> shared (cp.async), completing on an mbarrier --------
+__device__ __forceinline__ void cp_async4(void *smem_dst, const void *gsrc) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+// the barrier's current phase also waits for this thread's cp.async copies issued so far
+// (its pending count is raised now and lowered when they land)
+__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // ---- small warp-level helpers ----------------------------------------------------
 // barrier among `nthreads` threads (whole warps) using hardware barrier `id` (1..15)
 __device__ __forceinline__ void named_sync(int id, int nthreads) {
