@@ -422,8 +422,8 @@ def run_ours(args):
         dom = max(comps, key=lambda c: comp[c]["ms"])
         pk = ["prefill_prep_kernel", "prefill_chain_kernel"] if args.prefill_path == "split" \
             else ["prefill_tc_kernel"]
-        knames = {"prefill": pk, "decode": ["decode_kernel"], "verify": ["verify_kernel"],
-                  "commit": ["snapshot_kernel"], "verify_commit": ["verify_commit_kernel"]}[dom]
+        knames = {"prefill": pk, "decode": ["decode_kernel"], "verify": ["spec_kernel<verify>"],
+                  "commit": ["snapshot_kernel"], "verify_commit": ["spec_kernel<verify+commit>"]}[dom]
         kname = "+".join(knames)
         tr_units = {"prefill": (wl.T * H, wl.T * H), "decode": (wl.n_seq * H, wl.n_seq * H),
                     "verify": (wl.n_seq * H, wl.n_tok * H), "commit": (wl.n_commit, wl.n_commit),

@@ -431,8 +431,12 @@ struct CommitParams {
     int32_t tok0[kMaxSeqsPerLaunch + 1];  // previous batch offsets (relative)
 };
 
-// A persistent grid: CTA b owns the contiguous items [b per_cta, (b + 1) per_cta) of the
-// (sequence, head) list, so that its items share few sequences. Warp 0 is the producer:
+// A persistent grid of G CTAs over the (sequence, head) items, with the sequences in the
+// host's order of decreasing token count: CTA b takes ranks b, b + G, b + 2 G, ... of that
+// list, every second band of G ranks reversed (a snake), so that each CTA gets one item
+// of every band and the CTAs' token totals come out nearly equal (the heads of one
+// sequence share its token counts). The records of a CTA's items (slot, accepted count,
+// snapshot) are read once at its start. Warp 0 is the producer:
 // one bulk copy brings the next item's state (and conv window and weights) into shared
 // memory while the current item runs from registers, and the item's token rows come in
 // batches of TB by 3-D TMA tiles (channels x 1 head x TB rows) into two buffers, two
@@ -442,34 +446,42 @@ struct SpecParams {
     CUtensorMap pq, pk, pv, pg;       // the previous step's (replay; pq with the front-end only)
     DecodeParams p;                   // verify: token_states, conv_tok; pool read-only
     CommitParams c;                   // verify + commit only
-    int32_t n_items, per_cta;
+    int32_t n_items;
+    int32_t order[kMaxSeqsPerLaunch];   // sequences by decreasing token count
 };
 
 template <typename TIO> struct SpecShape {
     static constexpr int TB = sizeof(TIO) == 2 ? 8 : 4;   // tokens per batch
 };
-constexpr int kSpecSeqs = 16;         // sequence records per CTA (the host keeps ranges within it)
-
-struct SeqMeta {
-    int32_t slot, na, n_prev, n_tok, cnew, ok;
-    int64_t srow, jsnap;  // snapshot row, and the committed-token index after which it falls
+// item records per CTA (the host launches enough CTAs)
+template <bool CONV> struct SpecItems {
+    static constexpr int N = CONV ? 96 : 128;
 };
 
-template <int D, typename TIO> struct SpecSmem {
+struct ItemMeta {
+    int32_t s, slot;      // slot < 0: the item is out of range
+    int32_t na;           // accepted tokens to replay; bit 30: commit_new
+    int32_t jsnap;        // the committed-token index after which the snapshot falls, or -1
+    int64_t srow;         // snapshot row, or -1
+};
+constexpr int32_t kCnewBit = 1 << 30;
+
+template <int D, typename TIO, bool CONV> struct SpecSmem {
     static constexpr int TB = SpecShape<TIO>::TB;
     static constexpr uint32_t ROW = D * sizeof(TIO);
     static constexpr uint32_t ST = 0;                                  // state [D][D] fp32
     static constexpr uint32_t CW = ST + D * D * 4;                     // conv: q, k windows, q, k weights
     static constexpr uint32_t CW_K = D * (kMaxTaps - 1) * 4, CW_WQ = 2 * CW_K, CW_WK = CW_WQ + D * kMaxTaps * 4;
-    static constexpr uint32_t RAW0 = CW + CW_WK + D * kMaxTaps * 4;    // raw batches: q, k, v, g rows
+    static constexpr uint32_t RAW0 = CW + (CONV ? CW_WK + D * kMaxTaps * 4 : 0);   // raw batches: q, k, v, g
     static constexpr uint32_t RAW = TB * (3 * ROW + D * 4);
     static constexpr uint32_t BETA = RAW0 + 2 * RAW;                   // beta of the raw batches [2][TB]
     static constexpr uint32_t TV = BETA + 128;                         // token vectors [TB]
-    static constexpr uint32_t META = TV + TB * sizeof(TokVec<D>);      // SeqMeta [kSpecSeqs]
-    static constexpr uint32_t BARS = META + kSpecSeqs * sizeof(SeqMeta);   // state, raw 0, raw 1
+    static constexpr uint32_t META = TV + TB * sizeof(TokVec<D>);      // ItemMeta [SpecItems::N]
+    static constexpr uint32_t BARS = META + SpecItems<CONV>::N * sizeof(ItemMeta);   // state, raw 0, raw 1
     static constexpr uint32_t PROD = BARS + 32;                        // producer cursors
     static constexpr uint32_t BYTES = PROD + 32 + 128;                 // + alignment slack
     static_assert(RAW0 % 128 == 0 && RAW % 128 == 0 && (TB * ROW) % 128 == 0 && TV % 16 == 0, "alignment");
+    static_assert(D != 128 || sizeof(TIO) != 2 || 2 * (BYTES + 1024) <= 233472, "two CTAs per SM");
 };
 
 struct ItemInfo {
@@ -479,18 +491,26 @@ struct ItemInfo {
     int64_t srow, jsnap, prev_first, tok_first;
 };
 
+// rank of the CTA's k-th item in the sorted item list (the snake over bands of G)
+__device__ __forceinline__ int item_rank(int k, int n_items) {
+    const int G = gridDim.x, base = k * G, pos = blockIdx.x;
+    const int width = min(G, n_items - base);
+    return base + ((k & 1) ? width - 1 - pos : pos);
+}
+
+// the CTA's k-th item
 template <int D, typename TIO, bool COMMIT>
-__device__ __forceinline__ ItemInfo item_info(const SpecParams &P, const SeqMeta *meta, int s0, int it) {
+__device__ __forceinline__ ItemInfo item_info(const SpecParams &P, const ItemMeta *meta, int k) {
     constexpr int TB = SpecShape<TIO>::TB;
     ItemInfo I;
-    I.s = it / P.p.H;
-    I.h = it - I.s * P.p.H;
-    const SeqMeta &m = meta[I.s - s0];
+    const ItemMeta m = meta[k];
+    I.s = m.s;
+    I.h = item_rank(k, P.n_items) % P.p.H;
     I.slot = m.slot;
-    I.valid = m.ok != 0;
-    I.n_tok = m.n_tok;
-    I.na = COMMIT ? m.na : 0;
-    I.cnew = COMMIT && m.cnew != 0;
+    I.valid = m.slot >= 0;
+    I.n_tok = P.p.tok0[I.s + 1] - P.p.tok0[I.s];
+    I.na = COMMIT ? (m.na & ~kCnewBit) : 0;
+    I.cnew = COMMIT && (m.na & kCnewBit) != 0;
     I.srow = m.srow;
     I.jsnap = m.jsnap;
     I.nb0 = (I.na + TB - 1) / TB;
@@ -508,9 +528,9 @@ struct ProdCursor {
 // warp 0: issue the next batch of token rows (lane 0 the tiles, lanes c < nb a copy of
 // their token's beta; all complete on the buffer's mbarrier)
 template <int D, typename TIO, bool CONV, bool COMMIT>
-__device__ __forceinline__ void produce_batch(const SpecParams &P, uint8_t *sm, const SeqMeta *meta, int s0,
-                                              int i0, int n_local) {
-    using SM = SpecSmem<D, TIO>;
+__device__ __forceinline__ void produce_batch(const SpecParams &P, uint8_t *sm, const ItemMeta *meta,
+                                              int n_local) {
+    using SM = SpecSmem<D, TIO, CONV>;
     constexpr int TB = SM::TB;
     ProdCursor *cur = reinterpret_cast<ProdCursor *>(sm + SM::PROD);
     const int lane = threadIdx.x & 31;
@@ -518,7 +538,7 @@ __device__ __forceinline__ void produce_batch(const SpecParams &P, uint8_t *sm, 
     ItemInfo I;
     for (;; ++kb, bb = 0) {
         if (kb >= n_local) return;
-        I = item_info<D, TIO, COMMIT>(P, meta, s0, i0 + kb);
+        I = item_info<D, TIO, COMMIT>(P, meta, kb);
         if (I.valid && bb < I.nbat) break;
     }
     const bool replay = bb < I.nb0;
@@ -552,12 +572,12 @@ __device__ __forceinline__ void produce_batch(const SpecParams &P, uint8_t *sm, 
 
 // thread 0: issue the state (and conv window and weights) of the next item that needs it
 template <int D, typename TIO, bool CONV, bool COMMIT>
-__device__ __forceinline__ void produce_state(const SpecParams &P, uint8_t *sm, const SeqMeta *meta, int s0,
-                                              int i0, int n_local) {
-    using SM = SpecSmem<D, TIO>;
+__device__ __forceinline__ void produce_state(const SpecParams &P, uint8_t *sm, const ItemMeta *meta,
+                                              int n_local) {
+    using SM = SpecSmem<D, TIO, CONV>;
     ProdCursor *cur = reinterpret_cast<ProdCursor *>(sm + SM::PROD);
     for (int ks = cur->ks; ks < n_local; ++ks) {
-        const ItemInfo I = item_info<D, TIO, COMMIT>(P, meta, s0, i0 + ks);
+        const ItemInfo I = item_info<D, TIO, COMMIT>(P, meta, ks);
         if (!I.valid || I.nbat == 0) continue;
         const DecodeParams &p = P.p;
         uint64_t *bar = reinterpret_cast<uint64_t *>(sm + SM::BARS);
@@ -617,7 +637,7 @@ __device__ __forceinline__ void convert_batch(TokVec<D> *tv, const uint8_t *raw,
 template <int D, typename TIO, bool CONV, bool COMMIT>
 __global__ void __launch_bounds__(DecodeShape<D>::NT, 2)
 spec_kernel(const __grid_constant__ SpecParams P) {
-    using SM = SpecSmem<D, TIO>;
+    using SM = SpecSmem<D, TIO, CONV>;
     using Sh = DecodeShape<D>;
     constexpr int TB = SM::TB;
     extern __shared__ uint8_t smem_raw[];
@@ -625,39 +645,42 @@ spec_kernel(const __grid_constant__ SpecParams P) {
     const DecodeParams &p = P.p;
     const CommitParams &c = P.c;
     TokVec<D> *tv = reinterpret_cast<TokVec<D> *>(sm + SM::TV);
-    SeqMeta *meta = reinterpret_cast<SeqMeta *>(sm + SM::META);
+    ItemMeta *meta = reinterpret_cast<ItemMeta *>(sm + SM::META);
     uint64_t *bar_s = reinterpret_cast<uint64_t *>(sm + SM::BARS), *bar_t = bar_s + 1;
     ProdCursor *cur = reinterpret_cast<ProdCursor *>(sm + SM::PROD);
     const int t = threadIdx.x, warp = t >> 5;
 
-    const int i0 = blockIdx.x * P.per_cta;
-    const int n_local = max(0, min(P.n_items, i0 + P.per_cta) - i0);
+    const int n_local = (int)blockIdx.x < P.n_items ? (P.n_items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     if (n_local == 0) return;
-    const int s0 = i0 / p.H, n_meta = (i0 + n_local - 1) / p.H - s0 + 1;
-    if (n_meta > kSpecSeqs) {                   // the host never launches this
+    if (n_local > SpecItems<CONV>::N) {         // the host never launches this
         if (t == 0) record_status(KDA_ERR_INVALID);
         return;
     }
-    // per-sequence records of this CTA's range
-    if (t < n_meta) {
-        const int s = s0 + t;
-        SeqMeta m;
+    // the records of this CTA's items, read in parallel once
+    for (int k = t; k < n_local; k += Sh::NT) {
+        const int r = item_rank(k, P.n_items);
+        const int s = P.order[r / p.H];
+        ItemMeta m;
+        m.s = s;
         m.slot = p.slots[s];
-        m.n_tok = p.tok0[s + 1] - p.tok0[s];
-        m.ok = m.slot >= 0 && m.slot < p.n_slots;
-        m.na = 0; m.n_prev = 0; m.cnew = 0; m.srow = -1; m.jsnap = -1;
+        m.na = 0;
+        m.jsnap = -1;
+        m.srow = -1;
+        bool ok = m.slot >= 0 && m.slot < p.n_slots;
         if (COMMIT) {
-            m.na = c.n_accept[s];
-            m.n_prev = c.tok0[s + 1] - c.tok0[s];
-            m.cnew = c.commit_new != nullptr && c.commit_new[s] != 0 && m.n_tok > 0;
+            const int32_t na = c.n_accept[s];
+            const int n_tok = p.tok0[s + 1] - p.tok0[s];
+            const bool cnew = c.commit_new != nullptr && c.commit_new[s] != 0 && n_tok > 0;
             if (c.snap_interval > 0 && c.snap_row != nullptr && c.snap_row[s] >= 0) {
                 m.srow = c.snap_row[s];
                 const int64_t p0 = c.pos[s];
-                m.jsnap = (p0 / c.snap_interval + 1) * c.snap_interval - p0 - 1;
+                m.jsnap = (int32_t)((p0 / c.snap_interval + 1) * c.snap_interval - p0 - 1);
             }
-            m.ok = m.ok && m.na >= 0 && m.na <= m.n_prev && m.srow < c.n_snap_rows;
+            ok = ok && na >= 0 && na <= c.tok0[s + 1] - c.tok0[s] && na < kCnewBit && m.srow < c.n_snap_rows;
+            m.na = na | (cnew ? kCnewBit : 0);
         }
-        meta[t] = m;
+        if (!ok) m.slot = -1;
+        meta[k] = m;
     }
     if (t == 0) {
         tc::bar_init(bar_s, 1);
@@ -667,10 +690,10 @@ spec_kernel(const __grid_constant__ SpecParams P) {
         cur->kb = 0; cur->bb = 0; cur->nb_issued = 0; cur->ks = 0; cur->ns_issued = 0;
     }
     __syncthreads();
-    if (t == 0) produce_state<D, TIO, CONV, COMMIT>(P, sm, meta, s0, i0, n_local);
+    if (t == 0) produce_state<D, TIO, CONV, COMMIT>(P, sm, meta, n_local);
     if (warp == 0) {
-        produce_batch<D, TIO, CONV, COMMIT>(P, sm, meta, s0, i0, n_local);
-        produce_batch<D, TIO, CONV, COMMIT>(P, sm, meta, s0, i0, n_local);
+        produce_batch<D, TIO, CONV, COMMIT>(P, sm, meta, n_local);
+        produce_batch<D, TIO, CONV, COMMIT>(P, sm, meta, n_local);
     }
 
     bool ok = true;
@@ -678,7 +701,7 @@ spec_kernel(const __grid_constant__ SpecParams P) {
     for (int kl = 0; kl < n_local && ok; ++kl) {
         int nbat;
         {
-            const ItemInfo I = item_info<D, TIO, COMMIT>(P, meta, s0, i0 + kl);
+            const ItemInfo I = item_info<D, TIO, COMMIT>(P, meta, kl);
             if (!I.valid) {
                 if (t == 0) record_status(KDA_ERR_RANGE);
                 continue;
@@ -699,11 +722,11 @@ spec_kernel(const __grid_constant__ SpecParams P) {
             win_load(w.k, cw + SM::CW_WK / 4 + t * K, cw + SM::CW_K / 4 + t * (K - 1), K);
         }
         __syncthreads();        // the state buffer is free
-        if (t == 0 && ok) produce_state<D, TIO, CONV, COMMIT>(P, sm, meta, s0, i0, n_local);
+        if (t == 0 && ok) produce_state<D, TIO, CONV, COMMIT>(P, sm, meta, n_local);
         for (int bi = 0; bi < nbat; ++bi) {
             // the item's fields are re-read from shared memory after every barrier rather
             // than held in registers through the steps
-            const ItemInfo I = item_info<D, TIO, COMMIT>(P, meta, s0, i0 + kl);
+            const ItemInfo I = item_info<D, TIO, COMMIT>(P, meta, kl);
             const bool replay = bi < I.nb0;
             const int j0 = (replay ? bi : bi - I.nb0) * TB;
             const int nb = min(TB, (replay ? I.na : I.n_tok) - j0);
@@ -719,7 +742,7 @@ spec_kernel(const __grid_constant__ SpecParams P) {
             ok = __syncthreads_and(ok && bok);   // vectors staged, raw buffer read
             if (!ok) break;
             ++g;
-            if (warp == 0) produce_batch<D, TIO, CONV, COMMIT>(P, sm, meta, s0, i0, n_local);
+            if (warp == 0) produce_batch<D, TIO, CONV, COMMIT>(P, sm, meta, n_local);
             for (int j = warp; j < nb; j += Sh::NW) token_finish<D>(tv[j], CONV, !replay);
             __syncthreads();
             const int64_t hh = I.h;
@@ -748,7 +771,7 @@ spec_kernel(const __grid_constant__ SpecParams P) {
             __syncthreads();                  // the vectors are free for the next batch
         }
         if (ok) {
-            const ItemInfo I = item_info<D, TIO, COMMIT>(P, meta, s0, i0 + kl);
+            const ItemInfo I = item_info<D, TIO, COMMIT>(P, meta, kl);
             if (I.cnew) {
                 store_state<D>(Pr, p.pool + ((int64_t)I.slot * p.H + I.h) * (int64_t)D * D);
                 if (CONV && t < D) conv_store(w, p, p.conv, I.slot, I.h, D, t);

@@ -17,7 +17,7 @@ import torch
 
 import synth
 from hybrid_linear_attention_04_b200 import kda as K
-from kda_cases import TOL_BF16, TOL_FP32, check_outputs, check_states, to_np
+from kda_cases import TOL_BF16, TOL_FP32, check_outputs, check_states, same_outputs, same_states, to_np
 from oracle import native
 
 pytestmark = pytest.mark.gpu
@@ -80,12 +80,18 @@ def test_verify_commit_matches_oracle(cuda_device, d, io, H, n_seq):
     assert torch.equal(got_pool[unused], c["pool"][unused])
 
 
-def test_verify_commit_bit_identical_to_verify_and_snapshot(cuda_device):
+def _exact(d, io):
+    """verify + commit runs the same SIMT step as kda_verify for every d and I/O type"""
+    return True
+
+
+@pytest.mark.parametrize("d,io", [(128, "bf16"), (128, "fp32"), (64, "bf16")])
+def test_verify_commit_equals_verify_and_snapshot(cuda_device, d, io):
     """The fused step equals kda_verify of the previous batch with per-token states,
     kda_snapshot of the accepted token's state into the slot, then kda_verify of this
     batch: committed states and outputs bit for bit."""
-    H, d, n_seq = 16, 128, 64
-    c = _case(801, n_seq, H, d, "bf16", cuda_device)
+    H, n_seq = 16, 64
+    c = _case(801, n_seq, H, d, io, cuda_device)
     pool_a = c["pool"].to(cuda_device)
     pool_b = pool_a.clone()
     # reference path
@@ -104,16 +110,18 @@ def test_verify_commit_bit_identical_to_verify_and_snapshot(cuda_device):
     # fused
     o = _fused(c, pool_b)
     assert K.kda_check_device_status() == 0
-    assert torch.equal(pool_a, pool_b)
-    assert torch.equal(o, o_ref)
+    ex = _exact(d, io)
+    assert same_states(pool_b, pool_a, ex)
+    assert same_outputs(o, o_ref, ex)
 
 
-def test_verify_commit_writes_block_boundary_snapshots(cuda_device):
+@pytest.mark.parametrize("io", ["bf16", "fp32"])
+def test_verify_commit_writes_block_boundary_snapshots(cuda_device, io):
     """Sequences whose committed tokens cross a multiple of snap_interval write the
-    state at that position to their snapshot row (bit-identical to the per-token
-    state of kda_verify); the others leave their row untouched."""
+    state at that position to their snapshot row (bit-identical to the per-token state
+    of kda_verify); the others leave their row untouched."""
     H, d, n_seq, snap = 4, 128, 24, 64
-    c = _case(901, n_seq, H, d, "bf16", cuda_device)
+    c = _case(901, n_seq, H, d, io, cuda_device)
     cp = c["cp"]
     # positions a few tokens before a boundary, so that some accepted prefixes cross it
     pos = [snap * (s + 1) - 1 - (s % 6) for s in range(n_seq)]
@@ -133,7 +141,7 @@ def test_verify_commit_writes_block_boundary_snapshots(cuda_device):
     for s in range(n_seq):
         j = snap * (pos[s] // snap + 1) - pos[s] - 1        # token index that lands on it
         if j < c["acc"][s]:
-            assert torch.equal(sn[s], ts[int(cp[s]) + j]), s
+            assert same_states(sn[s], ts[int(cp[s]) + j], _exact(d, io)), s
             crossed += 1
         else:
             assert torch.isnan(sn[s]).all(), s
@@ -170,15 +178,18 @@ def test_verify_commit_drain_and_range(cuda_device):
         check_states("drained state", got[slot].double().numpy()[None], st[None], TOL_BF16, (2, 3))
 
 
-def test_mixed_step_decode_append_and_verify_in_one_launch(cuda_device):
+@pytest.mark.parametrize("io", ["bf16", "fp32"])
+def test_mixed_step_decode_append_and_verify_in_one_launch(cuda_device, io):
     """One launch serving three kinds of sequences (continuous batching): plain decode
     (one token, committed), a short prefill appended to a live sequence (several tokens,
     committed) and speculative sequences (the previous step's accepted prefix committed,
     this step's drafts only verified). Committed states equal kda_decode / kda_verify's
-    per-token states bit for bit, outputs equal kda_verify's, and a block-boundary
+    per-token states and outputs equal kda_verify's bit for bit, and a block-boundary
     snapshot falling among appended tokens is written."""
     H, d, n_seq, snap = 8, 128, 12, 64
-    c = _case(1201, n_seq, H, d, "bf16", cuda_device)
+    c = _case(1201, n_seq, H, d, io, cuda_device)
+    ex = _exact(d, io)
+    odt = torch.bfloat16 if io == "bf16" else torch.float32
     cp, cd = c["cp"], c["cd"]
     kind = ["decode", "append", "verify"] * 4
     # decode and append sequences commit nothing of the previous batch
@@ -188,12 +199,12 @@ def test_mixed_step_decode_append_and_verify_in_one_launch(cuda_device):
         if kind[s] == "decode":
             lens[s] = 1
     cd = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
-    xc = synth.token_inputs(1202, int(cd[-1]), H, d, d, io="bf16")
+    xc = synth.token_inputs(1202, int(cd[-1]), H, d, d, io=io)
     dc = {k: v.to(cuda_device) for k, v in xc.items()}
     pos = [snap * (s + 1) - 2 for s in range(n_seq)]          # boundaries 2 tokens ahead
     sn = torch.full((n_seq, H, d, d), float("nan"), device=cuda_device)
     pool_b = c["pool"].to(cuda_device)
-    o = torch.empty((int(cd[-1]), H, d), dtype=torch.bfloat16, device=cuda_device)
+    o = torch.empty((int(cd[-1]), H, d), dtype=odt, device=cuda_device)
     cnew = torch.tensor([k != "verify" for k in kind], dtype=torch.uint8, device=cuda_device)
     K.kda_verify_commit(c["dp"], torch.tensor(acc, dtype=torch.int32, device=cuda_device), cp,
                         dc["q"], dc["k"], dc["v"], dc["g"], dc["beta"], cd, c["slots_d"], pool_b, o,
@@ -216,26 +227,26 @@ def test_mixed_step_decode_append_and_verify_in_one_launch(cuda_device):
     ts2 = torch.empty((int(cd[-1]), H, d, d), device=cuda_device)
     o_ref = torch.empty_like(o)
     K.kda_verify(dc["q"], dc["k"], dc["v"], dc["g"], dc["beta"], cd, c["slots_d"], pool_a, ts2, o_ref)
-    assert torch.equal(o, o_ref)
+    assert same_outputs(o, o_ref, ex)
     for s in range(n_seq):
         slot = c["slots"][s]
         if kind[s] == "verify":
-            assert torch.equal(pool_b[slot], pool_a[slot]), s
+            assert same_states(pool_b[slot], pool_a[slot], ex), s
             assert torch.isnan(sn[s]).all() or acc[s] >= 2
         else:
-            assert torch.equal(pool_b[slot], ts2[int(cd[s + 1]) - 1]), s   # after the last token
-            if lens[s] >= 2:                                              # boundary at token 1
-                assert torch.equal(sn[s], ts2[int(cd[s]) + 1]), s
+            assert same_states(pool_b[slot], ts2[int(cd[s + 1]) - 1], ex), s   # after the last token
+            if lens[s] >= 2:                                                  # boundary at token 1
+                assert same_states(sn[s], ts2[int(cd[s]) + 1], ex), s
             else:
                 assert torch.isnan(sn[s]).all(), s
     # the decode sequences equal kda_decode itself
     dec = [s for s in range(n_seq) if kind[s] == "decode"]
     rows = torch.tensor([int(cd[s]) for s in dec], device=cuda_device)
     pool_d = c["pool"].to(cuda_device)
-    od = torch.empty((len(dec), H, d), dtype=torch.bfloat16, device=cuda_device)
+    od = torch.empty((len(dec), H, d), dtype=odt, device=cuda_device)
     K.kda_decode(dc["q"][rows].contiguous(), dc["k"][rows].contiguous(), dc["v"][rows].contiguous(),
                  dc["g"][rows].contiguous(), dc["beta"][rows].contiguous(),
                  c["slots_d"][dec].contiguous(), pool_d, od)
     for i, s in enumerate(dec):
-        assert torch.equal(pool_d[c["slots"][s]], pool_b[c["slots"][s]])
-        assert torch.equal(od[i], o[int(cd[s])])
+        assert same_states(pool_b[c["slots"][s]], pool_d[c["slots"][s]], ex)
+        assert same_outputs(o[int(cd[s])], od[i], ex)
