@@ -134,7 +134,9 @@ __device__ __forceinline__ void conv_store(const ConvWin &w, const DecodeParams 
     win_store(w.k, dst + conv_index(2 * row + 1, p.H, h, D, c, K), K);
 }
 
-__device__ __forceinline__ float swish(float y) { return y / (1.f + expf(-y)); }
+// y sigmoid(y) with the fast exponential and division (a few ulp; the features go on as
+// bf16 or into fp32 sums whose own rounding is larger). y below about -87 gives 0.
+__device__ __forceinline__ float swish(float y) { return __fdividef(y, 1.f + __expf(-y)); }
 
 // Where the front-end's conv state goes while a batch is staged (front-end on only):
 // after every token into rows tok0 + j of `tok` (nullable), and after token snap_j
