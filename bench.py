@@ -666,8 +666,8 @@ def time_calls(fn, steps, warmup, dev):
 
 
 def run_workload(args):
-    """Single-workload timing lines (tiny fp32, ragged batch, 1M-token segments)
-    used for the design notes; the default run is the serving step."""
+    """Single-workload timing lines (tiny fp32, ragged batch, 1M-token segments, the q/k
+    front-end) used for the design notes and profiles; the default run is the serving step."""
     from hybrid_linear_attention_04_b200 import build as kbuild
     kbuild.build()
     from hybrid_linear_attention_04_b200 import kda as K
@@ -746,6 +746,8 @@ def run_workload(args):
         byts = T * H * (3 * D * 2 + D * 2 + D * 4 + 4) + (T // c["snap"] + 2 * n_seg) * H * D * D * 4
         out.update({"unit": "tok/s", "value": T / (ms * 1e-3), "ms": ms, "tokens": T,
                     "algorithmic_bytes": byts, "hbm_frac": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]})
+    elif args.workload == "frontend":
+        out.update(bench_frontend(K, dev, args.steps, args.warmup, peaks))
     st_ = K.kda_check_device_status()
     if st_ != 0:
         raise RuntimeError(K.kda_status_string(st_))
@@ -793,7 +795,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=2048)
     ap.add_argument("--ref-tokens", type=int, default=512)
-    ap.add_argument("--workload", choices=["serving", "tiny", "ragged", "long"], default="serving")
+    ap.add_argument("--workload", choices=["serving", "tiny", "ragged", "long", "frontend"], default="serving")
     ap.add_argument("--prefill-tokens", type=int, default=PREFILL_T,
                     help="prefill length of the serving step (smaller only for profiler captures)")
     ap.add_argument("--decode-seqs", type=int, default=N_SEQ,

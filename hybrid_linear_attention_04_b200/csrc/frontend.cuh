@@ -7,10 +7,10 @@
 // sequence's conv state is its last taps-1 raw inputs, oldest first, laid out
 // [2 (q, k), H, D, taps-1] per sequence.
 //
-// One warp per (sequence, C-token tile, head), four per CTA; lane l owns the D/32
-// consecutive channels from D/32 l for q and k, with their weights and conv windows in
+// One warp per (sequence, C-token tile, head, q or k), four per CTA; lane l owns the
+// D/32 consecutive channels from D/32 l, with their weights and conv windows in
 // registers (the window from the sequence's conv state for its first tile, from the
-// rows before it otherwise). Rows go in groups of four with all their loads issued
+// rows before it otherwise). Rows go in groups of eight with all their loads issued
 // first; each row's L2 norm is a warp reduction. The tile that ends on a snapshot
 // boundary writes the conv state there, the last tile the final conv state.
 #pragma once
@@ -35,10 +35,10 @@ struct FrontendParams {
 
 template <int D>
 struct FrontendShape {
-    static constexpr int WARPS = 4;          // independent (tile, head) items per CTA
+    static constexpr int WARPS = 4;          // independent (tile, head, q or k) items per CTA
     static constexpr int NT = 32 * WARPS;
-    static constexpr int CPL = D / 32;       // channels per lane: 4 lane .. (CPL lane + CPL - 1)
-    static constexpr int G = 4;              // rows whose loads are issued together
+    static constexpr int CPL = D / 32;       // channels per lane: CPL lane .. (CPL lane + CPL - 1)
+    static constexpr int G = CPL == 4 ? 4 : 8;   // rows whose loads are issued together
 };
 
 // CPL consecutive elements of a row (one vector access)
@@ -62,15 +62,19 @@ __device__ __forceinline__ void st_vec(TIO *p, const float (&x)[CPL], float s) {
     }
 }
 
+// One warp per (tile, head, q or k): the two tensors go through the same conv, Swish and
+// L2 norm independently, so each warp holds one tensor's weights and windows and keeps
+// G rows of loads in flight.
 template <int D, typename TIO>
-__global__ void __launch_bounds__(FrontendShape<D>::NT) qk_frontend_kernel(const __grid_constant__ FrontendParams P) {
+__global__ void __launch_bounds__(FrontendShape<D>::NT, 5) qk_frontend_kernel(const __grid_constant__ FrontendParams P) {
     using Sh = FrontendShape<D>;
     constexpr int CPL = Sh::CPL, G = Sh::G;
     const int H = P.H, K = P.taps, C = P.C;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t item = (int64_t)blockIdx.x * Sh::WARPS + warp;
-    const int h = (int)(item % H);
-    const int64_t row = item / H;
+    const int which = (int)(item & 1);                      // 0: q, 1: k
+    const int h = (int)((item >> 1) % H);
+    const int64_t row = (item >> 1) / H;
     // owner sequence: the last one whose first tile row is <= row (rows of different
     // sequences never collide; see prefill_split.cuh for the same indexing)
     auto first_row = [&](int i) { return (int64_t)(P.tok0[i] - P.tok_first) / C + i; };
@@ -86,77 +90,51 @@ __global__ void __launch_bounds__(FrontendShape<D>::NT) qk_frontend_kernel(const
     const int n = max(0, min(C, len - b * C));
     const int64_t t0 = (int64_t)P.tok0[i] + (int64_t)b * C;
     const int c0 = CPL * lane;
-    const TIO *q = static_cast<const TIO *>(P.q), *k = static_cast<const TIO *>(P.k);
+    const TIO *x = static_cast<const TIO *>(which ? P.k : P.q);
+    const float *wt = which ? P.wk : P.wq;
     // weights and windows of the lane's channels
-    Win cq[CPL], ck[CPL];
-    float hist[kMaxTaps - 1][2][CPL];      // the window before the tile, oldest first
-#pragma unroll
-    for (int j = 0; j < kMaxTaps - 1; ++j) {
-#pragma unroll
-        for (int e = 0; e < CPL; ++e) hist[j][0][e] = hist[j][1][e] = 0.f;
-        if (j < K - 1) {
-            if (b == 0) {
-                if (P.conv_in) {
-#pragma unroll
-                    for (int e = 0; e < CPL; ++e) {
-                        hist[j][0][e] = P.conv_in[conv_index(2 * i, H, h, D, c0 + e, K) + j];
-                        hist[j][1][e] = P.conv_in[conv_index(2 * i + 1, H, h, D, c0 + e, K) + j];
-                    }
-                }
-            } else {
-                const int64_t r = t0 - (K - 1) + j;             // inside this sequence (b * C >= K - 1)
-                ld_vec<TIO, CPL>(q + (r * H + h) * D + c0, hist[j][0]);
-                ld_vec<TIO, CPL>(k + (r * H + h) * D + c0, hist[j][1]);
-            }
-        }
-    }
+    Win cw[CPL];
 #pragma unroll
     for (int e = 0; e < CPL; ++e) {
-        const float sq[3] = {hist[0][0][e], hist[1][0][e], hist[2][0][e]};
-        const float sk[3] = {hist[0][1][e], hist[1][1][e], hist[2][1][e]};
-        win_load(cq[e], P.wq + ((int64_t)h * D + c0 + e) * K, sq, K);
-        win_load(ck[e], P.wk + ((int64_t)h * D + c0 + e) * K, sk, K);
-    }
-    TIO *qo = static_cast<TIO *>(P.q_out), *ko = static_cast<TIO *>(P.k_out);
-    for (int r0 = 0; r0 < n; r0 += G) {
-        float xq[G][CPL], xk[G][CPL];
+        float hist[kMaxTaps - 1] = {0.f, 0.f, 0.f};   // the window before the tile, oldest first
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-            if (r0 + g < n) {
-                const int64_t off = ((t0 + r0 + g) * H + h) * D + c0;
-                ld_vec<TIO, CPL>(q + off, xq[g]);
-                ld_vec<TIO, CPL>(k + off, xk[g]);
+        for (int j = 0; j < kMaxTaps - 1; ++j) {
+            if (j < K - 1) {
+                if (b == 0) {
+                    if (P.conv_in) hist[j] = P.conv_in[conv_index(2 * i + which, H, h, D, c0 + e, K) + j];
+                } else {
+                    const int64_t r = t0 - (K - 1) + j;         // inside this sequence (b * C >= K - 1)
+                    hist[j] = IO<TIO>::ld(x + (r * H + h) * D + c0 + e);
+                }
             }
         }
+        win_load(cw[e], wt + ((int64_t)h * D + c0 + e) * K, hist, K);
+    }
+    TIO *xo = static_cast<TIO *>(which ? P.k_out : P.q_out);
+    for (int r0 = 0; r0 < n; r0 += G) {
+        float xv[G][CPL];
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+            if (r0 + g < n) ld_vec<TIO, CPL>(x + ((t0 + r0 + g) * H + h) * D + c0, xv[g]);
 #pragma unroll
         for (int g = 0; g < G; ++g) {
             if (r0 + g < n) {
-                float zq[CPL], zk[CPL], sq = 0.f, sk = 0.f;
+                float z[CPL], ss = 0.f;
 #pragma unroll
                 for (int e = 0; e < CPL; ++e) {
-                    zq[e] = swish(conv_step(cq[e], K, xq[g][e]));
-                    zk[e] = swish(conv_step(ck[e], K, xk[g][e]));
-                    sq = fmaf(zq[e], zq[e], sq);
-                    sk = fmaf(zk[e], zk[e], sk);
+                    z[e] = swish(conv_step(cw[e], K, xv[g][e]));
+                    ss = fmaf(z[e], z[e], ss);
                 }
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    sq += __shfl_xor_sync(0xffffffffu, sq, o);
-                    sk += __shfl_xor_sync(0xffffffffu, sk, o);
-                }
-                const int64_t off = ((t0 + r0 + g) * H + h) * D + c0;
-                st_vec<TIO, CPL>(qo + off, zq, 1.f / fmaxf(sqrtf(sq), kNormEps));
-                st_vec<TIO, CPL>(ko + off, zk, 1.f / fmaxf(sqrtf(sk), kNormEps));
+                for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                st_vec<TIO, CPL>(xo + ((t0 + r0 + g) * H + h) * D + c0, z, 1.f / fmaxf(sqrtf(ss), kNormEps));
             }
         }
     }
     // conv states: at a snapshot boundary that ends this tile, and after the last token
     auto put = [&](float *dst, int64_t srow) {
 #pragma unroll
-        for (int e = 0; e < CPL; ++e) {
-            win_store(cq[e], dst + conv_index(2 * srow, H, h, D, c0 + e, K), K);
-            win_store(ck[e], dst + conv_index(2 * srow + 1, H, h, D, c0 + e, K), K);
-        }
+        for (int e = 0; e < CPL; ++e) win_store(cw[e], dst + conv_index(2 * srow + which, H, h, D, c0 + e, K), K);
     };
     const int64_t p_end = P.start_pos[i] + (int64_t)b * C + n;
     if (P.conv_snap && P.snap_interval > 0 && n == C && p_end % P.snap_interval == 0)

@@ -661,12 +661,12 @@ kda_status kda_qk_frontend(const kda_dims *dims, const kda_conv *conv, int32_t n
             P.snap_off[i] = offs[g0 + i];
         }
         const int64_t rows = ((int64_t)cu[g0 + ng] - cu[g0]) / C + ng;
-        if (rows * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+        if (2 * rows * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
         const bool bf = dims->io == KDA_IO_BF16;
         switch (D) {
-        case 32: st = bf ? launch_frontend<32, __nv_bfloat16>(P, rows * H, cs) : launch_frontend<32, float>(P, rows * H, cs); break;
-        case 64: st = bf ? launch_frontend<64, __nv_bfloat16>(P, rows * H, cs) : launch_frontend<64, float>(P, rows * H, cs); break;
-        default: st = bf ? launch_frontend<128, __nv_bfloat16>(P, rows * H, cs) : launch_frontend<128, float>(P, rows * H, cs); break;
+        case 32: st = bf ? launch_frontend<32, __nv_bfloat16>(P, 2 * rows * H, cs) : launch_frontend<32, float>(P, 2 * rows * H, cs); break;
+        case 64: st = bf ? launch_frontend<64, __nv_bfloat16>(P, 2 * rows * H, cs) : launch_frontend<64, float>(P, 2 * rows * H, cs); break;
+        default: st = bf ? launch_frontend<128, __nv_bfloat16>(P, 2 * rows * H, cs) : launch_frontend<128, float>(P, 2 * rows * H, cs); break;
         }
         if (st != KDA_OK) return st;
     }
