@@ -307,13 +307,22 @@ __device__ __forceinline__ void store_state(const StatePairs<D> &P, float *S) {
 
 // One recurrence step on the register-resident columns of this warp. With OUT =
 // false the output read (y and o) is skipped; the state arithmetic is the same
-// instruction for instruction, so both forms give bit-identical states. The
-// returned o (OUT) holds the lane's four columns; every lane of a column group has it.
+// instruction for instruction, so both forms give bit-identical states.
+//
+// The column sums over d_k reduce inside the lane (two row halves, then added), then over
+// the 8 lanes of a column group (rg = lane / 4) as a reduce-scatter: at each of lane bits
+// 2, 3, 4 (rg bits 0, 1, 2) a lane keeps half of its partial sums and adds the partner's
+// copy of them, so the 8 sums (x and y of 4 columns) end one per lane after 7 shuffles,
+// and the 4 x sums go back to every lane by 4 indexed shuffles. Every sum has the same
+// addition tree (rows paired by rg bit 0, then 1, then 2) in both forms and in every lane
+// that holds it, so OUT changes no bit of x. With OUT the lane whose rg is odd holds y of
+// column `oe` of its group and returns that column's output; the other lanes return 0.
 template <int D, bool OUT = true>
-__device__ __forceinline__ float4 kda_step(StatePairs<D> &P, const TokVec<D> &tv, float scale) {
+__device__ __forceinline__ float kda_step(StatePairs<D> &P, const TokVec<D> &tv, float scale, int &oe) {
     using L = TokLayout<D>;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int rg = lane >> 2, cg = lane & 3;
+    const bool b0 = rg & 1, b1 = (rg >> 1) & 1, b2 = (rg >> 2) & 1;
     const float *ap = tv.a + rg * L::STR, *kp = tv.k + rg * L::STR, *qp = tv.q + rg * L::STR;
     f2 xa[4] = {0ull, 0ull, 0ull, 0ull}, ya[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
@@ -347,16 +356,46 @@ __device__ __forceinline__ float4 kda_step(StatePairs<D> &P, const TokVec<D> &tv
             y[e] = ys.x + ys.y;
         }
     }
+    constexpr unsigned FULL = 0xffffffffu;
+    float xr[4], own = 0.f;
+    if (OUT) {
+        // sums v = (x0..x3, y0..y3): keep v[4 b0 ..], then [2 b1 ..] of those, then [b2]
+        float u1[4], u2[2];
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            x[e] += __shfl_xor_sync(0xffffffffu, x[e], off);
-            if (OUT) y[e] += __shfl_xor_sync(0xffffffffu, y[e], off);
+        for (int i = 0; i < 4; ++i) {
+            const float send = b0 ? x[i] : y[i], keep = b0 ? y[i] : x[i];
+            u1[i] = keep + __shfl_xor_sync(FULL, send, 4);
         }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const float send = b1 ? u1[i] : u1[2 + i], keep = b1 ? u1[2 + i] : u1[i];
+            u2[i] = keep + __shfl_xor_sync(FULL, send, 8);
+        }
+        {
+            const float send = b2 ? u2[0] : u2[1], keep = b2 ? u2[1] : u2[0];
+            own = keep + __shfl_xor_sync(FULL, send, 16);   // (b0 ? y : x)[2 b1 + b2]
+        }
+        // x_e sits in the lane of the group with rg = 2 (e >> 1) + 4 (e & 1)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) xr[e] = __shfl_sync(FULL, own, 4 * (2 * (e >> 1) + 4 * (e & 1)) + cg);
+    } else {
+        // sums v = (x0..x3): keep v[2 b0 ..], then [b1], then the full sum over b2
+        float u1[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const float send = b0 ? x[i] : x[2 + i], keep = b0 ? x[2 + i] : x[i];
+            u1[i] = keep + __shfl_xor_sync(FULL, send, 4);
+        }
+        const float send = b1 ? u1[0] : u1[1], keep = b1 ? u1[1] : u1[0];
+        const float u2 = keep + __shfl_xor_sync(FULL, send, 8);
+        own = u2 + __shfl_xor_sync(FULL, u2, 16);             // x[2 b0 + b1]
+        // x_e sits in the lanes with rg = (e >> 1) + 2 (e & 1) (and + 4)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) xr[e] = __shfl_sync(FULL, own, 4 * ((e >> 1) + 2 * (e & 1)) + cg);
+    }
     const float4 vv = *reinterpret_cast<const float4 *>(tv.v + 16 * warp + 4 * cg);
-    const float w0 = tv.beta * (vv.x - x[0]), w1 = tv.beta * (vv.y - x[1]);
-    const float w2 = tv.beta * (vv.z - x[2]), w3 = tv.beta * (vv.w - x[3]);
+    const float w0 = tv.beta * (vv.x - xr[0]), w1 = tv.beta * (vv.y - xr[1]);
+    const float w2 = tv.beta * (vv.z - xr[2]), w3 = tv.beta * (vv.w - xr[3]);
     const f2 ww[4] = {pk2(w0, w0), pk2(w1, w1), pk2(w2, w2), pk2(w3, w3)};
 #pragma unroll
     for (int i = 0; i < L::R / 4; ++i) {
@@ -368,13 +407,17 @@ __device__ __forceinline__ float4 kda_step(StatePairs<D> &P, const TokVec<D> &tv
             P[2 * i + 1][e] = fma2(k23, ww[e], P[2 * i + 1][e]);
         }
     }
-    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (OUT) {
-        o.x = scale * fmaf(tv.kq, w0, y[0]); o.y = scale * fmaf(tv.kq, w1, y[1]);
-        o.z = scale * fmaf(tv.kq, w2, y[2]); o.w = scale * fmaf(tv.kq, w3, y[3]);
+    oe = 2 * b1 + b2;
+    float o = 0.f;
+    if (OUT && b0) {
+        const float w = oe == 0 ? w0 : oe == 1 ? w1 : oe == 2 ? w2 : w3;
+        o = scale * fmaf(tv.kq, w, own);
     }
     return o;
 }
+
+// the lanes that hold an output after kda_step<D, true>: odd rg
+__device__ __forceinline__ bool out_lane() { return ((threadIdx.x >> 2) & 1) != 0; }
 
 // ---------------------------------------------------------------- decode
 // One token per (sequence, head): one CTA each, the state read and written once.
@@ -408,9 +451,10 @@ decode_kernel(const __grid_constant__ DecodeParams p) {
     __syncthreads();
     if (t < 32) token_finish<D>(tv, CONV, true);
     __syncthreads();
-    const float4 o = kda_step<D>(P, tv, p.scale);
+    int oe;
+    const float o = kda_step<D>(P, tv, p.scale, oe);
     store_state<D>(P, S);
-    if ((t & 31) < 4) IO<TIO>::st4(static_cast<TIO *>(p.o) + row * D + lane_col(), o);
+    if (out_lane()) IO<TIO>::st(static_cast<TIO *>(p.o) + row * D + lane_col() + oe, o);
 }
 
 // ---------------------------------------------------------------- verify, verify + commit
@@ -752,7 +796,8 @@ spec_kernel(const __grid_constant__ SpecParams P) {
                 const bool store_after = bi == I.nb0 - 1 && !I.cnew;
                 float *snap = js >= 0 ? c.snapshots + (I.srow * p.H + hh) * (int64_t)D * D : nullptr;
                 for (int j = 0; j < nb; ++j) {
-                    kda_step<D, false>(Pr, tv[j], 0.f);
+                    int oe;
+                    kda_step<D, false>(Pr, tv[j], 0.f, oe);
                     if (j == js) store_state<D>(Pr, snap);
                 }
                 if (store_after) {
@@ -763,9 +808,10 @@ spec_kernel(const __grid_constant__ SpecParams P) {
                 float *snap = js >= 0 ? c.snapshots + (I.srow * p.H + hh) * (int64_t)D * D : nullptr;
                 const int64_t row0 = (I.tok_first + j0) * p.H + hh;
                 for (int j = 0; j < nb; ++j) {
-                    const float4 o = kda_step<D>(Pr, tv[j], p.scale);
+                    int oe;
+                    const float o = kda_step<D>(Pr, tv[j], p.scale, oe);
                     const int64_t row = row0 + (int64_t)j * p.H;
-                    if ((t & 31) < 4) IO<TIO>::st4(static_cast<TIO *>(p.o) + row * D + lane_col(), o);
+                    if (out_lane()) IO<TIO>::st(static_cast<TIO *>(p.o) + row * D + lane_col() + oe, o);
                     if (!COMMIT) store_state<D>(Pr, p.token_states + row * (int64_t)D * D);
                     if (COMMIT && j == js) store_state<D>(Pr, snap);
                 }

@@ -110,12 +110,15 @@ __global__ void __launch_bounds__(FrontendShape<D>::NT, 5) qk_frontend_kernel(co
         }
         win_load(cw[e], wt + ((int64_t)h * D + c0 + e) * K, hist, K);
     }
-    TIO *xo = static_cast<TIO *>(which ? P.k_out : P.q_out);
+    // the lane's channels of the tile's rows: row r at src + r * stride (and likewise dst)
+    const int64_t stride = (int64_t)H * D;
+    const TIO *src = x + (t0 * H + h) * D + c0;
+    TIO *dst = static_cast<TIO *>(which ? P.k_out : P.q_out) + (t0 * H + h) * D + c0;
     for (int r0 = 0; r0 < n; r0 += G) {
         float xv[G][CPL];
 #pragma unroll
         for (int g = 0; g < G; ++g)
-            if (r0 + g < n) ld_vec<TIO, CPL>(x + ((t0 + r0 + g) * H + h) * D + c0, xv[g]);
+            if (r0 + g < n) ld_vec<TIO, CPL>(src + (r0 + g) * stride, xv[g]);
 #pragma unroll
         for (int g = 0; g < G; ++g) {
             if (r0 + g < n) {
@@ -127,7 +130,8 @@ __global__ void __launch_bounds__(FrontendShape<D>::NT, 5) qk_frontend_kernel(co
                 }
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-                st_vec<TIO, CPL>(xo + ((t0 + r0 + g) * H + h) * D + c0, z, 1.f / fmaxf(sqrtf(ss), kNormEps));
+                // 1 / max(|z|, eps) as rsqrt(max(|z|^2, eps^2))
+                st_vec<TIO, CPL>(dst + (r0 + g) * stride, z, rsqrtf(fmaxf(ss, kNormEps * kNormEps)));
             }
         }
     }
