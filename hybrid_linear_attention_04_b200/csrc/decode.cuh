@@ -1,8 +1,8 @@
 // KDA decode and speculative-verify kernels (sm_100a, SIMT, HBM-bound).
 //
-// One CTA owns one (sequence, head) state S [D x D] fp32 (d_v contiguous) and
-// streams it through registers once: 128-bit loads, gate, rank-1 delta
-// correction and output read in one pass, 128-bit stores.
+// A CTA owns one (sequence, head) state S [D x D] fp32 (d_v contiguous) at a time and
+// streams it through registers once: 128-bit loads, gate, rank-1 delta correction and
+// output read in one pass per token, 128-bit stores.
 //
 // Per token (Kimi K3 technical FAQ, "What is KDA": delta rule with a
 // per-channel forget gate; standard gated-delta form):
@@ -13,18 +13,17 @@
 //     o  = scale (y + (k . q) w)            (= scale * S^T q, read after update)
 //
 // The d_v columns of S evolve independently (w, the update and o are per column),
-// so warp w owns the 16 columns 16w .. 16w+15 over all d_k rows: lane l holds the
-// float4 of columns 16w + 4 (l % 4) .. +3 in rows l / 4 + 8 m, m < D / 8. The column
-// sums over d_k reduce inside the lane, then across the 8 lanes that share the
-// column group (three butterfly shuffles, so every lane holds the same sum); a
-// token step has no barrier and no shared-memory reduction. Decode, verify and the
-// commit replay run the same step function, so verify's state after its j-th token
-// is bit-identical to j decode calls.
+// so warp w owns the 16 columns 16w .. 16w+15 over all d_k rows: lane l holds columns
+// 16w + 4 (l % 4) .. +3 of rows l / 4 + 8 m, m < D / 8, as f32x2 pairs of rows. The
+// column sums over d_k reduce inside the lane, then across the 8 lanes that share the
+// column group (a reduce-scatter and a gather of shuffles); a token step has no barrier
+// and no shared-memory reduction. Decode, verify and the commit replay run the same
+// step function, so verify's state after its j-th token is bit-identical to j decode
+// calls.
 //
-// Token vectors are staged in shared memory a batch at a time: threads t < D own
-// channel t of q and k (and run the q/k front-end's conv window in token order),
-// threads t >= D channel t - D of v and g; each thread issues all its loads for the
-// batch before it uses any.
+// Token vectors sit in shared memory (decode: one token; verify: batches of TMA-loaded
+// rows): threads t < D own channel t of q and k (and run the q/k front-end's conv
+// window in token order), threads t >= D channel t - D of v and g.
 #pragma once
 #include "common.cuh"
 #include "tc_util.cuh"
