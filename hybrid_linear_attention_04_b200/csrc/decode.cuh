@@ -732,6 +732,17 @@ spec_kernel(const __grid_constant__ SpecParams P) {
         tc::bar_init(&bar_t[0], 1);
         tc::bar_init(&bar_t[1], 1);
         tc::bar_init_fence();
+        // the token-row descriptors, ahead of the first copies that use them
+        tc::tma_prefetch_desc(&P.mk);
+        tc::tma_prefetch_desc(&P.mv);
+        tc::tma_prefetch_desc(&P.mg);
+        if (p.q) tc::tma_prefetch_desc(&P.mq);
+        if (COMMIT && c.k) {
+            tc::tma_prefetch_desc(&P.pk);
+            tc::tma_prefetch_desc(&P.pv);
+            tc::tma_prefetch_desc(&P.pg);
+            if (CONV && c.q) tc::tma_prefetch_desc(&P.pq);
+        }
         cur->kb = 0; cur->bb = 0; cur->nb_issued = 0; cur->ks = 0; cur->ns_issued = 0;
     }
     __syncthreads();
