@@ -476,16 +476,17 @@ struct CommitParams {
     int32_t tok0[kMaxSeqsPerLaunch + 1];  // previous batch offsets (relative)
 };
 
-// A persistent grid of G CTAs over the (sequence, head) items, with the sequences in the
-// host's order of decreasing token count: CTA b takes ranks b, b + G, b + 2 G, ... of that
-// list, every second band of G ranks reversed (a snake), so that each CTA gets one item
-// of every band and the CTAs' token totals come out nearly equal (the heads of one
-// sequence share its token counts). The records of a CTA's items (slot, accepted count,
-// snapshot) are read once at its start. Warp 0 is the producer:
-// one bulk copy brings the next item's state (and conv window and weights) into shared
-// memory while the current item runs from registers, and the item's token rows come in
-// batches of TB by 3-D TMA tiles (channels x 1 head x TB rows) into two buffers, two
-// batches ahead across item boundaries.
+// G CTAs over the (sequence, head) items, with the sequences in the host's order of
+// decreasing token count: CTA b takes ranks b, b + G, b + 2 G, ... of that list, every
+// second band of G ranks reversed (a snake), so that each CTA gets one item of every band
+// and the CTAs' token totals come out nearly equal (the heads of one sequence share its
+// token counts). verify + commit runs a persistent grid (two CTAs per SM); verify runs
+// G = items, one CTA per item, longest first. The records of a CTA's items (slot,
+// accepted count, snapshot) are read once at its start. Warp 0 is the producer: one bulk
+// copy brings the next item's state (and conv window and weights) into shared memory
+// while the current item runs from registers, and the item's token rows come in batches
+// of TB by 3-D TMA tiles (channels x 1 head x TB rows) into two buffers, two batches ahead
+// across item boundaries.
 struct SpecParams {
     CUtensorMap mq, mk, mv, mg;       // this step's q, k, v, g rows: (D, H, rows), box (D, 1, TB)
     CUtensorMap pq, pk, pv, pg;       // the previous step's (replay; pq with the front-end only)
