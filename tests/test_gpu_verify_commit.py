@@ -250,3 +250,32 @@ def test_mixed_step_decode_append_and_verify_in_one_launch(cuda_device, io):
     for i, s in enumerate(dec):
         assert same_states(pool_b[c["slots"][s]], pool_d[c["slots"][s]], ex)
         assert same_outputs(o[int(cd[s])], od[i], ex)
+
+
+def test_verify_commit_empty_items_among_others(cuda_device):
+    """Sequences with nothing accepted and no drafts (no work at all), nothing accepted
+    only, or no drafts only, interleaved with the rest: the persistent grid's producer
+    skips the empty items while it prefetches across item boundaries, and every other
+    sequence still equals kda_verify + kda_snapshot + kda_verify bit for bit."""
+    H, d, n_seq = 4, 64, 300
+    c = _case(1301, n_seq, H, d, "bf16", cuda_device, lo=0, hi=8)
+    cp, cd = c["cp"], c["cd"]
+    assert (np.diff(cp) == 0).any() and (np.diff(cd) == 0).any()
+    pool_a = c["pool"].to(cuda_device)
+    pool_b = pool_a.clone()
+    dp, dc = c["dp"], c["dc"]
+    ts = torch.empty((max(1, int(cp[-1])), H, d, d), device=cuda_device)
+    K.kda_verify(dp["q"], dp["k"], dp["v"], dp["g"], dp["beta"], cp, c["slots_d"], pool_a, ts,
+                 torch.empty_like(dp["v"]))
+    keep = [s for s in range(n_seq) if c["acc"][s] > 0]
+    K.kda_snapshot(torch.tensor([int(cp[s]) + c["acc"][s] - 1 for s in keep], dtype=torch.int64,
+                                device=cuda_device),
+                   torch.tensor([c["slots"][s] for s in keep], dtype=torch.int64, device=cuda_device),
+                   ts, pool_a)
+    o_ref = torch.empty_like(dc["v"])
+    ts2 = torch.empty((max(1, int(cd[-1])), H, d, d), device=cuda_device)
+    K.kda_verify(dc["q"], dc["k"], dc["v"], dc["g"], dc["beta"], cd, c["slots_d"], pool_a, ts2, o_ref)
+    o = _fused(c, pool_b)
+    assert K.kda_check_device_status() == 0
+    assert torch.equal(pool_b, pool_a)
+    assert torch.equal(o, o_ref)
