@@ -374,6 +374,136 @@ kda_status kda_prefill(const kda_dims *dims, int32_t n_seq, const int32_t *cu,
     return KDA_OK;
 }
 
+// The fixed scratch's device address on the current device, looked up on the first call
+// that needs it there (host code only sees a stand-in for the symbol).
+static kda_status noalloc_scratch(void **scratch) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    static std::atomic<void *> addr[kMaxDevices];
+    *scratch = dev < kMaxDevices ? addr[dev].load(std::memory_order_acquire) : nullptr;
+    if (!*scratch) {
+        e = cudaGetSymbolAddress(scratch, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (dev < kMaxDevices) addr[dev].store(*scratch, std::memory_order_release);
+    }
+    return KDA_OK;
+}
+
+// One sub-call of a prefill that does not fit the scratch: sequences [s0, s1) whole, or
+// tokens [a, b) of sequence s0 alone (s1 = -1).
+struct PrefillPiece {
+    int s0, s1;
+    int64_t a, b;
+};
+
+// kda_prefill_noalloc when the call's packets exceed the scratch: consecutive sequences
+// are grouped while their packets fit; a sequence that alone exceeds it runs in windows of
+// whole chunks, its state handed from one window to the next through two state buffers at
+// the end of the scratch (fp32, exact), so that the chunks, and the results, are those of
+// one call with a workspace. Returns KDA_ERR_UNSUPPORTED, with nothing launched, when a
+// piece's beta would not be 16-byte aligned (H not a multiple of 4); the caller then runs
+// the single-launch path.
+static kda_status prefill_pieces(const kda_dims *dims, int32_t n_seq, const int32_t *cu,
+                                 const int64_t *start_pos, const void *q, const void *k,
+                                 const void *v, const float *g, const float *beta,
+                                 const float *state_in, float *state_out, void *o,
+                                 int32_t snap_interval, float *snapshots, void *scratch,
+                                 kda_stream_t stream) {
+    const int C = dims->chunk, H = dims->H, dk = dims->dk, dv = dims->dv;
+    const size_t state_bytes = (size_t)H * dk * dv * 4;
+    if (kNoallocScratchBytes < 2 * state_bytes) return KDA_ERR_UNSUPPORTED;
+    const size_t cap = kNoallocScratchBytes - 2 * state_bytes;
+    const int64_t max_rows = (int64_t)(cap / ((size_t)H * spl::PACKET));
+    if (max_rows < 2) return KDA_ERR_UNSUPPORTED;
+    // the argument checks of kda_prefill, before anything is launched
+    std::vector<int64_t> offs(n_seq + 1);
+    kda_status st = kda_snapshot_plan(n_seq, cu, start_pos, snap_interval, offs.data(), nullptr);
+    if (st != KDA_OK) return st;
+    if (snap_interval > 0) {
+        if (snap_interval % C != 0) return KDA_ERR_INVALID;
+        for (int s = 0; s < n_seq && start_pos; ++s)
+            if (start_pos[s] % C != 0) return KDA_ERR_INVALID;
+    }
+    const int64_t T = cu[n_seq];
+    if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID;
+    if (offs[n_seq] > 0 && !snapshots) return KDA_ERR_INVALID;
+    const void *ptrs[] = {q, k, v, g, beta, state_in, state_out, o, snapshots};
+    for (const void *ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
+    // the plan
+    std::vector<PrefillPiece> plan;
+    const int64_t wtok = (max_rows - 1) * C;          // a window's tokens: (wtok >> 6) + 1 rows
+    for (int s = 0; s < n_seq;) {
+        const int64_t len = cu[s + 1] - cu[s];
+        if ((len >> 6) + 1 > max_rows) {
+            for (int64_t a = 0; a < len; a += wtok) plan.push_back({s, -1, a, std::min(len, a + wtok)});
+            ++s;
+            continue;
+        }
+        int s1 = s;
+        int64_t tok = 0;
+        while (s1 < n_seq && s1 - s < kPrefillSeqs) {
+            const int64_t l1 = cu[s1 + 1] - cu[s1];
+            if (((tok + l1) >> 6) + (s1 - s + 1) > max_rows) break;
+            tok += l1;
+            ++s1;
+        }
+        plan.push_back({s, s1, 0, 0});
+        s = s1;
+    }
+    const int64_t beta_row = (int64_t)H * 4;
+    for (const PrefillPiece &pc : plan) {
+        const int64_t row0 = cu[pc.s0] + (pc.s1 < 0 ? pc.a : 0);
+        if ((row0 * beta_row) % 16 != 0) return KDA_ERR_UNSUPPORTED;
+    }
+    // the pieces, in order on the stream
+    const size_t io = dims->io == KDA_IO_BF16 ? 2 : 4;
+    const int64_t qrow = (int64_t)H * dk * io, vrow = (int64_t)H * dv * io, grow = (int64_t)H * dk * 4;
+    const int64_t srow = (int64_t)H * dk * dv;                 // floats per state or snapshot row
+    auto at = [](const void *p, int64_t bytes) -> const uint8_t * {
+        return p ? static_cast<const uint8_t *>(p) + bytes : nullptr;
+    };
+    float *buf[2] = {reinterpret_cast<float *>(static_cast<uint8_t *>(scratch) + cap),
+                     reinterpret_cast<float *>(static_cast<uint8_t *>(scratch) + cap + state_bytes)};
+    std::vector<int32_t> cu2;
+    std::vector<int64_t> start2;
+    int w = 0;                                                  // window index within its sequence
+    for (const PrefillPiece &pc : plan) {
+        const int s = pc.s0;
+        if (pc.s1 >= 0) {
+            const int n = pc.s1 - pc.s0;
+            cu2.assign(n + 1, 0);
+            for (int i = 0; i <= n; ++i) cu2[i] = cu[s + i] - cu[s];
+            const int64_t r0 = cu[s];
+            st = kda_prefill(dims, n, cu2.data(), start_pos ? start_pos + s : nullptr, at(q, r0 * qrow),
+                             at(k, r0 * qrow), at(v, r0 * vrow), reinterpret_cast<const float *>(at(g, r0 * grow)),
+                             reinterpret_cast<const float *>(at(beta, r0 * beta_row)),
+                             state_in ? state_in + s * srow : nullptr, state_out ? state_out + s * srow : nullptr,
+                             const_cast<uint8_t *>(at(o, r0 * vrow)), snap_interval,
+                             snapshots ? snapshots + offs[s] * srow : nullptr, scratch, cap, stream);
+            w = 0;
+        } else {
+            const int64_t len = cu[s + 1] - cu[s], p0 = start_pos ? start_pos[s] : 0;
+            const int64_t r0 = cu[s] + pc.a;
+            cu2.assign(2, 0);
+            cu2[1] = (int32_t)(pc.b - pc.a);
+            start2.assign(1, p0 + pc.a);
+            const int64_t snap0 = offs[s] + (snap_interval > 0 ? (p0 + pc.a) / snap_interval - p0 / snap_interval : 0);
+            const float *sin = pc.a == 0 ? (state_in ? state_in + s * srow : nullptr) : buf[(w + 1) & 1];
+            float *sout = pc.b == len ? (state_out ? state_out + s * srow : nullptr) : buf[w & 1];
+            st = kda_prefill(dims, 1, cu2.data(), start2.data(), at(q, r0 * qrow), at(k, r0 * qrow),
+                             at(v, r0 * vrow), reinterpret_cast<const float *>(at(g, r0 * grow)),
+                             reinterpret_cast<const float *>(at(beta, r0 * beta_row)), sin, sout,
+                             const_cast<uint8_t *>(at(o, r0 * vrow)), snap_interval,
+                             snapshots ? snapshots + snap0 * srow : nullptr, scratch, cap, stream);
+            w = pc.b == len ? 0 : w + 1;
+        }
+        if (st != KDA_OK) return st;
+    }
+    return KDA_OK;
+}
+
 kda_status kda_prefill_noalloc(const kda_dims *dims, int32_t n_seq, const int32_t *cu,
                                const int64_t *start_pos, const void *q, const void *k,
                                const void *v, const float *g, const float *beta,
@@ -383,18 +513,14 @@ kda_status kda_prefill_noalloc(const kda_dims *dims, int32_t n_seq, const int32_
     kda_status st = kda_prefill_workspace_size(dims, n_seq, cu, &need);
     if (st != KDA_OK) return st;
     void *scratch = nullptr;
-    if (need > 0 && need <= kNoallocScratchBytes) {
-        // the array's device address on the current device, looked up on the first call
-        // that needs it there (host code only sees a stand-in for the symbol)
-        int dev = 0;
-        cudaError_t e = cudaGetDevice(&dev);
-        if (e != cudaSuccess) return cuda_fail(e);
-        static std::atomic<void *> addr[kMaxDevices];
-        scratch = dev < kMaxDevices ? addr[dev].load(std::memory_order_acquire) : nullptr;
-        if (!scratch) {
-            e = cudaGetSymbolAddress(&scratch, g_noalloc_scratch);
-            if (e != cudaSuccess) return cuda_fail(e);
-            if (dev < kMaxDevices) addr[dev].store(scratch, std::memory_order_release);
+    if (need > 0) {
+        st = noalloc_scratch(&scratch);
+        if (st != KDA_OK) return st;
+        if (need > kNoallocScratchBytes) {
+            st = prefill_pieces(dims, n_seq, cu, start_pos, q, k, v, g, beta, state_in, state_out, o,
+                                snap_interval, snapshots, scratch, stream);
+            if (st != KDA_ERR_UNSUPPORTED) return st;
+            scratch = nullptr;                        // the single-launch path
         }
     }
     return kda_prefill(dims, n_seq, cu, start_pos, q, k, v, g, beta, state_in, state_out, o,

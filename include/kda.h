@@ -174,11 +174,15 @@ kda_status kda_prefill(const kda_dims *dims, int32_t n_seq, const int32_t *cu_se
 
 /*
  * kda_prefill_noalloc — kda_prefill without a caller workspace and without any
- * allocation: the two-launch path uses the library's fixed device scratch of
+ * allocation: the two-launch path runs on the library's fixed device scratch of
  * kda_prefill_noalloc_capacity() bytes (a module-level array, resident from the
- * library's first use on a device) whenever kda_prefill_workspace_size fits in
- * it, and the single-launch path otherwise. Arguments, layouts and errors as
- * kda_prefill. For callers that cannot allocate device memory at the point of
+ * library's first use on a device). When kda_prefill_workspace_size exceeds it, the
+ * call runs as several two-launch pieces on the stream: consecutive sequences whose
+ * workspace fits together, and a sequence too long for the scratch in windows of
+ * whole chunks, with its state handed between windows in fp32 through the scratch.
+ * The results are bit-identical to one kda_prefill call with a workspace. Only when a
+ * piece's beta pointer would not be 16-byte aligned (H not a multiple of 4) does it
+ * take the single-launch path instead. Arguments, layouts and errors as kda_prefill. For callers that cannot allocate device memory at the point of
  * the call (code running inside a captured or replayed stream region, or a host
  * that forbids allocation after start-up) and cannot set a workspace aside.
  * The scratch is shared by all calls on a device of this process and keeps the

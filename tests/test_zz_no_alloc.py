@@ -1,8 +1,9 @@
 """kda_prefill_noalloc: the prefill call that neither allocates nor takes a caller
-workspace. It runs the two-launch prefill on the library's fixed device scratch
-when the call's workspace fits there, the single-launch prefill otherwise; both
-are checked against the fp64 oracle (token recurrence; Kimi K3 technical FAQ,
-"What is KDA") and against kda_prefill with a caller workspace.
+workspace. It runs the two-launch prefill on the library's fixed device scratch:
+in one piece when the call's workspace fits there, else as pieces (groups of whole
+sequences, and windows of whole chunks of a sequence too long for the scratch). Both
+are checked against the fp64 oracle (token recurrence; Kimi K3 technical FAQ, "What is
+KDA") and bit for bit against kda_prefill with a caller workspace.
 """
 from __future__ import annotations
 
@@ -82,23 +83,45 @@ def test_fits_in_scratch_two_launches_and_matches(cuda_device):
 
 
 @pytest.mark.gpu
-def test_larger_than_scratch_runs_single_launch(cuda_device):
-    """1024 tokens x 64 heads need (16 + 1) x 64 packets (82 MB) > 64 MiB: one launch
-    of the on-chip kernel, bit-identical to kda_prefill without a workspace."""
+def test_larger_than_scratch_runs_in_windows(cuda_device):
+    """1024 tokens x 64 heads need (16 + 1) x 64 packets (82 MB) > 64 MiB: two windows
+    of the two-launch path (704 + 320 tokens, the state handed over in fp32 between them),
+    the oracle's results, and the same bits as kda_prefill with a full workspace."""
     T, H, d = 1024, 64, 128
     x, dev, cu = packed_inputs(63, [T], H, d, "bf16", cuda_device)
-    assert K.kda_prefill_workspace_size(dev["q"], dev["v"], cu) == (T // 64 + 1) * H * PACKET
+    need = K.kda_prefill_workspace_size(dev["q"], dev["v"], cu)
+    assert need == (T // 64 + 1) * H * PACKET > K.kda_prefill_noalloc_capacity()
+    s0 = synth.states(64, 1, H, d, d, std=0.1)
     n0 = K.kda_launch_count()
-    got = _run(K.kda_prefill_noalloc, x, dev, cu, H, d, None, None, 256)
-    assert K.kda_launch_count() - n0 == 1
-    ref = oracle_prefill(x, cu, None, None, 256)
+    got = _run(K.kda_prefill_noalloc, x, dev, cu, H, d, [128], s0, 256)
+    assert K.kda_launch_count() - n0 == 4
+    ref = oracle_prefill(x, cu, [128], s0, 256)
     tol = tol_for("bf16")
-    # outputs per (token, head) row as well as per head: from a zero state the first
-    # tokens' rows scale with q.k, and only an fp32-accurate decayed QK^T keeps them
-    # within the tolerance where that product nearly cancels
+    # outputs per (token, head) row as well as per head: the first tokens' rows scale
+    # with q.k, and only an fp32-accurate decayed QK^T keeps them within the tolerance
+    # where that product nearly cancels
     check_outputs("o", to_np(got[0]), ref[0], tol, cu)
     check_states("state", to_np(got[1]), ref[1], tol, (2, 3))
     check_states("snapshots", got[2].cpu().numpy(), ref[2], tol, (2, 3))
-    again = _run(K.kda_prefill, x, dev, cu, H, d, None, None, 256, workspace=None)
+    ws = torch.empty(need, dtype=torch.uint8, device=cuda_device)
+    again = _run(K.kda_prefill, x, dev, cu, H, d, [128], s0, 256, workspace=ws)
+    for a, b in zip(got, again):
+        assert torch.equal(a, b)
+
+
+@pytest.mark.gpu
+def test_ragged_batch_larger_than_scratch_in_pieces(cuda_device):
+    """A ragged 64-head batch whose packets exceed the scratch: short sequences grouped,
+    a long one in windows, zero-length and resumed sequences among them; the same bits as
+    kda_prefill with a full workspace (outputs, final states, snapshots)."""
+    lens, H, d = [130, 0, 1500, 64, 700, 1], 64, 128
+    x, dev, cu = packed_inputs(65, lens, H, d, "bf16", cuda_device)
+    need = K.kda_prefill_workspace_size(dev["q"], dev["v"], cu)
+    assert need > K.kda_prefill_noalloc_capacity()
+    start = [0, 64, 256, 0, 512, 0]
+    s0 = synth.states(66, len(lens), H, d, d, std=0.1)
+    got = _run(K.kda_prefill_noalloc, x, dev, cu, H, d, start, s0, 128)
+    ws = torch.empty(need, dtype=torch.uint8, device=cuda_device)
+    again = _run(K.kda_prefill, x, dev, cu, H, d, start, s0, 128, workspace=ws)
     for a, b in zip(got, again):
         assert torch.equal(a, b)
