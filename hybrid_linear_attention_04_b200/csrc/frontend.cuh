@@ -64,12 +64,13 @@ __device__ __forceinline__ void st_vec(TIO *p, const float (&x)[CPL], float s) {
 
 // One warp per (tile, head, q or k): the two tensors go through the same conv, Swish and
 // L2 norm independently, so each warp holds one tensor's weights and windows and keeps
-// G rows of loads in flight.
-template <int D, typename TIO>
+// G rows of loads in flight. The tap count K is a template parameter, so that the window's
+// shift through an unrolled row group is register renaming rather than moves.
+template <int D, typename TIO, int K>
 __global__ void __launch_bounds__(FrontendShape<D>::NT, 5) qk_frontend_kernel(const __grid_constant__ FrontendParams P) {
     using Sh = FrontendShape<D>;
     constexpr int CPL = Sh::CPL, G = Sh::G;
-    const int H = P.H, K = P.taps, C = P.C;
+    const int H = P.H, C = P.C;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t item = (int64_t)blockIdx.x * Sh::WARPS + warp;
     const int which = (int)(item & 1);                      // 0: q, 1: k

@@ -215,7 +215,12 @@ template <int D, typename TIO>
 static kda_status launch_frontend(const FrontendParams &P, int64_t n_items, cudaStream_t st) {
     using Sh = FrontendShape<D>;
     if (!launch_gate()) return KDA_ERR_CUDA;
-    qk_frontend_kernel<D, TIO><<<(unsigned)((n_items + Sh::WARPS - 1) / Sh::WARPS), Sh::NT, 0, st>>>(P);
+    const unsigned grid = (unsigned)((n_items + Sh::WARPS - 1) / Sh::WARPS);
+    switch (P.taps) {
+    case 2: qk_frontend_kernel<D, TIO, 2><<<grid, Sh::NT, 0, st>>>(P); break;
+    case 3: qk_frontend_kernel<D, TIO, 3><<<grid, Sh::NT, 0, st>>>(P); break;
+    default: qk_frontend_kernel<D, TIO, 4><<<grid, Sh::NT, 0, st>>>(P); break;
+    }
     return last_launch_status();
 }
 
