@@ -141,10 +141,12 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
         tc::bar_init(bar_a, 1);
         tc::bar_init(bar_b, 1);
         tc::bar_init_fence();
-        tc::tma_prefetch_desc(&P.tm_q);
-        tc::tma_prefetch_desc(&P.tm_k);
-        tc::tma_prefetch_desc(&P.tm_v);
-        tc::tma_prefetch_desc(&P.tm_g);
+        if (n_chunks > 0) {
+            tc::tma_prefetch_desc(&P.tm_q);
+            tc::tma_prefetch_desc(&P.tm_k);
+            tc::tma_prefetch_desc(&P.tm_v);
+            tc::tma_prefetch_desc(&P.tm_g);
+        }
     }
     if (warp == 0) {
         tc::tmem_alloc(tmem_slot, TMEM_COLS);
@@ -623,12 +625,15 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// [T, H, 128] tensor, boxes of (inner, 1 head, 64 tokens)
+// [T, H, 128] tensor, boxes of (inner, 1 head, 64 tokens). An empty or absent array gets
+// a zeroed map: a call without tokens has no chunk, so no launch reads it.
 inline bool encode_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint32_t esize, int H,
                        int64_t T, uint32_t box_inner, CUtensorMapSwizzle sw) {
+    std::memset(m, 0, sizeof(*m));
+    if (!base || T <= 0) return true;
     auto enc = tensor_map_encoder();
     if (!enc) return false;
-    cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)(T > 0 ? T : 1)};
+    cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)T};
     cuuint64_t strides[2] = {(cuuint64_t)128 * esize, (cuuint64_t)H * 128 * esize};
     cuuint32_t box[3] = {box_inner, 1, 64};
     cuuint32_t estr[3] = {1, 1, 1};
