@@ -659,6 +659,17 @@ __global__ void __launch_bounds__(256, 1) prefill_chain_kernel(const __grid_cons
             u[q4] = *reinterpret_cast<const uint4 *>(pkt + u_piece(half, wh, q4, r_w));
     };
     if (wwarp && n_chunks > 0) load_u(0);
+    // U of chunk ci into L2 two chunks ahead, so that the register loads of it (one chunk
+    // ahead, just before the end barrier) hit L2 rather than HBM: -6 % on the chain
+    auto prefetch_u = [&](int ci) {
+        if ((lane & 7) == 0) {
+            const uint8_t *pkt = packet(ci);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(pkt + u_piece(half, wh, q4, r_w)) : "memory");
+        }
+    };
+    if (wwarp && n_chunks > 1) prefetch_u(1);
 
     const uint64_t dSM = tc::desc_mn(sbase + C_SM, 0, 16384);
     const uint64_t dW = tc::desc_mn(sbase + C_W, 0, 8192);
@@ -732,6 +743,7 @@ __global__ void __launch_bounds__(256, 1) prefill_chain_kernel(const __grid_cons
             }
         }
         float ov[32];          // O of chunk ci - 1 (O warps)
+        if (wwarp && ci + 2 < n_chunks) prefetch_u(ci + 2);
         if (wwarp) {
             // ---- W = U - W' Sm (token rows in TMEM lanes 64-127)
             ok = tc::bar_wait(bar_r1, (uint32_t)(ci & 1));
