@@ -543,7 +543,7 @@ def bench_tiny(K, dev, steps, warmup):
     byts = prefill_bytes_general(c["T"], 1, 0, 0, io_bytes=4, d=c["d"], heads=c["H"])
     return {"ms": round(ms, 5), "value": round(ms * 1e3, 2), "unit": "us/call",
             "tok_per_s": c["T"] / (ms * 1e-3), "algorithmic_bytes": byts,
-            "bound": "launch latency", "launches_per_call": launches,
+            "bound": "latency (one CTA per head walks the chunks)", "launches_per_call": launches,
             "workload": "B=1, H=2, T=64, d=32, chunk 16, fp32 throughout, zero initial state"}
 
 

@@ -6,7 +6,12 @@
 // D x 32 fp32 state slice in shared memory across chunks. Per chunk it follows
 // the chunk form in prefill_common.cuh with exact pairwise decays
 // exp(b_rc - b_ic) (no reference-point factorisation, so no range condition
-// on the gates) and a forward substitution for the unit lower-triangular solve.
+// on the gates), taken as 2^x of the cumsum in log2 units, and a forward
+// substitution for the unit lower-triangular solve: one thread per d_v column with
+// the column in registers, each solved row subtracted from the rows below it.
+// Where a chunk's inputs are at most 16 values per thread and tensor, the next
+// chunk's loads are issued into registers before this chunk's arithmetic, so
+// their latency is hidden (the small shapes, whose chunks are latency-bound).
 #pragma once
 #include "prefill_common.cuh"
 
@@ -60,32 +65,74 @@ prefill_simt_kernel(const __grid_constant__ PrefillParams p) {
         S[e] = p.state_in ? p.state_in[(((int64_t)s * H + h) * D + c) * D + j0 + j] : 0.f;
     }
     int64_t snap_row = sq.snap_off;
+    constexpr float LOG2E = 1.4426950408889634f;
+
+    // inputs of chunk c0 into registers (element e = tid + NT u of the C x D and C x DVS
+    // tiles; rows >= n are zero: an identity token)
+    constexpr int PQ = C * D / NT, PV = C * DVS / NT;
+    constexpr bool PF = PQ <= 16;
+    float rq[PF ? PQ : 1], rk[PF ? PQ : 1], rg[PF ? PQ : 1], rv[PF ? PV : 1], rb = 0.f;
+    auto fetch = [&](int c0) {
+        const int n = min(C, sq.len - c0);
+#pragma unroll
+        for (int u = 0; u < (PF ? PQ : 0); ++u) {
+            const int e = tid + NT * u, r = e / D, c = e % D;
+            rq[u] = rk[u] = rg[u] = 0.f;
+            if (r < n) {
+                const int64_t off = ((int64_t)(sq.tok0 + c0 + r) * H + h) * D + c;
+                rq[u] = IO<TIO>::ld(qg + off);
+                rk[u] = IO<TIO>::ld(kg + off);
+                rg[u] = p.g[off];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < (PF ? PV : 0); ++u) {
+            const int e = tid + NT * u, r = e / DVS, j = e % DVS;
+            rv[u] = r < n ? IO<TIO>::ld(vg + ((int64_t)(sq.tok0 + c0 + r) * H + h) * D + j0 + j) : 0.f;
+        }
+        rb = tid < n ? p.beta[(int64_t)(sq.tok0 + c0 + tid) * H + h] : 0.f;
+    };
+    if (PF && sq.len > 0) fetch(0);
 
     for (int c0 = 0; c0 < sq.len; c0 += C) {
         const int n = min(C, sq.len - c0);
         __syncthreads();
-        // ---- load the chunk (rows >= n are zero: an identity token) ----
-        for (int e = tid; e < C * D; e += NT) {
-            const int r = e / D, c = e % D;
-            float qv = 0.f, kv = 0.f, gv = 0.f;
-            if (r < n) {
-                const int64_t off = ((int64_t)(sq.tok0 + c0 + r) * H + h) * D + c;
-                qv = IO<TIO>::ld(qg + off);
-                kv = IO<TIO>::ld(kg + off);
-                gv = p.g[off];
+        // ---- the chunk into shared memory (g in log2 units) ----
+        if (PF) {
+#pragma unroll
+            for (int u = 0; u < (PF ? PQ : 0); ++u) {
+                const int e = tid + NT * u, r = e / D, c = e % D;
+                Q[r * DP + c] = rq[u];
+                K[r * DP + c] = rk[u];
+                B[r * DP + c] = rg[u] * LOG2E;
             }
-            Q[r * DP + c] = qv;
-            K[r * DP + c] = kv;
-            B[r * DP + c] = gv;
+#pragma unroll
+            for (int u = 0; u < (PF ? PV : 0); ++u) V[tid + NT * u] = rv[u];
+            if (tid < C) bet[tid] = rb;
+            if (c0 + C < sq.len) fetch(c0 + C);      // lands while this chunk computes
+        } else {
+            for (int e = tid; e < C * D; e += NT) {
+                const int r = e / D, c = e % D;
+                float qv = 0.f, kv = 0.f, gv = 0.f;
+                if (r < n) {
+                    const int64_t off = ((int64_t)(sq.tok0 + c0 + r) * H + h) * D + c;
+                    qv = IO<TIO>::ld(qg + off);
+                    kv = IO<TIO>::ld(kg + off);
+                    gv = p.g[off];
+                }
+                Q[r * DP + c] = qv;
+                K[r * DP + c] = kv;
+                B[r * DP + c] = gv * LOG2E;
+            }
+            for (int e = tid; e < C * DVS; e += NT) {
+                const int r = e / DVS, j = e % DVS;
+                V[e] = r < n ? IO<TIO>::ld(vg + ((int64_t)(sq.tok0 + c0 + r) * H + h) * D + j0 + j) : 0.f;
+            }
+            for (int r = tid; r < C; r += NT)
+                bet[r] = r < n ? p.beta[(int64_t)(sq.tok0 + c0 + r) * H + h] : 0.f;
         }
-        for (int e = tid; e < C * DVS; e += NT) {
-            const int r = e / DVS, j = e % DVS;
-            V[e] = r < n ? IO<TIO>::ld(vg + ((int64_t)(sq.tok0 + c0 + r) * H + h) * D + j0 + j) : 0.f;
-        }
-        for (int r = tid; r < C; r += NT)
-            bet[r] = r < n ? p.beta[(int64_t)(sq.tok0 + c0 + r) * H + h] : 0.f;
         __syncthreads();
-        // ---- b = inclusive cumsum of g over the chunk, per channel ----
+        // ---- b = inclusive cumsum of g over the chunk, per channel (log2 units) ----
         for (int c = tid; c < D; c += NT) {
             float run = 0.f;
             for (int r = 0; r < C; ++r) {
@@ -93,7 +140,7 @@ prefill_simt_kernel(const __grid_constant__ PrefillParams p) {
                 B[r * DP + c] = run;
             }
             bC[c] = run;
-            gC[c] = expf(run);
+            gC[c] = tc::ex2(run);
         }
         __syncthreads();
         // ---- A_kk (scaled by beta_r) and A_qk with exact pairwise decays ----
@@ -102,7 +149,7 @@ prefill_simt_kernel(const __grid_constant__ PrefillParams p) {
             float kk = 0.f, qk = 0.f;
             if (i <= r) {
                 for (int c = 0; c < D; ++c) {
-                    const float ex = expf(B[r * DP + c] - B[i * DP + c]);
+                    const float ex = tc::ex2(B[r * DP + c] - B[i * DP + c]);
                     const float ki = K[i * DP + c] * ex;
                     kk = fmaf(K[r * DP + c], ki, kk);
                     qk = fmaf(Q[r * DP + c], ki, qk);
@@ -116,11 +163,11 @@ prefill_simt_kernel(const __grid_constant__ PrefillParams p) {
         for (int e = tid; e < C * D; e += NT) {
             const int r = e / D, c = e % D;
             const float b = B[r * DP + c];
-            const float ga = expf(b);
+            const float ga = tc::ex2(b);
             const float kv = K[r * DP + c];
             Q[r * DP + c] *= ga;
             K[r * DP + c] = kv * ga;
-            B[r * DP + c] = kv * expf(bC[c] - b);
+            B[r * DP + c] = kv * tc::ex2(bC[c] - b);
         }
         __syncthreads();
         // ---- right-hand side: beta (V - (K . Gamma) S_0) ----
@@ -131,18 +178,18 @@ prefill_simt_kernel(const __grid_constant__ PrefillParams p) {
             W[e] = bet[r] * (V[e] - acc);
         }
         __syncthreads();
-        // ---- forward substitution: W <- (I + Diag(beta) A_kk)^{-1} W ----
-        {
-            const int j = tid >> 3, part = tid & 7;
-            for (int r = 1; r < C; ++r) {
-                float acc = 0.f;
-                for (int i = part; i < r; i += 8) acc = fmaf(Akk[r * CP + i], W[i * DVS + j], acc);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-                if (part == 0) W[r * DVS + j] -= acc;
-                __syncwarp();
-            }
+        // ---- forward substitution: W <- (I + Diag(beta) A_kk)^{-1} W, one thread per
+        // column: row i, once solved, is subtracted from every row below it ----
+        if (tid < DVS) {
+            float w[C];
+#pragma unroll
+            for (int r = 0; r < C; ++r) w[r] = W[r * DVS + tid];
+#pragma unroll
+            for (int i = 0; i < C - 1; ++i)
+#pragma unroll
+                for (int r = i + 1; r < C; ++r) w[r] = fmaf(-Akk[r * CP + i], w[i], w[r]);
+#pragma unroll
+            for (int r = 0; r < C; ++r) W[r * DVS + tid] = w[r];
         }
         __syncthreads();
         // ---- outputs: scale [ (Q . Gamma) S_0 + A_qk W ] ----
