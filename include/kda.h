@@ -153,7 +153,8 @@ kda_status kda_prefill_workspace_size(const kda_dims *dims, int32_t n_seq,
  *               that keeps every intermediate on chip. Results agree to
  *               rounding, not bit for bit, between the two. The workspace must
  *               not be used by other work until the call's kernels finish.
- * A zero-length sequence writes state_out = state_in and no snapshots.
+ * A zero-length sequence writes state_out = state_in and no snapshots; in a call
+ * without tokens (cu_seqlens all zero) q, k, v, g, beta and o may be NULL.
  * Errors (before launch): KDA_ERR_INVALID, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGN,
  * KDA_ERR_WORKSPACE (non-null workspace below kda_prefill_workspace_size).
  * Gate range on the tensor-core path: with b_r = g_0 + ... + g_r summed over a
