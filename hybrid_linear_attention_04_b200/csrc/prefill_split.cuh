@@ -727,8 +727,7 @@ __global__ void __launch_bounds__(256, 1) prefill_chain_kernel(const __grid_cons
         const uint32_t sstg = sbase + st * STAGE;
         const uint32_t col_r1 = C_COL_R1 + 64 * (ci & 1);
         const float *eC = reinterpret_cast<const float *>(stg + PK_VEC) + 128, *gC = eC + 128;
-        // ---- round 1: [Qh; W'] Sm -> rows 0-63 O, rows 64-127 W'Sm; then the loads of
-        // chunk ci + NSTAGE - 1 (its stage was released at the end of chunk ci - 1)
+        // ---- round 1: [Qh; W'] Sm -> rows 0-63 O, rows 64-127 W'Sm
         if (tid == 0) {
             tc::fence_after_sync();
             constexpr uint32_t id1 = tc::idesc_bf16(128, 64, false, true);
@@ -737,10 +736,6 @@ __global__ void __launch_bounds__(256, 1) prefill_chain_kernel(const __grid_cons
             for (int k = 0; k < 8; ++k)
                 tc::mma_bf16(tbase + col_r1, dQW + (k >> 2) * 1024 + (k & 3) * 2, dSM + 128 * k, id1, k > 0);
             tc::mma_commit(bar_r1);
-            if (issued < n_chunks) {
-                issue_loads(issued);
-                ++issued;
-            }
         }
         float ov[32];          // O of chunk ci - 1 (O warps)
         if (wwarp && ci + 2 < n_chunks) prefetch_u(ci + 2);
@@ -810,9 +805,13 @@ __global__ void __launch_bounds__(256, 1) prefill_chain_kernel(const __grid_cons
             }
         }
         tc::fence_before_sync();
-        __syncthreads();
+        const bool mid_ok = __syncthreads_and(ok);
         // ---- round 2: D = Kb^T W (commit bar_d), then O += A_qk W (M=128; A rows 64-127 are
-        // the bytes after A_qk and land in TMEM lanes 64-127, not read again; commit bar_o)
+        // the bytes after A_qk and land in TMEM lanes 64-127, not read again; commit bar_o);
+        // then the loads of chunk ci + NSTAGE - 1 into the stage of chunk ci - 1. Its last
+        // readers were that chunk's MMAs, which completed before this chunk's round 1 did
+        // (one thread issues every MMA, and a commit covers all earlier ones), and the W warps
+        // saw round 1 complete before the barrier above.
         if (tid == 0) {
             tc::fence_after_sync();
             constexpr uint32_t id_o = tc::idesc_bf16(128, 64, false, true);
@@ -825,6 +824,10 @@ __global__ void __launch_bounds__(256, 1) prefill_chain_kernel(const __grid_cons
 #pragma unroll
             for (int k = 0; k < 4; ++k) tc::mma_bf16(tbase + col_r1, dAQK + 2 * k, dW + 128 * k, id_o, 1);
             tc::mma_commit(bar_o);
+            if (mid_ok && issued < n_chunks) {
+                issue_loads(issued);
+                ++issued;
+            }
         }
         // ---- while this chunk's MMAs run: the W warps send half 1 of a pending snapshot
         if (wwarp && snap_pend >= 0 && snap_half == 1) {
