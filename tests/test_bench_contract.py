@@ -51,3 +51,23 @@ def test_algorithmic_bytes_per_unit():
     assert bench.decode_bytes(1) == H * (2 * D * D * 4 + 1540)
     assert bench.verify_bytes(2, 5) == 2 * state + 5 * H * (D * D * 4 + 1540)
     assert bench.commit_bytes(3) == 3 * 2 * state
+
+
+def test_end_to_end_windows_cover_the_call_and_its_snapshot_rows():
+    """The end-to-end leg runs the 8192-token prefill as windows with start positions: the
+    windows tile the call, and each window's snapshot rows (the host plan with its start
+    position) are the slice of the whole call's rows that the bench hands it."""
+    import numpy as np
+    from hybrid_linear_attention_04_b200 import kda as K
+    T, W, snap = bench.PREFILL_T, bench.E2E_WIN, bench.SNAP
+    assert W % snap == 0 and W % 64 == 0
+    offs, pos = K.kda_snapshot_plan(np.array([0, T], np.int32), None, snap)
+    wins = [(a, min(T, a + W)) for a in range(0, T, W)]
+    assert wins[0][0] == 0 and wins[-1][1] == T
+    assert all(b == c for (_, b), (c, _) in zip(wins, wins[1:]))
+    rows = []
+    for a, b in wins:
+        o, p = K.kda_snapshot_plan(np.array([0, b - a], np.int32), np.array([a], np.int64), snap)
+        assert list(p) == list(pos[a // snap:b // snap])
+        rows += list(range(a // snap, a // snap + int(o[-1])))
+    assert rows == list(range(int(offs[-1])))
