@@ -132,7 +132,8 @@ def _host_array(x, dtype):
 
 
 def _hptr(a):
-    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+    # the caller keeps `a` alive for the duration of the library call
+    return None if a is None else ctypes.c_void_p(a.ctypes.data)
 
 
 def _io(t):
@@ -159,29 +160,33 @@ def _expect(t, name, dtype, rows, tail, required=True):
         if required and rows > 0:
             raise KDAError(1, f"{name} is required")
         return
-    if not isinstance(t, torch.Tensor):
-        raise KDAError(1, f"{name} must be a tensor")
-    if t.dtype != dtype:
-        raise KDAError(1, f"{name} must be {dtype}, not {t.dtype}")
-    if t.dim() != 1 + len(tail) or tuple(t.shape[1:]) != tuple(tail):
-        raise KDAError(1, f"{name} must be shaped [n, {', '.join(map(str, tail))}], not {list(t.shape)}")
-    if t.shape[0] < rows:
-        raise KDAError(1, f"{name} has {t.shape[0]} rows; the call uses {rows}")
+    try:
+        shape, dt = t.shape, t.dtype
+    except AttributeError:
+        raise KDAError(1, f"{name} must be a tensor") from None
+    if dt is not dtype or len(shape) != len(tail) + 1 or shape[1:] != tail or shape[0] < rows:
+        if dt is not dtype:
+            raise KDAError(1, f"{name} must be {dtype}, not {dt}")
+        if len(shape) != len(tail) + 1 or shape[1:] != tail:
+            raise KDAError(1, f"{name} must be shaped [n, {', '.join(map(str, tail))}], not {list(shape)}")
+        raise KDAError(1, f"{name} has {shape[0]} rows; the call uses {rows}")
 
 
 def _expect_tokens(q, k, v, g, beta, o, T, tag=""):
     """Packed token arrays of T rows: q, k [T, H, dk] and v, o [T, H, dv] in q's I/O type,
     g [T, H, dk] and beta [T, H] fp32 (o may be None where the call writes none)."""
     _io(q)
+    io = q.dtype
     H, dk = q.shape[-2], q.shape[-1]
     dv = v.shape[-1] if v is not None else dk
-    _expect(q, tag + "q", q.dtype, T, (H, dk))
-    _expect(k, tag + "k", q.dtype, T, (H, dk))
-    _expect(v, tag + "v", q.dtype, T, (H, dv))
-    _expect(g, tag + "g", _F32, T, (H, dk))
+    hk, hv = (H, dk), (H, dv)
+    _expect(q, tag + "q", io, T, hk)
+    _expect(k, tag + "k", io, T, hk)
+    _expect(v, tag + "v", io, T, hv)
+    _expect(g, tag + "g", _F32, T, hk)
     _expect(beta, tag + "beta", _F32, T, (H,))
     if o is not None:
-        _expect(o, tag + "o", q.dtype, T, (H, dv))
+        _expect(o, tag + "o", io, T, hv)
     return H, dk, dv
 
 
