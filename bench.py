@@ -537,11 +537,31 @@ def bench_tiny(K, dev, steps, warmup):
     K.kda_prefill(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], cu, o, state_out=so,
                   chunk=c["chunk"], workspace=None)
     launches = K.kda_launch_count() - n0
-    ms = time_calls(lambda: K.kda_prefill(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], cu, o,
-                                          state_out=so, chunk=c["chunk"], workspace=None),
-                    steps, warmup, dev)
+    def call():
+        K.kda_prefill(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], cu, o, state_out=so,
+                      chunk=c["chunk"], workspace=None)
+    ms = time_calls(call, steps, warmup, dev)
+    # the same call captured once in a CUDA graph and replayed: the device time per call
+    # without the host's per-call work (argument checks, marshalling, launch)
+    graph_us = None
+    try:
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            call()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(10):
+                call()
+        graph_us = round(time_calls(graph.replay, max(3, steps // 10), warmup, dev) * 1e2, 2)
+        del graph
+    except Exception:                 # graph capture unavailable: report the eager time only
+        graph_us = None
     byts = prefill_bytes_general(c["T"], 1, 0, 0, io_bytes=4, d=c["d"], heads=c["H"])
     return {"ms": round(ms, 5), "value": round(ms * 1e3, 2), "unit": "us/call",
+            "graph_replay_us_per_call": graph_us,
             "tok_per_s": c["T"] / (ms * 1e-3), "algorithmic_bytes": byts,
             "bound": "latency (one CTA per head walks the chunks)", "launches_per_call": launches,
             "workload": "B=1, H=2, T=64, d=32, chunk 16, fp32 throughout, zero initial state"}
@@ -731,16 +751,10 @@ def run_workload(args):
         n = K.kda_prefill_workspace_size(xd["q"], xd["v"], cu, C)
         return torch.empty(n, dtype=torch.uint8, device=dev) if n else None
     if args.workload == "tiny":
-        c = wl["tiny_fp32"]
-        x = synth.token_inputs(c["seed"], c["T"], c["H"], c["d"], c["d"], io="fp32")
-        xd = {k: v.to(dev) for k, v in x.items()}
-        o = torch.empty_like(xd["v"])
-        so = torch.empty((1, c["H"], c["d"], c["d"]), device=dev)
-        cu = np.array([0, c["T"]], dtype=np.int32)
-        ms = time_calls(lambda: K.kda_prefill(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], cu, o,
-                                              state_out=so, chunk=c["chunk"], workspace=None),
-                        args.steps, args.warmup, dev)
-        out.update({"unit": "us/call", "value": ms * 1e3, "tokens": c["T"]})
+        r = bench_tiny(K, dev, args.steps, args.warmup)
+        out.update({"unit": "us/call", "value": r["value"],
+                    "graph_replay_us_per_call": r["graph_replay_us_per_call"],
+                    "tokens": wl["tiny_fp32"]["T"]})
     elif args.workload == "ragged":
         c = wl["ragged_prefix_32"]
         plan = synth.ragged_plan(c["seed"], c["n_seq"], c["mu"], c["sigma"], c["lo"], c["hi"],
